@@ -1,0 +1,320 @@
+"""CPU oracle for the ResidualQuant KV-cache hot path.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only
+callers.  The product library (``librq``) never imports, links or executes
+anything here, and this package imports nothing from the product.
+
+The arithmetic lives in plain C (``rqo.c``, single-threaded, built with
+``-ffp-contract=off``); this module only marshals numpy arrays.  Citations
+``[RQ §x]`` refer to "ResidualQuant: KV Cache Quantization for Looped
+Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+
+Array conventions (all C-contiguous):
+  x      uint16 bf16 bits, [L, N, D]: loop l, row n (rows are (b, h, t) in
+         that nesting order), channel d.  Loop L-1 is the final-loop anchor.
+  codes  uint32 [N, D*bits/32]; meta uint32 [N, D/group] (fp16 scale in the
+         low half, fp16 offset in the high half); alpha uint16 [N] (bf16).
+
+Parity unpinned: nothing here is pinned against learned rotations, real
+model KV, or the pages' accuracy / NMSE / throughput numbers; the pins are
+closed forms, invariants, brute force and the pages' storage accounting.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rqo.c")
+_LIB_PATH = os.path.join(_HERE, "librqo.so")
+
+POLICY_LAST = "last"   # shared anchor at the final loop [RQ §3.2]
+POLICY_NEXT = "next"   # chain toward the final loop [RQ §5.2 "Next-loop"]
+
+GCC_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+             "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile rqo.c into librqo.so next to it (gcc, no fused multiply-add)."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(_SRC),
+                                                  os.path.getmtime(os.path.join(_HERE, "rqo.h"))))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_D = ctypes.c_double
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        h = ctypes.CDLL(build())
+        sig = {
+            "rqo_bf16_to_f32": ([ctypes.c_uint16], _F),
+            "rqo_f32_to_bf16": ([_F], ctypes.c_uint16),
+            "rqo_f16_to_f32": ([ctypes.c_uint16], _F),
+            "rqo_f32_to_f16": ([_F], ctypes.c_uint16),
+            "rqo_rot_scale": ([_I], _F),
+            "rqo_fwht_f32": ([_P, _I], None),
+            "rqo_fwht_f64": ([_P, _I], None),
+            "rqo_fwht_rows_f64": ([_P, _I64, _I], None),
+            "rqo_dot_f32": ([_P, _P, _I], _F),
+            "rqo_quantize": ([_P, _I, _I, _I, _P, _P, _P], None),
+            "rqo_encode_anchor": ([_P, _I, _I, _I, _P, _P, _P], None),
+            "rqo_encode_residual_rot": ([_P, _P, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_residual": ([_P, _P, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_anchor_rows": ([_P, _I64, _I, _I, _I, _P, _P, _P], None),
+            "rqo_encode_residual_rows": ([_P, _P, _I64, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_dequant_codes_f64": ([_P, _P, _I, _I, _I, _P], None),
+            "rqo_dequant_rows_f64": ([_P, _P, _I64, _I, _I, _I, _P], None),
+            "rqo_attention_f64": ([_P, _P, _P, _I64, _P, _P, _I, _D, _P], None),
+            "rqo_effective_bits": ([_I, _P, _P, _I, _I, _I], _D),
+            "rqo_component_reads": ([_I, _I], _I64),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(h, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = h
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+# --------------------------------------------------------------------------
+# Scalar / row-level entry points (used by the pins)
+# --------------------------------------------------------------------------
+
+def f32_to_f16_bits(v: float) -> int:
+    return int(lib().rqo_f32_to_f16(float(v)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(lib().rqo_f16_to_f32(int(h)))
+
+
+def f32_to_bf16_bits(v: float) -> int:
+    return int(lib().rqo_f32_to_bf16(float(v)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(lib().rqo_bf16_to_f32(int(h)))
+
+
+def rot_scale(D: int) -> float:
+    return float(lib().rqo_rot_scale(D))
+
+
+def fwht_f32(z: np.ndarray) -> np.ndarray:
+    """Normalised Hadamard transform of each row of z (fp32, canonical order)."""
+    z = np.array(z, dtype=np.float32, order="C", copy=True)
+    D = z.shape[-1]
+    flat = z.reshape(-1, D)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        lib().rqo_fwht_f32(_ptr(row), D)
+        flat[r] = row
+    return flat.reshape(z.shape)
+
+
+def fwht_f64(z: np.ndarray) -> np.ndarray:
+    z = np.array(z, dtype=np.float64, order="C", copy=True)
+    D = z.shape[-1]
+    n = z.size // D
+    lib().rqo_fwht_rows_f64(_ptr(z), n, D)
+    return z
+
+
+def dot_f32(a: np.ndarray, b: np.ndarray) -> float:
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    b = np.ascontiguousarray(b, dtype=np.float32)
+    return float(lib().rqo_dot_f32(_ptr(a), _ptr(b), a.shape[-1]))
+
+
+def quantize(z: np.ndarray, bits: int, group: int):
+    """Affine-quantise one rotated fp32 row: (words, meta, deq)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    D = z.shape[-1]
+    words = np.zeros(D * bits // 32, np.uint32)
+    meta = np.zeros(D // group, np.uint32)
+    deq = np.zeros(D, np.float32)
+    lib().rqo_quantize(_ptr(z), D, bits, group, _ptr(words), _ptr(meta), _ptr(deq))
+    return words, meta, deq
+
+
+def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int):
+    """Residual encoder on an already-rotated fp32 row: (words, meta, alpha_bits, zhat)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    ref = np.ascontiguousarray(ref, dtype=np.float32)
+    D = z.shape[-1]
+    words = np.zeros(D * bits // 32, np.uint32)
+    meta = np.zeros(D // group, np.uint32)
+    alpha = np.zeros(1, np.uint16)
+    zhat = np.zeros(D, np.float32)
+    lib().rqo_encode_residual_rot(_ptr(z), _ptr(ref), D, bits, group, _ptr(words),
+                                  _ptr(meta), _ptr(alpha), _ptr(zhat))
+    return words, meta, int(alpha[0]), zhat
+
+
+def unpack_codes(words: np.ndarray, bits: int, D: int) -> np.ndarray:
+    """Codes of packed rows [..., D*bits/32] -> [..., D] (uint8)."""
+    per_word = 32 // bits
+    w = np.asarray(words, dtype=np.uint32)
+    idx = np.arange(D)
+    sh = (bits * (idx % per_word)).astype(np.uint32)
+    return ((w[..., idx // per_word] >> sh) & np.uint32((1 << bits) - 1)).astype(np.uint8)
+
+
+def meta_scale_zero(meta: np.ndarray):
+    """fp16 (scale, offset) of packed metadata words, as float32 arrays."""
+    m = np.asarray(meta, dtype=np.uint32)
+    s = (m & 0xFFFF).astype(np.uint16).view(np.float16).astype(np.float32)
+    z = (m >> 16).astype(np.uint16).view(np.float16).astype(np.float32)
+    return s, z
+
+
+# --------------------------------------------------------------------------
+# Layer-side encoder
+# --------------------------------------------------------------------------
+
+def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
+                policy: str = POLICY_LAST) -> List[Dict[str, np.ndarray]]:
+    """Encode every loop of one (layer, K|V) side.
+
+    x: uint16 [L, N, D].  Returns per loop l a dict with 'codes', 'meta',
+    'alpha' (None for the anchor) and 'zhat' (fp32 reconstructed rotated row,
+    the value a chained predecessor references).
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    L, N, D = x.shape
+    out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
+    a = L - 1
+    enc = {"codes": np.zeros((N, D * bits[a] // 32), np.uint32),
+           "meta": np.zeros((N, D // group[a]), np.uint32),
+           "alpha": None,
+           "zhat": np.zeros((N, D), np.float32)}
+    lib().rqo_encode_anchor_rows(_ptr(x[a]), N, D, bits[a], group[a], _ptr(enc["codes"]),
+                                 _ptr(enc["meta"]), _ptr(enc["zhat"]))
+    out[a] = enc
+    order = range(L - 2, -1, -1)
+    for r in order:
+        ref = out[a]["zhat"] if policy == POLICY_LAST else out[r + 1]["zhat"]
+        enc = {"codes": np.zeros((N, D * bits[r] // 32), np.uint32),
+               "meta": np.zeros((N, D // group[r]), np.uint32),
+               "alpha": np.zeros(N, np.uint16),
+               "zhat": np.zeros((N, D), np.float32)}
+        lib().rqo_encode_residual_rows(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D,
+                                       bits[r], group[r], _ptr(enc["codes"]),
+                                       _ptr(enc["meta"]), _ptr(enc["alpha"]),
+                                       _ptr(enc["zhat"]))
+        out[r] = enc
+    return out  # type: ignore[return-value]
+
+
+def _levels_f64(enc: Dict[str, np.ndarray], bits: int, group: int, D: int) -> np.ndarray:
+    N = enc["codes"].shape[0]
+    out = np.zeros((N, D), np.float64)
+    lib().rqo_dequant_rows_f64(_ptr(enc["codes"]), _ptr(enc["meta"]), N, D, bits, group,
+                               _ptr(out))
+    return out
+
+
+def reconstruct_rotated(encs: List[Dict[str, np.ndarray]], loop: int, bits: Sequence[int],
+                        group: Sequence[int], policy: str = POLICY_LAST) -> np.ndarray:
+    """fp64 rotated reconstruction Z^_loop [RQ App. G.2]:
+    Z^_anchor = A; Z^_r = alpha~_r * Z^_ref + D(c_r), ref = anchor (Last-loop)
+    or Z^_{r+1} (Next-loop chain)."""
+    L = len(encs)
+    D = encs[L - 1]["zhat"].shape[1]
+    a = L - 1
+    zA = _levels_f64(encs[a], bits[a], group[a], D)
+    if loop == a:
+        return zA
+    if policy == POLICY_LAST:
+        al = encs[loop]["alpha"].astype(np.uint32) << 16
+        al = al.view(np.float32).astype(np.float64)[:, None]
+        return al * zA + _levels_f64(encs[loop], bits[loop], group[loop], D)
+    z = zA
+    for r in range(a - 1, loop - 1, -1):
+        al = (encs[r]["alpha"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        z = al[:, None] * z + _levels_f64(encs[r], bits[r], group[r], D)
+    return z
+
+
+def reconstruct(encs, loop, bits, group, policy=POLICY_LAST) -> np.ndarray:
+    """fp64 reconstruction in the original domain: X^ = H^T Z^ (H symmetric)."""
+    return fwht_f64(reconstruct_rotated(encs, loop, bits, group, policy))
+
+
+def attention(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, kcur: np.ndarray,
+              vcur: np.ndarray, scale: float) -> np.ndarray:
+    """fp64 softmax attention of one query over T past rows plus the current token."""
+    q = np.ascontiguousarray(q, np.float64)
+    khat = np.ascontiguousarray(khat, np.float64)
+    vhat = np.ascontiguousarray(vhat, np.float64)
+    kcur = np.ascontiguousarray(kcur, np.float64)
+    vcur = np.ascontiguousarray(vcur, np.float64)
+    D = q.shape[-1]
+    T = khat.shape[0]
+    out = np.zeros(D, np.float64)
+    lib().rqo_attention_f64(_ptr(q), _ptr(khat), _ptr(vhat), T, _ptr(kcur), _ptr(vcur), D,
+                            float(scale), _ptr(out))
+    return out
+
+
+def bf16_bits_to_f64(a: np.ndarray) -> np.ndarray:
+    return (np.asarray(a, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def decode_attention(khat: np.ndarray, vhat: np.ndarray, q_bits: np.ndarray,
+                     seq_lens: Sequence[int], kcur_bits: np.ndarray, vcur_bits: np.ndarray,
+                     scale: Optional[float] = None) -> np.ndarray:
+    """fp64 decode attention for one loop [RQ §4.2 Decode].
+
+    khat, vhat: fp64 [B, H, T, D] reconstructed past keys / values (original
+    domain); q_bits, kcur_bits, vcur_bits: bf16 bits [B, H, D]; seq_lens[b]
+    past tokens of sequence b.  Returns fp64 [B, H, D]."""
+    B, H, T, D = khat.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    q = bf16_bits_to_f64(q_bits)
+    kc = bf16_bits_to_f64(kcur_bits)
+    vc = bf16_bits_to_f64(vcur_bits)
+    out = np.zeros((B, H, D), np.float64)
+    for b in range(B):
+        n = int(seq_lens[b])
+        for h in range(H):
+            out[b, h] = attention(q[b, h], khat[b, h, :n], vhat[b, h, :n], kc[b, h], vc[b, h],
+                                  scale)
+    return out
+
+
+def effective_bits(bits: Sequence[int], group: Sequence[int], D: int, meta_bits: int,
+                   residual: bool) -> float:
+    L = len(bits)
+    b = np.ascontiguousarray(bits, np.int32)
+    g = np.ascontiguousarray(group, np.int32)
+    return float(lib().rqo_effective_bits(L, _ptr(b), _ptr(g), D, meta_bits, int(residual)))
+
+
+def component_reads(L: int, chained: bool) -> int:
+    return int(lib().rqo_component_reads(L, int(chained)))

@@ -1,0 +1,317 @@
+/*
+ * rqo.c -- CPU oracle for the ResidualQuant KV-cache hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY (see rqo.h).  Plain scalar loops, one row at a
+ * time, in the order the method states them.  Build with
+ *   gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * so that no multiply-add is fused except the explicit fmaf() calls.
+ *
+ * Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
+ * Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+ */
+#include "rqo.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Number formats                                                           */
+/* ------------------------------------------------------------------------ */
+
+float rqo_bf16_to_f32(uint16_t h) {
+  /* bfloat16 is the upper half of an IEEE binary32. */
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+uint16_t rqo_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u); /* NaN stays NaN */
+  /* Drop the low 16 bits, rounding to nearest with ties to even. */
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+float rqo_f16_to_f32(uint16_t h) {
+  /* binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+  int sign = h >> 15;
+  int e = (h >> 10) & 0x1F;
+  int m = h & 0x3FF;
+  float v;
+  if (e == 0)
+    v = ldexpf((float)m, -24);                 /* subnormal: m * 2^-24 */
+  else if (e == 31)
+    v = m ? NAN : INFINITY;
+  else
+    v = ldexpf((float)(m + 1024), e - 25);     /* (1 + m/1024) * 2^(e-15) */
+  return sign ? -v : v;
+}
+
+uint16_t rqo_f32_to_f16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  float a = fabsf(f);
+  if (isnan(a)) return sign | 0x7E00u;
+  if (isinf(a)) return sign | 0x7C00u;
+  if (a < 0x1p-14f) {
+    /* Subnormal range: the unit in the last place is 2^-24.  a * 2^24 is an
+     * exact power-of-two scaling; rintf rounds half to even.  A result of
+     * 1024 is exactly the encoding of the smallest normal, 2^-14. */
+    float m = rintf(a * 0x1p24f);
+    return sign | (uint16_t)m;
+  }
+  int e;
+  (void)frexpf(a, &e);       /* a in [2^(e-1), 2^e) */
+  e -= 1;                    /* a in [2^e, 2^(e+1)), ulp = 2^(e-10) */
+  float m = rintf(ldexpf(a, 10 - e));   /* in [1024, 2048] */
+  if (m == 2048.0f) {
+    m = 1024.0f;
+    e += 1;
+  }
+  if (e > 15) return sign | 0x7C00u;   /* overflow rounds to infinity */
+  return sign | (uint16_t)((e + 15) << 10) | (uint16_t)(m - 1024.0f);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rotation: normalised Sylvester-Hadamard [RQ §3.3, App. G.1, App. G.2]     */
+/* ------------------------------------------------------------------------ */
+
+float rqo_rot_scale(int D) { return (float)(1.0 / sqrt((double)D)); }
+
+void rqo_fwht_f32(float* z, int D) {
+  for (int h = 1; h < D; h *= 2)
+    for (int i = 0; i < D; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        float a = z[j], b = z[j + h];
+        z[j] = a + b;
+        z[j + h] = a - b;
+      }
+  const float c = rqo_rot_scale(D);
+  for (int i = 0; i < D; ++i) z[i] = z[i] * c;
+}
+
+void rqo_fwht_f64(double* z, int D) {
+  for (int h = 1; h < D; h *= 2)
+    for (int i = 0; i < D; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        double a = z[j], b = z[j + h];
+        z[j] = a + b;
+        z[j + h] = a - b;
+      }
+  const double c = 1.0 / sqrt((double)D);
+  for (int i = 0; i < D; ++i) z[i] *= c;
+}
+
+void rqo_fwht_rows_f64(double* z, int64_t n, int D) {
+  for (int64_t r = 0; r < n; ++r) rqo_fwht_f64(z + r * D, D);
+}
+
+/* ------------------------------------------------------------------------ */
+/* LS coefficient dot product in its canonical order                        */
+/* ------------------------------------------------------------------------ */
+
+float rqo_dot_f32(const float* a, const float* b, int D) {
+  float p[8];
+  const int P = D / 32;
+  for (int l = 0; l < P; ++l) {
+    float acc = 0.0f;
+    for (int k = 0; k < 32; ++k) acc = fmaf(a[32 * l + k], b[32 * l + k], acc);
+    p[l] = acc;
+  }
+  for (int off = P / 2; off >= 1; off /= 2) {
+    float q[8];
+    for (int l = 0; l < P; ++l) q[l] = p[l] + p[l ^ off];
+    for (int l = 0; l < P; ++l) p[l] = q[l];
+  }
+  return p[0];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group-wise affine quantisation [RQ §2.1]                                  */
+/* ------------------------------------------------------------------------ */
+
+void rqo_quantize(const float* z, int D, int bits, int group, uint32_t* words,
+                  uint32_t* meta, float* deq) {
+  const int qmax = (1 << bits) - 1;
+  const int per_word = 32 / bits;
+  for (int w = 0; w < D * bits / 32; ++w) words[w] = 0u;
+
+  for (int g0 = 0, j = 0; g0 < D; g0 += group, ++j) {
+    /* Range of the group. */
+    float mn = z[g0], mx = z[g0];
+    for (int i = g0 + 1; i < g0 + group; ++i) {
+      if (z[i] < mn) mn = z[i];
+      if (z[i] > mx) mx = z[i];
+    }
+    mn = mn + 0.0f; /* a zero range end is taken as +0 */
+    mx = mx + 0.0f;
+
+    /* Scale and offset, stored as fp16; levels are z~ + k s~, k = 0..qmax. */
+    const float s = (mx - mn) / (float)qmax;
+    const uint16_t sh = rqo_f32_to_f16(s);
+    const uint16_t zh = rqo_f32_to_f16(mn);
+    const float st = rqo_f16_to_f32(sh);
+    const float zt = rqo_f16_to_f32(zh);
+    const float inv = (st > 0.0f) ? 1.0f / st : 0.0f;
+    meta[j] = (uint32_t)sh | ((uint32_t)zh << 16);
+
+    /* Nearest level: round half to even, clamped to the code range. */
+    for (int i = g0; i < g0 + group; ++i) {
+      float u = (z[i] - zt) * inv;
+      if (u < 0.0f) u = 0.0f;
+      if (u > (float)qmax) u = (float)qmax;
+      const uint32_t code = (uint32_t)rintf(u);
+      words[i / per_word] |= code << (bits * (i % per_word));
+      deq[i] = fmaf(st, (float)code, zt);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Anchor and residual encoders [RQ §3.2, §3.3, §3.4, App. G.1, App. G.2]    */
+/* ------------------------------------------------------------------------ */
+
+void rqo_encode_anchor(const uint16_t* x, int D, int bits, int group,
+                       uint32_t* words, uint32_t* meta, float* zhat) {
+  float z[256];
+  for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[i]);
+  rqo_fwht_f32(z, D);
+  rqo_quantize(z, D, bits, group, words, meta, zhat);
+}
+
+void rqo_encode_residual_rot(const float* z, const float* ref, int D, int bits,
+                             int group, uint32_t* words, uint32_t* meta,
+                             uint16_t* alpha, float* zhat) {
+  /* Least-squares scale of the reference: alpha = <X_r, R>/||R||^2. */
+  const float d_zr = rqo_dot_f32(z, ref, D);
+  const float d_rr = rqo_dot_f32(ref, ref, D);
+  const float a = (d_rr > 0.0f) ? d_zr / d_rr : 0.0f;
+  const uint16_t ab = rqo_f32_to_bf16(a);
+  const float at = rqo_bf16_to_f32(ab);
+  *alpha = ab;
+
+  /* Residual against the stored (bf16) coefficient, then affine quantise. */
+  float e[256], deq[256];
+  for (int i = 0; i < D; ++i) e[i] = fmaf(-at, ref[i], z[i]);
+  rqo_quantize(e, D, bits, group, words, meta, deq);
+
+  /* Reconstructed rotated row (the reference of a chained predecessor). */
+  for (int i = 0; i < D; ++i) zhat[i] = fmaf(at, ref[i], deq[i]);
+}
+
+void rqo_encode_residual(const uint16_t* x, const float* ref, int D, int bits,
+                         int group, uint32_t* words, uint32_t* meta,
+                         uint16_t* alpha, float* zhat) {
+  float z[256];
+  for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[i]);
+  rqo_fwht_f32(z, D);
+  rqo_encode_residual_rot(z, ref, D, bits, group, words, meta, alpha, zhat);
+}
+
+void rqo_encode_anchor_rows(const uint16_t* x, int64_t n, int D, int bits,
+                            int group, uint32_t* words, uint32_t* meta,
+                            float* zhat) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r)
+    rqo_encode_anchor(x + r * D, D, bits, group, words + r * W, meta + r * G,
+                      zhat + r * D);
+}
+
+void rqo_encode_residual_rows(const uint16_t* x, const float* ref, int64_t n,
+                              int D, int bits, int group, uint32_t* words,
+                              uint32_t* meta, uint16_t* alpha, float* zhat) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r)
+    rqo_encode_residual(x + r * D, ref + r * D, D, bits, group, words + r * W,
+                        meta + r * G, alpha + r, zhat + r * D);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Reconstruction and attention in fp64 [RQ §4.1, App. G.2]                  */
+/* ------------------------------------------------------------------------ */
+
+void rqo_dequant_codes_f64(const uint32_t* words, const uint32_t* meta, int D,
+                           int bits, int group, double* out) {
+  const uint32_t qmax = (1u << bits) - 1u;
+  const int per_word = 32 / bits;
+  for (int i = 0; i < D; ++i) {
+    const uint32_t code = (words[i / per_word] >> (bits * (i % per_word))) & qmax;
+    const uint32_t m = meta[i / group];
+    const double s = rqo_f16_to_f32((uint16_t)(m & 0xFFFFu));
+    const double z = rqo_f16_to_f32((uint16_t)(m >> 16));
+    out[i] = s * (double)code + z;
+  }
+}
+
+void rqo_dequant_rows_f64(const uint32_t* words, const uint32_t* meta,
+                          int64_t n, int D, int bits, int group, double* out) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r)
+    rqo_dequant_codes_f64(words + r * W, meta + r * G, D, bits, group,
+                          out + r * D);
+}
+
+void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
+                       int64_t T, const double* kcur, const double* vcur, int D,
+                       double scale, double* out) {
+  double* s = (double*)malloc(sizeof(double) * (size_t)(T + 1));
+  double m;
+  {
+    double d = 0.0;
+    for (int i = 0; i < D; ++i) d += q[i] * kcur[i];
+    s[T] = scale * d;
+    m = s[T];
+  }
+  for (int64_t t = 0; t < T; ++t) {
+    double d = 0.0;
+    for (int i = 0; i < D; ++i) d += q[i] * khat[t * D + i];
+    s[t] = scale * d;
+    if (s[t] > m) m = s[t];
+  }
+  double l = exp(s[T] - m);
+  for (int i = 0; i < D; ++i) out[i] = l * vcur[i];
+  for (int64_t t = 0; t < T; ++t) {
+    const double p = exp(s[t] - m);
+    l += p;
+    for (int i = 0; i < D; ++i) out[i] += p * vhat[t * D + i];
+  }
+  for (int i = 0; i < D; ++i) out[i] /= l;
+  free(s);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Storage and access accounting [RQ §5.1, App. A.3, App. D]                */
+/* ------------------------------------------------------------------------ */
+
+double rqo_effective_bits(int L, const int* bits, const int* group, int D,
+                          int meta_bits, int residual) {
+  double total = 0.0;
+  for (int r = 0; r < L; ++r)
+    total += (double)bits[r] + (double)meta_bits / (double)group[r];
+  if (residual) total += (double)(L - 1) * 16.0 / (double)D;
+  return total / (double)L;
+}
+
+int64_t rqo_component_reads(int L, int chained) {
+  /* Loops are 0..L-1 with the anchor at L-1 (Last-loop / Next-loop).  The
+   * anchor loop reads one component.  Under the shared anchor every other
+   * loop reads the anchor and its own residual; under the chain, loop r
+   * reads its residual, every residual between it and the anchor, and the
+   * anchor. */
+  int64_t total = 0;
+  for (int r = 0; r < L; ++r) {
+    if (r == L - 1)
+      total += 1;
+    else if (!chained)
+      total += 2;
+    else
+      total += (L - 1 - r) + 1;
+  }
+  return total;
+}

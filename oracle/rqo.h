@@ -1,0 +1,131 @@
+/*
+ * rqo.h -- CPU oracle for the ResidualQuant KV-cache hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (librq) never calls it and shares no code, header, table or helper with it.
+ *
+ * Plain, single-threaded, deliberately slow C.  Every function follows one
+ * passage of the method's description, cited as
+ *   [RQ §x]  = "ResidualQuant: KV Cache Quantization for Looped Transformers
+ *              with 2-Bit Residuals" (paperpeel.com/paper/2610.10381), section x.
+ *
+ * Precision: the quantities that decide an integer (a code, a min/max, the
+ * fp16 metadata, the bf16 LS coefficient) are computed in fp32 in one fixed,
+ * documented order, so the GPU path can be held to bit-exact agreement.
+ * Reconstruction and attention are computed in fp64.
+ *
+ * Packed formats (the storage contract both sides implement independently):
+ *   codes : channel i of a row lives in 32-bit word i / (32/b), bits
+ *           [b*(i % (32/b)), +b), little-endian words.
+ *   meta  : one 32-bit word per group: low half = fp16 scale s~,
+ *           high half = fp16 offset z~.
+ *   alpha : bf16 bits of the LS coefficient, one per (token, head).
+ */
+#ifndef RQO_H
+#define RQO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Number conversions, written from the IEEE-754 binary16 / bfloat16
+ * definitions (round to nearest, ties to even). */
+float    rqo_bf16_to_f32(uint16_t h);
+uint16_t rqo_f32_to_bf16(float f);
+float    rqo_f16_to_f32(uint16_t h);
+uint16_t rqo_f32_to_f16(float f);
+
+/* fp32 normalisation constant of the D x D Sylvester-Hadamard matrix:
+ * round-to-nearest fp32 of 1/sqrt(D). */
+float rqo_rot_scale(int D);
+
+/* z <- H z, H the normalised Sylvester-Hadamard matrix [RQ §3.3, App. G.2].
+ * fp32, stages h = 1, 2, ..., D/2, each pair (a, b) -> (a + b, a - b),
+ * then one fp32 multiply by rqo_rot_scale(D). */
+void rqo_fwht_f32(float* z, int D);
+
+/* Same transform in fp64, normalised by 1/sqrt(D) in fp64; H = H^T = H^-1. */
+void rqo_fwht_f64(double* z, int D);
+void rqo_fwht_rows_f64(double* z, int64_t n, int D);
+
+/* Canonical-order fp32 dot product used for the LS coefficient:
+ * the D channels are split into P = D/32 consecutive slices of 32; each
+ * slice is summed serially with fused multiply-add starting from +0; the P
+ * partial sums are then combined by a butterfly: for off = P/2, ..., 1,
+ * p[l] <- p[l] + p[l ^ off].  Returns p[0].  Requires D % 32 == 0. */
+float rqo_dot_f32(const float* a, const float* b, int D);
+
+/* Group-wise affine quantisation of one rotated row [RQ §2.1]:
+ * per group of g consecutive channels: mn, mx; s = (mx - mn)/(2^b - 1);
+ * s~ = fp16(s), z~ = fp16(mn); inv = 1/s~ (0 if s~ == 0);
+ * u = (z - z~) * inv; c = rint_half_even(clamp(u, 0, 2^b - 1));
+ * deq = fma(s~, c, z~).  Writes packed words (D*b/32), meta (D/g), deq (D). */
+void rqo_quantize(const float* z, int D, int bits, int group,
+                  uint32_t* words, uint32_t* meta, float* deq);
+
+/* Anchor of the final loop [RQ §3.2 Last-loop policy, §3.4, App. G.2]:
+ * Z = H x (x bf16), quantised with the anchor's bits and group.
+ * zhat receives the dequantised rotated anchor A (fp32). */
+void rqo_encode_anchor(const uint16_t* x, int D, int bits, int group,
+                       uint32_t* words, uint32_t* meta, float* zhat);
+
+/* Residual loop from an already rotated fp32 row z and reference ref
+ * (rotated, dequantised) [RQ §3.2 scaling coefficient, App. G.1]:
+ * alpha = <z, ref>/<ref, ref> (0 when <ref, ref> == 0), both dots by
+ * rqo_dot_f32, one IEEE division; alpha~ = bf16(alpha);
+ * E = fma(-alpha~, ref, z); E quantised with (bits, group);
+ * zhat = fma(alpha~, ref, deq(E)) is the reconstructed rotated row. */
+void rqo_encode_residual_rot(const float* z, const float* ref, int D, int bits,
+                             int group, uint32_t* words, uint32_t* meta,
+                             uint16_t* alpha, float* zhat);
+
+/* Same, from a bf16 row x (rotated here with rqo_fwht_f32). */
+void rqo_encode_residual(const uint16_t* x, const float* ref, int D, int bits,
+                         int group, uint32_t* words, uint32_t* meta,
+                         uint16_t* alpha, float* zhat);
+
+/* Row-batched forms of the two encoders: n rows, row-major. */
+void rqo_encode_anchor_rows(const uint16_t* x, int64_t n, int D, int bits,
+                            int group, uint32_t* words, uint32_t* meta,
+                            float* zhat);
+void rqo_encode_residual_rows(const uint16_t* x, const float* ref, int64_t n,
+                              int D, int bits, int group, uint32_t* words,
+                              uint32_t* meta, uint16_t* alpha, float* zhat);
+
+/* fp64 value of the stored levels of one packed row: s~ * c + z~. */
+void rqo_dequant_codes_f64(const uint32_t* words, const uint32_t* meta, int D,
+                           int bits, int group, double* out);
+void rqo_dequant_rows_f64(const uint32_t* words, const uint32_t* meta,
+                          int64_t n, int D, int bits, int group, double* out);
+
+/* Softmax attention of one query against T rows, fp64 [RQ §4.1, §4.2,
+ * App. G.1]: s_t = scale * q.k_t for t < T, plus the current token
+ * s_cur = scale * q.k_cur; p = softmax(s); out = sum_t p_t v_t + p_cur v_cur.
+ * khat and vhat are T x D row-major (original domain). */
+void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
+                       int64_t T, const double* kcur, const double* vcur,
+                       int D, double scale, double* out);
+
+/* Effective bits per KV element [RQ App. A.3]: codes, scales, offsets and LS
+ * coefficients, averaged over the L loops of a group.  bits[r], group[r] for
+ * r = 0..L-1 (loop L-1 is the anchor); meta_bits = bits of (scale + offset)
+ * per group; residual != 0 adds one 16-bit coefficient per (token, head) for
+ * each of the L-1 non-anchor loops. */
+double rqo_effective_bits(int L, const int* bits, const int* group, int D,
+                          int meta_bits, int residual);
+
+/* Logical compressed-component reads needed to reconstruct every loop of a
+ * group of L loops [RQ App. D, logical reference count]:
+ * shared anchor (First-/Last-loop): 2L - 1; chained (Previous-/Next-loop):
+ * L(L+1)/2.  chained selects the policy. */
+int64_t rqo_component_reads(int L, int chained);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQO_H */

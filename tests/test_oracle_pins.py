@@ -1,0 +1,413 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a closed form, an invariant, a library
+routine, brute force on tiny inputs, or a number the ResidualQuant pages print
+(tests/golden/pages_storage.txt), chosen so that a dropped term, a wrong sign
+or index, or a transposed operand in the oracle fails at least one of them.
+"""
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = (s.strip() for s in line.split("="))
+                vals[k] = float(v)
+    return vals
+
+
+# ---------------------------------------------------------------- formats --
+
+def _probe_floats(rng, n=4000):
+    v = np.concatenate([
+        rng.standard_normal(n).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(n) * 1e-5).astype(np.float32),          # fp16 subnormals
+        (rng.standard_normal(n) * 1e-8).astype(np.float32),          # flush-to-zero region
+        (rng.standard_normal(n) * 3e4).astype(np.float32),           # near fp16 overflow
+        np.array([0.0, -0.0, 65504.0, 65519.0, 65520.0, 65536.0, 1e30, 6.1e-5, 5.96e-8,
+                  2.98e-8, 2.9802322e-08, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11], np.float32),
+    ])
+    # exact ties of fp16: k + 0.5 ulp patterns
+    k = rng.integers(1024, 2048, 200).astype(np.float32)
+    ties = ((k + np.float32(0.5)) * np.float32(2.0 ** -10)).astype(np.float32)
+    return np.concatenate([v, ties, -ties])
+
+
+def test_f16_round_trip_matches_numpy(oracle_mod):
+    """fp32 -> fp16 (RN-even) and fp16 -> fp32 agree with numpy's IEEE conversions."""
+    rng = np.random.default_rng(0)
+    v = _probe_floats(rng)
+    with np.errstate(over="ignore"):
+        want = v.astype(np.float16).view(np.uint16)
+    got = np.array([oracle_mod.f32_to_f16_bits(x) for x in v], np.uint16)
+    np.testing.assert_array_equal(got, want)
+    allbits = np.arange(0, 1 << 16, 97, dtype=np.uint32).astype(np.uint16)
+    ref = allbits.view(np.float16).astype(np.float32)
+    mine = np.array([oracle_mod.f16_bits_to_f32(int(b)) for b in allbits], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan)
+    np.testing.assert_array_equal(mine[~nan], ref[~nan])
+
+
+def test_bf16_round_trip_matches_torch(oracle_mod):
+    rng = np.random.default_rng(1)
+    v = _probe_floats(rng)
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle_mod.f32_to_bf16_bits(x) for x in v], np.uint16)
+    np.testing.assert_array_equal(got, want)
+    for b in [0x0000, 0x8000, 0x3F80, 0xC2F7, 0x0001, 0x7F7F]:
+        assert oracle_mod.bf16_bits_to_f32(b) == float(
+            torch.from_numpy(np.array([b], np.uint16).view(np.int16)).view(torch.bfloat16).float()[0])
+
+
+# --------------------------------------------------------------- rotation --
+
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
+def test_fwht_equals_scipy_hadamard(oracle_mod, D):
+    """H x by the butterfly equals scipy's Sylvester matrix / sqrt(D) times x."""
+    rng = np.random.default_rng(D)
+    x = rng.standard_normal((5, D)).astype(np.float32)
+    H = scipy.linalg.hadamard(D).astype(np.float64) / np.sqrt(D)
+    want = x.astype(np.float64) @ H.T
+    got = oracle_mod.fwht_f32(x)
+    assert np.max(np.abs(got - want)) <= 1e-6 * np.max(np.abs(want))
+    got64 = oracle_mod.fwht_f64(x)
+    assert np.max(np.abs(got64 - want)) <= 1e-13 * np.max(np.abs(want))
+
+
+def test_fwht_sign_pattern_popcount(oracle_mod):
+    """Row i of H is (-1)^popcount(i & j) / sqrt(D): transform each basis vector."""
+    D = 64
+    eye = np.eye(D, dtype=np.float32)
+    Ht = oracle_mod.fwht_f32(eye)          # row i = H e_i = column i of H
+    i, j = np.meshgrid(np.arange(D), np.arange(D), indexing="ij")
+    pc = np.vectorize(lambda v: bin(v).count("1"))(i & j)
+    want = np.where(pc % 2 == 0, 1.0, -1.0) / 8.0
+    np.testing.assert_array_equal(Ht, want.astype(np.float32))
+
+
+def test_fwht_involution_exact_d64(oracle_mod):
+    """H H^T = I; exact for D=64 on small integers because 1/sqrt(64) = 1/8."""
+    rng = np.random.default_rng(2)
+    x = rng.integers(-50, 50, (8, 64)).astype(np.float32)
+    np.testing.assert_array_equal(oracle_mod.fwht_f32(oracle_mod.fwht_f32(x)), x)
+    e0 = np.zeros(64, np.float32)
+    e0[0] = 1
+    np.testing.assert_array_equal(oracle_mod.fwht_f32(e0), np.full(64, 0.125, np.float32))
+
+
+def test_rot_scale_is_rounded_inverse_sqrt(oracle_mod):
+    for D in (32, 64, 128, 256):
+        assert oracle_mod.rot_scale(D) == float(np.float32(1.0 / np.sqrt(np.float64(D))))
+
+
+def test_rotation_preserves_scores(oracle_mod):
+    """q.k = (Hq).(Hk) with quantisation bypassed (orthogonality)."""
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((16, 128))
+    k = rng.standard_normal((16, 128)) * np.exp(0.5 * rng.standard_normal(128))
+    s0 = np.sum(q * k, axis=1)
+    s1 = np.sum(oracle_mod.fwht_f64(q) * oracle_mod.fwht_f64(k), axis=1)
+    assert np.max(np.abs(s1 - s0)) <= 1e-12 * np.max(np.abs(s0))
+    s2 = np.sum(oracle_mod.fwht_f32(q).astype(np.float64) * oracle_mod.fwht_f32(k), axis=1)
+    assert np.max(np.abs(s2 - s0)) <= 1e-6 * np.sum(np.abs(q) * np.abs(k), axis=1).max()
+
+
+# ------------------------------------------------------------- dot product --
+
+def test_dot_exact_on_integers(oracle_mod):
+    rng = np.random.default_rng(4)
+    for D in (32, 64, 128, 256):
+        a = rng.integers(-300, 300, D)
+        b = rng.integers(-300, 300, D)
+        assert oracle_mod.dot_f32(a.astype(np.float32), b.astype(np.float32)) == float(np.dot(a, b))
+
+
+def test_dot_within_summation_bound(oracle_mod):
+    rng = np.random.default_rng(5)
+    for D in (64, 128):
+        a = rng.standard_normal(D).astype(np.float32)
+        b = rng.standard_normal(D).astype(np.float32)
+        exact = float(np.dot(a.astype(np.float64), b.astype(np.float64)))
+        bound = (D + 8) * 2.0 ** -24 * float(np.sum(np.abs(a.astype(np.float64) * b)))
+        assert abs(oracle_mod.dot_f32(a, b) - exact) <= bound
+        # swapping the operands cannot change the value
+        assert oracle_mod.dot_f32(a, b) == oracle_mod.dot_f32(b, a)
+
+
+# ------------------------------------------------------------ quantisation --
+
+def test_int2_ramp_uses_all_four_levels(oracle_mod):
+    """Affine INT2 has the four levels o, o+s, o+2s, o+3s [RQ §2.1]."""
+    o, s = np.float32(-1.25), np.float32(0.5)   # fp16-exact
+    z = np.array([o + k * s for k in range(4)] * 8, np.float32)
+    words, meta, deq = oracle_mod.quantize(z, 2, 32)
+    codes = oracle_mod.unpack_codes(words, 2, 32)
+    np.testing.assert_array_equal(codes, np.tile(np.arange(4), 8))
+    sc, zz = oracle_mod.meta_scale_zero(meta)
+    assert sc[0] == s and zz[0] == o
+    np.testing.assert_array_equal(deq, z)
+
+
+def test_packing_bit_positions():
+    """Channel i -> word i/(32/b), bits [b*(i%(32/b)), +b) (hand-computed words)."""
+    import oracle
+    o = np.float32(0.0)
+    # INT4, 32 channels with codes 0..15 then 15..0, scale 1, offset 0.
+    z = np.array(list(range(16)) + list(range(15, -1, -1)), np.float32)
+    words, _, _ = oracle.quantize(z, 4, 32)
+    assert [hex(w) for w in words] == ["0x76543210", "0xfedcba98", "0x89abcdef", "0x1234567"]
+    # INT2, 16 channels: codes 3,0,1,2,... -> ((3)|(0<<2)|(1<<4)|(2<<6)) per byte = 0x93
+    z2 = np.array([3, 0, 1, 2] * 4 + [0, 0, 0, 3] * 4, np.float32) + o
+    w2, _, _ = oracle.quantize(z2, 2, 32)
+    assert [hex(w) for w in w2] == ["0x93939393", "0xc0c0c0c0"]
+
+
+def _tie_distance(u):
+    return np.abs(np.abs(u - np.floor(u)) - 0.5)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 32), (2, 16), (2, 64), (4, 64)])
+def test_codes_are_nearest_level_brute_force(oracle_mod, bits, group):
+    """Brute force over every level: the code is the nearest level (clamped),
+    except where the scaled value sits within 1e-4 of a half-way tie."""
+    rng = np.random.default_rng(bits * 100 + group)
+    qmax = (1 << bits) - 1
+    checked = 0
+    for trial in range(40):
+        z = (rng.standard_normal(128) * rng.uniform(0.01, 5)).astype(np.float32)
+        words, meta, deq = oracle_mod.quantize(z, bits, group)
+        codes = oracle_mod.unpack_codes(words, bits, 128).astype(np.int64)
+        sc, zz = oracle_mod.meta_scale_zero(meta)
+        for gi in range(128 // group):
+            sl = slice(gi * group, (gi + 1) * group)
+            zg = z[sl].astype(np.float64)
+            s, o = float(sc[gi]), float(zz[gi])
+            # metadata: fp16 of (max-min)/qmax and of min
+            assert sc[gi] == np.float16(np.float32(np.float32(zg.max() - zg.min()) / qmax))
+            assert zz[gi] == np.float16(np.float32(zg.min()))
+            levels = o + s * np.arange(qmax + 1)
+            best = np.argmin(np.abs(zg[:, None] - levels[None, :]), axis=1)
+            u = (zg - o) / s
+            ok = _tie_distance(np.clip(u, 0, qmax)) > 1e-4
+            np.testing.assert_array_equal(codes[sl][ok], best[ok])
+            checked += ok.sum()
+            # the group's extremes land on the end codes
+            assert codes[sl][np.argmin(zg)] == 0 and codes[sl][np.argmax(zg)] == qmax
+            # every dequantised value is a level, within fp32 rounding of fma
+            np.testing.assert_allclose(deq[sl], levels[codes[sl]], rtol=0, atol=2e-7 * (abs(o) + s * qmax))
+            assert np.all(np.abs(zg - levels[codes[sl]]) <= 0.5 * s * (1 + 1e-3) + 1e-3 * s)
+    assert checked > 1000
+
+
+def test_constant_group_codes_zero(oracle_mod):
+    z = np.full(64, 0.8125, np.float32)
+    words, meta, deq = oracle_mod.quantize(z, 2, 32)
+    assert np.all(words == 0)
+    sc, zz = oracle_mod.meta_scale_zero(meta)
+    assert np.all(sc == 0) and np.all(zz == np.float32(0.8125))
+    np.testing.assert_array_equal(deq, z)
+
+
+# ---------------------------------------------------------- LS coefficient --
+
+def _anchor_row(oracle_mod, seed, D=128):
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal(D).astype(np.float32)
+    _, _, A = oracle_mod.quantize(z, 4, 32)
+    return A
+
+
+@pytest.mark.parametrize("c", [1.0, 0.5, 2.0, -0.25, 4.0])
+def test_scaled_reference_gives_alpha_c_and_zero_residual(oracle_mod, c):
+    """X_r = c R^ gives alpha = c and a zero residual [RQ §3.2, App. G.1]."""
+    A = _anchor_row(oracle_mod, 7)
+    z = (np.float32(c) * A).astype(np.float32)
+    words, meta, ab, zhat = oracle_mod.encode_residual_rot(z, A, 2, 32)
+    assert oracle_mod.bf16_bits_to_f32(ab) == c
+    assert np.all(words == 0)
+    sc, zz = oracle_mod.meta_scale_zero(meta)
+    assert np.all(sc == 0) and np.all(zz == 0)
+    np.testing.assert_array_equal(zhat, z)
+
+
+def test_alpha_is_bf16_of_least_squares(oracle_mod):
+    """alpha~ is the bf16 rounding of argmin_a ||z - a ref||^2 (within one bf16 step)."""
+    rng = np.random.default_rng(8)
+    for seed in range(30):
+        A = _anchor_row(oracle_mod, 100 + seed)
+        c = rng.uniform(0.7, 1.3)
+        z = (c * A + 0.3 * rng.standard_normal(128)).astype(np.float32)
+        _, _, ab, _ = oracle_mod.encode_residual_rot(z, A, 2, 32)
+        a64 = np.dot(z.astype(np.float64), A) / np.dot(A.astype(np.float64), A)
+        got = oracle_mod.bf16_bits_to_f32(ab)
+        assert abs(got - a64) <= 2.0 ** -8 * abs(a64)
+
+
+def test_zero_anchor_gives_alpha_zero(oracle_mod):
+    rng = np.random.default_rng(9)
+    z = rng.standard_normal(128).astype(np.float32)
+    ref = np.zeros(128, np.float32)
+    words, meta, ab, zhat = oracle_mod.encode_residual_rot(z, ref, 2, 32)
+    assert ab == 0
+    w2, m2, d2 = oracle_mod.quantize(z, 2, 32)
+    np.testing.assert_array_equal(words, w2)
+    np.testing.assert_array_equal(meta, m2)
+    np.testing.assert_array_equal(zhat, d2)
+
+
+def test_residual_beats_direct_quantisation(oracle_mod):
+    """The point of the method: on correlated loops, anchor + LS residual at INT2
+    reconstructs better than direct INT2 of the same loop [RQ §3.1, §3.2]."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=2, tokens=64)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_K, l, [0], [0, 1], 0, 64)).reshape(-1, 128)
+                  for l in range(4)])
+    encs = oracle_mod.encode_side(x, w.bits, w.group)
+    xs = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for r in range(3):
+        rec = oracle_mod.reconstruct(encs, r, w.bits, w.group)
+        direct = oracle_mod.encode_side(x[r:r + 1], (2,), (32,))
+        rec_d = oracle_mod.reconstruct(direct, 0, (2,), (32,))
+        err_res = np.sum((rec - xs[r]) ** 2)
+        err_dir = np.sum((rec_d - xs[r]) ** 2)
+        assert err_res < 0.5 * err_dir
+
+
+def test_chained_equals_shared_next_to_anchor(oracle_mod):
+    """Loop L-2 references the anchor under both policies: identical encodings;
+    the chain differs further away [RQ §5.2, App. D]."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["huginn_deep"].replace(batch=1, heads=1, tokens=16)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_V, l, [0], [0], 0, 16)).reshape(-1, 128)
+                  for l in range(w.loops)])
+    es = oracle_mod.encode_side(x, w.bits, w.group, "last")
+    ec = oracle_mod.encode_side(x, w.bits, w.group, "next")
+    r = w.loops - 2
+    for k in ("codes", "meta", "alpha"):
+        np.testing.assert_array_equal(es[r][k], ec[r][k])
+    assert not np.array_equal(es[0]["codes"], ec[0]["codes"])
+    # the chained reconstruction of loop r equals alpha_r * (reconstruction of r+1) + D(c_r)
+    z1 = oracle_mod.reconstruct_rotated(ec, 1, w.bits, w.group, "next")
+    z0 = oracle_mod.reconstruct_rotated(ec, 0, w.bits, w.group, "next")
+    lv = oracle_mod._levels_f64(ec[0], w.bits[0], w.group[0], 128)
+    a0 = oracle_mod.bf16_bits_to_f64(ec[0]["alpha"])[:, None]
+    np.testing.assert_allclose(z0, a0 * z1 + lv, rtol=0, atol=1e-12)
+
+
+def test_encoder_reference_row_matches_reconstruction(oracle_mod):
+    """The fp32 reconstructed row the encoder keeps (zhat) equals the fp64
+    reconstruction from the stored codes, alpha and metadata to fp32 rounding."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=1, tokens=32)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_K, l, [0], [0], 0, 32)).reshape(-1, 128)
+                  for l in range(4)])
+    encs = oracle_mod.encode_side(x, w.bits, w.group)
+    for r in range(4):
+        z = oracle_mod.reconstruct_rotated(encs, r, w.bits, w.group)
+        np.testing.assert_allclose(encs[r]["zhat"], z, rtol=2e-6, atol=2e-6)
+
+
+# --------------------------------------------------------------- attention --
+
+def _softmax_attention_numpy(q, K, V, kc, vc, scale):
+    s = np.concatenate([K @ q, [kc @ q]]) * scale
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    return p[:-1] @ V + p[-1] * vc
+
+
+def test_attention_matches_brute_force(oracle_mod):
+    rng = np.random.default_rng(10)
+    for T in (0, 1, 5, 37):
+        q, kc, vc = (rng.standard_normal(64) for _ in range(3))
+        K = rng.standard_normal((T, 64)) * 2
+        V = rng.standard_normal((T, 64))
+        got = oracle_mod.attention(q, K, V, kc, vc, 0.125)
+        want = _softmax_attention_numpy(q, K, V, kc, vc, 0.125)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases(oracle_mod):
+    rng = np.random.default_rng(11)
+    kc, vc = rng.standard_normal(128), rng.standard_normal(128)
+    # no past tokens: the current value alone
+    np.testing.assert_allclose(oracle_mod.attention(rng.standard_normal(128), np.zeros((0, 128)),
+                                                    np.zeros((0, 128)), kc, vc, 0.1), vc, rtol=1e-15)
+    # a zero query gives equal scores: the mean of all values
+    V = rng.standard_normal((9, 128))
+    got = oracle_mod.attention(np.zeros(128), rng.standard_normal((9, 128)), V, kc, vc, 0.1)
+    np.testing.assert_allclose(got, (V.sum(0) + vc) / 10, rtol=1e-12, atol=1e-14)
+
+
+def test_decode_units_are_independent(oracle_mod):
+    """Batch/head units do not interact: permuting heads permutes outputs."""
+    rng = np.random.default_rng(12)
+    B, H, T, D = 2, 3, 11, 64
+    kh, vh = rng.standard_normal((B, H, T, D)), rng.standard_normal((B, H, T, D))
+    bf = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    q, kc, vc = (bf(rng.standard_normal((B, H, D))) for _ in range(3))
+    out = oracle_mod.decode_attention(kh, vh, q, [T, 7], kc, vc)
+    perm = [2, 0, 1]
+    out2 = oracle_mod.decode_attention(kh[:, perm], vh[:, perm], q[:, perm], [T, 7], kc[:, perm],
+                                       vc[:, perm])
+    np.testing.assert_array_equal(out2, out[:, perm])
+
+
+# ---------------------------------------------------- storage and accesses --
+
+def test_effective_bits_match_pages():
+    """With the pages' 16-bit metadata per group, the accounting reproduces
+    every printed b_eff, the alpha overhead and the storage fractions."""
+    import oracle
+    g = _golden("pages_storage.txt")
+    D = 128
+    cfgs = {
+        "int2_g32": ((2, 2, 2, 2), (32, 32, 32, 32)),
+        "int2_g16": ((2, 2, 2, 2), (16, 16, 16, 16)),
+        "int24_g32": ((2, 2, 2, 4), (32, 32, 32, 32)),
+        "int24_g16": ((2, 2, 2, 4), (16, 16, 16, 32)),   # INT4 keeps g=32 [RQ §5.2]
+    }
+    for name, (bits, grp) in cfgs.items():
+        direct = oracle.effective_bits(bits, grp, D, 16, False)
+        resid = oracle.effective_bits(bits, grp, D, 16, True)
+        assert round(direct, 1) == g[f"beff_direct_{name}"], name
+        assert round(resid, 1) == g[f"beff_residual_{name}"], name
+    over = oracle.effective_bits((2,) * 4, (32,) * 4, D, 16, True) - oracle.effective_bits(
+        (2,) * 4, (32,) * 4, D, 16, False)
+    assert round(over, 3) == g["alpha_overhead_bits"]
+    b_rq = oracle.effective_bits((2, 2, 2, 4), (32,) * 4, D, 16, True)
+    assert round(b_rq / 16, 3) == g["storage_frac_int24_residual_g32"]
+    assert round(oracle.effective_bits((2,) * 4, (32,) * 4, D, 16, False) / 16, 3) == g[
+        "storage_frac_int2_direct_g32"]
+    assert round(1 - b_rq / 16, 3) == g["storage_reduction_int24"]
+    assert round(16 / b_rq, 1) == g["storage_ratio_int24"]
+
+
+def test_component_reads_match_pages():
+    import oracle
+    g = _golden("pages_storage.txt")
+    assert oracle.component_reads(4, True) == g["reads_chained_L4"]
+    assert oracle.component_reads(4, False) == g["reads_shared_L4"]
+    assert oracle.component_reads(32, True) == g["reads_chained_L32"]
+    assert oracle.component_reads(32, False) == g["reads_shared_L32"]
+    assert round(oracle.component_reads(4, True) / oracle.component_reads(4, False), 2) == g[
+        "reads_ratio_L4"]
+    assert round(oracle.component_reads(32, True) / oracle.component_reads(32, False), 2) == g[
+        "reads_ratio_L32"]
+    assert 8 * oracle.component_reads(4, True) == g["reads_chained_huginn_8x4"]
+    assert 8 * oracle.component_reads(4, False) == g["reads_shared_huginn_8x4"]
+    # closed forms L(L+1)/2 and 2L-1 for every L
+    for L in range(1, 40):
+        assert oracle.component_reads(L, True) == L * (L + 1) // 2
+        assert oracle.component_reads(L, False) == 2 * L - 1
