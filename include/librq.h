@@ -1,0 +1,222 @@
+/*
+ * librq.h -- C ABI of librq, a B200-native (sm_100a) implementation of the
+ * ResidualQuant KV-cache hot path for looped Transformers.
+ *
+ * Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
+ * Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+ *
+ * What is stored [RQ §3.2 Last-loop policy, §3.3, §3.4, App. G.2]:
+ *   For every past token and KV head of loop r, with Z = H x the normalised
+ *   Sylvester-Hadamard rotation of the bf16 row x:
+ *     anchor (final loop L-1):  A = deq(Q_bL(Z_{L-1}))
+ *     residual loop r < L-1:    alpha_r = <Z_r, R>/<R, R>, alpha~ = bf16(alpha_r),
+ *                               codes of Q_br(Z_r - alpha~ R)
+ *   where R = A (RQ_POLICY_LAST_LOOP, shared anchor) or R = Z^_{r+1}
+ *   (RQ_POLICY_NEXT_LOOP, the chained "Next-loop" reference [RQ §5.2]).
+ *   Q_b is group-wise affine quantisation [RQ §2.1]: per group of g
+ *   consecutive channels, s = (max - min)/(2^b - 1), s~ = fp16(s),
+ *   z~ = fp16(min), code = rint_even(clamp((z - z~) * (1/s~), 0, 2^b - 1)).
+ *   Reconstruction: Z^_r = alpha~_r R + s~ c + z~ and X^_r = H^T Z^_r.
+ *
+ * Storage contract (per layer and per side K | V; all offsets 256-B aligned;
+ * rows are [batch][kv_heads][token_stride] with token_stride =
+ * max_tokens rounded up to a multiple of 16):
+ *   codes of loop r : uint32 [rows][head_dim * bits[r] / 32]; channel i sits
+ *                     in word i / (32/b), bits [b*(i % (32/b)), +b)
+ *   meta of loop r  : uint32 [rows][head_dim / group[r]]; low half fp16
+ *                     scale s~, high half fp16 offset z~
+ *   alpha of loop r : bf16  [rows] (residual loops only)
+ *   Effective bits per element of loop r: bits[r] + 32/group[r]
+ *   (+ 16/head_dim for a residual loop).
+ *
+ * Conventions for every entry point:
+ *   - All pointers except rq_layout / rq_cache arguments are DEVICE pointers
+ *     unless stated; the caller owns all memory.  librq allocates nothing,
+ *     keeps no per-call state, and is safe to call from several host threads
+ *     on different streams.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on that stream.
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns an error and launches nothing.  Launch failures return
+ *     RQ_ERR_CUDA.  Device code never traps; conditions only the device can
+ *     see (a sequence length over its bound, a bounded wait that ran out) are
+ *     recorded in the decode workspace and reported by rq_workspace_error().
+ *   - bf16 / fp16 tensors are passed as raw 16-bit words.
+ */
+#ifndef LIBRQ_H
+#define LIBRQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RQ_ABI_VERSION 1
+#define RQ_MAX_LOOPS 32
+
+typedef enum rq_status {
+  RQ_OK = 0,
+  RQ_ERR_INVALID_ARG = 1,   /* null pointer, bad index, misaligned buffer ... */
+  RQ_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. head_dim 96)        */
+  RQ_ERR_CAPACITY = 3,      /* token range or sequence length over capacity  */
+  RQ_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+  RQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out             */
+  RQ_ERR_WORKSPACE = 6      /* workspace too small                            */
+} rq_status;
+
+/* Reference policy [RQ §3.2, §5.2]. */
+typedef enum rq_policy {
+  RQ_POLICY_LAST_LOOP = 0,  /* every loop r < L-1 references the final-loop anchor */
+  RQ_POLICY_NEXT_LOOP = 1   /* loop r references loop r+1 (chain to the anchor)    */
+} rq_policy;
+
+/* Shape and precision of a compressed KV cache.
+ *   num_layers  >= 1
+ *   num_loops   L in [1, RQ_MAX_LOOPS]; loop L-1 (0-based) is the anchor
+ *   batch, kv_heads >= 1
+ *   head_dim    D in {64, 128}
+ *   max_tokens  token capacity per (batch, head), >= 1
+ *   policy      rq_policy
+ *   bits[r]     2 or 4
+ *   group[r]    g in {16, 32, 64, 128}, g divides D, g * bits[r] >= 32
+ */
+typedef struct rq_layout {
+  int32_t num_layers;
+  int32_t num_loops;
+  int32_t batch;
+  int32_t kv_heads;
+  int32_t head_dim;
+  int32_t max_tokens;
+  int32_t policy;
+  int32_t reserved;            /* must be 0 */
+  int32_t bits[RQ_MAX_LOOPS];
+  int32_t group[RQ_MAX_LOOPS];
+} rq_layout;
+
+/* A cache bound to caller-owned device memory (filled by rq_cache_bind;
+ * treat as read-only).  Offsets are bytes within one (layer, side). */
+typedef struct rq_cache {
+  rq_layout layout;
+  void* k_base;                 /* num_layers * layer_bytes, K side */
+  void* v_base;                 /* num_layers * layer_bytes, V side */
+  uint64_t layer_bytes;
+  int64_t token_stride;
+  uint64_t codes_off[RQ_MAX_LOOPS];
+  uint64_t meta_off[RQ_MAX_LOOPS];
+  uint64_t alpha_off[RQ_MAX_LOOPS];  /* 0 for the anchor loop */
+} rq_cache;
+
+/* ABI version of the loaded library (RQ_ABI_VERSION at build time). */
+int32_t rq_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* rq_status_string(rq_status s);
+
+/* Checks every field of a layout.  RQ_OK, RQ_ERR_INVALID_ARG or
+ * RQ_ERR_UNSUPPORTED (head_dim or a bit width this build does not have). */
+rq_status rq_layout_validate(const rq_layout* layout);
+
+/* Bytes of ONE side (K or V) for all layers; 0 if the layout is invalid.
+ * The caller allocates this much twice (K and V). */
+uint64_t rq_cache_bytes(const rq_layout* layout);
+
+/* Bytes of one (layer, side): the stride between layers inside a side. */
+uint64_t rq_layer_bytes(const rq_layout* layout);
+
+/* Binds device buffers of rq_cache_bytes() each (256-byte aligned) to `out`.
+ * The buffers need no initialisation.  Host-only, launches nothing. */
+rq_status rq_cache_bind(const rq_layout* layout, void* k_base, void* v_base,
+                        rq_cache* out);
+
+/* Quantise-and-append the final-loop anchor [RQ §3.2, §3.4, §4.2 Prefill /
+ * Decode]: rows x (bf16, [batch][kv_heads][n][head_dim], contiguous) of
+ * loop L-1 are rotated, affine-quantised with bits[L-1] / group[L-1] and
+ * stored at token positions [t0, t0 + n) of `layer`, side kv (0 = K, 1 = V).
+ * n = 0 is a no-op.  t0 + n > max_tokens -> RQ_ERR_CAPACITY. */
+rq_status rq_quantize_anchor(const rq_cache* cache, int32_t layer, int32_t kv,
+                             const void* x, int32_t t0, int32_t n,
+                             void* stream);
+
+/* Quantise-and-append residual loop `loop` (0 <= loop < L-1) [RQ §3.2
+ * scaling coefficient, §3.3, App. G.1]: alpha, residual, rotation, affine
+ * quantisation and bit-packing of rows x (same layout as above).
+ * Stream-ordered precondition: the reference rows [t0, t0 + n) are stored
+ * already -- the anchor (LAST_LOOP) or loops loop+1 .. L-1 (NEXT_LOOP). */
+rq_status rq_quantize_append_residual(const rq_cache* cache, int32_t layer,
+                                      int32_t kv, int32_t loop, const void* x,
+                                      int32_t t0, int32_t n, void* stream);
+
+/* Reconstructs X^ of loop `loop` at positions [t0, t0 + n) in the original
+ * (unrotated) domain into out (fp32, [batch][kv_heads][n][head_dim]).
+ * For tests and export; not on the decode path [RQ App. G.2]. */
+rq_status rq_dequantize(const rq_cache* cache, int32_t layer, int32_t kv,
+                        int32_t loop, int32_t t0, int32_t n, float* out,
+                        void* stream);
+
+/* Workspace of rq_decode_attention for up to max_seq_len past tokens. */
+uint64_t rq_decode_workspace_bytes(const rq_layout* layout,
+                                   int32_t max_seq_len);
+
+/* Zeroes a decode workspace (cudaMemsetAsync).  Required once after
+ * allocation and after any call reported RQ_ERR_TIMEOUT; the kernels leave
+ * the workspace ready for the next call otherwise. */
+rq_status rq_decode_workspace_init(void* workspace, uint64_t ws_bytes,
+                                   void* stream);
+
+/* Compressed decode attention of loop `loop` for one query token per
+ * (batch, head) [RQ §4.1, §4.2 Decode, App. G.2]:
+ *   past keys/values t < seq_lens[b] are rebuilt on the fly from the packed
+ *   cache (anchor + the loop's residual; the whole chain under NEXT_LOOP),
+ *   scores use the rotated query (Hq) . Z^_K, values are accumulated in the
+ *   rotated domain and rotated back once; the current token's own k_cur /
+ *   v_cur (bf16, unrotated, [batch][kv_heads][head_dim]) are merged with the
+ *   softmax statistics.  Softmax and accumulation are fp32.
+ *   q        bf16 [batch][kv_heads][head_dim]
+ *   seq_lens int32 [batch] device array; values outside [0, max_seq_len] are
+ *            clamped and flagged (rq_workspace_error -> RQ_ERR_CAPACITY)
+ *   max_seq_len  host bound on seq_lens, <= max_tokens (sizes the grid)
+ *   softmax_scale  0 selects 1/sqrt(head_dim)
+ *   out      fp32 [batch][kv_heads][head_dim]
+ *   workspace  >= rq_decode_workspace_bytes(layout, max_seq_len), zeroed by
+ *            rq_decode_workspace_init once; calls sharing a workspace must be
+ *            ordered on one stream. */
+rq_status rq_decode_attention(const rq_cache* cache, int32_t layer,
+                              int32_t loop, const void* q,
+                              const int32_t* seq_lens, int32_t max_seq_len,
+                              const void* k_cur, const void* v_cur,
+                              float softmax_scale, float* out, void* workspace,
+                              uint64_t ws_bytes, void* stream);
+
+/* Uncompressed BF16 decode attention on the same split-K engine: the
+ * baseline the compressed path is measured against.
+ *   k, v  bf16 [batch][heads][token_stride][head_dim]
+ *   other arguments as rq_decode_attention; head_dim in {64, 128}. */
+uint64_t rq_decode_bf16_workspace_bytes(int32_t batch, int32_t heads,
+                                        int32_t head_dim, int32_t max_seq_len);
+rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads,
+                                   int32_t head_dim, const void* q,
+                                   const void* k, const void* v,
+                                   int64_t token_stride,
+                                   const int32_t* seq_lens,
+                                   int32_t max_seq_len, const void* k_cur,
+                                   const void* v_cur, float softmax_scale,
+                                   float* out, void* workspace,
+                                   uint64_t ws_bytes, void* stream);
+
+/* Reads and clears the device-side error word of a decode workspace
+ * (synchronises `stream`).  RQ_OK, RQ_ERR_CAPACITY (a seq_lens entry was out
+ * of range) or RQ_ERR_TIMEOUT (a bounded wait ran out; re-initialise the
+ * workspace). */
+rq_status rq_workspace_error(void* workspace, uint64_t ws_bytes, void* stream);
+
+/* Number of split-K partitions rq_decode_attention uses for this shape on
+ * the current device (for tests and benchmarks). */
+int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBRQ_H */

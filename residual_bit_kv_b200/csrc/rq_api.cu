@@ -1,0 +1,460 @@
+// rq_api.cu -- host side of the librq C ABI: argument validation, storage
+// layout, split-K sizing and kernel launches.  See include/librq.h.
+//
+// Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
+// Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+#include <math.h>
+#include <string.h>
+
+#include "rq_internal.cuh"
+
+namespace {
+
+using namespace rq;
+
+constexpr uint64_t kAlign = 256;
+constexpr int kMaxSplits = 1024;
+constexpr int kMaxStages = 4;
+constexpr size_t kRingBudget = 100 * 1024;   // stage ring per CTA: two or more CTAs per SM
+
+inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+inline bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+inline rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline int64_t token_stride_of(const rq_layout* l) {
+  return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), 16));
+}
+
+// Byte offsets of every array inside one (layer, side); returns layer bytes.
+uint64_t layout_offsets(const rq_layout* l, uint64_t* codes, uint64_t* meta, uint64_t* alpha) {
+  const uint64_t rows = static_cast<uint64_t>(l->batch) * l->kv_heads * token_stride_of(l);
+  const int L = l->num_loops, D = l->head_dim;
+  uint64_t off = 0;
+  // anchor (loop L-1) first, then residual loops 0 .. L-2
+  for (int k = 0; k < L; ++k) {
+    const int r = (k == 0) ? L - 1 : k - 1;
+    codes[r] = off;
+    off = align_up(off + rows * (D * l->bits[r] / 32) * 4, kAlign);
+    meta[r] = off;
+    off = align_up(off + rows * (D / l->group[r]) * 4, kAlign);
+    if (r != L - 1) {
+      alpha[r] = off;
+      off = align_up(off + rows * 2, kAlign);
+    } else {
+      alpha[r] = 0;
+    }
+  }
+  return align_up(off, kAlign);
+}
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return sms > 0 ? sms : 148;
+}
+
+int chunks_of(int32_t max_seq_len) { return (max_seq_len + kChunk - 1) / kChunk; }
+
+int max_splits_of(int32_t max_seq_len) {
+  int c = chunks_of(max_seq_len);
+  if (c < 1) c = 1;
+  return c > kMaxSplits ? kMaxSplits : c;
+}
+
+// Split count minimising (waves of CTAs) x (chunks per CTA), the time model
+// of a bandwidth-bound grid whose CTAs stream equal token ranges.
+void choose_splits(int bh, int32_t max_seq_len, int ctas_per_sm, int* splits, int* cps) {
+  const int chunks = chunks_of(max_seq_len);
+  if (chunks == 0) {
+    *splits = 1;
+    *cps = 0;
+    return;
+  }
+  const int64_t slots = static_cast<int64_t>(device_sms()) * (ctas_per_sm > 0 ? ctas_per_sm : 1);
+  const int smax = max_splits_of(max_seq_len);
+  double best = 1e300;
+  int best_s = 1;
+  for (int s = 1; s <= smax; ++s) {
+    const int c = (chunks + s - 1) / s;
+    if (s > 1 && (chunks + c - 1) / c != s) continue;   // would leave empty splits
+    const int64_t waves = (static_cast<int64_t>(bh) * s + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) * c + 0.01 * s;
+    if (cost < best) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  *splits = best_s;
+  *cps = (chunks + best_s - 1) / best_s;
+}
+
+struct WsLayout {
+  uint64_t err, counters, partials, total;
+};
+
+WsLayout ws_layout(int64_t bh, int D, int32_t max_seq_len) {
+  WsLayout w;
+  w.err = 0;
+  w.counters = kAlign;
+  w.partials = align_up(w.counters + static_cast<uint64_t>(bh) * 4, kAlign);
+  w.total = align_up(w.partials + static_cast<uint64_t>(bh) * max_splits_of(max_seq_len) *
+                                      (D + 2) * 4,
+                     kAlign);
+  return w;
+}
+
+const unsigned char* side_base(const rq_cache* c, int layer, int kv) {
+  const unsigned char* b = static_cast<const unsigned char*>(kv ? c->v_base : c->k_base);
+  return b + static_cast<uint64_t>(layer) * c->layer_bytes;
+}
+
+Comp comp_of(const rq_cache* c, int layer, int kv, int r) {
+  const unsigned char* b = side_base(c, layer, kv);
+  Comp k;
+  k.codes = reinterpret_cast<const uint32_t*>(b + c->codes_off[r]);
+  k.meta = reinterpret_cast<const uint32_t*>(b + c->meta_off[r]);
+  k.alpha = (r == c->layout.num_loops - 1)
+                ? nullptr
+                : reinterpret_cast<const uint16_t*>(b + c->alpha_off[r]);
+  k.bits = c->layout.bits[r];
+  k.group = c->layout.group[r];
+  return k;
+}
+
+// Reference chain used to reconstruct loop `loop`: [loop, ..., anchor]
+// (LAST_LOOP: [loop, anchor]; the anchor loop alone is [anchor]).
+int chain_of(const rq_cache* c, int layer, int kv, int loop, Comp* out) {
+  const int L = c->layout.num_loops;
+  int n = 0;
+  if (loop == L - 1) {
+    out[n++] = comp_of(c, layer, kv, L - 1);
+  } else if (c->layout.policy == RQ_POLICY_LAST_LOOP) {
+    out[n++] = comp_of(c, layer, kv, loop);
+    out[n++] = comp_of(c, layer, kv, L - 1);
+  } else {
+    for (int r = loop; r < L; ++r) out[n++] = comp_of(c, layer, kv, r);
+  }
+  return n;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+rq_status check_cache(const rq_cache* c, int32_t layer, int32_t kv) {
+  if (c == nullptr || c->k_base == nullptr || c->v_base == nullptr) return RQ_ERR_INVALID_ARG;
+  if (rq_layout_validate(&c->layout) != RQ_OK) return RQ_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= c->layout.num_layers) return RQ_ERR_INVALID_ARG;
+  if (kv != 0 && kv != 1) return RQ_ERR_INVALID_ARG;
+  return RQ_OK;
+}
+
+rq_status check_range(const rq_cache* c, int32_t t0, int32_t n) {
+  if (t0 < 0 || n < 0) return RQ_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(t0) + n > c->layout.max_tokens) return RQ_ERR_CAPACITY;
+  return RQ_OK;
+}
+
+float rot_scale_of(int D) { return static_cast<float>(1.0 / sqrt(static_cast<double>(D))); }
+
+float scale_log2_of(float softmax_scale, int D) {
+  const double s = softmax_scale == 0.0f ? 1.0 / sqrt(static_cast<double>(D)) : softmax_scale;
+  return static_cast<float>(s * 1.4426950408889634);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t rq_abi_version(void) { return RQ_ABI_VERSION; }
+
+const char* rq_status_string(rq_status s) {
+  switch (s) {
+    case RQ_OK: return "RQ_OK";
+    case RQ_ERR_INVALID_ARG: return "RQ_ERR_INVALID_ARG";
+    case RQ_ERR_UNSUPPORTED: return "RQ_ERR_UNSUPPORTED";
+    case RQ_ERR_CAPACITY: return "RQ_ERR_CAPACITY";
+    case RQ_ERR_CUDA: return "RQ_ERR_CUDA";
+    case RQ_ERR_TIMEOUT: return "RQ_ERR_TIMEOUT";
+    case RQ_ERR_WORKSPACE: return "RQ_ERR_WORKSPACE";
+  }
+  return "RQ_ERR_UNKNOWN";
+}
+
+rq_status rq_layout_validate(const rq_layout* l) {
+  if (l == nullptr) return RQ_ERR_INVALID_ARG;
+  if (l->num_layers < 1 || l->num_loops < 1 || l->num_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
+  if (l->batch < 1 || l->kv_heads < 1 || l->max_tokens < 1) return RQ_ERR_INVALID_ARG;
+  if (l->policy != RQ_POLICY_LAST_LOOP && l->policy != RQ_POLICY_NEXT_LOOP) return RQ_ERR_INVALID_ARG;
+  if (l->reserved != 0) return RQ_ERR_INVALID_ARG;
+  if (!is_pow2(l->head_dim) || l->head_dim < 32 || l->head_dim > 256) return RQ_ERR_INVALID_ARG;
+  if (l->head_dim != 64 && l->head_dim != 128) return RQ_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(l->batch) * l->kv_heads > 65535) return RQ_ERR_UNSUPPORTED;
+  if (l->max_tokens > (1 << 30)) return RQ_ERR_UNSUPPORTED;
+  for (int r = 0; r < l->num_loops; ++r) {
+    const int b = l->bits[r], g = l->group[r];
+    if (b != 2 && b != 4) return RQ_ERR_INVALID_ARG;
+    if (!is_pow2(g) || g < 16 || g > 128 || g > l->head_dim) return RQ_ERR_INVALID_ARG;
+    if (g * b < 32) return RQ_ERR_INVALID_ARG;
+  }
+  return RQ_OK;
+}
+
+uint64_t rq_layer_bytes(const rq_layout* l) {
+  if (rq_layout_validate(l) != RQ_OK) return 0;
+  uint64_t c[RQ_MAX_LOOPS], m[RQ_MAX_LOOPS], a[RQ_MAX_LOOPS];
+  return layout_offsets(l, c, m, a);
+}
+
+uint64_t rq_cache_bytes(const rq_layout* l) {
+  const uint64_t lb = rq_layer_bytes(l);
+  return lb * (lb ? static_cast<uint64_t>(l->num_layers) : 0);
+}
+
+rq_status rq_cache_bind(const rq_layout* l, void* k_base, void* v_base, rq_cache* out) {
+  if (out == nullptr || k_base == nullptr || v_base == nullptr) return RQ_ERR_INVALID_ARG;
+  const rq_status st = rq_layout_validate(l);
+  if (st != RQ_OK) return st;
+  if (!aligned(k_base, kAlign) || !aligned(v_base, kAlign)) return RQ_ERR_INVALID_ARG;
+  memset(out, 0, sizeof(*out));
+  out->layout = *l;
+  out->k_base = k_base;
+  out->v_base = v_base;
+  out->layer_bytes = layout_offsets(l, out->codes_off, out->meta_off, out->alpha_off);
+  out->token_stride = token_stride_of(l);
+  return RQ_OK;
+}
+
+rq_status rq_quantize_anchor(const rq_cache* c, int32_t layer, int32_t kv, const void* x,
+                             int32_t t0, int32_t n, void* stream) {
+  rq_status st = check_cache(c, layer, kv);
+  if (st != RQ_OK) return st;
+  if ((st = check_range(c, t0, n)) != RQ_OK) return st;
+  if (n == 0) return RQ_OK;
+  if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
+  const rq_layout& l = c->layout;
+  const int a = l.num_loops - 1;
+  unsigned char* base = const_cast<unsigned char*>(side_base(c, layer, kv));
+  QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = static_cast<const uint16_t*>(x);
+  p.bh = l.batch * l.kv_heads;
+  p.n = n;
+  p.t0 = t0;
+  p.tstride = c->token_stride;
+  p.codes = reinterpret_cast<uint32_t*>(base + c->codes_off[a]);
+  p.meta = reinterpret_cast<uint32_t*>(base + c->meta_off[a]);
+  p.alpha = nullptr;
+  p.nref = 0;
+  p.rot_scale = rot_scale_of(l.head_dim);
+  return cuda_status(launch_quantize(p, l.head_dim, l.bits[a], l.group[a], as_stream(stream)));
+}
+
+rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t kv, int32_t loop,
+                                      const void* x, int32_t t0, int32_t n, void* stream) {
+  rq_status st = check_cache(c, layer, kv);
+  if (st != RQ_OK) return st;
+  const rq_layout& l = c->layout;
+  if (loop < 0 || loop >= l.num_loops - 1) return RQ_ERR_INVALID_ARG;
+  if ((st = check_range(c, t0, n)) != RQ_OK) return st;
+  if (n == 0) return RQ_OK;
+  if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
+  unsigned char* base = const_cast<unsigned char*>(side_base(c, layer, kv));
+  QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = static_cast<const uint16_t*>(x);
+  p.bh = l.batch * l.kv_heads;
+  p.n = n;
+  p.t0 = t0;
+  p.tstride = c->token_stride;
+  p.codes = reinterpret_cast<uint32_t*>(base + c->codes_off[loop]);
+  p.meta = reinterpret_cast<uint32_t*>(base + c->meta_off[loop]);
+  p.alpha = reinterpret_cast<uint16_t*>(base + c->alpha_off[loop]);
+  // Reference: the anchor (Last-loop) or the chain loop+1 .. anchor (Next-loop).
+  Comp chain[RQ_MAX_LOOPS];
+  const int len = chain_of(c, layer, kv, loop, chain);   // [loop, ref...]
+  p.nref = len - 1;
+  for (int i = 1; i < len; ++i) p.ref[i - 1] = chain[i];
+  p.rot_scale = rot_scale_of(l.head_dim);
+  return cuda_status(
+      launch_quantize(p, l.head_dim, l.bits[loop], l.group[loop], as_stream(stream)));
+}
+
+rq_status rq_dequantize(const rq_cache* c, int32_t layer, int32_t kv, int32_t loop, int32_t t0,
+                        int32_t n, float* out, void* stream) {
+  rq_status st = check_cache(c, layer, kv);
+  if (st != RQ_OK) return st;
+  const rq_layout& l = c->layout;
+  if (loop < 0 || loop >= l.num_loops) return RQ_ERR_INVALID_ARG;
+  if ((st = check_range(c, t0, n)) != RQ_OK) return st;
+  if (n == 0) return RQ_OK;
+  if (out == nullptr || !aligned(out, 16)) return RQ_ERR_INVALID_ARG;
+  DequantParams p;
+  memset(&p, 0, sizeof(p));
+  p.bh = l.batch * l.kv_heads;
+  p.n = n;
+  p.t0 = t0;
+  p.tstride = c->token_stride;
+  p.ncomp = chain_of(c, layer, kv, loop, p.comp);
+  p.rot_scale = rot_scale_of(l.head_dim);
+  p.out = out;
+  return cuda_status(launch_dequantize(p, l.head_dim, as_stream(stream)));
+}
+
+uint64_t rq_decode_workspace_bytes(const rq_layout* l, int32_t max_seq_len) {
+  if (rq_layout_validate(l) != RQ_OK || max_seq_len < 0) return 0;
+  return ws_layout(static_cast<int64_t>(l->batch) * l->kv_heads, l->head_dim, max_seq_len).total;
+}
+
+uint64_t rq_decode_bf16_workspace_bytes(int32_t batch, int32_t heads, int32_t head_dim,
+                                        int32_t max_seq_len) {
+  if (batch < 1 || heads < 1 || (head_dim != 64 && head_dim != 128) || max_seq_len < 0) return 0;
+  return ws_layout(static_cast<int64_t>(batch) * heads, head_dim, max_seq_len).total;
+}
+
+rq_status rq_decode_workspace_init(void* ws, uint64_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes == 0) return RQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, as_stream(stream)));
+}
+
+rq_status rq_workspace_error(void* ws, uint64_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < 4) return RQ_ERR_INVALID_ARG;
+  uint32_t h = 0;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaMemcpyAsync(&h, ws, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && h != 0) {
+    e = cudaMemsetAsync(ws, 0, 4, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return RQ_ERR_CUDA;
+  if (h & kErrTimeout) return RQ_ERR_TIMEOUT;
+  if (h & kErrSeqLen) return RQ_ERR_CAPACITY;
+  return RQ_OK;
+}
+
+static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t loop,
+                                    int32_t max_seq_len, DecodeParams* p, int* D) {
+  const rq_layout& l = c->layout;
+  memset(p, 0, sizeof(*p));
+  p->bh = l.batch * l.kv_heads;
+  p->heads = l.kv_heads;
+  p->tstride = c->token_stride;
+  p->ncomp = chain_of(c, layer, 0, loop, p->k);
+  (void)chain_of(c, layer, 1, loop, p->v);
+  p->max_seq_len = max_seq_len;
+  p->rot_scale = rot_scale_of(l.head_dim);
+  *D = l.head_dim;
+  p->stage_bytes = decode_stage_bytes(*p, *D);
+  int stages = static_cast<int>(kRingBudget / p->stage_bytes);
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 1 && 2 * kRingBudget >= p->stage_bytes) stages = 1;
+  if (stages < 1) return RQ_ERR_UNSUPPORTED;
+  p->stages = stages;
+  int occ = 0;
+  if (decode_occupancy(*D, false, decode_dyn_smem(*D, stages, p->stage_bytes), &occ) !=
+      cudaSuccess)
+    return RQ_ERR_CUDA;
+  choose_splits(p->bh, max_seq_len, occ, &p->splits, &p->chunks_per_split);
+  return RQ_OK;
+}
+
+int32_t rq_decode_splits(const rq_layout* l, int32_t max_seq_len) {
+  if (rq_layout_validate(l) != RQ_OK || max_seq_len < 0) return 0;
+  // Shape-only: a cache bound to dummy (aligned, never dereferenced) bases.
+  rq_cache c;
+  if (rq_cache_bind(l, reinterpret_cast<void*>(kAlign), reinterpret_cast<void*>(kAlign), &c) !=
+      RQ_OK)
+    return 0;
+  DecodeParams p;
+  int D = 0;
+  // loop 0 is the most expensive loop to decode (longest chain)
+  if (fill_decode_params(&c, 0, 0, max_seq_len, &p, &D) != RQ_OK) return 0;
+  return p.splits;
+}
+
+rq_status rq_decode_attention(const rq_cache* c, int32_t layer, int32_t loop, const void* q,
+                              const int32_t* seq_lens, int32_t max_seq_len, const void* k_cur,
+                              const void* v_cur, float softmax_scale, float* out,
+                              void* workspace, uint64_t ws_bytes, void* stream) {
+  rq_status st = check_cache(c, layer, 0);
+  if (st != RQ_OK) return st;
+  const rq_layout& l = c->layout;
+  if (loop < 0 || loop >= l.num_loops) return RQ_ERR_INVALID_ARG;
+  if (q == nullptr || seq_lens == nullptr || k_cur == nullptr || v_cur == nullptr ||
+      out == nullptr || workspace == nullptr)
+    return RQ_ERR_INVALID_ARG;
+  if (max_seq_len < 0) return RQ_ERR_INVALID_ARG;
+  if (max_seq_len > l.max_tokens) return RQ_ERR_CAPACITY;
+  if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return RQ_ERR_INVALID_ARG;
+  if (!aligned(workspace, kAlign)) return RQ_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(static_cast<int64_t>(l.batch) * l.kv_heads, l.head_dim, max_seq_len);
+  if (ws_bytes < w.total) return RQ_ERR_WORKSPACE;
+  DecodeParams p;
+  int D = 0;
+  if ((st = fill_decode_params(c, layer, loop, max_seq_len, &p, &D)) != RQ_OK) return st;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.q = static_cast<const uint16_t*>(q);
+  p.kcur = static_cast<const uint16_t*>(k_cur);
+  p.vcur = static_cast<const uint16_t*>(v_cur);
+  p.seq_lens = seq_lens;
+  p.scale_log2 = scale_log2_of(softmax_scale, D);
+  p.out = out;
+  p.err = reinterpret_cast<uint32_t*>(ws + w.err);
+  p.counters = reinterpret_cast<uint32_t*>(ws + w.counters);
+  p.partials = reinterpret_cast<float*>(ws + w.partials);
+  return cuda_status(launch_decode(p, D, as_stream(stream)));
+}
+
+rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads, int32_t head_dim, const void* q,
+                                   const void* k, const void* v, int64_t token_stride,
+                                   const int32_t* seq_lens, int32_t max_seq_len,
+                                   const void* k_cur, const void* v_cur, float softmax_scale,
+                                   float* out, void* workspace, uint64_t ws_bytes,
+                                   void* stream) {
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > 65535)
+    return RQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return RQ_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || seq_lens == nullptr || k_cur == nullptr ||
+      v_cur == nullptr || out == nullptr || workspace == nullptr)
+    return RQ_ERR_INVALID_ARG;
+  if (max_seq_len < 0 || token_stride < max_seq_len || token_stride < 1) return RQ_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(workspace, kAlign))
+    return RQ_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return RQ_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(static_cast<int64_t>(batch) * heads, head_dim, max_seq_len);
+  if (ws_bytes < w.total) return RQ_ERR_WORKSPACE;
+  DecodeBf16Params p;
+  memset(&p, 0, sizeof(p));
+  p.bh = batch * heads;
+  p.heads = heads;
+  p.tstride = token_stride;
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.q = static_cast<const uint16_t*>(q);
+  p.kcur = static_cast<const uint16_t*>(k_cur);
+  p.vcur = static_cast<const uint16_t*>(v_cur);
+  p.seq_lens = seq_lens;
+  p.max_seq_len = max_seq_len;
+  p.scale_log2 = scale_log2_of(softmax_scale, head_dim);
+  p.out = out;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.err = reinterpret_cast<uint32_t*>(ws + w.err);
+  p.counters = reinterpret_cast<uint32_t*>(ws + w.counters);
+  p.partials = reinterpret_cast<float*>(ws + w.partials);
+  p.stage_bytes = static_cast<uint32_t>(2 * kChunk * head_dim * 2);
+  int stages = static_cast<int>(kRingBudget / p.stage_bytes);
+  if (stages > kMaxStages) stages = kMaxStages;
+  p.stages = stages;
+  int occ = 0;
+  if (decode_occupancy(head_dim, true, decode_dyn_smem(head_dim, stages, p.stage_bytes), &occ) !=
+      cudaSuccess)
+    return RQ_ERR_CUDA;
+  choose_splits(p.bh, max_seq_len, occ, &p.splits, &p.chunks_per_split);
+  return cuda_status(launch_decode_bf16(p, head_dim, as_stream(stream)));
+}
+
+}  // extern "C"

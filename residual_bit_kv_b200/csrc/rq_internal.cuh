@@ -1,0 +1,200 @@
+// rq_internal.cuh -- device helpers and kernel parameter blocks shared by the
+// librq translation units (never installed; the public ABI is librq.h).
+//
+// Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
+// Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "librq.h"
+
+namespace rq {
+
+// Device-side error bits recorded in the decode workspace.
+constexpr uint32_t kErrSeqLen = 1u;    // a seq_lens entry was outside [0, max_seq_len]
+constexpr uint32_t kErrTimeout = 2u;   // a bounded mbarrier wait ran out
+
+// Tokens per pipeline stage of the decode kernels.
+constexpr int kChunk = 64;
+constexpr int kDecodeThreads = 128;
+
+// ---------------------------------------------------------------------------
+// Parameter blocks
+// ---------------------------------------------------------------------------
+
+// One packed component (anchor or one residual loop) of one side.
+struct Comp {
+  const uint32_t* codes;   // [rows][D*bits/32]
+  const uint32_t* meta;    // [rows][D/group]
+  const uint16_t* alpha;   // [rows] bf16, nullptr for the anchor
+  int32_t bits;
+  int32_t group;
+};
+
+struct QuantParams {
+  const uint16_t* x;       // bf16 [B*H][n][D]
+  int32_t bh;              // B*H
+  int32_t n;
+  int32_t t0;
+  int64_t tstride;
+  uint32_t* codes;         // destination component
+  uint32_t* meta;
+  uint16_t* alpha;         // nullptr for the anchor
+  // Reference chain, nearest first: for LAST_LOOP one entry (the anchor);
+  // for NEXT_LOOP loops loop+1 .. L-1 (the anchor last).
+  int32_t nref;
+  Comp ref[RQ_MAX_LOOPS];
+  float rot_scale;         // fp32(1/sqrt(D))
+};
+
+struct DequantParams {
+  int32_t bh, n, t0;
+  int64_t tstride;
+  int32_t ncomp;           // chain: [0] = the loop itself ... [ncomp-1] = anchor
+  Comp comp[RQ_MAX_LOOPS];
+  float rot_scale;
+  float* out;              // fp32 [B*H][n][D]
+};
+
+struct DecodeParams {
+  int32_t bh;              // B*H
+  int32_t heads;
+  int64_t tstride;
+  int32_t ncomp;           // [0] = the loop's own residual ... [ncomp-1] = anchor
+  Comp k[RQ_MAX_LOOPS];
+  Comp v[RQ_MAX_LOOPS];
+  const uint16_t* q;       // bf16 [B*H][D]
+  const uint16_t* kcur;
+  const uint16_t* vcur;
+  const int32_t* seq_lens; // [B]
+  int32_t max_seq_len;
+  float scale_log2;        // softmax scale * log2(e)
+  float rot_scale;
+  float* out;              // fp32 [B*H][D]
+  // workspace
+  float* partials;         // [B*H][splits][D+2]
+  uint32_t* counters;      // [B*H]
+  uint32_t* err;           // [1]
+  int32_t splits;
+  int32_t chunks_per_split;
+  int32_t stages;
+  uint32_t stage_bytes;
+};
+
+struct DecodeBf16Params {
+  int32_t bh, heads;
+  int64_t tstride;
+  const uint16_t* k;       // bf16 [B*H][tstride][D]
+  const uint16_t* v;
+  const uint16_t* q;
+  const uint16_t* kcur;
+  const uint16_t* vcur;
+  const int32_t* seq_lens;
+  int32_t max_seq_len;
+  float scale_log2;
+  float* out;
+  float* partials;
+  uint32_t* counters;
+  uint32_t* err;
+  int32_t splits;
+  int32_t chunks_per_split;
+  int32_t stages;
+  uint32_t stage_bytes;
+};
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in the .cu files)
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
+                            cudaStream_t s);
+cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t s);
+cudaError_t launch_decode_bf16(const DecodeBf16Params& p, int D,
+                               cudaStream_t s);
+// bytes of one pipeline stage for a decode call
+uint32_t decode_stage_bytes(const DecodeParams& p, int D);
+// dynamic shared memory of a decode launch (stage ring or merge scratch)
+size_t decode_dyn_smem(int D, int stages, uint32_t stage_bytes);
+// resident CTAs per SM of a decode kernel at this dynamic shared memory
+cudaError_t decode_occupancy(int D, bool bf16, size_t dyn_smem, int* ctas_per_sm);
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
+  return __uint_as_float(h << 16);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(count)
+               : "memory");
+}
+
+// Make barrier initialisation visible to the async (bulk-copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
+                                                      uint32_t bytes) {
+  asm volatile(
+      "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a phase of an mbarrier: gives up after ~2^22 polls (well
+// over a second with the back-off), records kErrTimeout and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint32_t* err) {
+  for (uint32_t it = 0; it < (1u << 22); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (it > 16) __nanosleep(256);
+  }
+  atomicOr(err, kErrTimeout);
+  return false;
+}
+
+// Bulk (non-tensor) asynchronous copy global -> this CTA's shared memory,
+// completing `bytes` of transaction count on `bar`.  No multicast.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src,
+                                              uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+}  // namespace rq

@@ -18,3 +18,23 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def librq_built():
+    """Builds (if stale) and loads the in-tree librq.so; GPU tests need a device."""
+    import torch
+    from residual_bit_kv_b200 import build
+    build.build()
+    import residual_bit_kv_b200.librq as L
+    L.load()
+    return L
+
+
+@pytest.fixture(scope="session")
+def cuda_dev(librq_built):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+    return torch.device("cuda")

@@ -1,0 +1,193 @@
+"""Test harness: builds packed caches through the C ABI and the matching
+oracle encodings from the same seeded inputs.
+
+Inputs come from residual_bit_kv_b200.synth (bit-identical on CPU and CUDA);
+expected values come only from the oracle.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle
+import residual_bit_kv_b200.librq as L
+import residual_bit_kv_b200.synth as synth
+
+SIDES = (synth.SIDE_K, synth.SIDE_V)
+
+
+def policy_code(policy: str) -> int:
+    return L.RQ_POLICY_LAST_LOOP if policy == "last" else L.RQ_POLICY_NEXT_LOOP
+
+
+def layout_of(w: synth.Workload, policy: str = "last", layers: Optional[int] = None,
+              max_tokens: Optional[int] = None) -> L.rq_layout:
+    return L.make_layout(layers or w.layers, w.loops, w.batch, w.heads, w.head_dim,
+                         max_tokens or (w.tokens + 1), w.bits, w.group, policy_code(policy))
+
+
+def append_order(w: synth.Workload, policy: str) -> List[int]:
+    """Anchor first, then residual loops (descending, as the chain requires)."""
+    return [w.loops - 1] + list(range(w.loops - 2, -1, -1))
+
+
+@dataclasses.dataclass
+class GpuCache:
+    w: synth.Workload
+    policy: str
+    layout: L.rq_layout
+    cache: L.rq_cache
+    kbuf: torch.Tensor
+    vbuf: torch.Tensor
+    inputs: Dict  # (layer, side, loop) -> bf16 [B, H, T, D] cuda tensor (if kept)
+
+
+def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
+                    keep_inputs: bool = True, tokens: Optional[int] = None,
+                    max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None
+                    ) -> GpuCache:
+    """Generates every loop's K/V on the GPU and quantise-appends them through
+    the C ABI in the order the policy requires.  append_chunks splits the
+    token range into consecutive appends (e.g. prefill then single tokens)."""
+    T = w.tokens if tokens is None else tokens
+    lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens)
+    nbytes = L.rq_cache_bytes(lay)
+    assert nbytes > 0
+    kbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    vbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    cache = L.rq_cache_bind(lay, kbuf, vbuf)
+    inputs = {}
+    bounds = [0] + list(np.cumsum(append_chunks)) if append_chunks else [0, T]
+    assert bounds[-1] == T
+    for layer in layers:
+        for side in SIDES:
+            xs = {loop: synth.kv_full(w, layer, side, loop, 0, T, device="cuda", chunk_b=4)
+                  for loop in range(w.loops)}
+            for a, b in zip(bounds[:-1], bounds[1:]):
+                if b == a:
+                    continue
+                for loop in append_order(w, policy):
+                    x = xs[loop][:, :, a:b].contiguous()
+                    if loop == w.loops - 1:
+                        L.rq_quantize_anchor(cache, layer, side, x, a, b - a)
+                    else:
+                        L.rq_quantize_append_residual(cache, layer, side, loop, x, a, b - a)
+            if keep_inputs:
+                for loop, x in xs.items():
+                    inputs[(layer, side, loop)] = x
+            del xs
+    torch.cuda.synchronize()
+    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs)
+
+
+def gpu_component(gc: GpuCache, layer: int, side: int, loop: int) -> Dict[str, np.ndarray]:
+    """Packed arrays of one component as numpy [B, H, tstride, ...] views."""
+    c = gc.cache
+    w = gc.w
+    buf = gc.kbuf if side == synth.SIDE_K else gc.vbuf
+    base = layer * c.layer_bytes
+    ts = c.token_stride
+    rows = w.batch * w.heads * ts
+    D = w.head_dim
+    W = D * w.bits[loop] // 32
+    G = D // w.group[loop]
+
+    def grab(off, n_bytes):
+        return buf[base + off: base + off + n_bytes].cpu().numpy()
+
+    out = {
+        "codes": grab(c.codes_off[loop], rows * W * 4).view(np.uint32).reshape(w.batch, w.heads, ts, W),
+        "meta": grab(c.meta_off[loop], rows * G * 4).view(np.uint32).reshape(w.batch, w.heads, ts, G),
+        "alpha": None,
+    }
+    if loop != w.loops - 1:
+        out["alpha"] = grab(c.alpha_off[loop], rows * 2).view(np.uint16).reshape(w.batch, w.heads, ts)
+    return out
+
+
+def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
+                  hsel: Sequence[int], t0: int, t1: int, policy: str = "last",
+                  x_loops: Optional[List[np.ndarray]] = None):
+    """Oracle encodings of the selected rows.  Returns (encs, x) where
+    x is uint16 [L, nb*nh*(t1-t0), D]."""
+    if x_loops is None:
+        cs = synth.key_channel_scale(w, layer) if side == synth.SIDE_K else None
+        x_loops = [synth.bits_of(synth.kv(w, layer, side, loop, bsel, hsel, t0, t1, "cpu", cs))
+                   .reshape(-1, w.head_dim) for loop in range(w.loops)]
+    x = np.stack(x_loops)
+    return oracle.encode_side(x, w.bits, w.group, policy), x
+
+
+def assert_component_equal(gpu: Dict[str, np.ndarray], enc: Dict[str, np.ndarray], shape,
+                           what: str) -> None:
+    """Bit-exact comparison of codes, metadata and LS coefficients."""
+    for key in ("codes", "meta", "alpha"):
+        g = gpu[key]
+        o = enc[key]
+        if o is None:
+            assert g is None
+            continue
+        g = np.ascontiguousarray(g).reshape(o.shape)
+        bad = np.count_nonzero(g != o)
+        assert bad == 0, f"{what} {key}: {bad} of {o.size} words differ"
+
+
+def decode_inputs(w: synth.Workload, layer: int, loop: int, device="cuda"):
+    q = synth.query(w, layer, loop, device)
+    kc = synth.current_token(w, layer, synth.SIDE_K, loop, device)
+    vc = synth.current_token(w, layer, synth.SIDE_V, loop, device)
+    return q.contiguous(), kc.contiguous(), vc.contiguous()
+
+
+class Workspace:
+    def __init__(self, layout: L.rq_layout, max_seq_len: int):
+        self.bytes = L.rq_decode_workspace_bytes(layout, max_seq_len)
+        assert self.bytes > 0
+        self.buf = torch.empty(self.bytes, dtype=torch.uint8, device="cuda")
+        L.rq_decode_workspace_init(self.buf, self.bytes)
+
+
+def gpu_decode(gc: GpuCache, layer: int, loop: int, seq_lens: Sequence[int], max_seq_len: int,
+               ws: Optional[Workspace] = None, scale: float = 0.0):
+    w = gc.w
+    q, kc, vc = decode_inputs(w, layer, loop)
+    sl = torch.tensor(list(seq_lens), dtype=torch.int32, device="cuda")
+    out = torch.empty(w.batch, w.heads, w.head_dim, dtype=torch.float32, device="cuda")
+    ws = ws or Workspace(gc.layout, max_seq_len)
+    L.rq_decode_attention(gc.cache, layer, loop, q, sl, max_seq_len, kc, vc, scale, out, ws.buf,
+                          ws.bytes)
+    torch.cuda.synchronize()
+    status = L.rq_workspace_error(ws.buf, ws.bytes)
+    return out.cpu().numpy().astype(np.float64), status
+
+
+def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
+                  hsel: Sequence[int], seq_lens: Sequence[int], policy: str = "last",
+                  inputs: Optional[Dict] = None, scale: Optional[float] = None) -> np.ndarray:
+    """fp64 oracle decode for the selected (b, h): [len(bsel), len(hsel), D]."""
+    T = max(int(seq_lens[b]) for b in bsel)
+    D = w.head_dim
+    outs = []
+    rec = {}
+    for side in SIDES:
+        xl = None
+        if inputs is not None:
+            xl = [synth.bits_of(inputs[(layer, side, l)][list(bsel)][:, list(hsel), :T].cpu())
+                  .reshape(-1, D) for l in range(w.loops)]
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl)
+        rec[side] = oracle.reconstruct(encs, loop, w.bits, w.group, policy).reshape(
+            len(bsel), len(hsel), T, D)
+    q = synth.bits_of(synth.query(w, layer, loop)).reshape(w.batch, w.heads, D)
+    kc = synth.bits_of(synth.current_token(w, layer, synth.SIDE_K, loop))
+    vc = synth.bits_of(synth.current_token(w, layer, synth.SIDE_V, loop))
+    bi, hi = np.ix_(list(bsel), list(hsel))
+    return oracle.decode_attention(rec[0], rec[1], q[bi, hi], [seq_lens[b] for b in bsel],
+                                   kc[bi, hi], vc[bi, hi], scale)
+
+
+def attn_tolerance(ref: np.ndarray) -> float:
+    """max-abs error bound: 2e-3 * max|out| (per the method's parity target)."""
+    return 2e-3 * float(np.max(np.abs(ref)))

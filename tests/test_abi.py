@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments on the host and sizes storage exactly."""
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L(librq_built):
+    return librq_built
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "librq.h")).read()
+    return sorted(set(re.findall(r"\b(rq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    lib = L.load()
+    names = _header_functions()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.SYMBOLS)
+    assert L.rq_abi_version() == 1
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.rq_status_string(s).startswith("RQ_")
+
+
+def _lay(L, **kw):
+    base = dict(num_layers=1, num_loops=4, batch=8, kv_heads=16, head_dim=128, max_tokens=4096,
+                bits=(2, 2, 2, 4), group=(32, 32, 32, 32))
+    base.update(kw)
+    return L.make_layout(**base)
+
+
+def test_layout_validation(L):
+    assert L.rq_layout_validate(_lay(L)) == L.RQ_OK
+    bad = [dict(num_loops=0), dict(num_loops=33), dict(batch=0), dict(head_dim=48),
+           dict(bits=(3, 2, 2, 4)), dict(group=(8, 32, 32, 32)), dict(group=(32, 32, 32, 256)),
+           dict(max_tokens=0), dict(num_layers=0)]
+    for kw in bad:
+        assert L.rq_layout_validate(_lay(L, **kw)) == L.RQ_ERR_INVALID_ARG, kw
+    assert L.rq_layout_validate(_lay(L, head_dim=256)) == L.RQ_ERR_UNSUPPORTED
+    assert L.rq_layout_validate(_lay(L, head_dim=32)) == L.RQ_ERR_UNSUPPORTED
+    lay = _lay(L)
+    lay.policy = 7
+    assert L.rq_layout_validate(lay) == L.RQ_ERR_INVALID_ARG
+    assert L.rq_cache_bytes(_lay(L, batch=0)) == 0
+
+
+@pytest.mark.parametrize("bits,group", [((2, 2, 2, 4), (32,) * 4), ((4, 2, 2, 4), (32,) * 4),
+                                        ((2,) * 7 + (4,), (64,) * 8), ((2, 2, 2, 4), (16, 16, 16, 32))])
+def test_cache_bytes_equal_effective_bits(L, bits, group):
+    """Stored bytes = sum over loops of (b + 32/g + [residual] 16/D) bits per
+    element, the oracle's accounting with fp16 scale + fp16 offset (32-bit metadata)."""
+    T = 4096
+    lay = _lay(L, num_loops=len(bits), bits=bits, group=group, max_tokens=T)
+    elems = 8 * 16 * T * 128
+    beff = oracle.effective_bits(bits, group, 128, 32, True)
+    want = beff * len(bits) * elems / 8
+    got = L.rq_layer_bytes(lay)
+    assert want <= got <= want + 256 * 3 * len(bits)     # only alignment padding on top
+    assert L.rq_cache_bytes(_lay(L, num_layers=3, num_loops=len(bits), bits=bits, group=group,
+                                 max_tokens=T)) == 3 * got
+
+
+def test_host_checks_reject_before_launch(L):
+    """Invalid arguments return an error status without touching the device."""
+    lay = _lay(L, max_tokens=100)
+    nb = L.rq_cache_bytes(lay)
+    assert L.rq_decode_workspace_bytes(lay, 100) > 0
+    with pytest.raises(L.RQError) as e:
+        L.rq_cache_bind(lay, 0, 0)
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+    with pytest.raises(L.RQError) as e:
+        L.rq_cache_bind(lay, 4096 + 8, 8192)          # misaligned base
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+    cache = L.rq_cache_bind(lay, 1 << 20, 1 << 30)    # never dereferenced below
+    for args, status in [((0, 0, 1 << 12, 90, 20), L.RQ_ERR_CAPACITY),
+                         ((0, 0, 1 << 12, -1, 2), L.RQ_ERR_INVALID_ARG),
+                         ((1, 0, 1 << 12, 0, 2), L.RQ_ERR_INVALID_ARG),
+                         ((0, 2, 1 << 12, 0, 2), L.RQ_ERR_INVALID_ARG),
+                         ((0, 0, None, 0, 2), L.RQ_ERR_INVALID_ARG),
+                         ((0, 0, (1 << 12) + 2, 0, 2), L.RQ_ERR_INVALID_ARG)]:
+        with pytest.raises(L.RQError) as e:
+            L.rq_quantize_anchor(cache, *args, stream=0)
+        assert e.value.status == status, args
+    with pytest.raises(L.RQError) as e:
+        L.rq_quantize_append_residual(cache, 0, 0, 3, 1 << 12, 0, 2, stream=0)   # 3 is the anchor
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+    with pytest.raises(L.RQError) as e:
+        L.rq_decode_attention(cache, 0, 0, 256, 256, 101, 256, 256, 0.0, 256, 256, 1 << 30,
+                              stream=0)
+    assert e.value.status == L.RQ_ERR_CAPACITY
+    with pytest.raises(L.RQError) as e:
+        L.rq_decode_attention(cache, 0, 0, 256, 256, 100, 256, 256, 0.0, 256, 256, 16, stream=0)
+    assert e.value.status == L.RQ_ERR_WORKSPACE
+    with pytest.raises(L.RQError) as e:
+        L.rq_decode_attention(cache, 0, 4, 256, 256, 100, 256, 256, 0.0, 256, 256, 1 << 30,
+                              stream=0)
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+    with pytest.raises(L.RQError) as e:
+        L.rq_decode_attention_bf16(1, 1, 96, 256, 256, 256, 10, 256, 10, 256, 256, 0.0, 256, 256,
+                                   1 << 20, stream=0)
+    assert e.value.status == L.RQ_ERR_UNSUPPORTED
+
+
+def test_no_cpu_fallback_in_product():
+    """The product package never imports the oracle."""
+    pkg = os.path.join(ROOT, "residual_bit_kv_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "rqo_" not in src, f

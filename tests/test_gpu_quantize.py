@@ -1,0 +1,135 @@
+"""GPU quantise-and-append through the C ABI vs the oracle: packed codes,
+fp16 metadata and bf16 LS coefficients must be bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import residual_bit_kv_b200.synth as synth
+from rq_harness import (SIDES, assert_component_equal, build_gpu_cache, gpu_component,
+                        oracle_encode)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_all(gc, layer=0, tokens=None, bsel=None, hsel=None, from_gpu_inputs=True):
+    w = gc.w
+    T = w.tokens if tokens is None else tokens
+    bsel = list(range(w.batch)) if bsel is None else bsel
+    hsel = list(range(w.heads)) if hsel is None else hsel
+    for side in SIDES:
+        xl = None
+        if from_gpu_inputs:
+            xl = [synth.bits_of(gc.inputs[(layer, side, l)][bsel][:, hsel].cpu()).reshape(-1, w.head_dim)
+                  for l in range(w.loops)]
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, gc.policy, xl)
+        for loop in range(w.loops):
+            g = gpu_component(gc, layer, side, loop)
+            gsel = {k: (None if v is None else v[np.ix_(bsel, hsel)][:, :, :T]) for k, v in g.items()}
+            assert_component_equal(gsel, encs[loop], None, f"side {side} loop {loop}")
+
+
+def test_generator_identical_on_cuda(cuda_dev):
+    """The shared generator draws the same bf16 values on the GPU and the host."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=50)
+    for side in SIDES:
+        for loop in range(w.loops):
+            a = synth.kv_full(w, 0, side, loop, 0, 50, device="cuda").cpu()
+            b = synth.kv_full(w, 0, side, loop, 0, 50, device="cpu")
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(synth.query(w, 0, 1, "cuda").cpu().view(torch.int16),
+                       synth.query(w, 0, 1, "cpu").view(torch.int16))
+
+
+def test_tiny_reference_bit_exact(cuda_dev):
+    """Tiny reference workload (2 loops, D=64, 256 tokens): every stored bit."""
+    gc = build_gpu_cache(synth.WORKLOADS["tiny"])
+    _check_all(gc, from_gpu_inputs=False)
+
+
+@pytest.mark.parametrize("bits,group,policy", [
+    ((2, 2, 2, 4), (32, 32, 32, 32), "last"),
+    ((4, 2, 2, 4), (32, 32, 32, 32), "last"),
+    ((2, 2, 2, 4), (16, 16, 16, 32), "last"),
+    ((2, 2, 4, 4), (64, 64, 16, 16), "last"),
+    ((2, 2, 2, 4), (128, 32, 64, 128), "next"),
+    ((2, 4, 2, 4), (32, 32, 32, 64), "next"),
+])
+def test_ragged_shapes_bit_exact(cuda_dev, bits, group, policy):
+    """Several warps, a ragged row tail and every bit-width / group size."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=203, bits=bits, group=group)
+    gc = build_gpu_cache(w, policy=policy)
+    _check_all(gc)
+
+
+def test_head_dim_64_chained_bit_exact(cuda_dev):
+    w = synth.WORKLOADS["huginn_deep"].replace(batch=1, heads=3, tokens=77, head_dim=64, loops=5,
+                                               bits=(2, 2, 4, 2, 4), group=(32, 16, 64, 64, 32),
+                                               sigma=(0.4, 0.3, 0.2, 0.1))
+    gc = build_gpu_cache(w, policy="next")
+    _check_all(gc)
+
+
+def test_appends_match_prefill(cuda_dev):
+    """Prefill followed by single-token appends at t0 = T, T+1, ... stores the
+    same bits as the oracle's whole-sequence encoding (rows are independent)."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=2, tokens=133)
+    gc = build_gpu_cache(w, append_chunks=[128, 1, 1, 3])
+    _check_all(gc)
+
+
+def test_edge_rows(cuda_dev):
+    """Zero rows (zero anchor -> alpha 0, constant groups -> codes 0), a row
+    equal to a power-of-two multiple of the anchor, and huge/small magnitudes."""
+    import residual_bit_kv_b200.librq as L
+    from rq_harness import layout_of
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=1, tokens=8)
+    lay = layout_of(w, max_tokens=8)
+    nb = L.rq_cache_bytes(lay)
+    kb = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    vb = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    cache = L.rq_cache_bind(lay, kb, vb)
+    g = torch.Generator().manual_seed(0)
+    anchor = torch.randn(1, 1, 8, 128, generator=g)
+    anchor[0, 0, 0] = 0.0                       # zero anchor row
+    anchor[0, 0, 1] = 3.0                       # constant row
+    anchor[0, 0, 5] *= 1e3
+    anchor[0, 0, 6] *= 1e-3
+    xs = {3: anchor.to(torch.bfloat16)}
+    for r in range(3):
+        x = anchor * 0.9 + 0.2 * torch.randn(1, 1, 8, 128, generator=g)
+        x[0, 0, 2] = anchor[0, 0, 2] * 2.0      # exact multiple of the anchor input
+        x[0, 0, 3] = 0.0
+        xs[r] = x.to(torch.bfloat16)
+    for side in (0, 1):
+        L.rq_quantize_anchor(cache, 0, side, xs[3].cuda(), 0, 8)
+        for r in (2, 1, 0):
+            L.rq_quantize_append_residual(cache, 0, side, r, xs[r].cuda(), 0, 8)
+    torch.cuda.synchronize()
+    x = np.stack([synth.bits_of(xs[l]).reshape(-1, 128) for l in range(4)])
+    encs = oracle.encode_side(x, w.bits, w.group)
+    from rq_harness import GpuCache
+    gc = GpuCache(w, "last", lay, cache, kb, vb, {})
+    for side in (0, 1):
+        for loop in range(4):
+            gcomp = gpu_component(gc, 0, side, loop)
+            gsel = {k: (None if v is None else v[:, :, :8]) for k, v in gcomp.items()}
+            assert_component_equal(gsel, encs[loop], None, f"edge loop {loop}")
+    assert encs[0]["alpha"][0] == 0                       # zero anchor -> alpha 0
+
+
+def test_dequantize_matches_oracle(cuda_dev):
+    import residual_bit_kv_b200.librq as L
+    for policy in ("last", "next"):
+        w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=2, tokens=150)
+        gc = build_gpu_cache(w, policy=policy)
+        for side in SIDES:
+            encs, _ = oracle_encode(w, 0, side, [0, 1], [0, 1], 0, 150, policy)
+            for loop in range(w.loops):
+                out = torch.empty(2, 2, 100, 128, dtype=torch.float32, device="cuda")
+                L.rq_dequantize(gc.cache, 0, side, loop, 25, 100, out)
+                torch.cuda.synchronize()
+                ref = oracle.reconstruct(encs, loop, w.bits, w.group, policy).reshape(2, 2, 150, 128)
+                ref = ref[:, :, 25:125]
+                err = np.max(np.abs(out.cpu().numpy() - ref))
+                assert err <= 2e-6 * np.max(np.abs(ref)) + 1e-7, (policy, side, loop, err)
