@@ -1,0 +1,586 @@
+#!/usr/bin/env python3
+"""Benchmark of the ResidualQuant decode step on B200.
+
+One step = one decode step of the 16k-context Ouro-like workload: for each of
+24 layers and 4 loops, compressed decode attention for every sequence of the
+batch (96 launches), then the quantise-and-append of the new token's K/V for
+every loop of every layer (anchor + 3 LS residuals, K and V: 192 launches).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rq|reference]
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle on a
+bounded sample of the same workload.  Under torchrun (N > 1) every rank runs
+the full per-GPU workload on its own sequences (weak scaling; (batch, head)
+units are independent, so no collective touches the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import residual_bit_kv_b200.synth as synth  # noqa: E402
+
+METRIC = "decode-attn tokens/s at 16k ctx"
+WORKLOAD = "ouro_16k"
+QUANT_WORKLOAD = "quantize_prefill"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- plumbing --
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws):
+    if ws <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.path is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def profile_traffic(kernel_file: str, profile_name: str):
+    """Per-launch DRAM traffic from a committed ncu summary, if it was taken on
+    the kernel source as it stands (else None)."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_sha or not m_tr:
+        return None
+    if m_sha.group(1) != file_sha(os.path.join(ROOT, "residual_bit_kv_b200", "csrc", kernel_file)):
+        return None
+    return float(m_tr.group(1))
+
+
+# ----------------------------------------------------------- byte accounting --
+
+def component_bytes_per_row(w, loop, policy="last"):
+    """Packed bytes of one (token, head) row of every component loop `loop`
+    reads, for one side (codes + fp16 scale/offset + bf16 LS coefficient)."""
+    D = w.head_dim
+    A = w.loops - 1
+    comps = [A] if loop == A else ([loop, A] if policy == "last" else list(range(loop, w.loops)))
+    tot = 0
+    for r in comps:
+        tot += D * w.bits[r] // 8 + (D // w.group[r]) * 4 + (2 if r != A else 0)
+    return tot
+
+
+def decode_call_bytes(w, loop, seq_len, policy="last"):
+    """Algorithmic bytes of one decode call: packed K and V of every past
+    token, plus q, k_cur, v_cur (bf16) and the fp32 output."""
+    bh = w.batch * w.heads
+    return bh * (2 * seq_len * component_bytes_per_row(w, loop, policy) + w.head_dim * (2 * 3 + 4))
+
+
+def quant_call_bytes(w, loop, n):
+    """Algorithmic bytes of one quantise call over n tokens: the bf16 input,
+    the packed output, and for a residual the packed anchor re-read."""
+    rows = w.batch * w.heads * n
+    D = w.head_dim
+    A = w.loops - 1
+    out = D * w.bits[loop] // 8 + (D // w.group[loop]) * 4 + (2 if loop != A else 0)
+    ref = 0 if loop == A else D * w.bits[A] // 8 + (D // w.group[A]) * 4
+    return rows * (2 * D + out + ref)
+
+
+# --------------------------------------------------------------- rq engine --
+
+class Engine:
+    """Resident packed caches of every layer plus the step's inputs."""
+
+    def __init__(self, w, device, seed_offset=0, keep_bf16_layers=0):
+        import residual_bit_kv_b200.librq as L
+        self.L = L
+        self.w = w = w.replace(seed=w.seed + seed_offset)
+        self.dev = device
+        T = w.tokens
+        self.lay = L.make_layout(w.layers, w.loops, w.batch, w.heads, w.head_dim, T + 16,
+                                 w.bits, w.group, L.RQ_POLICY_LAST_LOOP)
+        nb = L.rq_cache_bytes(self.lay)
+        self.kbuf = torch.empty(nb, dtype=torch.uint8, device=device)
+        self.vbuf = torch.empty(nb, dtype=torch.uint8, device=device)
+        self.cache = L.rq_cache_bind(self.lay, self.kbuf, self.vbuf)
+        self.bf16 = {}
+        for layer in range(w.layers):
+            for side in (0, 1):
+                xs = {}
+                for loop in [w.loops - 1] + list(range(w.loops - 2, -1, -1)):
+                    x = synth.kv_full(w, layer, side, loop, 0, T, device=device, chunk_b=4)
+                    if loop == w.loops - 1:
+                        L.rq_quantize_anchor(self.cache, layer, side, x, 0, T)
+                    else:
+                        L.rq_quantize_append_residual(self.cache, layer, side, loop, x, 0, T)
+                    if layer < keep_bf16_layers:
+                        xs[loop] = x
+                    else:
+                        del x
+                for loop, x in xs.items():
+                    # bf16 baseline buffer [B, H, T+16, D] with room for the appended token
+                    buf = torch.empty(w.batch, w.heads, T + 16, w.head_dim, dtype=torch.bfloat16,
+                                      device=device)
+                    buf[:, :, :T] = x
+                    self.bf16[(layer, side, loop)] = buf
+                del xs
+            torch.cuda.synchronize(device)
+        # step inputs: per (layer, loop) query and the current token's K/V
+        self.q, self.kc, self.vc = {}, {}, {}
+        for layer in range(w.layers):
+            for loop in range(w.loops):
+                self.q[(layer, loop)] = synth.query(w, layer, loop, device).contiguous()
+                self.kc[(layer, loop)] = synth.current_token(w, layer, 0, loop, device).contiguous()
+                self.vc[(layer, loop)] = synth.current_token(w, layer, 1, loop, device).contiguous()
+        self.seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
+        self.out = torch.empty(w.layers, w.loops, w.batch, w.heads, w.head_dim,
+                               dtype=torch.float32, device=device)
+        self.ws_bytes = L.rq_decode_workspace_bytes(self.lay, T)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        L.rq_decode_workspace_init(self.ws, self.ws_bytes)
+        self.bws_bytes = L.rq_decode_bf16_workspace_bytes(w.batch, w.heads, w.head_dim, T)
+        self.bws = torch.zeros(self.bws_bytes, dtype=torch.uint8, device=device)
+        torch.cuda.synchronize(device)
+
+    def launches_per_step(self):
+        w = self.w
+        return w.layers * w.loops + w.layers * w.loops * 2
+
+    def step(self, stream, ev=None, q=None, kc=None, vc=None):
+        """One decode step.  ev: optional list collecting (start, end) event
+        pairs around each decode-attention launch."""
+        L, w, T = self.L, self.w, self.w.tokens
+        q = q or self.q
+        kc = kc or self.kc
+        vc = vc or self.vc
+        for layer in range(w.layers):
+            for loop in range(w.loops):
+                if ev is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                L.rq_decode_attention(self.cache, layer, loop, q[(layer, loop)], self.seq, T,
+                                      kc[(layer, loop)], vc[(layer, loop)], 0.0,
+                                      self.out[layer, loop], self.ws, self.ws_bytes, stream)
+                if ev is not None:
+                    e1.record(stream)
+                    ev.append((e0, e1, loop))
+            # after the final loop: quantise and append the new token (position T)
+            for side, cur in ((0, kc), (1, vc)):
+                A = w.loops - 1
+                L.rq_quantize_anchor(self.cache, layer, side, cur[(layer, A)], T, 1, stream)
+                for loop in range(w.loops - 2, -1, -1):
+                    L.rq_quantize_append_residual(self.cache, layer, side, loop,
+                                                  cur[(layer, loop)], T, 1, stream)
+
+    def bf16_step(self, stream, ev=None, nlayers_buf=4):
+        L, w, T = self.L, self.w, self.w.tokens
+        for layer in range(w.layers):
+            lb = layer % nlayers_buf
+            for loop in range(w.loops):
+                k = self.bf16[(lb, 0, loop)]
+                v = self.bf16[(lb, 1, loop)]
+                if ev is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                L.rq_decode_attention_bf16(w.batch, w.heads, w.head_dim, self.q[(layer, loop)], k,
+                                           v, T + 16, self.seq, T, self.kc[(layer, loop)],
+                                           self.vc[(layer, loop)], 0.0, self.out[layer, loop],
+                                           self.bws, self.bws_bytes, stream)
+                if ev is not None:
+                    e1.record(stream)
+                    ev.append((e0, e1, loop))
+            for loop in range(w.loops):
+                self.bf16[(lb, 0, loop)][:, :, T].copy_(self.kc[(layer, loop)], non_blocking=True)
+                self.bf16[(lb, 1, loop)][:, :, T].copy_(self.vc[(layer, loop)], non_blocking=True)
+
+
+def timed(fn, steps, warmup, stream, dist=None):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+# --------------------------------------------------------- oracle (CPU) legs --
+
+def oracle_decode_sample(w, pairs, loops):
+    """Times the oracle's decode of `pairs` (b, h) units for `loops` of layer 0:
+    reconstruction of every past row in fp64 and exact softmax attention.
+    Encoding the sample cache is set-up, not timed."""
+    import oracle
+    T = w.tokens
+    D = w.head_dim
+    encs = {}
+    for side in (0, 1):
+        cs = synth.key_channel_scale(w, 0) if side == 0 else None
+        xl = []
+        for loop in range(w.loops):
+            rows = [synth.bits_of(synth.kv(w, 0, side, loop, [b], [h], 0, T, "cpu", cs)).reshape(-1, D)
+                    for b, h in pairs]
+            xl.append(np.concatenate(rows))
+        encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
+    q = synth.bits_of(torch.stack([synth.query(w, 0, l) for l in range(w.loops)]))
+    kc = {l: synth.bits_of(synth.current_token(w, 0, 0, l)) for l in loops}
+    vc = {l: synth.bits_of(synth.current_token(w, 0, 1, l)) for l in loops}
+    t0 = time.perf_counter()
+    units = 0
+    for loop in loops:
+        kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(len(pairs), T, D)
+        vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(len(pairs), T, D)
+        for i, (b, h) in enumerate(pairs):
+            oracle.attention(oracle.bf16_bits_to_f64(q[loop, b, h]), kh[i], vh[i],
+                             oracle.bf16_bits_to_f64(kc[loop][b, h]),
+                             oracle.bf16_bits_to_f64(vc[loop][b, h]), 1.0 / np.sqrt(D))
+            units += 1
+    return time.perf_counter() - t0, units
+
+
+def cpu_baseline(w):
+    """Oracle decode on a bounded sample: 2 (batch, head) units x 4 loops of
+    layer 0 at the full 16k context, scaled to the step's 24*4*B*H units."""
+    pairs = [(0, 0), (w.batch - 1, w.heads - 1)]
+    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)))
+    step_units = w.layers * w.loops * w.batch * w.heads
+    step_s = secs / units * step_units
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens} "
+                      f"({secs:.1f} s), scaled to {step_units} units per step"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[WORKLOAD]
+    pairs = [(0, 0)]
+    for _ in range(args.warmup):
+        oracle_decode_sample(w, pairs, [w.loops - 1])
+    times = []
+    for _ in range(args.steps):
+        secs, units = oracle_decode_sample(w, pairs, [0])
+        times.append(secs / units)
+    per_unit = statistics.median(times)
+    step_units = w.layers * w.loops * w.batch * w.heads
+    step_s = per_unit * step_units
+    value = w.batch / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based generator)",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: 1 (batch,head) unit of loop 0, layer 0 at T=16384, "
+                                   f"scaled to {step_units} units"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: {w.layers} layers x {w.loops} loops, batch {w.batch}, "
+                        f"{w.heads} KV heads, head_dim {w.head_dim}, {w.tokens} past tokens, "
+                        f"bits {list(w.bits)}, group {w.group[0]}, Last-loop anchor",
+            "global_batch": w.batch, "seq_len": w.tokens,
+            "l2": "inputs larger than L2: every decode call streams >= 0.67 GB of packed KV",
+            "parallelism": "replicated workload per GPU (batch/head units independent)"}
+
+
+# --------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="rq", choices=["rq", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the BF16 baseline kernel")
+    ap.add_argument("--layers", type=int, default=None, help="override layer count (debug)")
+    args = ap.parse_args()
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    dist = init_dist(ws)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from residual_bit_kv_b200 import build
+    build.build()
+    w = synth.WORKLOADS[WORKLOAD]
+    if args.layers:
+        w = w.replace(layers=args.layers)
+    nbuf = 0 if args.no_bf16 else 4
+    eng = Engine(w, dev, seed_offset=1000 * rank, keep_bf16_layers=nbuf)
+    w = eng.w
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- main timed region: the decode step, per-launch events on the decode kernel
+    ev = []
+    for _ in range(args.warmup):
+        eng.step(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            eng.step(stream, ev)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.summary()
+    dec_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
+    dec_bytes = args.steps * w.layers * sum(decode_call_bytes(w, l, w.tokens) for l in range(w.loops))
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    per_loop = {}
+    for l in range(w.loops):
+        t_l = sum(a.elapsed_time(b) for a, b, ll in ev if ll == l) / (args.steps * w.layers)
+        per_loop[str(l)] = {"us": t_l * 1e3,
+                            "gbs": decode_call_bytes(w, l, w.tokens) / (t_l * 1e-3) / 1e9}
+    hbm, hbm_kind = peaks()
+    n_launch_dec = args.steps * w.layers * w.loops
+    traffic = profile_traffic("rq_decode.cu", "decode_kernel_ouro_16k.md")
+
+    # ---- end to end: host buffers, H2D of the step's inputs, D2H of the outputs
+    pin = {k: v.cpu().pin_memory() for k, v in eng.q.items()}
+    pkc = {k: v.cpu().pin_memory() for k, v in eng.kc.items()}
+    pvc = {k: v.cpu().pin_memory() for k, v in eng.vc.items()}
+    hout = torch.empty(eng.out.shape, dtype=torch.float32).pin_memory()
+    dq = {k: torch.empty_like(v) for k, v in eng.q.items()}
+    dkc = {k: torch.empty_like(v) for k, v in eng.kc.items()}
+    dvc = {k: torch.empty_like(v) for k, v in eng.vc.items()}
+
+    def e2e_step():
+        for k in pin:
+            dq[k].copy_(pin[k], non_blocking=True)
+            dkc[k].copy_(pkc[k], non_blocking=True)
+            dvc[k].copy_(pvc[k], non_blocking=True)
+        eng.step(stream, None, dq, dkc, dvc)
+        hout.copy_(eng.out, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, args.steps, args.warmup, stream, dist)
+    h2d = sum(v.numel() * 2 for v in pin.values()) * 3
+    d2h = hout.numel() * 4
+
+    # ---- BF16 baseline kernel on identical K/V (4 distinct layer buffers cycled)
+    bf16 = None
+    if not args.no_bf16:
+        bev = []
+        bms = timed(lambda: eng.bf16_step(stream), args.steps, args.warmup, stream, dist)
+        eng.bf16_step(stream, bev)
+        torch.cuda.synchronize()
+        bdec_ms = sum(a.elapsed_time(b) for a, b, _ in bev)
+        bbytes = w.layers * w.loops * w.batch * w.heads * (
+            2 * w.tokens * w.head_dim * 2 + w.head_dim * (2 * 3 + 4))
+        bf16 = {"tokens_per_s": w.batch * 1e3 / bms, "ms_per_step": bms,
+                "decode_gbs": bbytes / (bdec_ms * 1e-3) / 1e9,
+                "frac_of_hbm": bbytes / (bdec_ms * 1e-3) / 1e9 / hbm,
+                "bytes_per_step": bbytes,
+                "note": "same split-K engine on uncompressed bf16 K/V; 4 distinct layer buffers"}
+
+    # ---- prefill-sized quantise (anchor + 3 residuals, K and V), separate workload
+    quant = None
+    if rank == 0 or ws > 1:
+        quant = bench_quantize(dev, stream, args, hbm)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        value = ws * w.batch * 1e3 / ms
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded counter-based generator; Ouro-like looped KV)",
+            "config": config_of(w),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic,
+                         "kernel": "decode_kernel<128>", "peak_kind": hbm_kind,
+                         "bytes_per_step": dec_bytes / args.steps},
+            "decode_per_loop": per_loop,
+            "decode_hbm_frac_of_8tbs": achieved / 8000.0,
+            "e2e": {"value": ws * w.batch * 1e3 / e2e_ms, "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * eng.launches_per_step(),
+            "clocks": clocks,
+            "bf16_baseline": bf16,
+            "quantize": quant,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_quantize(dev, stream, args, hbm):
+    """Quantise-and-append of a 16k-token prefill: anchor then 3 residual loops,
+    for K and V (8 launches per pass).  Reports input GB/s and the fraction of
+    HBM for the bytes the pass must move."""
+    import residual_bit_kv_b200.librq as L
+    w = synth.WORKLOADS[QUANT_WORKLOAD]
+    T = w.tokens
+    lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T, w.bits, w.group,
+                        L.RQ_POLICY_LAST_LOOP)
+    nb = L.rq_cache_bytes(lay)
+    kb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    vb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    cache = L.rq_cache_bind(lay, kb, vb)
+    xs = {(s, l): synth.kv_full(w, 0, s, l, 0, T, device=dev, chunk_b=1)
+          for s in (0, 1) for l in range(w.loops)}
+    ev = []
+
+    def one(record=False):
+        for s in (0, 1):
+            for l in [w.loops - 1] + list(range(w.loops - 2, -1, -1)):
+                if record:
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                if l == w.loops - 1:
+                    L.rq_quantize_anchor(cache, 0, s, xs[(s, l)], 0, T, stream)
+                else:
+                    L.rq_quantize_append_residual(cache, 0, s, l, xs[(s, l)], 0, T, stream)
+                if record:
+                    b.record(stream)
+                    ev.append((a, b, l))
+
+    ms = timed(one, args.steps, args.warmup, stream)
+    one(True)
+    torch.cuda.synchronize()
+    inp = 2 * w.loops * w.batch * w.heads * T * w.head_dim * 2
+    req = 2 * sum(quant_call_bytes(w, l, T) for l in range(w.loops))
+    kern_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
+    res_ms = sum(a.elapsed_time(b) for a, b, l in ev if l != w.loops - 1)
+    res_bytes = 2 * sum(quant_call_bytes(w, l, T) for l in range(w.loops - 1))
+    return {"workload": f"{w.name}: batch {w.batch}, {w.heads} heads, {T} tokens, {w.loops} loops, "
+                        f"bits {list(w.bits)}, g {w.group[0]}, K and V",
+            "ms_per_pass": ms, "input_gbs": inp / (ms * 1e-3) / 1e9,
+            "required_gbs": req / (kern_ms * 1e-3) / 1e9,
+            "frac_of_hbm": req / (kern_ms * 1e-3) / 1e9 / hbm,
+            "residual_kernel_gbs": res_bytes / (res_ms * 1e-3) / 1e9,
+            "residual_codes_per_pass": 2 * (w.loops - 1) * w.batch * w.heads * T * w.head_dim}
+
+
+if __name__ == "__main__":
+    sys.exit(main())
