@@ -517,6 +517,7 @@ def main():
                          "kernel": "decode_kernel<128>", "peak_kind": hbm_kind,
                          "bytes_per_step": dec_bytes / args.steps},
             "decode_per_loop": per_loop,
+            "decode_splits_loop0": eng.L.rq_decode_splits(eng.lay, w.tokens),
             "decode_hbm_frac_of_8tbs": achieved / 8000.0,
             "e2e": {"value": ws * w.batch * 1e3 / e2e_ms, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -66,24 +66,32 @@ int max_splits_of(int32_t max_seq_len) {
   return c > kMaxSplits ? kMaxSplits : c;
 }
 
-// Split count minimising (waves of CTAs) x (chunks per CTA), the time model
-// of a bandwidth-bound grid whose CTAs stream equal token ranges.
-void choose_splits(int bh, int32_t max_seq_len, int ctas_per_sm, int* splits, int* cps) {
-  const int chunks = chunks_of(max_seq_len);
+// Split count for a grid of bh * splits CTAs, each streaming `cps` chunks.
+// Time model: (waves of resident CTAs) x (chunks per CTA); splits start at
+// the count that fills every resident slot once, so a small batch still
+// occupies the whole GPU.  Splits never exceed max_splits_of() (the
+// workspace bound) and never leave an empty split.
+void choose_splits(int bh, int32_t max_seq_len, int chunk, int ctas_per_sm, int* splits,
+                   int* cps) {
+  const int chunks = (max_seq_len + chunk - 1) / chunk;
   if (chunks == 0) {
     *splits = 1;
     *cps = 0;
     return;
   }
   const int64_t slots = static_cast<int64_t>(device_sms()) * (ctas_per_sm > 0 ? ctas_per_sm : 1);
-  const int smax = max_splits_of(max_seq_len);
+  int smax = max_splits_of(max_seq_len);
+  if (smax > chunks) smax = chunks;
+  int smin = static_cast<int>((slots + bh - 1) / bh);
+  if (smin > smax) smin = smax;
+  if (smin < 1) smin = 1;
   double best = 1e300;
-  int best_s = 1;
-  for (int s = 1; s <= smax; ++s) {
+  int best_s = smin;
+  for (int s = smin; s <= smax; ++s) {
     const int c = (chunks + s - 1) / s;
-    if (s > 1 && (chunks + c - 1) / c != s) continue;   // would leave empty splits
+    if ((chunks + c - 1) / c != s) continue;   // would leave empty splits
     const int64_t waves = (static_cast<int64_t>(bh) * s + slots - 1) / slots;
-    const double cost = static_cast<double>(waves) * c + 0.01 * s;
+    const double cost = static_cast<double>(waves) * c * (1.0 + 1e-3 * s);
     if (cost < best) {
       best = cost;
       best_s = s;
@@ -348,17 +356,22 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
   p->max_seq_len = max_seq_len;
   p->rot_scale = rot_scale_of(l.head_dim);
   *D = l.head_dim;
-  p->stage_bytes = decode_stage_bytes(*p, *D);
-  int stages = static_cast<int>(kRingBudget / p->stage_bytes);
-  if (stages > kMaxStages) stages = kMaxStages;
-  if (stages < 1 && 2 * kRingBudget >= p->stage_bytes) stages = 1;
-  if (stages < 1) return RQ_ERR_UNSUPPORTED;
+  int stages = 0, occ = 0, chunk = kChunk;
+  if (fast_decode_plan(*p, *D, kRingBudget, kMaxStages, &stages, &occ)) {
+    p->use_fast = 1;
+    chunk = fast_chunk();
+  } else {
+    p->use_fast = 0;
+    p->stage_bytes = decode_stage_bytes(*p, *D);
+    stages = static_cast<int>(kRingBudget / p->stage_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 1 && 2 * kRingBudget >= p->stage_bytes) stages = 1;
+    if (stages < 1) return RQ_ERR_UNSUPPORTED;
+    if (decode_occupancy(*D, decode_dyn_smem(*D, stages, p->stage_bytes), &occ) != cudaSuccess)
+      return RQ_ERR_CUDA;
+  }
   p->stages = stages;
-  int occ = 0;
-  if (decode_occupancy(*D, false, decode_dyn_smem(*D, stages, p->stage_bytes), &occ) !=
-      cudaSuccess)
-    return RQ_ERR_CUDA;
-  choose_splits(p->bh, max_seq_len, occ, &p->splits, &p->chunks_per_split);
+  choose_splits(p->bh, max_seq_len, chunk, occ, &p->splits, &p->chunks_per_split);
   return RQ_OK;
 }
 
@@ -406,7 +419,8 @@ rq_status rq_decode_attention(const rq_cache* c, int32_t layer, int32_t loop, co
   p.err = reinterpret_cast<uint32_t*>(ws + w.err);
   p.counters = reinterpret_cast<uint32_t*>(ws + w.counters);
   p.partials = reinterpret_cast<float*>(ws + w.partials);
-  return cuda_status(launch_decode(p, D, as_stream(stream)));
+  return cuda_status(p.use_fast ? launch_decode_fast(p, D, as_stream(stream))
+                                : launch_decode(p, D, as_stream(stream)));
 }
 
 rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads, int32_t head_dim, const void* q,
@@ -445,15 +459,14 @@ rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads, int32_t head_di
   p.err = reinterpret_cast<uint32_t*>(ws + w.err);
   p.counters = reinterpret_cast<uint32_t*>(ws + w.counters);
   p.partials = reinterpret_cast<float*>(ws + w.partials);
-  p.stage_bytes = static_cast<uint32_t>(2 * kChunk * head_dim * 2);
+  p.stage_bytes = bf16_stage_bytes(head_dim);
   int stages = static_cast<int>(kRingBudget / p.stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) stages = 2;
   p.stages = stages;
   int occ = 0;
-  if (decode_occupancy(head_dim, true, decode_dyn_smem(head_dim, stages, p.stage_bytes), &occ) !=
-      cudaSuccess)
-    return RQ_ERR_CUDA;
-  choose_splits(p.bh, max_seq_len, occ, &p.splits, &p.chunks_per_split);
+  if (bf16_occupancy(head_dim, stages, &occ) != cudaSuccess) return RQ_ERR_CUDA;
+  choose_splits(p.bh, max_seq_len, bf16_chunk(head_dim), occ, &p.splits, &p.chunks_per_split);
   return cuda_status(launch_decode_bf16(p, head_dim, as_stream(stream)));
 }
 

@@ -1,5 +1,7 @@
-// rq_decode.cu -- split-K decode attention over the packed ResidualQuant
-// cache, and the uncompressed BF16 decode kernel on the same engine.
+// rq_decode.cu -- generic split-K decode attention over the packed
+// ResidualQuant cache: any chain of components with run-time bit widths and
+// group sizes.  Layouts compiled into rq_decode_fast.cu take the
+// warp-specialised kernel instead; this one covers every other layout.
 //
 // Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
 // Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
@@ -21,14 +23,10 @@
 // the workspace; the last CTA of a (batch, head) -- elected by an atomic
 // counter, no waiting -- merges the splits and the current token's bf16
 // k/v [RQ §4.2 Decode], applies H^T once and writes the output.
-#include <math.h>
-
-#include "rq_internal.cuh"
+#include "rq_decode_common.cuh"
 
 namespace rq {
 namespace {
-
-constexpr float kNegInf = -INFINITY;
 
 template <int D>
 struct Geom {
@@ -38,18 +36,6 @@ struct Geom {
   static constexpr int TT = kChunk / TPC;     // tokens per thread per chunk
   static constexpr int NSLOT = kDecodeThreads / P;
 };
-
-// Exact small-integer -> float conversion: 0x4B000000 | c is 2^23 + c.
-__device__ __forceinline__ float code_to_float(uint32_t c) {
-  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
-}
-
-__device__ __forceinline__ void unpack_meta(uint32_t mw, float& s, float& z) {
-  const __half2 h = *reinterpret_cast<const __half2*>(&mw);
-  const float2 f = __half22float2(h);
-  s = f.x;
-  z = f.y;
-}
 
 // Per-component shared-memory offsets inside one pipeline stage.
 struct StageMap {
@@ -145,122 +131,6 @@ __device__ __forceinline__ void comp_acc(const uint32_t* cw, const uint32_t* mro
     const uint32_t c = (w[ch / PER_WORD] >> (BITS * (ch % PER_WORD))) & QMAX;
     acc[ch] = fmaf(ch < 16 ? w0 : w1, code_to_float(c), acc[ch]);
   }
-}
-
-__device__ __forceinline__ int log2_pow2(int v) { return 31 - __clz(v); }
-
-// In-place normalised-free Hadamard butterflies over D values in shared
-// memory, D threads participating (thread t < D).
-template <int D>
-__device__ __forceinline__ void smem_fwht(float* v) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int h = 1; h < D; h <<= 1) {
-    if (t < D && (t & h) == 0) {
-      const float a = v[t], b = v[t + h];
-      v[t] = a + b;
-      v[t + h] = a - b;
-    }
-    __syncthreads();
-  }
-}
-
-// Reduction of the per-slot online-softmax states of a CTA into one partial
-// (m, l, acc[D]) in the workspace, then the last-CTA merge of all splits with
-// the current token.  `stage_mem` is free scratch of at least
-// (NSLOT*D + 2*NSLOT) floats.  ROT: apply H^T to the merged accumulator.
-template <int D, bool ROT>
-__device__ __forceinline__ void finish(float m, float l, float (&acc)[32], int slice,
-                                       int slot, float* stage_mem, int bhi, int split,
-                                       int splits, float* partials, uint32_t* counters,
-                                       const uint16_t* q, const uint16_t* kcur,
-                                       const uint16_t* vcur, float scale_log2,
-                                       float rot_scale, float* out, float* svec,
-                                       float* sred) {
-  using G = Geom<D>;
-  float* red = stage_mem;                       // [NSLOT][D]
-  float* mred = red + G::NSLOT * D;             // [NSLOT]
-  float* lred = mred + G::NSLOT;                // [NSLOT]
-  const int t = threadIdx.x;
-  if (slice == 0) {
-    mred[slot] = m;
-    lred[slot] = l;
-  }
-  __syncthreads();
-  float M = kNegInf;
-  for (int s = 0; s < G::NSLOT; ++s) M = fmaxf(M, mred[s]);
-  const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - M);
-  float4* dst = reinterpret_cast<float4*>(red + slot * D + slice * 32);
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    dst[i] = make_float4(acc[4 * i] * f, acc[4 * i + 1] * f, acc[4 * i + 2] * f,
-                         acc[4 * i + 3] * f);
-  __syncthreads();
-  float* part = partials + (static_cast<size_t>(bhi) * splits + split) * (D + 2);
-  if (t < D) {
-    float sum = 0.0f;
-    for (int s = 0; s < G::NSLOT; ++s) sum += red[s * D + t];
-    part[2 + t] = sum;
-  }
-  if (t == 0) {
-    float L = 0.0f;
-    for (int s = 0; s < G::NSLOT; ++s)
-      L += (mred[s] == kNegInf) ? 0.0f : lred[s] * fast_exp2(mred[s] - M);
-    part[0] = M;
-    part[1] = L;
-  }
-  // Publish the partial, then count this split in.
-  __threadfence();
-  __syncthreads();
-  __shared__ uint32_t s_last;
-  if (t == 0) s_last = (atomicAdd(counters + bhi, 1u) == static_cast<uint32_t>(splits - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // ---- last CTA of this (batch, head): merge ----
-  // Current token score q.k_cur in the original domain [RQ §3.2, §4.2].
-  float qk = 0.0f;
-  if (t < D) qk = bf16_bits_to_f32(q[static_cast<size_t>(bhi) * D + t]) *
-                  bf16_bits_to_f32(kcur[static_cast<size_t>(bhi) * D + t]);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
-  if ((t & 31) == 0) sred[t >> 5] = qk;
-  __syncthreads();
-  const float s_cur = (sred[0] + sred[1] + sred[2] + sred[3]) * scale_log2;
-  const float* pbase = partials + static_cast<size_t>(bhi) * splits * (D + 2);
-  float Mx = s_cur;
-  for (int s = 0; s < splits; ++s) Mx = fmaxf(Mx, __ldcg(pbase + s * (D + 2)));
-  float Lx = fast_exp2(s_cur - Mx);
-  float ax = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = __ldcg(pbase + s * (D + 2));
-    if (ms == kNegInf) continue;
-    const float fs = fast_exp2(ms - Mx);
-    Lx += __ldcg(pbase + s * (D + 2) + 1) * fs;
-    if (t < D) ax += __ldcg(pbase + s * (D + 2) + 2 + t) * fs;
-  }
-  if (t < D) svec[t] = ax;
-  __syncthreads();
-  if constexpr (ROT) smem_fwht<D>(svec);
-  if (t < D) {
-    const float pc = fast_exp2(s_cur - Mx);
-    const float v = ROT ? svec[t] * rot_scale : svec[t];
-    out[static_cast<size_t>(bhi) * D + t] =
-        (v + pc * bf16_bits_to_f32(vcur[static_cast<size_t>(bhi) * D + t])) / Lx;
-  }
-  if (t == 0) counters[bhi] = 0u;   // ready for the next call
-}
-
-// Sequence length of batch row b, clamped to [0, max_seq_len] and flagged.
-__device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int max_seq_len,
-                                          uint32_t* err) {
-  int n = seq_lens[b];
-  if (n < 0 || n > max_seq_len) {
-    if (threadIdx.x == 0) atomicOr(err, kErrSeqLen);
-    n = n < 0 ? 0 : max_seq_len;
-  }
-  return n;
 }
 
 template <int D>
@@ -441,146 +311,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
   for (int ch = 0; ch < 32; ++ch) acc[ch] += (ch < 16) ? cst0 : cst1;
   __syncthreads();
-  finish<D, true>(m, l, acc, slice, slot, reinterpret_cast<float*>(smem), bhi, split,
-                  p.splits, p.partials, p.counters, p.q, p.kcur, p.vcur, p.scale_log2,
-                  p.rot_scale, p.out, svec, sred);
-}
-
-// Uncompressed bf16 rows: K and V [B*H][tstride][D].
-template <int D>
-__global__ void __launch_bounds__(kDecodeThreads)
-    decode_bf16_kernel(const __grid_constant__ DecodeBf16Params p) {
-  using G = Geom<D>;
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t full_bar[8];
-  __shared__ float svec[D];
-  __shared__ float sred[4];
-  __shared__ int s_abort;
-
-  const int t = threadIdx.x;
-  const int lane = t & 31, warp = t >> 5;
-  const int slice = lane % G::P;
-  const int tw = lane / G::P;
-  const int slot = warp * G::TPW + tw;
-  const int split = blockIdx.x;
-  const int bhi = blockIdx.y;
-  const int b = bhi / p.heads;
-  const int S = p.stages;
-  constexpr uint32_t kRowBytes = D * 2;
-
-  const int n = seq_len_of(p.seq_lens, b, p.max_seq_len, p.err);
-  const int t_begin = split * p.chunks_per_split * kChunk;
-  const int t_end = min(n, t_begin + p.chunks_per_split * kChunk);
-  const int nchunks = t_end > t_begin ? (t_end - t_begin + kChunk - 1) / kChunk : 0;
-
-  if (t == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full_bar[s], 1);
-    fence_barrier_init();
-    s_abort = 0;
-  }
-  __syncthreads();
-  const size_t row0 = static_cast<size_t>(bhi) * p.tstride;
-  auto issue = [&](int i) {
-    const int s = i % S;
-    const int t0 = t_begin + i * kChunk;
-    const int nt = min(kChunk, t_end - t0);
-    unsigned char* st = smem + static_cast<size_t>(s) * p.stage_bytes;
-    mbar_arrive_expect_tx(&full_bar[s], 2u * nt * kRowBytes);
-    bulk_copy_g2s(st, p.k + (row0 + t0) * D, nt * kRowBytes, &full_bar[s]);
-    bulk_copy_g2s(st + kChunk * kRowBytes, p.v + (row0 + t0) * D, nt * kRowBytes,
-                  &full_bar[s]);
-  };
-  int issued = 0;
-  if (t == 0) {
-    for (; issued < min(S, nchunks); ++issued) issue(issued);
-  }
-  float q[32];
-  {
-    const uint16_t* qr = p.q + static_cast<size_t>(bhi) * D + slice * 32;
-#pragma unroll
-    for (int ch = 0; ch < 32; ++ch) q[ch] = bf16_bits_to_f32(qr[ch]) * p.scale_log2;
-  }
-  float m = kNegInf, l = 0.0f;
-  float acc[32];
-#pragma unroll
-  for (int ch = 0; ch < 32; ++ch) acc[ch] = 0.0f;
-
-  int i = 0;
-  for (; i < nchunks; ++i) {
-    const int s = i % S;
-    if (!mbar_wait(&full_bar[s], (i / S) & 1, p.err)) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    const unsigned char* st = smem + static_cast<size_t>(s) * p.stage_bytes;
-    const int nt = min(kChunk, t_end - (t_begin + i * kChunk));
-    float sc[G::TT];
-#pragma unroll
-    for (int tt = 0; tt < G::TT; ++tt) {
-      const int j = tt * G::TPC + warp * G::TPW + tw;
-      const uint4* kr = reinterpret_cast<const uint4*>(st + j * kRowBytes + slice * 64);
-      float part = 0.0f;
-#pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) {
-        const uint4 v = kr[i4];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          part = fmaf(q[i4 * 8 + 2 * e], __uint_as_float(w[e] << 16), part);
-          part = fmaf(q[i4 * 8 + 2 * e + 1], __uint_as_float(w[e] & 0xFFFF0000u), part);
-        }
-      }
-#pragma unroll
-      for (int off = G::P / 2; off >= 1; off >>= 1)
-        part += __shfl_xor_sync(0xffffffffu, part, off);
-      sc[tt] = (j < nt) ? part : kNegInf;
-    }
-    float mc = sc[0];
-#pragma unroll
-    for (int tt = 1; tt < G::TT; ++tt) mc = fmaxf(mc, sc[tt]);
-    if (mc > m) {
-      const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
-      l *= f;
-#pragma unroll
-      for (int ch = 0; ch < 32; ++ch) acc[ch] *= f;
-      m = mc;
-    }
-#pragma unroll
-    for (int tt = 0; tt < G::TT; ++tt) {
-      const int j = tt * G::TPC + warp * G::TPW + tw;
-      if (sc[tt] == kNegInf) continue;
-      const float pt = fast_exp2(sc[tt] - m);
-      l += pt;
-      const uint4* vr =
-          reinterpret_cast<const uint4*>(st + kChunk * kRowBytes + j * kRowBytes + slice * 64);
-#pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) {
-        const uint4 v = vr[i4];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc[i4 * 8 + 2 * e] = fmaf(pt, __uint_as_float(w[e] << 16), acc[i4 * 8 + 2 * e]);
-          acc[i4 * 8 + 2 * e + 1] =
-              fmaf(pt, __uint_as_float(w[e] & 0xFFFF0000u), acc[i4 * 8 + 2 * e + 1]);
-        }
-      }
-    }
-    __syncthreads();
-    if (t == 0 && issued < nchunks) issue(issued++);
-  }
-  if (s_abort) {
-    if (t == 0) {
-      for (int k = i; k < issued; ++k) (void)mbar_wait(&full_bar[k % S], (k / S) & 1, p.err);
-    }
-    __syncthreads();
-    m = kNegInf;
-    l = 0.0f;
-#pragma unroll
-    for (int ch = 0; ch < 32; ++ch) acc[ch] = 0.0f;
-  }
-  __syncthreads();
-  finish<D, false>(m, l, acc, slice, slot, reinterpret_cast<float*>(smem), bhi, split,
-                   p.splits, p.partials, p.counters, p.q, p.kcur, p.vcur, p.scale_log2,
-                   1.0f, p.out, svec, sred);
+  finish_split<D, kDecodeThreads, Geom<D>::NSLOT, true>(
+      m, l, acc, slice, slot, reinterpret_cast<float*>(smem), bhi, split, p.splits, p.partials,
+      p.counters, p.q, p.kcur, p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred);
 }
 
 template <int D>
@@ -608,32 +341,18 @@ size_t decode_dyn_smem(int D, int stages, uint32_t stage_bytes) {
   return ring > scr ? ring : scr;
 }
 
-cudaError_t decode_occupancy(int D, bool bf16, size_t dyn_smem, int* ctas_per_sm) {
+cudaError_t decode_occupancy(int D, size_t dyn_smem, int* ctas_per_sm) {
   cudaError_t e;
-  if (bf16) {
-    if (D == 64) {
-      e = set_smem(decode_bf16_kernel<64>, dyn_smem);
-      if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_bf16_kernel<64>,
-                                                          kDecodeThreads, dyn_smem);
-    } else {
-      e = set_smem(decode_bf16_kernel<128>, dyn_smem);
-      if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_bf16_kernel<128>,
-                                                          kDecodeThreads, dyn_smem);
-    }
+  if (D == 64) {
+    e = set_smem(decode_kernel<64>, dyn_smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_kernel<64>,
+                                                        kDecodeThreads, dyn_smem);
   } else {
-    if (D == 64) {
-      e = set_smem(decode_kernel<64>, dyn_smem);
-      if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_kernel<64>,
-                                                          kDecodeThreads, dyn_smem);
-    } else {
-      e = set_smem(decode_kernel<128>, dyn_smem);
-      if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_kernel<128>,
-                                                          kDecodeThreads, dyn_smem);
-    }
+    e = set_smem(decode_kernel<128>, dyn_smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_kernel<128>,
+                                                        kDecodeThreads, dyn_smem);
   }
   return e;
 }
@@ -649,23 +368,6 @@ cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t s) {
     cudaError_t e = set_smem(decode_kernel<128>, dyn);
     if (e != cudaSuccess) return e;
     decode_kernel<128><<<grid, kDecodeThreads, dyn, s>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_decode_bf16(const DecodeBf16Params& p, int D, cudaStream_t s) {
-  const size_t dyn = decode_dyn_smem(D, p.stages, p.stage_bytes);
-  const dim3 grid(p.splits, p.bh);
-  if (D == 64) {
-    cudaError_t e = set_smem(decode_bf16_kernel<64>, dyn);
-    if (e != cudaSuccess) return e;
-    decode_bf16_kernel<64><<<grid, kDecodeThreads, dyn, s>>>(p);
-  } else if (D == 128) {
-    cudaError_t e = set_smem(decode_bf16_kernel<128>, dyn);
-    if (e != cudaSuccess) return e;
-    decode_bf16_kernel<128><<<grid, kDecodeThreads, dyn, s>>>(p);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -1,0 +1,152 @@
+// rq_decode_common.cuh -- pieces shared by the decode kernels: the
+// end-of-split reduction, the last-CTA merge with the current token and the
+// final inverse rotation [RQ §4.1, §4.2 Decode, App. G.2].
+//
+// Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
+// Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
+#pragma once
+
+#include <math.h>
+
+#include "rq_internal.cuh"
+
+namespace rq {
+
+constexpr float kNegInf = -INFINITY;
+
+// Exact small-integer -> float conversion: 0x4B000000 | c is 2^23 + c.
+__device__ __forceinline__ float code_to_float(uint32_t c) {
+  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
+}
+
+__device__ __forceinline__ void unpack_meta(uint32_t mw, float& s, float& z) {
+  const __half2 h = *reinterpret_cast<const __half2*>(&mw);
+  const float2 f = __half22float2(h);
+  s = f.x;
+  z = f.y;
+}
+
+__device__ __forceinline__ int log2_pow2(int v) { return 31 - __clz(v); }
+
+// In-place Hadamard butterflies (unnormalised) over D values in shared
+// memory; every thread of the CTA must call it.
+template <int D>
+__device__ __forceinline__ void smem_fwht(float* v) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    if (t < D && (t & h) == 0) {
+      const float a = v[t], b = v[t + h];
+      v[t] = a + b;
+      v[t + h] = a - b;
+    }
+    __syncthreads();
+  }
+}
+
+// Sequence length of batch row b, clamped to [0, max_seq_len] and flagged.
+__device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int max_seq_len,
+                                          uint32_t* err) {
+  int n = seq_lens[b];
+  if (n < 0 || n > max_seq_len) {
+    if (threadIdx.x == 0) atomicOr(err, kErrSeqLen);
+    n = n < 0 ? 0 : max_seq_len;
+  }
+  return n;
+}
+
+// End of a split.  Every thread of the CTA (NT threads) calls this.  Threads
+// with slot >= 0 own the online-softmax state (m, l, acc[32]) of token slot
+// `slot` for channels [32*slice, 32*slice+32).  The slots are reduced into one
+// partial (m, l, acc[D]) in the workspace; the last CTA of the (batch, head)
+// then merges every split with the current token and writes the output,
+// applying H^T once when ROT.  `scratch` holds NSLOT*D + 2*NSLOT floats.
+template <int D, int NT, int NSLOT, bool ROT>
+__device__ __forceinline__ void finish_split(float m, float l, const float (&acc)[32], int slice,
+                                             int slot, float* scratch, int bhi, int split,
+                                             int splits, float* partials, uint32_t* counters,
+                                             const uint16_t* q, const uint16_t* kcur,
+                                             const uint16_t* vcur, float scale_log2,
+                                             float rot_scale, float* out, float* svec,
+                                             float* sred) {
+  float* red = scratch;                 // [NSLOT][D]
+  float* mred = red + NSLOT * D;        // [NSLOT]
+  float* lred = mred + NSLOT;           // [NSLOT]
+  const int t = threadIdx.x;
+  if (slot >= 0 && slice == 0) {
+    mred[slot] = m;
+    lred[slot] = l;
+  }
+  __syncthreads();
+  float M = kNegInf;
+  for (int s = 0; s < NSLOT; ++s) M = fmaxf(M, mred[s]);
+  if (slot >= 0) {
+    const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - M);
+    float4* dst = reinterpret_cast<float4*>(red + slot * D + slice * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(acc[4 * i] * f, acc[4 * i + 1] * f, acc[4 * i + 2] * f,
+                           acc[4 * i + 3] * f);
+  }
+  __syncthreads();
+  float* part = partials + (static_cast<size_t>(bhi) * splits + split) * (D + 2);
+  if (t < D) {
+    float sum = 0.0f;
+    for (int s = 0; s < NSLOT; ++s) sum += red[s * D + t];
+    part[2 + t] = sum;
+  }
+  if (t == 0) {
+    float L = 0.0f;
+    for (int s = 0; s < NSLOT; ++s)
+      L += (mred[s] == kNegInf) ? 0.0f : lred[s] * fast_exp2(mred[s] - M);
+    part[0] = M;
+    part[1] = L;
+  }
+  // Publish the partial, then count this split in (no waiting on other CTAs).
+  __threadfence();
+  __syncthreads();
+  __shared__ uint32_t s_last;
+  if (t == 0) s_last = (atomicAdd(counters + bhi, 1u) == static_cast<uint32_t>(splits - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- last CTA of this (batch, head): merge ----
+  // Current token score q.k_cur, original domain [RQ §3.2, §4.2].
+  float qk = 0.0f;
+  if (t < D)
+    qk = bf16_bits_to_f32(q[static_cast<size_t>(bhi) * D + t]) *
+         bf16_bits_to_f32(kcur[static_cast<size_t>(bhi) * D + t]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
+  if ((t & 31) == 0) sred[t >> 5] = qk;
+  __syncthreads();
+  float s_cur = 0.0f;
+  for (int w = 0; w < (D + 31) / 32; ++w) s_cur += sred[w];
+  s_cur *= scale_log2;
+  const float* pbase = partials + static_cast<size_t>(bhi) * splits * (D + 2);
+  float Mx = s_cur;
+  for (int s = 0; s < splits; ++s) Mx = fmaxf(Mx, __ldcg(pbase + s * (D + 2)));
+  float Lx = fast_exp2(s_cur - Mx);
+  float ax = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float ms = __ldcg(pbase + s * (D + 2));
+    if (ms == kNegInf) continue;
+    const float fs = fast_exp2(ms - Mx);
+    Lx += __ldcg(pbase + s * (D + 2) + 1) * fs;
+    if (t < D) ax += __ldcg(pbase + s * (D + 2) + 2 + t) * fs;
+  }
+  __syncthreads();   // everyone is done reading sred / svec
+  if (t < D) svec[t] = ax;
+  __syncthreads();
+  if constexpr (ROT) smem_fwht<D>(svec);
+  if (t < D) {
+    const float pc = fast_exp2(s_cur - Mx);
+    const float v = ROT ? svec[t] * rot_scale : svec[t];
+    out[static_cast<size_t>(bhi) * D + t] =
+        (v + pc * bf16_bits_to_f32(vcur[static_cast<size_t>(bhi) * D + t])) / Lx;
+  }
+  if (t == 0) counters[bhi] = 0u;   // ready for the next call
+}
+
+}  // namespace rq

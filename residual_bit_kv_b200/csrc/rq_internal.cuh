@@ -83,6 +83,7 @@ struct DecodeParams {
   int32_t chunks_per_split;
   int32_t stages;
   uint32_t stage_bytes;
+  int32_t use_fast;        // warp-specialised kernel for a compiled layout
 };
 
 struct DecodeBf16Params {
@@ -113,15 +114,25 @@ struct DecodeBf16Params {
 cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
                             cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s);
+// generic compressed decode (any chain of bits / groups), chunk kChunk
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t s);
+// warp-specialised decode for compiled layouts, chunk fast_chunk()
+bool fast_decode_plan(const DecodeParams& p, int D, size_t ring_budget, int max_stages,
+                      int* stages, int* ctas_per_sm);
+cudaError_t launch_decode_fast(const DecodeParams& p, int D, cudaStream_t s);
+int fast_chunk();
+// uncompressed bf16 decode, chunk bf16_chunk(D)
 cudaError_t launch_decode_bf16(const DecodeBf16Params& p, int D,
                                cudaStream_t s);
+uint32_t bf16_stage_bytes(int D);
+int bf16_chunk(int D);
+cudaError_t bf16_occupancy(int D, int stages, int* occ);
 // bytes of one pipeline stage for a decode call
 uint32_t decode_stage_bytes(const DecodeParams& p, int D);
 // dynamic shared memory of a decode launch (stage ring or merge scratch)
 size_t decode_dyn_smem(int D, int stages, uint32_t stage_bytes);
-// resident CTAs per SM of a decode kernel at this dynamic shared memory
-cudaError_t decode_occupancy(int D, bool bf16, size_t dyn_smem, int* ctas_per_sm);
+// resident CTAs per SM of the generic decode kernel at this dynamic shared memory
+cudaError_t decode_occupancy(int D, size_t dyn_smem, int* ctas_per_sm);
 
 // ---------------------------------------------------------------------------
 // Device helpers
@@ -153,6 +164,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
           smem_addr(bar)),
       "r"(bytes)
       : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
