@@ -407,7 +407,11 @@ def main():
     ap.add_argument("--impl", default="rq", choices=["rq", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-bf16", action="store_true", help="skip the BF16 baseline kernel")
-    ap.add_argument("--layers", type=int, default=None, help="override layer count (debug)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers (default 24); smaller values give a profiling-sized case")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per step (default 16); smaller values give a profiling-sized case")
+    ap.add_argument("--no-quant", action="store_true", help="skip the prefill quantise leg")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -420,6 +424,8 @@ def main():
     w = synth.WORKLOADS[WORKLOAD]
     if args.layers:
         w = w.replace(layers=args.layers)
+    if args.batch:
+        w = w.replace(batch=args.batch)
     nbuf = 0 if args.no_bf16 else 4
     eng = Engine(w, dev, seed_offset=1000 * rank, keep_bf16_layers=nbuf)
     w = eng.w
@@ -497,7 +503,7 @@ def main():
 
     # ---- prefill-sized quantise (anchor + 3 residuals, K and V), separate workload
     quant = None
-    if rank == 0 or ws > 1:
+    if not args.no_quant:
         quant = bench_quantize(dev, stream, args, hbm)
 
     cpu = None
