@@ -23,6 +23,7 @@ closed forms, invariants, brute force and the pages' storage accounting.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import subprocess
 from typing import Dict, List, Optional, Sequence
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "rqo_attention_f64": ([_P, _P, _P, _I64, _P, _P, _I, _D, _P], None),
             "rqo_effective_bits": ([_I, _P, _P, _I, _I, _I], _D),
             "rqo_component_reads": ([_I, _I], _I64),
+            "rqo_code_pos": ([_I, _I, _P, _P], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(h, name)
@@ -175,13 +177,24 @@ def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int):
     return words, meta, int(alpha[0]), zhat
 
 
+@functools.lru_cache(maxsize=None)
+def code_positions(bits: int, D: int):
+    """(word, shift) of every channel of a packed row (rqo_code_pos)."""
+    wi = np.zeros(D, np.int64)
+    sh = np.zeros(D, np.uint32)
+    w = ctypes.c_int()
+    s = ctypes.c_int()
+    for i in range(D):
+        lib().rqo_code_pos(i, bits, ctypes.byref(w), ctypes.byref(s))
+        wi[i], sh[i] = w.value, s.value
+    return wi, sh
+
+
 def unpack_codes(words: np.ndarray, bits: int, D: int) -> np.ndarray:
     """Codes of packed rows [..., D*bits/32] -> [..., D] (uint8)."""
-    per_word = 32 // bits
+    wi, sh = code_positions(bits, D)
     w = np.asarray(words, dtype=np.uint32)
-    idx = np.arange(D)
-    sh = (bits * (idx % per_word)).astype(np.uint32)
-    return ((w[..., idx // per_word] >> sh) & np.uint32((1 << bits) - 1)).astype(np.uint8)
+    return ((w[..., wi] >> sh) & np.uint32((1 << bits) - 1)).astype(np.uint8)
 
 
 def meta_scale_zero(meta: np.ndarray):

@@ -136,10 +136,24 @@ float rqo_dot_f32(const float* a, const float* b, int D) {
 /* Group-wise affine quantisation [RQ §2.1]                                  */
 /* ------------------------------------------------------------------------ */
 
+/* Storage position of channel i of a row (word index, bit shift).
+ * b = 2: word i/16, bits 2*(i%16).
+ * b = 4: channels come in blocks of 16 (i = 16u + v); word 2u + ((v>>1)&1),
+ *        nibble 2*(v>>2) + (v&1), i.e. bits 4*nibble. */
+void rqo_code_pos(int i, int bits, int* word, int* shift) {
+  if (bits == 2) {
+    *word = i / 16;
+    *shift = 2 * (i % 16);
+  } else {
+    const int u = i / 16, v = i % 16;
+    *word = 2 * u + ((v >> 1) & 1);
+    *shift = 4 * (2 * (v >> 2) + (v & 1));
+  }
+}
+
 void rqo_quantize(const float* z, int D, int bits, int group, uint32_t* words,
                   uint32_t* meta, float* deq) {
   const int qmax = (1 << bits) - 1;
-  const int per_word = 32 / bits;
   for (int w = 0; w < D * bits / 32; ++w) words[w] = 0u;
 
   for (int g0 = 0, j = 0; g0 < D; g0 += group, ++j) {
@@ -167,7 +181,9 @@ void rqo_quantize(const float* z, int D, int bits, int group, uint32_t* words,
       if (u < 0.0f) u = 0.0f;
       if (u > (float)qmax) u = (float)qmax;
       const uint32_t code = (uint32_t)rintf(u);
-      words[i / per_word] |= code << (bits * (i % per_word));
+      int wi, bit;
+      rqo_code_pos(i, bits, &wi, &bit);
+      words[wi] |= code << bit;
       deq[i] = fmaf(st, (float)code, zt);
     }
   }
@@ -239,9 +255,10 @@ void rqo_encode_residual_rows(const uint16_t* x, const float* ref, int64_t n,
 void rqo_dequant_codes_f64(const uint32_t* words, const uint32_t* meta, int D,
                            int bits, int group, double* out) {
   const uint32_t qmax = (1u << bits) - 1u;
-  const int per_word = 32 / bits;
   for (int i = 0; i < D; ++i) {
-    const uint32_t code = (words[i / per_word] >> (bits * (i % per_word))) & qmax;
+    int wi, sh;
+    rqo_code_pos(i, bits, &wi, &sh);
+    const uint32_t code = (words[wi] >> sh) & qmax;
     const uint32_t m = meta[i / group];
     const double s = rqo_f16_to_f32((uint16_t)(m & 0xFFFFu));
     const double z = rqo_f16_to_f32((uint16_t)(m >> 16));

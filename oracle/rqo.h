@@ -16,8 +16,11 @@
  * Reconstruction and attention are computed in fp64.
  *
  * Packed formats (the storage contract both sides implement independently):
- *   codes : channel i of a row lives in 32-bit word i / (32/b), bits
- *           [b*(i % (32/b)), +b), little-endian words.
+ *   codes : b = 2: channel i of a row lives in 32-bit word i/16, bits
+ *           [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v,
+ *           word 2u + ((v>>1)&1), bits [4*(2*(v>>2) + (v&1)), +4); this
+ *           order puts the same channels in the same byte lanes for both
+ *           widths.  Little-endian 32-bit words.
  *   meta  : one 32-bit word per group: low half = fp16 scale s~,
  *           high half = fp16 offset z~.
  *   alpha : bf16 bits of the LS coefficient, one per (token, head).
@@ -58,6 +61,9 @@ void rqo_fwht_rows_f64(double* z, int64_t n, int D);
  * partial sums are then combined by a butterfly: for off = P/2, ..., 1,
  * p[l] <- p[l] + p[l ^ off].  Returns p[0].  Requires D % 32 == 0. */
 float rqo_dot_f32(const float* a, const float* b, int D);
+
+/* Word index and bit shift of channel i in a packed row of `bits`-bit codes. */
+void rqo_code_pos(int i, int bits, int* word, int* shift);
 
 /* Group-wise affine quantisation of one rotated row [RQ §2.1]:
  * per group of g consecutive channels: mn, mx; s = (mx - mn)/(2^b - 1);

@@ -68,7 +68,6 @@ template <int BITS>
 __device__ __forceinline__ float comp_dot(const uint32_t* cw, const uint32_t* mrow,
                                           int slice, int gshift, const float (&q)[32],
                                           float qsa, float qsb) {
-  constexpr int PER_WORD = 32 / BITS;
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   uint32_t w[BITS];
   if constexpr (BITS == 4) {
@@ -81,7 +80,7 @@ __device__ __forceinline__ float comp_dot(const uint32_t* cw, const uint32_t* mr
   float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
   for (int ch = 0; ch < 32; ++ch) {
-    const uint32_t c = (w[ch / PER_WORD] >> (BITS * (ch % PER_WORD))) & QMAX;
+    const uint32_t c = (w[slice_word<BITS>(ch)] >> slice_shift<BITS>(ch)) & QMAX;
     if (ch < 16)
       a0 = fmaf(q[ch], code_to_float(c), a0);
     else
@@ -103,7 +102,6 @@ template <int BITS>
 __device__ __forceinline__ void comp_acc(const uint32_t* cw, const uint32_t* mrow,
                                          int slice, int gshift, float pk, float (&acc)[32],
                                          float& cst0, float& cst1) {
-  constexpr int PER_WORD = 32 / BITS;
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   uint32_t w[BITS];
   if constexpr (BITS == 4) {
@@ -128,7 +126,7 @@ __device__ __forceinline__ void comp_acc(const uint32_t* cw, const uint32_t* mro
   cst1 = fmaf(pk, z1, cst1);
 #pragma unroll
   for (int ch = 0; ch < 32; ++ch) {
-    const uint32_t c = (w[ch / PER_WORD] >> (BITS * (ch % PER_WORD))) & QMAX;
+    const uint32_t c = (w[slice_word<BITS>(ch)] >> slice_shift<BITS>(ch)) & QMAX;
     acc[ch] = fmaf(ch < 16 ? w0 : w1, code_to_float(c), acc[ch]);
   }
 }

@@ -26,20 +26,26 @@
 namespace rq {
 namespace {
 
-constexpr int kWarps = 8;                      // compute warps per CTA
+constexpr int kWarps = 8;                      // BF16 kernel: compute warps per CTA
 constexpr int kThreads = (kWarps + 1) * 32;    // + producer warp
 constexpr int kMaxRing = 4;
 
-template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_, int TC_ = 128>
+constexpr int kCWarps = 4;                     // compressed kernel: warps per CTA
+constexpr int kCThreads = kCWarps * 32;
+constexpr int kCChunk = 64;                    // tokens per stage
+constexpr int kCMinCtas = 5;                   // register target: CTAs per SM
+constexpr size_t kCRingBudget = 40 * 1024;     // stage ring per CTA (several CTAs per SM)
+
+template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
 struct Spec {
-  static constexpr int D = D_, NC = NC_, TC = TC_;
+  static constexpr int D = D_, NC = NC_, TC = kCChunk;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
   __host__ __device__ static constexpr int wpr(int c) { return D_ * bits(c) / 32; }
   __host__ __device__ static constexpr int gpr(int c) { return D_ / group(c); }
   __host__ __device__ static constexpr uint32_t comp_bytes(int c) {
-    return TC_ * (wpr(c) * 4 + gpr(c) * 4 + (has_alpha(c) ? 2 : 0));
+    return TC * (wpr(c) * 4 + gpr(c) * 4 + (has_alpha(c) ? 2 : 0));
   }
   __host__ __device__ static constexpr uint32_t side_bytes() {
     uint32_t s = 0;
@@ -53,28 +59,25 @@ struct Spec {
     return o;
   }
   __host__ __device__ static constexpr uint32_t meta_off(int side, int c) {
-    return codes_off(side, c) + TC_ * wpr(c) * 4;
+    return codes_off(side, c) + TC * wpr(c) * 4;
   }
   __host__ __device__ static constexpr uint32_t alpha_off(int side, int c) {
-    return meta_off(side, c) + TC_ * gpr(c) * 4;
+    return meta_off(side, c) + TC * gpr(c) * 4;
   }
-  static constexpr bool has4 = AB_ == 4 || (NC_ > 1 && RB_ == 4);
-  static constexpr bool has2 = AB_ == 2 || (NC_ > 1 && RB_ == 2);
 };
 
-// Fixed-point rotated query of one lane's 32 channels, in the byte orders the
-// unpacked code words come in.
+// Fixed-point rotated query of one lane's 32 channels as int8 limb bytes in
+// the quad order of the unpacked codes: quad (k, s) holds channels
+// 16k + s + {0, 4, 8, 12} (the same for 2-bit and 4-bit codes).
 struct QLimbs {
-  int e4h[4], o4h[4], e4l[4], o4l[4];   // 4-bit words: channels 8k+{0,2,4,6} / 8k+{1,3,5,7}
-  int q2h[2][4], q2l[2][4];             // 2-bit words: channels 16k+s+{0,4,8,12}
-  float sq[2];                          // sum of q~ over channels 0-15 / 16-31
+  int h[2][4], l[2][4];
+  float sq[2];   // sum of q~ over channels 0-15 / 16-31
 };
 
 __device__ __forceinline__ int pack_bytes(int a, int b, int c, int d) {
   return (a & 0xFF) | ((b & 0xFF) << 8) | ((c & 0xFF) << 16) | (d << 24);
 }
 
-template <bool H4, bool H2>
 __device__ __forceinline__ void build_limbs(const float* qrow, float inv_sigma, QLimbs& ql) {
   int hi[32], lo[32];
   float s0 = 0.0f, s1 = 0.0f;
@@ -88,25 +91,14 @@ __device__ __forceinline__ void build_limbs(const float* qrow, float inv_sigma, 
   }
   ql.sq[0] = s0;
   ql.sq[1] = s1;
-  if constexpr (H4) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      ql.e4h[k] = pack_bytes(hi[8 * k], hi[8 * k + 2], hi[8 * k + 4], hi[8 * k + 6]);
-      ql.o4h[k] = pack_bytes(hi[8 * k + 1], hi[8 * k + 3], hi[8 * k + 5], hi[8 * k + 7]);
-      ql.e4l[k] = pack_bytes(lo[8 * k], lo[8 * k + 2], lo[8 * k + 4], lo[8 * k + 6]);
-      ql.o4l[k] = pack_bytes(lo[8 * k + 1], lo[8 * k + 3], lo[8 * k + 5], lo[8 * k + 7]);
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int b = 16 * k + s;
+      ql.h[k][s] = pack_bytes(hi[b], hi[b + 4], hi[b + 8], hi[b + 12]);
+      ql.l[k][s] = pack_bytes(lo[b], lo[b + 4], lo[b + 8], lo[b + 12]);
     }
-  }
-  if constexpr (H2) {
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int b = 16 * k + s;
-        ql.q2h[k][s] = pack_bytes(hi[b], hi[b + 4], hi[b + 8], hi[b + 12]);
-        ql.q2l[k][s] = pack_bytes(lo[b], lo[b + 4], lo[b + 8], lo[b + 12]);
-      }
-  }
 }
 
 // q~ . D(c) over one lane's 32 channels of token j of a component, in sigma
@@ -116,25 +108,19 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
                                       int slice, const QLimbs& ql) {
   constexpr int WPR = D * BITS / 32, GPR = D / G;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + j * WPR + slice * BITS;
-  int ah0 = 0, al0 = 0, ah1 = 0, al1 = 0;
+  int ah[2] = {0, 0}, al[2] = {0, 0};   // per 16-channel block
   if constexpr (BITS == 4) {
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int lo = static_cast<int>(w[k] & 0x0F0F0F0Fu);
-      const int hi = static_cast<int>((w[k] >> 4) & 0x0F0F0F0Fu);
-      if (G == 16 && k >= 2) {
-        ah1 = __dp4a(ql.e4h[k], lo, ah1);
-        ah1 = __dp4a(ql.o4h[k], hi, ah1);
-        al1 = __dp4a(ql.e4l[k], lo, al1);
-        al1 = __dp4a(ql.o4l[k], hi, al1);
-      } else {
-        ah0 = __dp4a(ql.e4h[k], lo, ah0);
-        ah0 = __dp4a(ql.o4h[k], hi, ah0);
-        al0 = __dp4a(ql.e4l[k], lo, al0);
-        al0 = __dp4a(ql.o4l[k], hi, al0);
-      }
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int k = k4 >> 1, h = k4 & 1;
+      const int lo = static_cast<int>(w[k4] & 0x0F0F0F0Fu);          // quad s = 2h
+      const int hi = static_cast<int>((w[k4] >> 4) & 0x0F0F0F0Fu);   // quad s = 2h + 1
+      ah[k] = __dp4a(ql.h[k][2 * h], lo, ah[k]);
+      al[k] = __dp4a(ql.l[k][2 * h], lo, al[k]);
+      ah[k] = __dp4a(ql.h[k][2 * h + 1], hi, ah[k]);
+      al[k] = __dp4a(ql.l[k][2 * h + 1], hi, al[k]);
     }
   } else {
     const uint2 v = *reinterpret_cast<const uint2*>(cw);
@@ -144,27 +130,23 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const int x = static_cast<int>((w[k] >> (2 * s)) & 0x03030303u);
-        if (G == 16 && k == 1) {
-          ah1 = __dp4a(ql.q2h[k][s], x, ah1);
-          al1 = __dp4a(ql.q2l[k][s], x, al1);
-        } else {
-          ah0 = __dp4a(ql.q2h[k][s], x, ah0);
-          al0 = __dp4a(ql.q2l[k][s], x, al0);
-        }
+        ah[k] = __dp4a(ql.h[k][s], x, ah[k]);
+        al[k] = __dp4a(ql.l[k][s], x, al[k]);
       }
   }
   const uint32_t* mr = reinterpret_cast<const uint32_t*>(meta) + j * GPR;
   float s0, z0;
   if constexpr (G >= 32) {
     unpack_meta(mr[(slice * 32) / G], s0, z0);
-    return s0 * static_cast<float>(ah0 * 256 + al0) + z0 * (ql.sq[0] + ql.sq[1]);
+    return s0 * static_cast<float>((ah[0] + ah[1]) * 256 + (al[0] + al[1])) +
+           z0 * (ql.sq[0] + ql.sq[1]);
   } else {
     float s1, z1;
     const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
     unpack_meta(mw.x, s0, z0);
     unpack_meta(mw.y, s1, z1);
-    return s0 * static_cast<float>(ah0 * 256 + al0) + z0 * ql.sq[0] +
-           (s1 * static_cast<float>(ah1 * 256 + al1) + z1 * ql.sq[1]);
+    return s0 * static_cast<float>(ah[0] * 256 + al[0]) + z0 * ql.sq[0] +
+           (s1 * static_cast<float>(ah[1] * 256 + al[1]) + z1 * ql.sq[1]);
   }
 }
 
@@ -175,8 +157,9 @@ __device__ __forceinline__ float2 code_pair(uint32_t a, uint32_t b, uint32_t mas
   return __fadd2_rn(v, make_float2(-8388608.0f, -8388608.0f));
 }
 
-// acc += pk * D(c) over one lane's 32 channels of token j.  acc2[4b + c]
-// holds channels (8b + c, 8b + c + 4).
+// acc += pk * D(c) over one lane's 32 channels of token j.  acc2[8k + c] holds
+// channels (16k + c, 16k + c + 4) and acc2[8k + 4 + c] channels
+// (16k + 8 + c, 16k + 12 + c), c = 0..3.
 template <int D, int BITS, int G>
 __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned char* meta, int j,
                                      int slice, float pk, float2 (&acc2)[16], float (&cst)[2]) {
@@ -193,47 +176,43 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
     unpack_meta(mw.x, s0, z0);
     unpack_meta(mw.y, s1, z1);
   }
-  const float w0 = pk * s0, w1 = pk * s1;
   cst[0] = fmaf(pk, z0, cst[0]);
   cst[1] = fmaf(pk, z1, cst[1]);
+  const float wk[2] = {pk * s0, pk * s1};
   if constexpr (BITS == 4) {
+    // word 2k + h, nibble n holds channel 16k + 4(n>>1) + 2h + (n&1); the
+    // pairs (n, n+2) sit at the same bits of (w, w>>8) and (w>>16, w>>24).
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float2 ws[2][4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float sc = 1.0f / static_cast<float>(1u << (4 * c));
-      ws[0][c] = make_float2(w0 * sc, w0 * sc);
-      ws[1][c] = make_float2(w1 * sc, w1 * sc);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t hi = w[k] >> 16;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float2 x = code_pair(w[k], hi, 0xFu << (4 * c));
-        acc2[4 * k + c] = __ffma2_rn(ws[(G == 16 && k >= 2) ? 1 : 0][c], x, acc2[4 * k + c]);
-      }
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int k = k4 >> 1, h = k4 & 1;
+      const float wt = (G >= 32) ? wk[0] : wk[k];
+      const float2 w0 = make_float2(wt, wt);
+      const float2 w1 = make_float2(wt * 0.0625f, wt * 0.0625f);
+      const uint32_t w8 = w[k4] >> 8, w16 = w[k4] >> 16, w24 = w[k4] >> 24;
+      acc2[8 * k + 2 * h] = __ffma2_rn(w0, code_pair(w[k4], w8, 0x0Fu), acc2[8 * k + 2 * h]);
+      acc2[8 * k + 2 * h + 1] =
+          __ffma2_rn(w1, code_pair(w[k4], w8, 0xF0u), acc2[8 * k + 2 * h + 1]);
+      acc2[8 * k + 4 + 2 * h] =
+          __ffma2_rn(w0, code_pair(w16, w24, 0x0Fu), acc2[8 * k + 4 + 2 * h]);
+      acc2[8 * k + 4 + 2 * h + 1] =
+          __ffma2_rn(w1, code_pair(w16, w24, 0xF0u), acc2[8 * k + 4 + 2 * h + 1]);
     }
   } else {
     const uint2 v = *reinterpret_cast<const uint2*>(cw);
     const uint32_t w[2] = {v.x, v.y};
-    float2 ws[2][4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float sc = 1.0f / static_cast<float>(1u << (2 * c));
-      ws[0][c] = make_float2(w0 * sc, w0 * sc);
-      ws[1][c] = make_float2(w1 * sc, w1 * sc);
-    }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
+      const float wt = (G >= 32) ? wk[0] : wk[k];
       const uint32_t w8 = w[k] >> 8, w16 = w[k] >> 16, w24 = w[k] >> 24;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        const float sc = wt * (1.0f / static_cast<float>(1u << (2 * c)));
+        const float2 wc = make_float2(sc, sc);
         const uint32_t m = 3u << (2 * c);
-        const float2& wt = ws[(G == 16 && k == 1) ? 1 : 0][c];
-        acc2[8 * k + c] = __ffma2_rn(wt, code_pair(w[k], w8, m), acc2[8 * k + c]);
-        acc2[8 * k + 4 + c] = __ffma2_rn(wt, code_pair(w16, w24, m), acc2[8 * k + 4 + c]);
+        acc2[8 * k + c] = __ffma2_rn(wc, code_pair(w[k], w8, m), acc2[8 * k + c]);
+        acc2[8 * k + 4 + c] = __ffma2_rn(wc, code_pair(w16, w24, m), acc2[8 * k + 4 + c]);
       }
     }
   }
@@ -268,11 +247,13 @@ __device__ __forceinline__ void value_comps(const unsigned char* st, int j, int 
 __device__ __forceinline__ void unpair(const float2 (&acc2)[16], const float (&cst)[2],
                                        float (&acc)[32]) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b)
+  for (int k = 0; k < 2; ++k)
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      acc[8 * b + c] = acc2[4 * b + c].x + cst[b / 2];
-      acc[8 * b + c + 4] = acc2[4 * b + c].y + cst[b / 2];
+      acc[16 * k + c] = acc2[8 * k + c].x + cst[k];
+      acc[16 * k + c + 4] = acc2[8 * k + c].y + cst[k];
+      acc[16 * k + 8 + c] = acc2[8 * k + 4 + c].x + cst[k];
+      acc[16 * k + 12 + c] = acc2[8 * k + 4 + c].y + cst[k];
     }
 }
 
@@ -290,7 +271,7 @@ __device__ __forceinline__ Range split_range(int n, int split, int cps, int tc) 
 }
 
 // Producer loop (one lane): waits for a free stage, then issues the chunk's
-// copies.  issue(i, stage) returns nothing; `bytes(i)` the expected bytes.
+// copies.
 template <int S_MAX, typename Bytes, typename Issue>
 __device__ __forceinline__ int produce(int nchunks, int S, uint64_t* full, uint64_t* empty,
                                        uint32_t* err, volatile int* abort_flag, Bytes bytes,
@@ -318,39 +299,78 @@ __device__ __forceinline__ void drain(int issued, int S, uint64_t* full, uint32_
     (void)mbar_wait(&full[k % S], (k / S) & 1, err);
 }
 
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Compressed decode.  Every warp consumes every stage; the warp that releases
+// a stage last (a shared-memory counter, no waiting) issues that stage's
+// refill with the chunk S ahead.
 template <class SP>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kCThreads, kCMinCtas)
     decode_fast_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int D = SP::D, NC = SP::NC, TC = SP::TC;
-  constexpr int P = D / 32, TPW = 32 / P, TPC = kWarps * TPW, TT = TC / TPC;
-  constexpr int NSLOT = kWarps * TPW;
-  static_assert(TT * TPC == TC, "chunk must be a multiple of the tokens per pass");
+  constexpr int P = D / 32, TPW = 32 / P, TPC = kCWarps * TPW, TT = TC / TPC;
+  constexpr int NSLOT = kCWarps * TPW;
+  static_assert(TT >= 1 && TT * TPC == TC, "chunk must be a multiple of the tokens per pass");
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t full_bar[kMaxRing], empty_bar[kMaxRing];
+  __shared__ uint64_t full_bar[kMaxRing];
+  __shared__ uint32_t s_release[kMaxRing];
   __shared__ float svec[D];
-  __shared__ float sred[kThreads / 32];
+  __shared__ float sred[kCThreads / 32];
   __shared__ volatile int s_abort;
+  __shared__ int s_issued;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const bool producer = warp == kWarps;
   const int slice = lane % P, tw = lane / P;
   const int split = blockIdx.x, bhi = blockIdx.y;
   const int S = p.stages;
   const int n = seq_len_of(p.seq_lens, bhi / p.heads, p.max_seq_len, p.err);
   const Range R = split_range(n, split, p.chunks_per_split, TC);
+  const size_t row0 = static_cast<size_t>(bhi) * p.tstride;
+
+  // Copies of chunk i into stage s (one lane).
+  auto issue = [&](int i, int s) {
+    const int t0 = R.t_begin + i * TC;
+    const uint32_t ntc = static_cast<uint32_t>((min(TC, R.t_end - t0) + 7) & ~7);
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      bytes += 2u * ntc * (SP::wpr(c) * 4 + SP::gpr(c) * 4 + (SP::has_alpha(c) ? 2 : 0));
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&full_bar[s], bytes);
+    unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+      const Comp* cs = side == 0 ? p.k : p.v;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        bulk_copy_g2s(st + SP::codes_off(side, c), cs[c].codes + (row0 + t0) * SP::wpr(c),
+                      ntc * SP::wpr(c) * 4, &full_bar[s]);
+        bulk_copy_g2s(st + SP::meta_off(side, c), cs[c].meta + (row0 + t0) * SP::gpr(c),
+                      ntc * SP::gpr(c) * 4, &full_bar[s]);
+        if (SP::has_alpha(c))
+          bulk_copy_g2s(st + SP::alpha_off(side, c), cs[c].alpha + row0 + t0, ntc * 2,
+                        &full_bar[s]);
+      }
+    }
+  };
 
   if (t == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kWarps);
+      s_release[s] = 0u;
     }
     fence_barrier_init();
     s_abort = 0;
+    const int first = min(S, R.nchunks);
+    for (int i = 0; i < first; ++i) issue(i, i);
+    s_issued = first;
   }
   if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
   __syncthreads();
   smem_fwht<D>(svec);
-  // max |q'| for the fixed-point scale
+  // Fixed-point scale of q' = H q * softmax scale * log2 e.
   const float qscale = p.rot_scale * p.scale_log2;
   float amax = (t < D) ? fabsf(svec[t] * qscale) : 0.0f;
 #pragma unroll
@@ -358,119 +378,88 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (lane == 0) sred[warp] = amax;
   __syncthreads();
   amax = 0.0f;
-  for (int w = 0; w < kThreads / 32; ++w) amax = fmaxf(amax, sred[w]);
+#pragma unroll
+  for (int w = 0; w < kCThreads / 32; ++w) amax = fmaxf(amax, sred[w]);
   const float sigma = amax > 0.0f ? amax / 32639.0f : 1.0f;
 
+  QLimbs ql;
+  build_limbs(svec + slice * 32, qscale / sigma, ql);
+  float2 acc2[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+  float cst[2] = {0.0f, 0.0f};
   float m = kNegInf, l = 0.0f;
-  float acc[32];
-  int slot = -1;
-  if (producer) {
-    if (lane == 0) {
-      const size_t row0 = static_cast<size_t>(bhi) * p.tstride;
-      auto bytes = [&](int i) -> uint32_t {
-        const int t0 = R.t_begin + i * TC;
-        const uint32_t ntc = static_cast<uint32_t>((min(TC, R.t_end - t0) + 7) & ~7);
-        uint32_t b = 0;
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-          b += 2u * ntc * (SP::wpr(c) * 4 + SP::gpr(c) * 4 + (SP::has_alpha(c) ? 2 : 0));
-        return b;
-      };
-      auto issue = [&](int i, int s) {
-        const int t0 = R.t_begin + i * TC;
-        const uint32_t ntc = static_cast<uint32_t>((min(TC, R.t_end - t0) + 7) & ~7);
-        unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
-#pragma unroll
-        for (int side = 0; side < 2; ++side) {
-          const Comp* cs = side == 0 ? p.k : p.v;
-#pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            bulk_copy_g2s(st + SP::codes_off(side, c), cs[c].codes + (row0 + t0) * SP::wpr(c),
-                          ntc * SP::wpr(c) * 4, &full_bar[s]);
-            bulk_copy_g2s(st + SP::meta_off(side, c), cs[c].meta + (row0 + t0) * SP::gpr(c),
-                          ntc * SP::gpr(c) * 4, &full_bar[s]);
-            if (SP::has_alpha(c))
-              bulk_copy_g2s(st + SP::alpha_off(side, c), cs[c].alpha + row0 + t0, ntc * 2,
-                            &full_bar[s]);
-          }
-        }
-      };
-      const int issued =
-          produce<kMaxRing>(R.nchunks, S, full_bar, empty_bar, p.err, &s_abort, bytes, issue);
-      if (s_abort) drain(issued, S, full_bar, p.err);
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-  } else {
-    slot = warp * TPW + tw;
-    QLimbs ql;
-    build_limbs<SP::has4, SP::has2>(svec + slice * 32, 1.0f / sigma * qscale, ql);
-    float2 acc2[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc2[i] = make_float2(0.0f, 0.0f);
-    float cst[2] = {0.0f, 0.0f};
 
-    for (int i = 0; i < R.nchunks; ++i) {
-      const int s = i % S;
-      if (!mbar_wait(&full_bar[s], (i / S) & 1, p.err)) s_abort = 1;
-      if (s_abort) break;
-      const unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
-      const int nt = min(TC, R.t_end - (R.t_begin + i * TC));
-      float sc[TT];
+  for (int i = 0; i < R.nchunks; ++i) {
+    const int s = i % S;
+    if (!mbar_wait(&full_bar[s], (i / S) & 1, p.err)) s_abort = 1;
+    if (s_abort) break;
+    const unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
+    const int nt = min(TC, R.t_end - (R.t_begin + i * TC));
+    float sc[TT];
 #pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        const int j = tt * TPC + warp * TPW + tw;
-        float part = 0.0f, kap = 1.0f;
-        score_comps<SP>(st, j, slice, ql, part, kap);
+    for (int tt = 0; tt < TT; ++tt) {
+      const int j = tt * TPC + warp * TPW + tw;
+      float part = 0.0f, kap = 1.0f;
+      score_comps<SP>(st, j, slice, ql, part, kap);
 #pragma unroll
-        for (int off = P / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        sc[tt] = (j < nt) ? part * sigma : kNegInf;
-      }
-      float mc = sc[0];
-#pragma unroll
-      for (int tt = 1; tt < TT; ++tt) mc = fmaxf(mc, sc[tt]);
-      if (mc > m) {
-        const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
-        const float2 f2 = make_float2(f, f);
-        l *= f;
-        cst[0] *= f;
-        cst[1] *= f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc2[k] = __fmul2_rn(acc2[k], f2);
-        m = mc;
-      }
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        const int j = tt * TPC + warp * TPW + tw;
-        if (sc[tt] == kNegInf) continue;
-        const float pt = fast_exp2(sc[tt] - m);
-        l += pt;
-        float kap = pt;
-        value_comps<SP>(st, j, slice, kap, acc2, cst);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      for (int off = P / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      sc[tt] = (j < nt) ? part * sigma : kNegInf;
     }
-    if (s_abort) {
-      m = kNegInf;
-      l = 0.0f;
-    }
-    unpair(acc2, cst, acc);
-    if (s_abort) {
+    float mc = sc[0];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+    for (int tt = 1; tt < TT; ++tt) mc = fmaxf(mc, sc[tt]);
+    if (mc > m) {
+      const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
+      const float2 f2 = make_float2(f, f);
+      l *= f;
+      cst[0] *= f;
+      cst[1] *= f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc2[k] = __fmul2_rn(acc2[k], f2);
+      m = mc;
+    }
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) {
+      const int j = tt * TPC + warp * TPW + tw;
+      if (sc[tt] == kNegInf) continue;
+      const float pt = fast_exp2(sc[tt] - m);
+      l += pt;
+      value_comps<SP>(st, j, slice, pt, acc2, cst);
+    }
+    // Release the stage; the last warp to do so refills it.
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      const uint32_t r = atomicAdd(&s_release[s], 1u);
+      if (r % kCWarps == kCWarps - 1 && i + S < R.nchunks && !s_abort) {
+        __threadfence_block();
+        issue(i + S, s);
+        atomicAdd(&s_issued, 1);
+      }
     }
   }
+  float acc[32];
+  unpair(acc2, cst, acc);
+  if (s_abort) {
+    m = kNegInf;
+    l = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) acc[k] = 0.0f;
+  }
   __syncthreads();
-  finish_split<D, kThreads, NSLOT, true>(m, l, acc, slice, slot, reinterpret_cast<float*>(smem),
-                                         bhi, split, p.splits, p.partials, p.counters, p.q, p.kcur,
-                                         p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred);
+  if (s_abort && t == 0) drain(s_issued, S, full_bar, p.err);
+  __syncthreads();
+  finish_split<D, kCThreads, NSLOT, true>(m, l, acc, slice, warp * TPW + tw,
+                                          reinterpret_cast<float*>(smem), bhi, split, p.splits,
+                                          p.partials, p.counters, p.q, p.kcur, p.vcur,
+                                          p.scale_log2, p.rot_scale, p.out, svec, sred);
 }
 
 // ---------------------------------------------------------------- BF16 --
 
 template <int D>
-constexpr int bf16_tc() { return D == 64 ? 128 : 64; }
+__host__ __device__ constexpr int bf16_tc() { return D == 64 ? 128 : 64; }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -619,24 +608,25 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <typename K>
-cudaError_t prep(K kernel, size_t dyn, int* occ) {
+cudaError_t prep(K kernel, size_t dyn, int* occ, int threads = kThreads) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(dyn));
   if (e != cudaSuccess) return e;
   if (occ != nullptr)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kernel, kThreads, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kernel, threads, dyn);
   return e;
 }
 
+// merge scratch of a kernel with `warps` compute warps: NSLOT*(D+2) floats
 template <int D>
-constexpr size_t scratch_floats() {
-  return static_cast<size_t>(kWarps * (32 / (D / 32))) * (D + 2);
+constexpr size_t scratch_floats(int warps = kWarps) {
+  return static_cast<size_t>(warps * (32 / (D / 32))) * (D + 2);
 }
 
 template <class SP>
 size_t dyn_bytes(int stages) {
   const size_t ring = static_cast<size_t>(stages) * SP::stage_bytes();
-  const size_t scr = scratch_floats<SP::D>() * sizeof(float);
+  const size_t scr = scratch_floats<SP::D>(kCWarps) * sizeof(float);
   return ring > scr ? ring : scr;
 }
 
@@ -651,15 +641,15 @@ struct FastEntry {
 template <class SP>
 cudaError_t launch_spec(const DecodeParams& p, cudaStream_t s) {
   const size_t dyn = dyn_bytes<SP>(p.stages);
-  cudaError_t e = prep(decode_fast_kernel<SP>, dyn, nullptr);
+  cudaError_t e = prep(decode_fast_kernel<SP>, dyn, nullptr, kCThreads);
   if (e != cudaSuccess) return e;
-  decode_fast_kernel<SP><<<dim3(p.splits, p.bh), kThreads, dyn, s>>>(p);
+  decode_fast_kernel<SP><<<dim3(p.splits, p.bh), kCThreads, dyn, s>>>(p);
   return cudaGetLastError();
 }
 
 template <class SP>
 cudaError_t occ_spec(int stages, int* occ) {
-  return prep(decode_fast_kernel<SP>, dyn_bytes<SP>(stages), occ);
+  return prep(decode_fast_kernel<SP>, dyn_bytes<SP>(stages), occ, kCThreads);
 }
 
 #define RQ_FAST(D, NC, RB, RG, AB, AG)                                                        \
@@ -709,7 +699,8 @@ bool fast_decode_plan(const DecodeParams& p, int D, size_t ring_budget, int max_
                       int* stages, int* ctas_per_sm) {
   const FastEntry* f = find_fast(p, D);
   if (f == nullptr) return false;
-  int s = static_cast<int>(ring_budget / f->stage_bytes);
+  (void)ring_budget;
+  int s = static_cast<int>(kCRingBudget / f->stage_bytes);
   if (s > max_stages) s = max_stages;
   if (s > kMaxRing) s = kMaxRing;
   if (s < 2) s = 2;
@@ -731,7 +722,7 @@ uint32_t bf16_stage_bytes(int D) {
   return D == 64 ? 2u * bf16_tc<64>() * 64 * 2 : 2u * bf16_tc<128>() * 128 * 2;
 }
 int bf16_chunk(int D) { return D == 64 ? bf16_tc<64>() : bf16_tc<128>(); }
-int fast_chunk() { return 128; }
+int fast_chunk() { return kCChunk; }
 
 cudaError_t bf16_occupancy(int D, int stages, int* occ) {
   const size_t ring = static_cast<size_t>(stages) * bf16_stage_bytes(D);

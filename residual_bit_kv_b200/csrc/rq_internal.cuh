@@ -138,6 +138,21 @@ cudaError_t decode_occupancy(int D, size_t dyn_smem, int* ctas_per_sm);
 // Device helpers
 // ---------------------------------------------------------------------------
 
+// Storage order of packed codes.  A lane's 32-channel slice of a row starts
+// at word slice*BITS; inside it channel ch (0..31) sits at
+//   BITS = 2: word ch/16, bits 2*(ch%16)
+//   BITS = 4: word 2*(ch/16) + ((ch%16 >> 1) & 1), nibble 2*((ch%16) >> 2) + (ch & 1)
+// so that, for both widths, masking bytes of the words yields the channel
+// quads {s, s+4, s+8, s+12} of each 16-channel block.
+template <int BITS>
+__host__ __device__ constexpr int slice_word(int ch) {
+  return BITS == 2 ? ch / 16 : 2 * (ch / 16) + (((ch % 16) >> 1) & 1);
+}
+template <int BITS>
+__host__ __device__ constexpr int slice_shift(int ch) {
+  return BITS == 2 ? 2 * (ch % 16) : 4 * (2 * ((ch % 16) >> 2) + (ch & 1));
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
   return __uint_as_float(h << 16);
 }

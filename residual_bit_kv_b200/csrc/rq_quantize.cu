@@ -57,7 +57,6 @@ template <int BITS>
 __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t crow,
                                             int slice, int D, float (&o)[32]) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
-  constexpr int PER_WORD = 32 / BITS;
   const uint32_t* w = c.codes + crow * (D * BITS / 32) + slice * BITS;
   uint32_t words[BITS];
 #pragma unroll
@@ -78,7 +77,7 @@ __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t crow,
   const float z1 = __half2float(__ushort_as_half((unsigned short)(mw1 >> 16)));
 #pragma unroll
   for (int ch = 0; ch < 32; ++ch) {
-    const uint32_t code = (words[ch / PER_WORD] >> (BITS * (ch % PER_WORD))) & QMAX;
+    const uint32_t code = (words[slice_word<BITS>(ch)] >> slice_shift<BITS>(ch)) & QMAX;
     const float cf = static_cast<float>(code);
     o[ch] = (ch < 16) ? __fmaf_rn(s0, cf, z0) : __fmaf_rn(s1, cf, z1);
   }
@@ -113,7 +112,6 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
                                                bool active, uint32_t* codes_row,
                                                uint32_t* meta_row) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
-  constexpr int PER_WORD = 32 / BITS;
   constexpr int GL = G < 32 ? G : 32;    // group part held by this lane
   constexpr int NG = 32 / GL;            // group parts per lane
   constexpr int LPG = G > 32 ? G / 32 : 1;  // lanes sharing a group
@@ -152,7 +150,7 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
       // u + 1.5*2^23 rounds u to the nearest integer, ties to even, and
       // leaves that integer in the low mantissa bits.
       const uint32_t code = __float_as_uint(__fadd_rn(u, 12582912.0f)) & QMAX;
-      words[ch / PER_WORD] |= code << (BITS * (ch % PER_WORD));
+      words[slice_word<BITS>(ch)] |= code << slice_shift<BITS>(ch);
     }
   }
   if (!active) return;

@@ -160,13 +160,15 @@ def test_int2_ramp_uses_all_four_levels(oracle_mod):
 
 
 def test_packing_bit_positions():
-    """Channel i -> word i/(32/b), bits [b*(i%(32/b)), +b) (hand-computed words)."""
+    """Storage order (hand-computed words): 2-bit channel i -> word i/16, bits
+    2*(i%16); 4-bit channel 16u+v -> word 2u+((v>>1)&1), nibble 2*(v>>2)+(v&1)."""
     import oracle
     o = np.float32(0.0)
-    # INT4, 32 channels with codes 0..15 then 15..0, scale 1, offset 0.
+    # INT4, 32 channels with codes 0..15 then 15..0, scale 1, offset 0:
+    # word 0 holds channels 0,1,4,5,8,9,12,13 in nibbles 0..7, word 1 the rest.
     z = np.array(list(range(16)) + list(range(15, -1, -1)), np.float32)
     words, _, _ = oracle.quantize(z, 4, 32)
-    assert [hex(w) for w in words] == ["0x76543210", "0xfedcba98", "0x89abcdef", "0x1234567"]
+    assert [hex(w) for w in words] == ["0xdc985410", "0xfeba7632", "0x2367abef", "0x14589cd"]
     # INT2, 16 channels: codes 3,0,1,2,... -> ((3)|(0<<2)|(1<<4)|(2<<6)) per byte = 0x93
     z2 = np.array([3, 0, 1, 2] * 4 + [0, 0, 0, 3] * 4, np.float32) + o
     w2, _, _ = oracle.quantize(z2, 2, 32)
