@@ -15,6 +15,7 @@ using namespace rq;
 constexpr uint64_t kAlign = 256;
 constexpr int kMaxSplits = 1024;
 constexpr int kMaxStages = 4;
+constexpr double kCtaOverheadChunks = 4.0;   // per-CTA fixed cost, in chunk times
 constexpr size_t kRingBudget = 100 * 1024;   // stage ring per CTA: two or more CTAs per SM
 
 inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
@@ -67,7 +68,8 @@ int max_splits_of(int32_t max_seq_len) {
 }
 
 // Split count for a grid of bh * splits CTAs, each streaming `cps` chunks.
-// Time model: (waves of resident CTAs) x (chunks per CTA); splits start at
+// Time model: (waves of resident CTAs) x (chunks per CTA + a fixed per-CTA
+// cost of set-up, first-chunk latency and merge); splits start at
 // the count that fills every resident slot once, so a small batch still
 // occupies the whole GPU.  Splits never exceed max_splits_of() (the
 // workspace bound) and never leave an empty split.
@@ -91,7 +93,7 @@ void choose_splits(int bh, int32_t max_seq_len, int chunk, int ctas_per_sm, int*
     const int c = (chunks + s - 1) / s;
     if ((chunks + c - 1) / c != s) continue;   // would leave empty splits
     const int64_t waves = (static_cast<int64_t>(bh) * s + slots - 1) / slots;
-    const double cost = static_cast<double>(waves) * c * (1.0 + 1e-3 * s);
+    const double cost = static_cast<double>(waves) * (c + kCtaOverheadChunks) * (1.0 + 1e-3 * s);
     if (cost < best) {
       best = cost;
       best_s = s;

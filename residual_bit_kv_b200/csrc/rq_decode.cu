@@ -335,7 +335,8 @@ uint32_t decode_stage_bytes(const DecodeParams& p, int D) {
 
 size_t decode_dyn_smem(int D, int stages, uint32_t stage_bytes) {
   const size_t ring = static_cast<size_t>(stages) * stage_bytes;
-  const size_t scr = D == 64 ? scratch_bytes<64>() : scratch_bytes<128>();
+  size_t scr = D == 64 ? scratch_bytes<64>() : scratch_bytes<128>();
+  if (scr < 3 * 1024 * sizeof(float)) scr = 3 * 1024 * sizeof(float);   // split headers
   return ring > scr ? ring : scr;
 }
 

@@ -60,7 +60,8 @@ __device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int ma
 // `slot` for channels [32*slice, 32*slice+32).  The slots are reduced into one
 // partial (m, l, acc[D]) in the workspace; the last CTA of the (batch, head)
 // then merges every split with the current token and writes the output,
-// applying H^T once when ROT.  `scratch` holds NSLOT*D + 2*NSLOT floats.
+// applying H^T once when ROT.  `scratch` holds max(NSLOT*D + 2*NSLOT,
+// 3*splits) floats.
 template <int D, int NT, int NSLOT, bool ROT>
 __device__ __forceinline__ void finish_split(float m, float l, const float (&acc)[32], int slice,
                                              int slot, float* scratch, int bhi, int split,
@@ -120,23 +121,40 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
   if ((t & 31) == 0) sred[t >> 5] = qk;
+  // Split headers (m, l) into shared memory (the scratch is free now).
+  const float* pbase = partials + static_cast<size_t>(bhi) * splits * (D + 2);
+  float* sm_m = scratch;              // [splits]
+  float* sm_l = scratch + splits;     // [splits]
+  float* sm_f = scratch + 2 * splits; // [splits]
+  for (int s = t; s < splits; s += NT) {
+    sm_m[s] = __ldcg(pbase + static_cast<size_t>(s) * (D + 2));
+    sm_l[s] = __ldcg(pbase + static_cast<size_t>(s) * (D + 2) + 1);
+  }
   __syncthreads();
   float s_cur = 0.0f;
   for (int w = 0; w < (D + 31) / 32; ++w) s_cur += sred[w];
   s_cur *= scale_log2;
-  const float* pbase = partials + static_cast<size_t>(bhi) * splits * (D + 2);
   float Mx = s_cur;
-  for (int s = 0; s < splits; ++s) Mx = fmaxf(Mx, __ldcg(pbase + s * (D + 2)));
+  for (int s = 0; s < splits; ++s) Mx = fmaxf(Mx, sm_m[s]);
+  for (int s = t; s < splits; s += NT)
+    sm_f[s] = (sm_m[s] == kNegInf) ? 0.0f : fast_exp2(sm_m[s] - Mx);
+  __syncthreads();
   float Lx = fast_exp2(s_cur - Mx);
+  for (int s = 0; s < splits; ++s) Lx = fmaf(sm_l[s], sm_f[s], Lx);
   float ax = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = __ldcg(pbase + s * (D + 2));
-    if (ms == kNegInf) continue;
-    const float fs = fast_exp2(ms - Mx);
-    Lx += __ldcg(pbase + s * (D + 2) + 1) * fs;
-    if (t < D) ax += __ldcg(pbase + s * (D + 2) + 2 + t) * fs;
+  if (t < D) {
+    const float* col = pbase + 2 + t;
+    int s = 0;
+    for (; s + 8 <= splits; s += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(col + static_cast<size_t>(s + u) * (D + 2));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ax = fmaf(v[u], sm_f[s + u], ax);
+    }
+    for (; s < splits; ++s) ax = fmaf(__ldcg(col + static_cast<size_t>(s) * (D + 2)), sm_f[s], ax);
   }
-  __syncthreads();   // everyone is done reading sred / svec
+  __syncthreads();   // everyone is done reading svec / the scratch
   if (t < D) svec[t] = ax;
   __syncthreads();
   if constexpr (ROT) smem_fwht<D>(svec);

@@ -35,6 +35,7 @@ constexpr int kCThreads = kCWarps * 32;
 constexpr int kCChunk = 64;                    // tokens per stage
 constexpr int kCMinCtas = 5;                   // register target: CTAs per SM
 constexpr size_t kCRingBudget = 40 * 1024;     // stage ring per CTA (several CTAs per SM)
+constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, up to 1024 splits
 
 template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
 struct Spec {
@@ -73,6 +74,34 @@ struct QLimbs {
   int h[2][4], l[2][4];
   float sq[2];   // sum of q~ over channels 0-15 / 16-31
 };
+
+// Unnormalised Hadamard butterflies over a row held by P = D/32 lanes, lane
+// `slice` holding channels 32*slice .. 32*slice+31 (stages h = 1..16 inside
+// the lane, then across lanes by xor-shuffles).
+template <int D>
+__device__ __forceinline__ void fwht_lanes(float (&z)[32], int slice) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float a = z[j], b = z[j + h];
+        z[j] = a + b;
+        z[j + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int hl = 1; hl < D / 32; hl <<= 1) {
+    const bool upper = (slice & hl) != 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, z[k], hl);
+      z[k] = upper ? o - z[k] : z[k] + o;
+    }
+  }
+}
 
 __device__ __forceinline__ int pack_bytes(int a, int b, int c, int d) {
   return (a & 0xFF) | ((b & 0xFF) << 8) | ((c & 0xFF) << 16) | (d << 24);
@@ -367,23 +396,37 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
     for (int i = 0; i < first; ++i) issue(i, i);
     s_issued = first;
   }
-  if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
-  __syncthreads();
-  smem_fwht<D>(svec);
-  // Fixed-point scale of q' = H q * softmax scale * log2 e.
+  // q' = H q * softmax scale * log2 e, rotated in registers by the P lanes of
+  // each token slot (every slot holds the same query), then its fixed-point
+  // scale from max |q'|.
+  float qv[32];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + static_cast<size_t>(bhi) * D + slice * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = src[i];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qv[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+        qv[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+  }
+  fwht_lanes<D>(qv, slice);
   const float qscale = p.rot_scale * p.scale_log2;
-  float amax = (t < D) ? fabsf(svec[t] * qscale) : 0.0f;
+  float amax = 0.0f;
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if (lane == 0) sred[warp] = amax;
-  __syncthreads();
-  amax = 0.0f;
+  for (int i = 0; i < 32; ++i) {
+    qv[i] *= qscale;
+    amax = fmaxf(amax, fabsf(qv[i]));
+  }
 #pragma unroll
-  for (int w = 0; w < kCThreads / 32; ++w) amax = fmaxf(amax, sred[w]);
+  for (int off = P / 2; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   const float sigma = amax > 0.0f ? amax / 32639.0f : 1.0f;
-
   QLimbs ql;
-  build_limbs(svec + slice * 32, qscale / sigma, ql);
+  build_limbs(qv, 1.0f / sigma, ql);
+  __syncthreads();   // barrier initialisation is visible to every warp
   float2 acc2[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc2[i] = make_float2(0.0f, 0.0f);
@@ -626,7 +669,8 @@ constexpr size_t scratch_floats(int warps = kWarps) {
 template <class SP>
 size_t dyn_bytes(int stages) {
   const size_t ring = static_cast<size_t>(stages) * SP::stage_bytes();
-  const size_t scr = scratch_floats<SP::D>(kCWarps) * sizeof(float);
+  size_t scr = scratch_floats<SP::D>(kCWarps) * sizeof(float);
+  if (scr < kMergeScratch) scr = kMergeScratch;
   return ring > scr ? ring : scr;
 }
 
@@ -683,7 +727,8 @@ const FastEntry* find_fast(const DecodeParams& p, int D) {
 template <int D>
 cudaError_t launch_bf16_t(const DecodeBf16Params& p, cudaStream_t s) {
   const size_t ring = static_cast<size_t>(p.stages) * (2 * bf16_tc<D>() * D * 2);
-  const size_t scr = scratch_floats<D>() * sizeof(float);
+  size_t scr = scratch_floats<D>() * sizeof(float);
+  if (scr < kMergeScratch) scr = kMergeScratch;
   const size_t dyn = ring > scr ? ring : scr;
   cudaError_t e = prep(decode_bf16_fast_kernel<D>, dyn, nullptr);
   if (e != cudaSuccess) return e;
