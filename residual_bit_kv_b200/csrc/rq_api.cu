@@ -342,6 +342,7 @@ rq_status rq_workspace_error(void* ws, uint64_t ws_bytes, void* stream) {
   }
   if (e != cudaSuccess) return RQ_ERR_CUDA;
   if (h & kErrTimeout) return RQ_ERR_TIMEOUT;
+  if (h & kErrRange) return RQ_ERR_UNSUPPORTED;
   if (h & kErrSeqLen) return RQ_ERR_CAPACITY;
   return RQ_OK;
 }

@@ -40,6 +40,7 @@ constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, u
 template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
 struct Spec {
   static constexpr int D = D_, NC = NC_, TC = kCChunk;
+  static constexpr int RB = RB_, AB = AB_;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
@@ -179,69 +180,115 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
   }
 }
 
-// Exact c * 2^p pairs: (x & mask) | 2^23-bits, minus 2^23.
-__device__ __forceinline__ float2 code_pair(uint32_t a, uint32_t b, uint32_t mask) {
-  const float2 v = make_float2(__uint_as_float((a & mask) | 0x4B000000u),
-                               __uint_as_float((b & mask) | 0x4B000000u));
-  return __fadd2_rn(v, make_float2(-8388608.0f, -8388608.0f));
+// Value path.  Two codes of one 32-bit word are OR-ed into the mantissas of
+// two f16 halves of 1024 (0x6400): half value 1024 + c * 2^p, exact for
+// p + bits <= 10.  Each half is multiplied by an f16 weight
+// w_p = f16(p_t * kappa * s~ * 2^(kWeightExp - p)) with an fp32 accumulator
+// (fma.rn.f32.f16: the f16 x f16 product is exact in fp32).  The 1024 * w_p
+// part is removed at the end from the exact running sum of the p = 0 weights
+// per component type and 16-channel half: w_p = w_0 * 2^-p exactly while the
+// weights stay in the f16 normal range.
+constexpr int kWeightExp = 8;
+constexpr float kWeightScale = 256.0f;          // 2^kWeightExp
+constexpr float kWeightMax = 65504.0f;          // largest finite f16
+
+__device__ __forceinline__ float fma_h(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;"
+      : "=f"(d)
+      : "h"(static_cast<unsigned short>(a)), "h"(static_cast<unsigned short>(b)), "f"(c));
+  return d;
 }
 
-// acc += pk * D(c) over one lane's 32 channels of token j.  acc2[8k + c] holds
-// channels (16k + c, 16k + c + 4) and acc2[8k + 4 + c] channels
-// (16k + 8 + c, 16k + 12 + c), c = 0..3.
-template <int D, int BITS, int G>
+__device__ __forceinline__ uint32_t f16_bits(float x) {
+  return __half_as_ushort(__float2half_rn(x));
+}
+
+// Half-word position (bits) of the channel paired at 16-channel-block offset v
+// in the value path: 2-bit codes at 2*(v%4) (word or word >> 8), 4-bit codes
+// at 4*(v&1) (word or word >> 8).
+template <int BITS>
+__host__ __device__ constexpr int vpos(int v) {
+  return BITS == 2 ? 2 * (v % 4) : 4 * (v & 1);
+}
+
+// acc += w * D(c) over one lane's 32 channels of token j.  pk = p_t * kappa;
+// TYPE selects the weight-sum slot (0: residual layout, 1: anchor layout).
+template <int D, int BITS, int G, int TYPE>
 __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned char* meta, int j,
-                                     int slice, float pk, float2 (&acc2)[16], float (&cst)[2]) {
+                                     int slice, float pk, float (&acc)[32], float (&cst)[2],
+                                     float (&wsum)[2][2], uint32_t& range_err) {
   constexpr int WPR = D * BITS / 32, GPR = D / G;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + j * WPR + slice * BITS;
   const uint32_t* mr = reinterpret_cast<const uint32_t*>(meta) + j * GPR;
-  float s0, z0, s1, z1;
+  float sc[2], zc[2];
   if constexpr (G >= 32) {
-    unpack_meta(mr[(slice * 32) / G], s0, z0);
-    s1 = s0;
-    z1 = z0;
+    unpack_meta(mr[(slice * 32) / G], sc[0], zc[0]);
+    sc[1] = sc[0];
+    zc[1] = zc[0];
   } else {
     const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
-    unpack_meta(mw.x, s0, z0);
-    unpack_meta(mw.y, s1, z1);
+    unpack_meta(mw.x, sc[0], zc[0]);
+    unpack_meta(mw.y, sc[1], zc[1]);
   }
-  cst[0] = fmaf(pk, z0, cst[0]);
-  cst[1] = fmaf(pk, z1, cst[1]);
-  const float wk[2] = {pk * s0, pk * s1};
+  constexpr int NPOS = BITS == 2 ? 4 : 2;   // positions 0,2,4,6 or 0,4
+  uint32_t wt[2][NPOS];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    cst[h] = fmaf(pk, zc[h], cst[h]);
+    if (G >= 32 && h == 1) {
+#pragma unroll
+      for (int q = 0; q < NPOS; ++q) wt[1][q] = wt[0][q];
+      wsum[TYPE][1] = fma_h(wt[1][0], 0x3C00u, wsum[TYPE][1]);
+      continue;
+    }
+    float w = pk * sc[h] * kWeightScale;
+    if (!(w <= kWeightMax)) {   // outside the f16 range of the weights
+      range_err = 1u;
+      w = 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < NPOS; ++q)
+      wt[h][q] = f16_bits(w * (1.0f / static_cast<float>(1u << (q * (BITS == 2 ? 2 : 4)))));
+    wsum[TYPE][h] = fma_h(wt[h][0], 0x3C00u, wsum[TYPE][h]);   // + exact f16 value
+  }
   if constexpr (BITS == 4) {
-    // word 2k + h, nibble n holds channel 16k + 4(n>>1) + 2h + (n&1); the
-    // pairs (n, n+2) sit at the same bits of (w, w>>8) and (w>>16, w>>24).
+    // word 2k + hh, nibble n: channel 16k + 4(n>>1) + 2hh + (n&1); nibbles n
+    // and n+4 share a half-word position, 0 or 4 in (word) / (word >> 8).
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
-      const int k = k4 >> 1, h = k4 & 1;
-      const float wt = (G >= 32) ? wk[0] : wk[k];
-      const float2 w0 = make_float2(wt, wt);
-      const float2 w1 = make_float2(wt * 0.0625f, wt * 0.0625f);
-      const uint32_t w8 = w[k4] >> 8, w16 = w[k4] >> 16, w24 = w[k4] >> 24;
-      acc2[8 * k + 2 * h] = __ffma2_rn(w0, code_pair(w[k4], w8, 0x0Fu), acc2[8 * k + 2 * h]);
-      acc2[8 * k + 2 * h + 1] =
-          __ffma2_rn(w1, code_pair(w[k4], w8, 0xF0u), acc2[8 * k + 2 * h + 1]);
-      acc2[8 * k + 4 + 2 * h] =
-          __ffma2_rn(w0, code_pair(w16, w24, 0x0Fu), acc2[8 * k + 4 + 2 * h]);
-      acc2[8 * k + 4 + 2 * h + 1] =
-          __ffma2_rn(w1, code_pair(w16, w24, 0xF0u), acc2[8 * k + 4 + 2 * h + 1]);
+      const int k = k4 >> 1, hh = k4 & 1;
+      const uint32_t w8 = w[k4] >> 8;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        const uint32_t src = n < 2 ? w[k4] : w8;
+        const uint32_t mask = (n & 1) ? 0x00F000F0u : 0x000F000Fu;
+        const uint32_t x = (src & mask) | 0x64006400u;
+        const int ch = 16 * k + 4 * (n >> 1) + 2 * hh + (n & 1);
+        const uint32_t wq = wt[G >= 32 ? 0 : k][n & 1];
+        acc[ch] = fma_h(x & 0xFFFFu, wq, acc[ch]);
+        acc[ch + 8] = fma_h(x >> 16, wq, acc[ch + 8]);
+      }
     }
   } else {
+    // word k, 2-bit field f (f < 8 in the low half, f + 8 in the high half):
+    // fields 0..3 at bits 2f of the word, fields 4..7 at bits 2(f-4) of word >> 8.
     const uint2 v = *reinterpret_cast<const uint2*>(cw);
     const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const float wt = (G >= 32) ? wk[0] : wk[k];
-      const uint32_t w8 = w[k] >> 8, w16 = w[k] >> 16, w24 = w[k] >> 24;
+      const uint32_t w8 = w[k] >> 8;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float sc = wt * (1.0f / static_cast<float>(1u << (2 * c)));
-        const float2 wc = make_float2(sc, sc);
-        const uint32_t m = 3u << (2 * c);
-        acc2[8 * k + c] = __ffma2_rn(wc, code_pair(w[k], w8, m), acc2[8 * k + c]);
-        acc2[8 * k + 4 + c] = __ffma2_rn(wc, code_pair(w16, w24, m), acc2[8 * k + 4 + c]);
+      for (int f = 0; f < 8; ++f) {
+        const int q = f & 3;
+        const uint32_t src = f < 4 ? w[k] : w8;
+        const uint32_t mask = (3u << (2 * q)) | (3u << (16 + 2 * q));
+        const uint32_t x = (src & mask) | 0x64006400u;
+        const uint32_t wq = wt[G >= 32 ? 0 : k][q];
+        acc[16 * k + f] = fma_h(x & 0xFFFFu, wq, acc[16 * k + f]);
+        acc[16 * k + 8 + f] = fma_h(x >> 16, wq, acc[16 * k + 8 + f]);
       }
     }
   }
@@ -263,27 +310,31 @@ __device__ __forceinline__ void score_comps(const unsigned char* st, int j, int 
 
 template <class SP, int C = 0>
 __device__ __forceinline__ void value_comps(const unsigned char* st, int j, int slice, float kap,
-                                            float2 (&acc2)[16], float (&cst)[2]) {
+                                            float (&acc)[32], float (&cst)[2],
+                                            float (&wsum)[2][2], uint32_t& range_err) {
   if constexpr (C < SP::NC) {
-    vacc<SP::D, SP::bits(C), SP::group(C)>(st + SP::codes_off(1, C), st + SP::meta_off(1, C), j,
-                                           slice, kap, acc2, cst);
+    vacc<SP::D, SP::bits(C), SP::group(C), (C == SP::NC - 1) ? 1 : 0>(
+        st + SP::codes_off(1, C), st + SP::meta_off(1, C), j, slice, kap, acc, cst, wsum,
+        range_err);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(st + SP::alpha_off(1, C))[j]);
-    value_comps<SP, C + 1>(st, j, slice, kap, acc2, cst);
+    value_comps<SP, C + 1>(st, j, slice, kap, acc, cst, wsum, range_err);
   }
 }
 
-__device__ __forceinline__ void unpair(const float2 (&acc2)[16], const float (&cst)[2],
-                                       float (&acc)[32]) {
+// Final value of the accumulators: remove the 1024 * w_p offsets of each
+// component type (residual layout RB, anchor layout AB) and the weight scale,
+// add the z~ terms.
+template <int RB, int AB, bool HAS_R>
+__device__ __forceinline__ void finish_values(float (&acc)[32], const float (&cst)[2],
+                                              const float (&wsum)[2][2]) {
 #pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      acc[16 * k + c] = acc2[8 * k + c].x + cst[k];
-      acc[16 * k + c + 4] = acc2[8 * k + c].y + cst[k];
-      acc[16 * k + 8 + c] = acc2[8 * k + 4 + c].x + cst[k];
-      acc[16 * k + 12 + c] = acc2[8 * k + 4 + c].y + cst[k];
-    }
+  for (int ch = 0; ch < 32; ++ch) {
+    const int v = ch % 16, h = ch / 16;
+    float off = 1024.0f * wsum[1][h] / static_cast<float>(1u << vpos<AB>(v));
+    if (HAS_R) off += 1024.0f * wsum[0][h] / static_cast<float>(1u << vpos<RB>(v));
+    acc[ch] = (acc[ch] - off) * (1.0f / kWeightScale) + cst[h];
+  }
 }
 
 // Token range of this CTA's split.
@@ -427,10 +478,12 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   QLimbs ql;
   build_limbs(qv, 1.0f / sigma, ql);
   __syncthreads();   // barrier initialisation is visible to every warp
-  float2 acc2[16];
+  float acc[32];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+  for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
   float cst[2] = {0.0f, 0.0f};
+  float wsum[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+  uint32_t range_err = 0u;
   float m = kNegInf, l = 0.0f;
 
   for (int i = 0; i < R.nchunks; ++i) {
@@ -454,12 +507,15 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
     for (int tt = 1; tt < TT; ++tt) mc = fmaxf(mc, sc[tt]);
     if (mc > m) {
       const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
-      const float2 f2 = make_float2(f, f);
       l *= f;
       cst[0] *= f;
       cst[1] *= f;
+      wsum[0][0] *= f;
+      wsum[0][1] *= f;
+      wsum[1][0] *= f;
+      wsum[1][1] *= f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) acc2[k] = __fmul2_rn(acc2[k], f2);
+      for (int k = 0; k < 32; ++k) acc[k] *= f;
       m = mc;
     }
 #pragma unroll
@@ -468,7 +524,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       if (sc[tt] == kNegInf) continue;
       const float pt = fast_exp2(sc[tt] - m);
       l += pt;
-      value_comps<SP>(st, j, slice, pt, acc2, cst);
+      value_comps<SP>(st, j, slice, pt, acc, cst, wsum, range_err);
     }
     // Release the stage; the last warp to do so refills it.
     __syncwarp();
@@ -482,8 +538,8 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       }
     }
   }
-  float acc[32];
-  unpair(acc2, cst, acc);
+  finish_values<SP::RB, SP::AB, (SP::NC > 1)>(acc, cst, wsum);
+  if (range_err) atomicOr(p.err, kErrRange);
   if (s_abort) {
     m = kNegInf;
     l = 0.0f;

@@ -17,6 +17,7 @@ namespace rq {
 // Device-side error bits recorded in the decode workspace.
 constexpr uint32_t kErrSeqLen = 1u;    // a seq_lens entry was outside [0, max_seq_len]
 constexpr uint32_t kErrTimeout = 2u;   // a bounded mbarrier wait ran out
+constexpr uint32_t kErrRange = 4u;     // a value weight left the f16 range (group scale too large)
 
 // Tokens per pipeline stage of the decode kernels.
 constexpr int kChunk = 64;
