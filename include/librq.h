@@ -18,14 +18,20 @@
  *   z~ = fp16(min), code = rint_even(clamp((z - z~) * (1/s~), 0, 2^b - 1)).
  *   Reconstruction: Z^_r = alpha~_r R + s~ c + z~ and X^_r = H^T Z^_r.
  *
- * Storage contract (per layer and per side K | V; all offsets 256-B aligned;
- * rows are [batch][kv_heads][token_stride] with token_stride =
- * max_tokens rounded up to a multiple of 16):
- *   codes of loop r : uint32 [rows][head_dim * bits[r] / 32]; channel i sits
- *                     in word i / (32/b), bits [b*(i % (32/b)), +b)
- *   meta of loop r  : uint32 [rows][head_dim / group[r]]; low half fp16
- *                     scale s~, high half fp16 offset z~
- *   alpha of loop r : bf16  [rows] (residual loops only)
+ * Storage contract (per layer and per side K | V):
+ *   Tokens are stored in records of RQ_BLOCK_TOKENS = 64 consecutive tokens.
+ *   Loop r of (row = batch*kv_heads index b*H + h, block k) is one record at
+ *   byte offset comp_off[r] + (row * token_stride/64 + k) * rec_bytes[r] of
+ *   the (layer, side) region; token_stride is max_tokens rounded up to 64.
+ *   A record holds, contiguously:
+ *     codes  uint32 [64][head_dim * bits[r] / 32]
+ *     meta   uint32 [64][head_dim / group[r]]; low half fp16 scale s~,
+ *            high half fp16 offset z~
+ *     alpha  bf16   [64]             (residual loops only)
+ *   so a 64-token decode stage of one component is one contiguous copy.
+ *   Code order inside a token's row: b = 2: channel i in word i/16, bits
+ *   [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v, word
+ *   2u + ((v>>1)&1), bits [4*(2*(v>>2) + (v&1)), +4).  Little-endian words.
  *   Effective bits per element of loop r: bits[r] + 32/group[r]
  *   (+ 16/head_dim for a residual loop).
  *
@@ -55,6 +61,7 @@ extern "C" {
 
 #define RQ_ABI_VERSION 1
 #define RQ_MAX_LOOPS 32
+#define RQ_BLOCK_TOKENS 64
 
 typedef enum rq_status {
   RQ_OK = 0,
@@ -99,13 +106,12 @@ typedef struct rq_layout {
  * treat as read-only).  Offsets are bytes within one (layer, side). */
 typedef struct rq_cache {
   rq_layout layout;
-  void* k_base;                 /* num_layers * layer_bytes, K side */
-  void* v_base;                 /* num_layers * layer_bytes, V side */
+  void* k_base;                      /* num_layers * layer_bytes, K side */
+  void* v_base;                      /* num_layers * layer_bytes, V side */
   uint64_t layer_bytes;
-  int64_t token_stride;
-  uint64_t codes_off[RQ_MAX_LOOPS];
-  uint64_t meta_off[RQ_MAX_LOOPS];
-  uint64_t alpha_off[RQ_MAX_LOOPS];  /* 0 for the anchor loop */
+  int64_t token_stride;              /* max_tokens rounded up to RQ_BLOCK_TOKENS */
+  uint64_t comp_off[RQ_MAX_LOOPS];   /* first record of loop r (256-B aligned) */
+  uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 64-token record of loop r */
 } rq_cache;
 
 /* ABI version of the loaded library (RQ_ABI_VERSION at build time). */

@@ -27,29 +27,30 @@ inline rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 inline int64_t token_stride_of(const rq_layout* l) {
-  return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), 16));
+  return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), kBlock));
 }
 
-// Byte offsets of every array inside one (layer, side); returns layer bytes.
-uint64_t layout_offsets(const rq_layout* l, uint64_t* codes, uint64_t* meta, uint64_t* alpha) {
-  const uint64_t rows = static_cast<uint64_t>(l->batch) * l->kv_heads * token_stride_of(l);
-  const int L = l->num_loops, D = l->head_dim;
+inline uint32_t record_bytes(const rq_layout* l, int r) {
+  const int D = l->head_dim;
+  const uint32_t per_token = (D * l->bits[r] / 32) * 4 + (D / l->group[r]) * 4 +
+                             (r != l->num_loops - 1 ? 2 : 0);
+  return kBlock * per_token;   // a multiple of 128 bytes
+}
+
+// Byte offset of every component's first record inside one (layer, side);
+// returns the layer bytes.  Anchor (loop L-1) first, then loops 0 .. L-2.
+uint64_t layout_offsets(const rq_layout* l, uint64_t* comp_off, uint32_t* rec_bytes) {
+  const uint64_t records = static_cast<uint64_t>(l->batch) * l->kv_heads *
+                           (token_stride_of(l) / kBlock);
+  const int L = l->num_loops;
   uint64_t off = 0;
-  // anchor (loop L-1) first, then residual loops 0 .. L-2
   for (int k = 0; k < L; ++k) {
     const int r = (k == 0) ? L - 1 : k - 1;
-    codes[r] = off;
-    off = align_up(off + rows * (D * l->bits[r] / 32) * 4, kAlign);
-    meta[r] = off;
-    off = align_up(off + rows * (D / l->group[r]) * 4, kAlign);
-    if (r != L - 1) {
-      alpha[r] = off;
-      off = align_up(off + rows * 2, kAlign);
-    } else {
-      alpha[r] = 0;
-    }
+    comp_off[r] = off;
+    rec_bytes[r] = record_bytes(l, r);
+    off = align_up(off + records * rec_bytes[r], kAlign);
   }
-  return align_up(off, kAlign);
+  return off;
 }
 
 int device_sms() {
@@ -124,15 +125,12 @@ const unsigned char* side_base(const rq_cache* c, int layer, int kv) {
 }
 
 Comp comp_of(const rq_cache* c, int layer, int kv, int r) {
-  const unsigned char* b = side_base(c, layer, kv);
   Comp k;
-  k.codes = reinterpret_cast<const uint32_t*>(b + c->codes_off[r]);
-  k.meta = reinterpret_cast<const uint32_t*>(b + c->meta_off[r]);
-  k.alpha = (r == c->layout.num_loops - 1)
-                ? nullptr
-                : reinterpret_cast<const uint16_t*>(b + c->alpha_off[r]);
+  k.base = const_cast<unsigned char*>(side_base(c, layer, kv)) + c->comp_off[r];
+  k.rec_bytes = c->rec_bytes[r];
   k.bits = c->layout.bits[r];
   k.group = c->layout.group[r];
+  k.has_alpha = (r != c->layout.num_loops - 1) ? 1 : 0;
   return k;
 }
 
@@ -215,8 +213,9 @@ rq_status rq_layout_validate(const rq_layout* l) {
 
 uint64_t rq_layer_bytes(const rq_layout* l) {
   if (rq_layout_validate(l) != RQ_OK) return 0;
-  uint64_t c[RQ_MAX_LOOPS], m[RQ_MAX_LOOPS], a[RQ_MAX_LOOPS];
-  return layout_offsets(l, c, m, a);
+  uint64_t c[RQ_MAX_LOOPS];
+  uint32_t rb[RQ_MAX_LOOPS];
+  return layout_offsets(l, c, rb);
 }
 
 uint64_t rq_cache_bytes(const rq_layout* l) {
@@ -233,7 +232,7 @@ rq_status rq_cache_bind(const rq_layout* l, void* k_base, void* v_base, rq_cache
   out->layout = *l;
   out->k_base = k_base;
   out->v_base = v_base;
-  out->layer_bytes = layout_offsets(l, out->codes_off, out->meta_off, out->alpha_off);
+  out->layer_bytes = layout_offsets(l, out->comp_off, out->rec_bytes);
   out->token_stride = token_stride_of(l);
   return RQ_OK;
 }
@@ -247,17 +246,14 @@ rq_status rq_quantize_anchor(const rq_cache* c, int32_t layer, int32_t kv, const
   if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
   const rq_layout& l = c->layout;
   const int a = l.num_loops - 1;
-  unsigned char* base = const_cast<unsigned char*>(side_base(c, layer, kv));
   QuantParams p;
   memset(&p, 0, sizeof(p));
   p.x = static_cast<const uint16_t*>(x);
   p.bh = l.batch * l.kv_heads;
   p.n = n;
   p.t0 = t0;
-  p.tstride = c->token_stride;
-  p.codes = reinterpret_cast<uint32_t*>(base + c->codes_off[a]);
-  p.meta = reinterpret_cast<uint32_t*>(base + c->meta_off[a]);
-  p.alpha = nullptr;
+  p.nblk = c->token_stride / kBlock;
+  p.dst = comp_of(c, layer, kv, a);
   p.nref = 0;
   p.rot_scale = rot_scale_of(l.head_dim);
   return cuda_status(launch_quantize(p, l.head_dim, l.bits[a], l.group[a], as_stream(stream)));
@@ -272,17 +268,14 @@ rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t 
   if ((st = check_range(c, t0, n)) != RQ_OK) return st;
   if (n == 0) return RQ_OK;
   if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
-  unsigned char* base = const_cast<unsigned char*>(side_base(c, layer, kv));
   QuantParams p;
   memset(&p, 0, sizeof(p));
   p.x = static_cast<const uint16_t*>(x);
   p.bh = l.batch * l.kv_heads;
   p.n = n;
   p.t0 = t0;
-  p.tstride = c->token_stride;
-  p.codes = reinterpret_cast<uint32_t*>(base + c->codes_off[loop]);
-  p.meta = reinterpret_cast<uint32_t*>(base + c->meta_off[loop]);
-  p.alpha = reinterpret_cast<uint16_t*>(base + c->alpha_off[loop]);
+  p.nblk = c->token_stride / kBlock;
+  p.dst = comp_of(c, layer, kv, loop);
   // Reference: the anchor (Last-loop) or the chain loop+1 .. anchor (Next-loop).
   Comp chain[RQ_MAX_LOOPS];
   const int len = chain_of(c, layer, kv, loop, chain);   // [loop, ref...]
@@ -307,7 +300,7 @@ rq_status rq_dequantize(const rq_cache* c, int32_t layer, int32_t kv, int32_t lo
   p.bh = l.batch * l.kv_heads;
   p.n = n;
   p.t0 = t0;
-  p.tstride = c->token_stride;
+  p.nblk = c->token_stride / kBlock;
   p.ncomp = chain_of(c, layer, kv, loop, p.comp);
   p.rot_scale = rot_scale_of(l.head_dim);
   p.out = out;
@@ -353,7 +346,7 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
   memset(p, 0, sizeof(*p));
   p->bh = l.batch * l.kv_heads;
   p->heads = l.kv_heads;
-  p->tstride = c->token_stride;
+  p->nblk = c->token_stride / kBlock;
   p->ncomp = chain_of(c, layer, 0, loop, p->k);
   (void)chain_of(c, layer, 1, loop, p->v);
   p->max_seq_len = max_seq_len;

@@ -56,7 +56,7 @@ __host__ __device__ inline void build_stage_map(const DecodeParams& p, int D,
       m.meta[side][c] = off;
       off += kChunk * (D / cs[c].group) * 4;
       m.alpha[side][c] = off;
-      if (cs[c].alpha != nullptr) off += kChunk * 2;
+      if (cs[c].has_alpha) off += kChunk * 2;
     }
   }
   m.bytes = off;
@@ -167,34 +167,22 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
   __syncthreads();
 
-  const size_t row0 = static_cast<size_t>(bhi) * p.tstride;
+  static_assert(kChunk == kBlock, "a decode stage is one storage record per component");
   auto issue = [&](int i) {
     const int s = i % S;
     const int t0 = t_begin + i * kChunk;
-    const int nt = min(kChunk, t_end - t0);
-    const int ntc = (nt + 7) & ~7;   // 16-byte granules of the bf16 coefficients
     unsigned char* st = smem + static_cast<size_t>(s) * p.stage_bytes;
     uint32_t bytes = 0;
     for (int side = 0; side < 2; ++side) {
       const Comp* cs = side == 0 ? p.k : p.v;
-      for (int c = 0; c < p.ncomp; ++c) {
-        bytes += ntc * (D * cs[c].bits / 32) * 4 + ntc * (D / cs[c].group) * 4;
-        if (cs[c].alpha != nullptr) bytes += ntc * 2;
-      }
+      for (int c = 0; c < p.ncomp; ++c) bytes += cs[c].rec_bytes;
     }
     mbar_arrive_expect_tx(&full_bar[s], bytes);
     for (int side = 0; side < 2; ++side) {
       const Comp* cs = side == 0 ? p.k : p.v;
-      for (int c = 0; c < p.ncomp; ++c) {
-        const int wpr = D * cs[c].bits / 32, gpr = D / cs[c].group;
-        bulk_copy_g2s(st + map.codes[side][c], cs[c].codes + (row0 + t0) * wpr,
-                      ntc * wpr * 4, &full_bar[s]);
-        bulk_copy_g2s(st + map.meta[side][c], cs[c].meta + (row0 + t0) * gpr,
-                      ntc * gpr * 4, &full_bar[s]);
-        if (cs[c].alpha != nullptr)
-          bulk_copy_g2s(st + map.alpha[side][c], cs[c].alpha + row0 + t0, ntc * 2,
-                        &full_bar[s]);
-      }
+      for (int c = 0; c < p.ncomp; ++c)
+        bulk_copy_g2s(st + map.codes[side][c], comp_record(cs[c], bhi, p.nblk, t0),
+                      cs[c].rec_bytes, &full_bar[s]);
     }
   };
   int issued = 0;

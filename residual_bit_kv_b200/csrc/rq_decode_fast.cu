@@ -189,7 +189,7 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
 // per component type and 16-channel half: w_p = w_0 * 2^-p exactly while the
 // weights stay in the f16 normal range.
 constexpr int kWeightExp = 8;
-constexpr float kWeightScale = 256.0f;          // 2^kWeightExp
+constexpr float kWeightScale = static_cast<float>(1 << kWeightExp);
 constexpr float kWeightMax = 65504.0f;          // largest finite f16
 
 __device__ __forceinline__ float fma_h(uint32_t a, uint32_t b, float c) {
@@ -407,32 +407,21 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   const int S = p.stages;
   const int n = seq_len_of(p.seq_lens, bhi / p.heads, p.max_seq_len, p.err);
   const Range R = split_range(n, split, p.chunks_per_split, TC);
-  const size_t row0 = static_cast<size_t>(bhi) * p.tstride;
+  static_assert(TC == kBlock, "a decode stage is one storage record per component");
 
-  // Copies of chunk i into stage s (one lane).
+  // Copies of chunk i into stage s (one lane): one record per component.
   auto issue = [&](int i, int s) {
     const int t0 = R.t_begin + i * TC;
-    const uint32_t ntc = static_cast<uint32_t>((min(TC, R.t_end - t0) + 7) & ~7);
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-      bytes += 2u * ntc * (SP::wpr(c) * 4 + SP::gpr(c) * 4 + (SP::has_alpha(c) ? 2 : 0));
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&full_bar[s], bytes);
+    mbar_arrive_expect_tx(&full_bar[s], SP::stage_bytes());
     unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
 #pragma unroll
     for (int side = 0; side < 2; ++side) {
       const Comp* cs = side == 0 ? p.k : p.v;
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        bulk_copy_g2s(st + SP::codes_off(side, c), cs[c].codes + (row0 + t0) * SP::wpr(c),
-                      ntc * SP::wpr(c) * 4, &full_bar[s]);
-        bulk_copy_g2s(st + SP::meta_off(side, c), cs[c].meta + (row0 + t0) * SP::gpr(c),
-                      ntc * SP::gpr(c) * 4, &full_bar[s]);
-        if (SP::has_alpha(c))
-          bulk_copy_g2s(st + SP::alpha_off(side, c), cs[c].alpha + row0 + t0, ntc * 2,
-                        &full_bar[s]);
-      }
+      for (int c = 0; c < NC; ++c)
+        bulk_copy_g2s(st + SP::codes_off(side, c), comp_record(cs[c], bhi, p.nblk, t0),
+                      SP::comp_bytes(c), &full_bar[s]);
     }
   };
 
@@ -775,6 +764,10 @@ const FastEntry* find_fast(const DecodeParams& p, int D) {
     if (f.D != D || f.NC != NC) continue;
     bool ok = p.k[NC - 1].bits == f.AB && p.k[NC - 1].group == f.AG;
     for (int c = 0; c + 1 < NC; ++c) ok = ok && p.k[c].bits == f.RB && p.k[c].group == f.RG;
+    // a stage is exactly one record per component and side
+    uint32_t rec = 0;
+    for (int c = 0; c < NC; ++c) rec += p.k[c].rec_bytes + p.v[c].rec_bytes;
+    ok = ok && rec == f.stage_bytes;
     if (ok) return &f;
   }
   return nullptr;

@@ -27,24 +27,42 @@ constexpr int kDecodeThreads = 128;
 // Parameter blocks
 // ---------------------------------------------------------------------------
 
-// One packed component (anchor or one residual loop) of one side.
+// One packed component (anchor or one residual loop) of one side, stored as
+// 64-token records [codes[64][D*bits/32] | meta[64][D/group] | alpha[64]].
 struct Comp {
-  const uint32_t* codes;   // [rows][D*bits/32]
-  const uint32_t* meta;    // [rows][D/group]
-  const uint16_t* alpha;   // [rows] bf16, nullptr for the anchor
+  unsigned char* base;     // record of (row 0, block 0)
+  uint32_t rec_bytes;      // bytes per record
   int32_t bits;
   int32_t group;
+  int32_t has_alpha;       // 0 for the anchor
 };
+
+constexpr int kBlock = RQ_BLOCK_TOKENS;
+
+// Record holding token t of row `row` (nblk = records per row).
+__host__ __device__ inline unsigned char* comp_record(const Comp& c, int64_t row, int64_t nblk,
+                                                      int64_t t) {
+  return c.base + (row * nblk + t / kBlock) * static_cast<int64_t>(c.rec_bytes);
+}
+__host__ __device__ inline uint32_t* rec_codes(unsigned char* rec, int D, int bits, int i) {
+  return reinterpret_cast<uint32_t*>(rec) + i * (D * bits / 32);
+}
+__host__ __device__ inline uint32_t* rec_meta(unsigned char* rec, int D, int bits, int group,
+                                              int i) {
+  return reinterpret_cast<uint32_t*>(rec) + kBlock * (D * bits / 32) + i * (D / group);
+}
+__host__ __device__ inline uint16_t* rec_alpha(unsigned char* rec, int D, int bits, int group,
+                                               int i) {
+  return reinterpret_cast<uint16_t*>(rec + kBlock * 4 * (D * bits / 32 + D / group)) + i;
+}
 
 struct QuantParams {
   const uint16_t* x;       // bf16 [B*H][n][D]
   int32_t bh;              // B*H
   int32_t n;
   int32_t t0;
-  int64_t tstride;
-  uint32_t* codes;         // destination component
-  uint32_t* meta;
-  uint16_t* alpha;         // nullptr for the anchor
+  int64_t nblk;            // records per row
+  Comp dst;                // destination component
   // Reference chain, nearest first: for LAST_LOOP one entry (the anchor);
   // for NEXT_LOOP loops loop+1 .. L-1 (the anchor last).
   int32_t nref;
@@ -54,7 +72,7 @@ struct QuantParams {
 
 struct DequantParams {
   int32_t bh, n, t0;
-  int64_t tstride;
+  int64_t nblk;
   int32_t ncomp;           // chain: [0] = the loop itself ... [ncomp-1] = anchor
   Comp comp[RQ_MAX_LOOPS];
   float rot_scale;
@@ -64,7 +82,7 @@ struct DequantParams {
 struct DecodeParams {
   int32_t bh;              // B*H
   int32_t heads;
-  int64_t tstride;
+  int64_t nblk;            // records per row
   int32_t ncomp;           // [0] = the loop's own residual ... [ncomp-1] = anchor
   Comp k[RQ_MAX_LOOPS];
   Comp v[RQ_MAX_LOOPS];

@@ -52,17 +52,19 @@ __device__ __forceinline__ void fwht_row(float (&z)[32], int slice) {
   }
 }
 
-// Stored levels fma(s~, code, z~) of one lane's 32 channels of a component.
+// Stored levels fma(s~, code, z~) of one lane's 32 channels of a component
+// at token t of row `row`.
 template <int BITS>
-__device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t crow,
+__device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t row, int64_t nblk, int64_t t,
                                             int slice, int D, float (&o)[32]) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
-  const uint32_t* w = c.codes + crow * (D * BITS / 32) + slice * BITS;
+  unsigned char* rec = comp_record(c, row, nblk, t);
+  const int i = static_cast<int>(t % kBlock);
+  const uint32_t* w = rec_codes(rec, D, BITS, i) + slice * BITS;
   uint32_t words[BITS];
 #pragma unroll
-  for (int i = 0; i < BITS; ++i) words[i] = w[i];
-  const int gpr = D / c.group;
-  const uint32_t* m = c.meta + crow * gpr;
+  for (int k = 0; k < BITS; ++k) words[k] = w[k];
+  const uint32_t* m = rec_meta(rec, D, BITS, c.group, i);
   uint32_t mw0, mw1;
   if (c.group >= 32) {
     mw0 = m[(slice * 32) / c.group];
@@ -83,24 +85,25 @@ __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t crow,
   }
 }
 
-__device__ __forceinline__ void deq_slice(const Comp& c, int64_t crow, int slice,
-                                          int D, float (&o)[32]) {
+__device__ __forceinline__ void deq_slice(const Comp& c, int64_t row, int64_t nblk, int64_t t,
+                                          int slice, int D, float (&o)[32]) {
   if (c.bits == 4)
-    deq_slice_t<4>(c, crow, slice, D, o);
+    deq_slice_t<4>(c, row, nblk, t, slice, D, o);
   else
-    deq_slice_t<2>(c, crow, slice, D, o);
+    deq_slice_t<2>(c, row, nblk, t, slice, D, o);
 }
 
-// Rotated reconstruction of a chain [0 .. n-1] (anchor last) at cache row
-// crow: Z = deq(anchor); for k = n-2 .. 0: Z = fma(alpha~_k, Z, deq_k).
-__device__ __forceinline__ void chain_slice(const Comp* comps, int n,
-                                            int64_t crow, int slice, int D,
-                                            float (&zr)[32]) {
-  deq_slice(comps[n - 1], crow, slice, D, zr);
+// Rotated reconstruction of a chain [0 .. n-1] (anchor last) at token t of
+// row `row`: Z = deq(anchor); for k = n-2 .. 0: Z = fma(alpha~_k, Z, deq_k).
+__device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t row, int64_t nblk,
+                                            int64_t t, int slice, int D, float (&zr)[32]) {
+  deq_slice(comps[n - 1], row, nblk, t, slice, D, zr);
   for (int k = n - 2; k >= 0; --k) {
     float d[32];
-    deq_slice(comps[k], crow, slice, D, d);
-    const float a = bf16_bits_to_f32(comps[k].alpha[crow]);
+    deq_slice(comps[k], row, nblk, t, slice, D, d);
+    const Comp& c = comps[k];
+    const float a = bf16_bits_to_f32(
+        *rec_alpha(comp_record(c, row, nblk, t), D, c.bits, c.group, static_cast<int>(t % kBlock)));
 #pragma unroll
     for (int ch = 0; ch < 32; ++ch) zr[ch] = __fmaf_rn(a, zr[ch], d[ch]);
   }
@@ -174,8 +177,6 @@ __global__ void __launch_bounds__(kQuantThreads)
     quantize_kernel(const __grid_constant__ QuantParams p) {
   constexpr int P = D / 32;
   constexpr int RPW = 32 / P;
-  constexpr int WPR = D * BITS / 32;
-  constexpr int GPR = D / G;
   const int lane = threadIdx.x & 31;
   const int slice = lane % P;
   const int64_t total = static_cast<int64_t>(p.bh) * p.n;
@@ -207,14 +208,14 @@ __global__ void __launch_bounds__(kQuantThreads)
     for (int k = 0; k < 32; ++k) z[k] = __fmul_rn(z[k], p.rot_scale);
 
     const int64_t bhi = active ? row / p.n : 0;
-    const int64_t crow = bhi * p.tstride + p.t0 + (active ? row % p.n : 0);
+    const int64_t t = p.t0 + (active ? row % p.n : 0);
 
-    if (p.alpha != nullptr) {
+    if (p.dst.has_alpha) {
       // Least-squares coefficient against the reconstructed reference
       // [RQ §3.2 scaling coefficient, App. G.1], then the residual.
       float ref[32];
       if (active) {
-        chain_slice(p.ref, p.nref, crow, slice, D, ref);
+        chain_slice(p.ref, p.nref, bhi, p.nblk, t, slice, D, ref);
       } else {
 #pragma unroll
         for (int k = 0; k < 32; ++k) ref[k] = 0.0f;
@@ -235,10 +236,14 @@ __global__ void __launch_bounds__(kQuantThreads)
       const float at = __bfloat162float(ab);
 #pragma unroll
       for (int k = 0; k < 32; ++k) z[k] = __fmaf_rn(-at, ref[k], z[k]);
-      if (active && slice == 0) p.alpha[crow] = __bfloat16_as_ushort(ab);
+      if (active && slice == 0)
+        *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock)) =
+            __bfloat16_as_ushort(ab);
     }
-    quantize_store<D, BITS, G>(z, slice, active, p.codes + crow * WPR,
-                               p.meta + crow * GPR);
+    unsigned char* rec = comp_record(p.dst, bhi, p.nblk, t);
+    const int i = static_cast<int>(t % kBlock);
+    quantize_store<D, BITS, G>(z, slice, active, rec_codes(rec, D, BITS, i),
+                               rec_meta(rec, D, BITS, G, i));
   }
 }
 
@@ -258,8 +263,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     const bool active = row < total;
     float z[32];
     if (active) {
-      const int64_t crow = (row / p.n) * p.tstride + p.t0 + row % p.n;
-      chain_slice(p.comp, p.ncomp, crow, slice, D, z);
+      chain_slice(p.comp, p.ncomp, row / p.n, p.nblk, p.t0 + row % p.n, slice, D, z);
     } else {
 #pragma unroll
       for (int k = 0; k < 32; ++k) z[k] = 0.0f;

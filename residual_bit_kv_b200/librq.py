@@ -13,6 +13,7 @@ import os
 from typing import Optional, Sequence
 
 RQ_MAX_LOOPS = 32
+RQ_BLOCK_TOKENS = 64
 RQ_POLICY_LAST_LOOP = 0
 RQ_POLICY_NEXT_LOOP = 1
 
@@ -50,9 +51,8 @@ class rq_cache(ctypes.Structure):
     _fields_ = [
         ("layout", rq_layout), ("k_base", ctypes.c_void_p), ("v_base", ctypes.c_void_p),
         ("layer_bytes", ctypes.c_uint64), ("token_stride", ctypes.c_int64),
-        ("codes_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
-        ("meta_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
-        ("alpha_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
+        ("comp_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
+        ("rec_bytes", ctypes.c_uint32 * RQ_MAX_LOOPS),
     ]
 
 

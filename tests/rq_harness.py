@@ -84,27 +84,28 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
 
 
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int) -> Dict[str, np.ndarray]:
-    """Packed arrays of one component as numpy [B, H, tstride, ...] views."""
+    """Packed arrays of one component, unblocked from the 64-token records into
+    numpy [B, H, token_stride, ...] arrays."""
     c = gc.cache
     w = gc.w
     buf = gc.kbuf if side == synth.SIDE_K else gc.vbuf
-    base = layer * c.layer_bytes
     ts = c.token_stride
-    rows = w.batch * w.heads * ts
+    blk = L.RQ_BLOCK_TOKENS
+    nrec = w.batch * w.heads * (ts // blk)
+    rb = c.rec_bytes[loop]
     D = w.head_dim
     W = D * w.bits[loop] // 32
     G = D // w.group[loop]
-
-    def grab(off, n_bytes):
-        return buf[base + off: base + off + n_bytes].cpu().numpy()
-
-    out = {
-        "codes": grab(c.codes_off[loop], rows * W * 4).view(np.uint32).reshape(w.batch, w.heads, ts, W),
-        "meta": grab(c.meta_off[loop], rows * G * 4).view(np.uint32).reshape(w.batch, w.heads, ts, G),
-        "alpha": None,
-    }
+    base = layer * c.layer_bytes + c.comp_off[loop]
+    recs = buf[base: base + nrec * rb].cpu().numpy().reshape(nrec, rb)
+    codes = recs[:, : blk * W * 4].copy().view(np.uint32).reshape(w.batch, w.heads, ts, W)
+    meta = recs[:, blk * W * 4: blk * (W + G) * 4].copy().view(np.uint32).reshape(
+        w.batch, w.heads, ts, G)
+    out = {"codes": codes, "meta": meta, "alpha": None}
     if loop != w.loops - 1:
-        out["alpha"] = grab(c.alpha_off[loop], rows * 2).view(np.uint16).reshape(w.batch, w.heads, ts)
+        a0 = blk * (W + G) * 4
+        out["alpha"] = recs[:, a0: a0 + blk * 2].copy().view(np.uint16).reshape(
+            w.batch, w.heads, ts)
     return out
 
 
