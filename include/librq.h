@@ -221,6 +221,32 @@ rq_status rq_workspace_error(void* workspace, uint64_t ws_bytes, void* stream);
  * the current device (for tests and benchmarks). */
 int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);
 
+/* rq_decode_attention for callers that cannot allocate device memory -- code
+ * embedded in a host framework that owns every allocation, or a serving loop
+ * that may not call cudaMalloc -- and so cannot provide a workspace.  The
+ * paper has no counterpart; this is an interface convenience.
+ *   Arguments, layouts and results are those of rq_decode_attention, minus
+ *   the workspace.  The split-K scratch is a fixed 8 MiB array inside this
+ *   library that every GPU which loads the library holds until exit.  The
+ *   call allocates nothing (no cudaMalloc / cudaFree).
+ *   The first call on a device looks up that array's address and zeroes it
+ *   (synchronously, with that device current): make that first call before
+ *   any CUDA-graph stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents; calls that overlap on the GPU (other streams, other host
+ *   threads) race on it and must be ordered by the caller.
+ *   If the split partials of a shape do not fit, fewer splits are used; if
+ *   one split per (batch, head) does not fit (batch * kv_heads * (head_dim+2)
+ *   * 4 bytes above ~8 MiB) the call returns RQ_ERR_WORKSPACE without
+ *   launching.  Device-side conditions (a seq_lens entry out of range is
+ *   clamped, as in rq_decode_attention) are not reported by this entry point. */
+rq_status rq_decode_attention_noalloc(const rq_cache* cache, int32_t layer,
+                                      int32_t loop, const void* q,
+                                      const int32_t* seq_lens,
+                                      int32_t max_seq_len, const void* k_cur,
+                                      const void* v_cur, float softmax_scale,
+                                      float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

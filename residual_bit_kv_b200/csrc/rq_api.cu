@@ -467,3 +467,11 @@ rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads, int32_t head_di
 }
 
 }  // extern "C"
+
+namespace rq {
+rq_status plan_decode(const rq_cache* c, int32_t layer, int32_t loop, int32_t max_seq_len,
+                      DecodeParams* p, int* D) {
+  return fill_decode_params(c, layer, loop, max_seq_len, p, D);
+}
+float decode_scale_log2(float softmax_scale, int D) { return scale_log2_of(softmax_scale, D); }
+}  // namespace rq

@@ -153,6 +153,12 @@ size_t decode_dyn_smem(int D, int stages, uint32_t stage_bytes);
 // resident CTAs per SM of the generic decode kernel at this dynamic shared memory
 cudaError_t decode_occupancy(int D, size_t dyn_smem, int* ctas_per_sm);
 
+// Host planning of a compressed decode call (pointers into the workspace are
+// left for the caller to set): component chain, kernel choice, stages, splits.
+rq_status plan_decode(const rq_cache* c, int32_t layer, int32_t loop, int32_t max_seq_len,
+                      DecodeParams* p, int* D);
+float decode_scale_log2(float softmax_scale, int D);
+
 // ---------------------------------------------------------------------------
 // Device helpers
 // ---------------------------------------------------------------------------

@@ -33,7 +33,7 @@ SYMBOLS = (
     "rq_layer_bytes", "rq_cache_bind", "rq_quantize_anchor", "rq_quantize_append_residual",
     "rq_dequantize", "rq_decode_workspace_bytes", "rq_decode_workspace_init",
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
-    "rq_workspace_error", "rq_decode_splits",
+    "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
 )
 
 
@@ -100,6 +100,8 @@ def load() -> ctypes.CDLL:
                                       _P, _P, _U64, _P], ctypes.c_int),
         "rq_workspace_error": ([_P, _U64, _P], ctypes.c_int),
         "rq_decode_splits": ([LP, _I32], _I32),
+        "rq_decode_attention_noalloc": ([CP, _I32, _I32, _P, _P, _I32, _P, _P, _F, _P, _P],
+                                        ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -230,3 +232,14 @@ def rq_workspace_error(workspace, ws_bytes: int, stream=None) -> int:
 
 def rq_decode_splits(layout: rq_layout, max_seq_len: int) -> int:
     return int(load().rq_decode_splits(ctypes.byref(layout), max_seq_len))
+
+
+def rq_decode_attention_noalloc(cache: rq_cache, layer: int, loop: int, q, seq_lens,
+                                max_seq_len: int, k_cur, v_cur, softmax_scale: float, out,
+                                stream=None) -> None:
+    """rq_decode_attention without a workspace, for callers that cannot
+    allocate device memory; see include/librq.h."""
+    _check(load().rq_decode_attention_noalloc(ctypes.byref(cache), layer, loop, _ptr(q),
+                                              _ptr(seq_lens), max_seq_len, _ptr(k_cur),
+                                              _ptr(v_cur), softmax_scale, _ptr(out),
+                                              _stream(stream)), "rq_decode_attention_noalloc")
