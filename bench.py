@@ -131,9 +131,21 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def profile_traffic(kernel_file: str, profile_name: str):
+DECODE_SOURCES = ("rq_decode_fast.cu", "rq_decode_common.cuh", "rq_internal.cuh")
+
+
+def sources_sha(files) -> str:
+    """sha256 over the kernel's source files (in the given order)."""
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "residual_bit_kv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profile_traffic(files, profile_name: str):
     """Per-launch DRAM traffic from a committed ncu summary, if it was taken on
-    the kernel source as it stands (else None)."""
+    the kernel sources as they stand (else None)."""
     path = os.path.join(ROOT, "profiles", profile_name)
     try:
         txt = open(path).read()
@@ -143,7 +155,7 @@ def profile_traffic(kernel_file: str, profile_name: str):
     m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     if not m_sha or not m_tr:
         return None
-    if m_sha.group(1) != file_sha(os.path.join(ROOT, "residual_bit_kv_b200", "csrc", kernel_file)):
+    if m_sha.group(1) != sources_sha(files):
         return None
     return float(m_tr.group(1))
 
@@ -462,7 +474,7 @@ def main():
                             "gbs": decode_call_bytes(w, l, w.tokens) / (t_l * 1e-3) / 1e9}
     hbm, hbm_kind = peaks()
     n_launch_dec = args.steps * w.layers * w.loops
-    traffic = profile_traffic("rq_decode.cu", "decode_kernel_ouro_16k.md")
+    traffic = profile_traffic(DECODE_SOURCES, "decode_kernel_ouro_16k.md")
 
     # ---- end to end: host buffers, H2D of the step's inputs, D2H of the outputs
     pin = {k: v.cpu().pin_memory() for k, v in eng.q.items()}
@@ -520,7 +532,7 @@ def main():
             "config": config_of(w),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
-                         "kernel": "decode_kernel<128>", "peak_kind": hbm_kind,
+                         "kernel": "decode_fast_kernel (all loops of the step)", "peak_kind": hbm_kind,
                          "bytes_per_step": dec_bytes / args.steps},
             "decode_per_loop": per_loop,
             "decode_splits_loop0": eng.L.rq_decode_splits(eng.lay, w.tokens),
