@@ -424,6 +424,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per step (default 16); smaller values give a profiling-sized case")
     ap.add_argument("--no-quant", action="store_true", help="skip the prefill quantise leg")
+    ap.add_argument("--no-ablation", action="store_true",
+                    help="skip the shared-vs-chained deep-recurrence decode ablation")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -514,9 +516,16 @@ def main():
                 "note": "same split-K engine on uncompressed bf16 K/V; 4 distinct layer buffers"}
 
     # ---- prefill-sized quantise (anchor + 3 residuals, K and V), separate workload
+    splits0 = eng.L.rq_decode_splits(eng.lay, w.tokens)
+    launches = args.steps * eng.launches_per_step()
     quant = None
     if not args.no_quant:
         quant = bench_quantize(dev, stream, args, hbm)
+    ablation = None
+    if not args.no_ablation:
+        del eng
+        torch.cuda.empty_cache()
+        ablation = bench_ablation(dev, stream, args, hbm)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -535,14 +544,15 @@ def main():
                          "kernel": "decode_fast_kernel (all loops of the step)", "peak_kind": hbm_kind,
                          "bytes_per_step": dec_bytes / args.steps},
             "decode_per_loop": per_loop,
-            "decode_splits_loop0": eng.L.rq_decode_splits(eng.lay, w.tokens),
+            "decode_splits_loop0": splits0,
             "decode_hbm_frac_of_8tbs": achieved / 8000.0,
             "e2e": {"value": ws * w.batch * 1e3 / e2e_ms, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * eng.launches_per_step(),
+            "gpu_launches": launches,
             "clocks": clocks,
             "bf16_baseline": bf16,
             "quantize": quant,
+            "ablation_shared_vs_chained": ablation,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -550,6 +560,60 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def bench_ablation(dev, stream, args, hbm):
+    """Deep-recurrence workload (8 loops, batch 32, 40 heads, 8192 tokens, g 64),
+    one layer: decode of all 8 loops under the shared final-loop anchor and under
+    the chained Next-loop reference (loop r reads the anchor and every residual
+    r..6), to measure the read-traffic gap [RQ §3.2, §5.2, App. D]."""
+    import residual_bit_kv_b200.librq as L
+    w = synth.WORKLOADS["huginn_deep"]
+    T = w.tokens
+    out = {"workload": f"{w.name}: 1 layer x {w.loops} loops, batch {w.batch}, {w.heads} heads, "
+                       f"{T} past tokens, bits {list(w.bits)}, group {w.group[0]}"}
+    for policy, name in ((L.RQ_POLICY_LAST_LOOP, "shared"), (L.RQ_POLICY_NEXT_LOOP, "chained")):
+        lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T + 16, w.bits, w.group,
+                            policy)
+        nb = L.rq_cache_bytes(lay)
+        kb = torch.empty(nb, dtype=torch.uint8, device=dev)
+        vb = torch.empty(nb, dtype=torch.uint8, device=dev)
+        cache = L.rq_cache_bind(lay, kb, vb)
+        for side in (0, 1):
+            for loop in [w.loops - 1] + list(range(w.loops - 2, -1, -1)):
+                x = synth.kv_full(w, 0, side, loop, 0, T, device=dev, chunk_b=2)
+                if loop == w.loops - 1:
+                    L.rq_quantize_anchor(cache, 0, side, x, 0, T, stream)
+                else:
+                    L.rq_quantize_append_residual(cache, 0, side, loop, x, 0, T, stream)
+                del x
+        q = [synth.query(w, 0, l, dev).contiguous() for l in range(w.loops)]
+        kc = [synth.current_token(w, 0, 0, l, dev).contiguous() for l in range(w.loops)]
+        vc = [synth.current_token(w, 0, 1, l, dev).contiguous() for l in range(w.loops)]
+        seq = torch.full((w.batch,), T, dtype=torch.int32, device=dev)
+        o = torch.empty(w.batch, w.heads, w.head_dim, dtype=torch.float32, device=dev)
+        wsb = L.rq_decode_workspace_bytes(lay, T)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        L.rq_decode_workspace_init(ws, wsb, stream)
+
+        def step():
+            for loop in range(w.loops):
+                L.rq_decode_attention(cache, 0, loop, q[loop], seq, T, kc[loop], vc[loop], 0.0, o,
+                                      ws, wsb, stream)
+
+        ms = timed(step, args.steps, args.warmup, stream)
+        pol = "last" if policy == L.RQ_POLICY_LAST_LOOP else "next"
+        byt = sum(decode_call_bytes(w, l, T, pol) for l in range(w.loops))
+        out[name] = {"ms_per_step": ms, "bytes_per_step": byt,
+                     "gbs": byt / (ms * 1e-3) / 1e9, "frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
+                     "component_reads": w.loops * 2 - 1 if name == "shared"
+                     else w.loops * (w.loops + 1) // 2}
+        del kb, vb, ws
+        torch.cuda.empty_cache()
+    out["speedup_shared_over_chained"] = out["chained"]["ms_per_step"] / out["shared"]["ms_per_step"]
+    out["bytes_ratio_chained_over_shared"] = (out["chained"]["bytes_per_step"] /
+                                              out["shared"]["bytes_per_step"])
+    return out
 
 
 def bench_quantize(dev, stream, args, hbm):

@@ -83,29 +83,35 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
     return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs)
 
 
-def gpu_component(gc: GpuCache, layer: int, side: int, loop: int) -> Dict[str, np.ndarray]:
+def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
+                  bsel: Optional[Sequence[int]] = None,
+                  hsel: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
     """Packed arrays of one component, unblocked from the 64-token records into
-    numpy [B, H, token_stride, ...] arrays."""
+    numpy [B, H, token_stride, ...] arrays (or [len(bsel), len(hsel), ...] for
+    a selection, copying only those rows off the device)."""
     c = gc.cache
     w = gc.w
     buf = gc.kbuf if side == synth.SIDE_K else gc.vbuf
     ts = c.token_stride
     blk = L.RQ_BLOCK_TOKENS
-    nrec = w.batch * w.heads * (ts // blk)
+    nb = ts // blk
     rb = c.rec_bytes[loop]
     D = w.head_dim
     W = D * w.bits[loop] // 32
     G = D // w.group[loop]
     base = layer * c.layer_bytes + c.comp_off[loop]
-    recs = buf[base: base + nrec * rb].cpu().numpy().reshape(nrec, rb)
-    codes = recs[:, : blk * W * 4].copy().view(np.uint32).reshape(w.batch, w.heads, ts, W)
-    meta = recs[:, blk * W * 4: blk * (W + G) * 4].copy().view(np.uint32).reshape(
-        w.batch, w.heads, ts, G)
+    bsel = list(range(w.batch)) if bsel is None else list(bsel)
+    hsel = list(range(w.heads)) if hsel is None else list(hsel)
+    rows = [b * w.heads + h for b in bsel for h in hsel]
+    allrec = buf[base: base + w.batch * w.heads * nb * rb].view(w.batch * w.heads, nb * rb)
+    recs = allrec[rows].cpu().numpy().reshape(len(rows) * nb, rb)
+    shp = (len(bsel), len(hsel), ts)
+    codes = recs[:, : blk * W * 4].copy().view(np.uint32).reshape(*shp, W)
+    meta = recs[:, blk * W * 4: blk * (W + G) * 4].copy().view(np.uint32).reshape(*shp, G)
     out = {"codes": codes, "meta": meta, "alpha": None}
     if loop != w.loops - 1:
         a0 = blk * (W + G) * 4
-        out["alpha"] = recs[:, a0: a0 + blk * 2].copy().view(np.uint16).reshape(
-            w.batch, w.heads, ts)
+        out["alpha"] = recs[:, a0: a0 + blk * 2].copy().view(np.uint16).reshape(*shp)
     return out
 
 

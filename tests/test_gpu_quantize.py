@@ -24,8 +24,8 @@ def _check_all(gc, layer=0, tokens=None, bsel=None, hsel=None, from_gpu_inputs=T
                   for l in range(w.loops)]
         encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, gc.policy, xl)
         for loop in range(w.loops):
-            g = gpu_component(gc, layer, side, loop)
-            gsel = {k: (None if v is None else v[np.ix_(bsel, hsel)][:, :, :T]) for k, v in g.items()}
+            g = gpu_component(gc, layer, side, loop, bsel, hsel)
+            gsel = {k: (None if v is None else v[:, :, :T]) for k, v in g.items()}
             assert_component_equal(gsel, encs[loop], None, f"side {side} loop {loop}")
 
 
