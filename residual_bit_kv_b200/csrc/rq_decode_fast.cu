@@ -40,7 +40,6 @@ constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, u
 template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
 struct Spec {
   static constexpr int D = D_, NC = NC_, TC = kCChunk;
-  static constexpr int RB = RB_, AB = AB_;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
@@ -180,17 +179,17 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
   }
 }
 
-// Value path.  Two codes of one 32-bit word are OR-ed into the mantissas of
-// two f16 halves of 1024 (0x6400): half value 1024 + c * 2^p, exact for
-// p + bits <= 10.  Each half is multiplied by an f16 weight
+// Value path.  Two codes of one 32-bit word are masked into the two 16-bit
+// halves of a register with the exponent field left at zero: each half is the
+// f16 subnormal c * 2^(p-24), exact, for a code at bits [p, p+bits) of the half
+// (p + bits <= 10).  Each half is multiplied by an f16 weight
 // w_p = f16(p_t * kappa * s~ * 2^(kWeightExp - p)) with an fp32 accumulator
-// (fma.rn.f32.f16: the f16 x f16 product is exact in fp32).  The 1024 * w_p
-// part is removed at the end from the exact running sum of the p = 0 weights
-// per component type and 16-channel half: w_p = w_0 * 2^-p exactly while the
-// weights stay in the f16 normal range.
+// (fma.rn.f32.f16: the product of two f16 values is exact in fp32), so every
+// channel accumulates p_t * kappa * s~ * c * 2^(kWeightExp - 24).
 constexpr int kWeightExp = 8;
 constexpr float kWeightScale = static_cast<float>(1 << kWeightExp);
 constexpr float kWeightMax = 65504.0f;          // largest finite f16
+constexpr float kValueUnscale = static_cast<float>(1 << (24 - kWeightExp));
 
 __device__ __forceinline__ float fma_h(uint32_t a, uint32_t b, float c) {
   float d;
@@ -204,20 +203,12 @@ __device__ __forceinline__ uint32_t f16_bits(float x) {
   return __half_as_ushort(__float2half_rn(x));
 }
 
-// Half-word position (bits) of the channel paired at 16-channel-block offset v
-// in the value path: 2-bit codes at 2*(v%4) (word or word >> 8), 4-bit codes
-// at 4*(v&1) (word or word >> 8).
-template <int BITS>
-__host__ __device__ constexpr int vpos(int v) {
-  return BITS == 2 ? 2 * (v % 4) : 4 * (v & 1);
-}
-
-// acc += w * D(c) over one lane's 32 channels of token j.  pk = p_t * kappa;
-// TYPE selects the weight-sum slot (0: residual layout, 1: anchor layout).
-template <int D, int BITS, int G, int TYPE>
+// acc += w * D(c) over one lane's 32 channels of token j (codes part; the z~
+// offsets go to cst per 16-channel half).  pk = p_t * kappa.
+template <int D, int BITS, int G>
 __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned char* meta, int j,
                                      int slice, float pk, float (&acc)[32], float (&cst)[2],
-                                     float (&wsum)[2][2], uint32_t& range_err) {
+                                     uint32_t& range_err) {
   constexpr int WPR = D * BITS / 32, GPR = D / G;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + j * WPR + slice * BITS;
   const uint32_t* mr = reinterpret_cast<const uint32_t*>(meta) + j * GPR;
@@ -231,17 +222,13 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
     unpack_meta(mw.x, sc[0], zc[0]);
     unpack_meta(mw.y, sc[1], zc[1]);
   }
-  constexpr int NPOS = BITS == 2 ? 4 : 2;   // positions 0,2,4,6 or 0,4
+  constexpr int NPOS = BITS == 2 ? 4 : 2;   // code positions 0,2,4,6 or 0,4
+  constexpr int NW = G >= 32 ? 1 : 2;       // distinct weights per lane
   uint32_t wt[2][NPOS];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     cst[h] = fmaf(pk, zc[h], cst[h]);
-    if (G >= 32 && h == 1) {
-#pragma unroll
-      for (int q = 0; q < NPOS; ++q) wt[1][q] = wt[0][q];
-      wsum[TYPE][1] = fma_h(wt[1][0], 0x3C00u, wsum[TYPE][1]);
-      continue;
-    }
+    if (h >= NW) continue;
     float w = pk * sc[h] * kWeightScale;
     if (!(w <= kWeightMax)) {   // outside the f16 range of the weights
       range_err = 1u;
@@ -250,7 +237,6 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
 #pragma unroll
     for (int q = 0; q < NPOS; ++q)
       wt[h][q] = f16_bits(w * (1.0f / static_cast<float>(1u << (q * (BITS == 2 ? 2 : 4)))));
-    wsum[TYPE][h] = fma_h(wt[h][0], 0x3C00u, wsum[TYPE][h]);   // + exact f16 value
   }
   if constexpr (BITS == 4) {
     // word 2k + hh, nibble n: channel 16k + 4(n>>1) + 2hh + (n&1); nibbles n
@@ -264,10 +250,9 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
         const uint32_t src = n < 2 ? w[k4] : w8;
-        const uint32_t mask = (n & 1) ? 0x00F000F0u : 0x000F000Fu;
-        const uint32_t x = (src & mask) | 0x64006400u;
+        const uint32_t x = src & ((n & 1) ? 0x00F000F0u : 0x000F000Fu);
         const int ch = 16 * k + 4 * (n >> 1) + 2 * hh + (n & 1);
-        const uint32_t wq = wt[G >= 32 ? 0 : k][n & 1];
+        const uint32_t wq = wt[NW == 1 ? 0 : k][n & 1];
         acc[ch] = fma_h(x & 0xFFFFu, wq, acc[ch]);
         acc[ch + 8] = fma_h(x >> 16, wq, acc[ch + 8]);
       }
@@ -284,9 +269,8 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
       for (int f = 0; f < 8; ++f) {
         const int q = f & 3;
         const uint32_t src = f < 4 ? w[k] : w8;
-        const uint32_t mask = (3u << (2 * q)) | (3u << (16 + 2 * q));
-        const uint32_t x = (src & mask) | 0x64006400u;
-        const uint32_t wq = wt[G >= 32 ? 0 : k][q];
+        const uint32_t x = src & ((3u << (2 * q)) | (3u << (16 + 2 * q)));
+        const uint32_t wq = wt[NW == 1 ? 0 : k][q];
         acc[16 * k + f] = fma_h(x & 0xFFFFu, wq, acc[16 * k + f]);
         acc[16 * k + 8 + f] = fma_h(x >> 16, wq, acc[16 * k + 8 + f]);
       }
@@ -311,30 +295,21 @@ __device__ __forceinline__ void score_comps(const unsigned char* st, int j, int 
 template <class SP, int C = 0>
 __device__ __forceinline__ void value_comps(const unsigned char* st, int j, int slice, float kap,
                                             float (&acc)[32], float (&cst)[2],
-                                            float (&wsum)[2][2], uint32_t& range_err) {
+                                            uint32_t& range_err) {
   if constexpr (C < SP::NC) {
-    vacc<SP::D, SP::bits(C), SP::group(C), (C == SP::NC - 1) ? 1 : 0>(
-        st + SP::codes_off(1, C), st + SP::meta_off(1, C), j, slice, kap, acc, cst, wsum,
-        range_err);
+    vacc<SP::D, SP::bits(C), SP::group(C)>(st + SP::codes_off(1, C), st + SP::meta_off(1, C), j,
+                                           slice, kap, acc, cst, range_err);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(st + SP::alpha_off(1, C))[j]);
-    value_comps<SP, C + 1>(st, j, slice, kap, acc, cst, wsum, range_err);
+    value_comps<SP, C + 1>(st, j, slice, kap, acc, cst, range_err);
   }
 }
 
-// Final value of the accumulators: remove the 1024 * w_p offsets of each
-// component type (residual layout RB, anchor layout AB) and the weight scale,
-// add the z~ terms.
-template <int RB, int AB, bool HAS_R>
-__device__ __forceinline__ void finish_values(float (&acc)[32], const float (&cst)[2],
-                                              const float (&wsum)[2][2]) {
+// Final value of the accumulators: undo the weight and subnormal scales and
+// add the z~ terms of each 16-channel half.
+__device__ __forceinline__ void finish_values(float (&acc)[32], const float (&cst)[2]) {
 #pragma unroll
-  for (int ch = 0; ch < 32; ++ch) {
-    const int v = ch % 16, h = ch / 16;
-    float off = 1024.0f * wsum[1][h] / static_cast<float>(1u << vpos<AB>(v));
-    if (HAS_R) off += 1024.0f * wsum[0][h] / static_cast<float>(1u << vpos<RB>(v));
-    acc[ch] = (acc[ch] - off) * (1.0f / kWeightScale) + cst[h];
-  }
+  for (int ch = 0; ch < 32; ++ch) acc[ch] = fmaf(acc[ch], kValueUnscale, cst[ch / 16]);
 }
 
 // Token range of this CTA's split.
@@ -471,7 +446,6 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
 #pragma unroll
   for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
   float cst[2] = {0.0f, 0.0f};
-  float wsum[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
   uint32_t range_err = 0u;
   float m = kNegInf, l = 0.0f;
 
@@ -499,10 +473,6 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       l *= f;
       cst[0] *= f;
       cst[1] *= f;
-      wsum[0][0] *= f;
-      wsum[0][1] *= f;
-      wsum[1][0] *= f;
-      wsum[1][1] *= f;
 #pragma unroll
       for (int k = 0; k < 32; ++k) acc[k] *= f;
       m = mc;
@@ -513,7 +483,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       if (sc[tt] == kNegInf) continue;
       const float pt = fast_exp2(sc[tt] - m);
       l += pt;
-      value_comps<SP>(st, j, slice, pt, acc, cst, wsum, range_err);
+      value_comps<SP>(st, j, slice, pt, acc, cst, range_err);
     }
     // Release the stage; the last warp to do so refills it.
     __syncwarp();
@@ -527,7 +497,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       }
     }
   }
-  finish_values<SP::RB, SP::AB, (SP::NC > 1)>(acc, cst, wsum);
+  finish_values(acc, cst);
   if (range_err) atomicOr(p.err, kErrRange);
   if (s_abort) {
     m = kNegInf;
