@@ -179,28 +179,17 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
   }
 }
 
-// Value path.  Two codes of one 32-bit word are masked into the two 16-bit
-// halves of a register with the exponent field left at zero: each half is the
-// f16 subnormal c * 2^(p-24), exact, for a code at bits [p, p+bits) of the half
-// (p + bits <= 10).  Each half is multiplied by an f16 weight
-// w_p = f16(p_t * kappa * s~ * 2^(kWeightExp - p)) with an fp32 accumulator
-// (fma.rn.f32.f16: the product of two f16 values is exact in fp32), so every
-// channel accumulates p_t * kappa * s~ * c * 2^(kWeightExp - 24).
-constexpr int kWeightExp = 8;
-constexpr float kWeightScale = static_cast<float>(1 << kWeightExp);
-constexpr float kWeightMax = 65504.0f;          // largest finite f16
-constexpr float kValueUnscale = static_cast<float>(1 << (24 - kWeightExp));
+// Value path.  A code masked out of its word with the rest of the register
+// (and so the exponent field) zero is the exact fp32 subnormal c * 2^(p-149),
+// p its bit position (p + bits <= 23).  One FFMA with the fp32 weight
+// w_p = p_t * kappa * s~ * 2^(kPosBias - p) adds p_t * kappa * s~ * c * 2^-40
+// to the channel's accumulator: one mask and one FMA per code, fp32 weights.
+constexpr int kPosBias = 109;                        // 2^(109 - p) <= 2^109 stays finite
+constexpr float kValueUnscale = 1099511627776.0f;    // 2^(149 - kPosBias) = 2^40
+constexpr float kWeightMax = 262144.0f;              // 2^18: weights above this are flagged
 
-__device__ __forceinline__ float fma_h(uint32_t a, uint32_t b, float c) {
-  float d;
-  asm("fma.rn.f32.f16 %0, %1, %2, %3;"
-      : "=f"(d)
-      : "h"(static_cast<unsigned short>(a)), "h"(static_cast<unsigned short>(b)), "f"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t f16_bits(float x) {
-  return __half_as_ushort(__float2half_rn(x));
+__device__ __forceinline__ float pow2_bias(int pos) {
+  return __uint_as_float(static_cast<uint32_t>(127 + kPosBias - pos) << 23);
 }
 
 // acc += w * D(c) over one lane's 32 channels of token j (codes part; the z~
@@ -222,57 +211,53 @@ __device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned 
     unpack_meta(mw.x, sc[0], zc[0]);
     unpack_meta(mw.y, sc[1], zc[1]);
   }
-  constexpr int NPOS = BITS == 2 ? 4 : 2;   // code positions 0,2,4,6 or 0,4
+  constexpr int NPOS = BITS == 2 ? 8 : 4;   // positions 0,2,..,14 or 0,4,8,12 (after >>16)
   constexpr int NW = G >= 32 ? 1 : 2;       // distinct weights per lane
-  uint32_t wt[2][NPOS];
+  float ws[2][NPOS];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     cst[h] = fmaf(pk, zc[h], cst[h]);
     if (h >= NW) continue;
-    float w = pk * sc[h] * kWeightScale;
-    if (!(w <= kWeightMax)) {   // outside the f16 range of the weights
+    float w = pk * sc[h];
+    if (!(fabsf(w) <= kWeightMax)) {
       range_err = 1u;
       w = 0.0f;
     }
 #pragma unroll
-    for (int q = 0; q < NPOS; ++q)
-      wt[h][q] = f16_bits(w * (1.0f / static_cast<float>(1u << (q * (BITS == 2 ? 2 : 4)))));
+    for (int q = 0; q < NPOS; ++q) ws[h][q] = w * pow2_bias(q * BITS);
   }
   if constexpr (BITS == 4) {
-    // word 2k + hh, nibble n: channel 16k + 4(n>>1) + 2hh + (n&1); nibbles n
-    // and n+4 share a half-word position, 0 or 4 in (word) / (word >> 8).
+    // word 2k + hh, nibble n: channel 16k + 4(n>>1) + 2hh + (n&1); nibbles
+    // 4..7 are read from word >> 16 at the positions of nibbles 0..3.
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
       const int k = k4 >> 1, hh = k4 & 1;
-      const uint32_t w8 = w[k4] >> 8;
+      const uint32_t w16 = w[k4] >> 16;
+      const float* wq = ws[NW == 1 ? 0 : k];
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
-        const uint32_t src = n < 2 ? w[k4] : w8;
-        const uint32_t x = src & ((n & 1) ? 0x00F000F0u : 0x000F000Fu);
+        const uint32_t m = 0xFu << (4 * n);
         const int ch = 16 * k + 4 * (n >> 1) + 2 * hh + (n & 1);
-        const uint32_t wq = wt[NW == 1 ? 0 : k][n & 1];
-        acc[ch] = fma_h(x & 0xFFFFu, wq, acc[ch]);
-        acc[ch + 8] = fma_h(x >> 16, wq, acc[ch + 8]);
+        acc[ch] = fmaf(wq[n], __uint_as_float(w[k4] & m), acc[ch]);
+        acc[ch + 8] = fmaf(wq[n], __uint_as_float(w16 & m), acc[ch + 8]);
       }
     }
   } else {
-    // word k, 2-bit field f (f < 8 in the low half, f + 8 in the high half):
-    // fields 0..3 at bits 2f of the word, fields 4..7 at bits 2(f-4) of word >> 8.
+    // word k: field f (channel 16k + f) at bits 2f; fields 8..15 are read from
+    // word >> 16 at the positions of fields 0..7.
     const uint2 v = *reinterpret_cast<const uint2*>(cw);
     const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const uint32_t w8 = w[k] >> 8;
+      const uint32_t w16 = w[k] >> 16;
+      const float* wq = ws[NW == 1 ? 0 : k];
 #pragma unroll
       for (int f = 0; f < 8; ++f) {
-        const int q = f & 3;
-        const uint32_t src = f < 4 ? w[k] : w8;
-        const uint32_t x = src & ((3u << (2 * q)) | (3u << (16 + 2 * q)));
-        const uint32_t wq = wt[NW == 1 ? 0 : k][q];
-        acc[16 * k + f] = fma_h(x & 0xFFFFu, wq, acc[16 * k + f]);
-        acc[16 * k + 8 + f] = fma_h(x >> 16, wq, acc[16 * k + 8 + f]);
+        const uint32_t m = 3u << (2 * f);
+        acc[16 * k + f] = fmaf(wq[f], __uint_as_float(w[k] & m), acc[16 * k + f]);
+        acc[16 * k + 8 + f] = fmaf(wq[f], __uint_as_float(w16 & m), acc[16 * k + 8 + f]);
       }
     }
   }
