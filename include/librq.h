@@ -19,16 +19,18 @@
  *   Reconstruction: Z^_r = alpha~_r R + s~ c + z~ and X^_r = H^T Z^_r.
  *
  * Storage contract (per layer and per side K | V):
- *   Tokens are stored in records of RQ_BLOCK_TOKENS = 64 consecutive tokens.
+ *   Tokens are stored in records of RQ_BLOCK_TOKENS = 32 consecutive tokens.
  *   Loop r of (row = batch*kv_heads index b*H + h, block k) is one record at
- *   byte offset comp_off[r] + (row * token_stride/64 + k) * rec_bytes[r] of
- *   the (layer, side) region; token_stride is max_tokens rounded up to 64.
+ *   byte offset comp_off[r] + (row * token_stride/32 + k) * rec_bytes[r] of
+ *   the (layer, side) region; token_stride is max_tokens rounded up to 64
+ *   (an even number of records per row).
  *   A record holds, contiguously:
- *     codes  uint32 [64][head_dim * bits[r] / 32]
- *     meta   uint32 [64][head_dim / group[r]]; low half fp16 scale s~,
+ *     codes  uint32 [32][head_dim * bits[r] / 32]
+ *     meta   uint32 [32][head_dim / group[r]]; low half fp16 scale s~,
  *            high half fp16 offset z~
- *     alpha  bf16   [64]             (residual loops only)
- *   so a 64-token decode stage of one component is one contiguous copy.
+ *     alpha  bf16   [32]             (residual loops only)
+ *   so a decode stage of one component (one or two records) is one
+ *   contiguous copy.
  *   Code order inside a token's row: b = 2: channel i in word i/16, bits
  *   [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v, word
  *   2u + ((v>>1)&1), bits [4*(2*(v>>2) + (v&1)), +4).  Little-endian words.
@@ -61,7 +63,7 @@ extern "C" {
 
 #define RQ_ABI_VERSION 1
 #define RQ_MAX_LOOPS 32
-#define RQ_BLOCK_TOKENS 64
+#define RQ_BLOCK_TOKENS 32
 
 typedef enum rq_status {
   RQ_OK = 0,
@@ -109,7 +111,7 @@ typedef struct rq_cache {
   void* k_base;                      /* num_layers * layer_bytes, K side */
   void* v_base;                      /* num_layers * layer_bytes, V side */
   uint64_t layer_bytes;
-  int64_t token_stride;              /* max_tokens rounded up to RQ_BLOCK_TOKENS */
+  int64_t token_stride;              /* max_tokens rounded up to 64 */
   uint64_t comp_off[RQ_MAX_LOOPS];   /* first record of loop r (256-B aligned) */
   uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 64-token record of loop r */
 } rq_cache;
@@ -213,8 +215,10 @@ rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads,
 
 /* Reads and clears the device-side error word of a decode workspace
  * (synchronises `stream`).  RQ_OK, RQ_ERR_CAPACITY (a seq_lens entry was out
- * of range) or RQ_ERR_TIMEOUT (a bounded wait ran out; re-initialise the
- * workspace). */
+ * of range), RQ_ERR_UNSUPPORTED (a value weight p_t * kappa * s~ reached
+ * 2^19, outside the range of the decode kernel's scaled accumulators; that
+ * call's output is not valid) or RQ_ERR_TIMEOUT (a bounded wait ran out;
+ * re-initialise the workspace). */
 rq_status rq_workspace_error(void* workspace, uint64_t ws_bytes, void* stream);
 
 /* Number of split-K partitions rq_decode_attention uses for this shape on

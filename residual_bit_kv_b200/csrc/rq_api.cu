@@ -27,14 +27,14 @@ inline rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 inline int64_t token_stride_of(const rq_layout* l) {
-  return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), kBlock));
+  return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), kRowTokens));
 }
 
 inline uint32_t record_bytes(const rq_layout* l, int r) {
   const int D = l->head_dim;
   const uint32_t per_token = (D * l->bits[r] / 32) * 4 + (D / l->group[r]) * 4 +
                              (r != l->num_loops - 1 ? 2 : 0);
-  return kBlock * per_token;   // a multiple of 128 bytes
+  return kBlock * per_token;   // a multiple of 64 bytes
 }
 
 // Byte offset of every component's first record inside one (layer, side);
@@ -353,10 +353,10 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
   p->rot_scale = rot_scale_of(l.head_dim);
   *D = l.head_dim;
   int stages = 0, occ = 0, chunk = kChunk;
-  if (fast_decode_plan(*p, *D, kRingBudget, kMaxStages, &stages, &occ)) {
+  if (fast_decode_plan(*p, *D, &stages, &chunk, &occ)) {
     p->use_fast = 1;
-    chunk = fast_chunk();
   } else {
+    chunk = kChunk;
     p->use_fast = 0;
     p->stage_bytes = decode_stage_bytes(*p, *D);
     stages = static_cast<int>(kRingBudget / p->stage_bytes);
@@ -367,6 +367,7 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
       return RQ_ERR_CUDA;
   }
   p->stages = stages;
+  p->chunk = chunk;
   choose_splits(p->bh, max_seq_len, chunk, occ, &p->splits, &p->chunks_per_split);
   return RQ_OK;
 }

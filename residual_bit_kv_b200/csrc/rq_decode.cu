@@ -8,9 +8,10 @@
 //
 // Work decomposition: one CTA (128 threads) per (batch*head, split); a split
 // is a contiguous range of past tokens.  Each CTA streams its range in chunks
-// of kChunk tokens: thread 0 issues one bulk asynchronous copy per packed
-// array (codes, metadata, LS coefficients of every component, K and V) into
-// an S-stage shared-memory ring, completing on a per-stage mbarrier; all
+// of kChunk tokens (two 32-token storage records): thread 0 issues one bulk
+// asynchronous copy per component and side (codes, metadata and LS
+// coefficients of two consecutive records are contiguous) into an S-stage
+// shared-memory ring, completing on a per-stage mbarrier; all
 // threads consume a stage, synchronise, and thread 0 refills it.
 //
 // Compute [RQ §4.1, App. G.2]: q' = H q is formed once per CTA and the
@@ -37,13 +38,18 @@ struct Geom {
   static constexpr int NSLOT = kDecodeThreads / P;
 };
 
-// Per-component shared-memory offsets inside one pipeline stage.
+// Per-component shared-memory layout of one pipeline stage: component c of
+// side `side` occupies kChunk/kBlock consecutive records (one copy) starting
+// at comp[side][c]; inside a record, codes start at 0, metadata at meta[..]
+// and LS coefficients at alpha[..].
 struct StageMap {
-  uint32_t codes[2][RQ_MAX_LOOPS];
+  uint32_t comp[2][RQ_MAX_LOOPS];
   uint32_t meta[2][RQ_MAX_LOOPS];
   uint32_t alpha[2][RQ_MAX_LOOPS];
   uint32_t bytes;
 };
+
+constexpr int kRecsPerStage = kChunk / kBlock;
 
 __host__ __device__ inline void build_stage_map(const DecodeParams& p, int D,
                                                 StageMap& m) {
@@ -51,15 +57,20 @@ __host__ __device__ inline void build_stage_map(const DecodeParams& p, int D,
   for (int side = 0; side < 2; ++side) {
     const Comp* cs = side == 0 ? p.k : p.v;
     for (int c = 0; c < p.ncomp; ++c) {
-      m.codes[side][c] = off;
-      off += kChunk * (D * cs[c].bits / 32) * 4;
-      m.meta[side][c] = off;
-      off += kChunk * (D / cs[c].group) * 4;
-      m.alpha[side][c] = off;
-      if (cs[c].has_alpha) off += kChunk * 2;
+      m.comp[side][c] = off;
+      m.meta[side][c] = kBlock * (D * cs[c].bits / 32) * 4;
+      m.alpha[side][c] = m.meta[side][c] + kBlock * (D / cs[c].group) * 4;
+      off += kRecsPerStage * cs[c].rec_bytes;
     }
   }
   m.bytes = off;
+}
+
+// Start of the record holding stage token j of component c.
+__device__ __forceinline__ const unsigned char* stage_rec(const unsigned char* st,
+                                                          const StageMap& m, const Comp& cp,
+                                                          int side, int c, int j) {
+  return st + m.comp[side][c] + (j / kBlock) * cp.rec_bytes;
 }
 
 // q'.D(c) over this lane's 32 channels of one token of one component:
@@ -167,7 +178,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
   __syncthreads();
 
-  static_assert(kChunk == kBlock, "a decode stage is one storage record per component");
+  // One copy of kRecsPerStage consecutive records per component and side
+  // (stages start at multiples of kChunk tokens, so they never leave the row).
   auto issue = [&](int i) {
     const int s = i % S;
     const int t0 = t_begin + i * kChunk;
@@ -175,14 +187,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
     uint32_t bytes = 0;
     for (int side = 0; side < 2; ++side) {
       const Comp* cs = side == 0 ? p.k : p.v;
-      for (int c = 0; c < p.ncomp; ++c) bytes += cs[c].rec_bytes;
+      for (int c = 0; c < p.ncomp; ++c) bytes += kRecsPerStage * cs[c].rec_bytes;
     }
     mbar_arrive_expect_tx(&full_bar[s], bytes);
     for (int side = 0; side < 2; ++side) {
       const Comp* cs = side == 0 ? p.k : p.v;
       for (int c = 0; c < p.ncomp; ++c)
-        bulk_copy_g2s(st + map.codes[side][c], comp_record(cs[c], bhi, p.nblk, t0),
-                      cs[c].rec_bytes, &full_bar[s]);
+        bulk_copy_g2s(st + map.comp[side][c], comp_record(cs[c], bhi, p.nblk, t0),
+                      kRecsPerStage * cs[c].rec_bytes, &full_bar[s]);
     }
   };
   int issued = 0;
@@ -223,17 +235,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
       const int j = tt * G::TPC + warp * G::TPW + tw;
       float part = 0.0f, kappa = 1.0f;
       for (int c = 0; c < p.ncomp; ++c) {
-        const int bits = p.k[c].bits;
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + map.codes[0][c]) +
-                             j * (D * bits / 32) + slice * bits;
-        const uint32_t* mr = reinterpret_cast<const uint32_t*>(st + map.meta[0][c]) +
-                             j * (D / p.k[c].group);
+        const int bits = p.k[c].bits, jl = j % kBlock;
+        const unsigned char* rec = stage_rec(st, map, p.k[c], 0, c, j);
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * (D * bits / 32) +
+                             slice * bits;
+        const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + map.meta[0][c]) +
+                             jl * (D / p.k[c].group);
         const float d = (bits == 4) ? comp_dot<4>(cw, mr, slice, log2_pow2(p.k[c].group), q, qsa, qsb)
                                     : comp_dot<2>(cw, mr, slice, log2_pow2(p.k[c].group), q, qsa, qsb);
         part = fmaf(kappa, d, part);
         if (c + 1 < p.ncomp)
-          kappa *= bf16_bits_to_f32(
-              reinterpret_cast<const uint16_t*>(st + map.alpha[0][c])[j]);
+          kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[0][c])[jl]);
       }
 #pragma unroll
       for (int off = G::P / 2; off >= 1; off >>= 1)
@@ -262,18 +274,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
       l += pt;
       float kappa = pt;
       for (int c = 0; c < p.ncomp; ++c) {
-        const int bits = p.v[c].bits;
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + map.codes[1][c]) +
-                             j * (D * bits / 32) + slice * bits;
-        const uint32_t* mr = reinterpret_cast<const uint32_t*>(st + map.meta[1][c]) +
-                             j * (D / p.v[c].group);
+        const int bits = p.v[c].bits, jl = j % kBlock;
+        const unsigned char* rec = stage_rec(st, map, p.v[c], 1, c, j);
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * (D * bits / 32) +
+                             slice * bits;
+        const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + map.meta[1][c]) +
+                             jl * (D / p.v[c].group);
         if (bits == 4)
           comp_acc<4>(cw, mr, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
         else
           comp_acc<2>(cw, mr, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
         if (c + 1 < p.ncomp)
-          kappa *= bf16_bits_to_f32(
-              reinterpret_cast<const uint16_t*>(st + map.alpha[1][c])[j]);
+          kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[1][c])[jl]);
       }
     }
     __syncthreads();   // stage s fully consumed

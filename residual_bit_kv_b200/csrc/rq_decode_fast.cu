@@ -1,14 +1,15 @@
-// rq_decode_fast.cu -- warp-specialised split-K decode attention for the
-// packed ResidualQuant cache (compile-time component layouts) and for the
-// uncompressed BF16 baseline.
+// rq_decode_fast.cu -- split-K decode attention for the packed ResidualQuant
+// cache with compile-time component layouts, and for the uncompressed BF16
+// baseline.
 //
 // Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
 // Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
 //
-// CTA = 8 compute warps + 1 producer warp.  The producer streams a split's
-// token range in chunks with bulk asynchronous copies (one per packed array)
-// into an S-stage shared-memory ring: full[s] completes on the copies' byte
-// count, empty[s] when all compute warps are done with the stage.
+// Compressed kernel: a CTA of 4 warps streams one (batch*head, split) token
+// range in stages of two 32-token storage records per component and side
+// (one bulk asynchronous copy each) through an S-stage shared-memory
+// ring.  Every warp consumes every stage; the warp that releases a stage last
+// issues its refill, S stages ahead.
 //
 // Scores [RQ §4.1, App. G.2]: q' = H q (pre-scaled by softmax scale and
 // log2 e) is held as 16-bit fixed point, q' ~= sigma * (256 h + l) with
@@ -16,11 +17,11 @@
 // (dp4a) of the unpacked code bytes with the limbs; the score of a token is
 // sigma * sum_c kappa_c (s~_c * dot_c + z~_c * sum q~), kappa the product of
 // the LS coefficients along the reference chain.
-// Values: codes are turned into exact floats c * 2^p by OR-ing them into the
-// mantissa of 2^23 and subtracting 2^23 (packed fp32 pairs), and accumulated
-// with packed fp32 FMAs against weights p_t * kappa * s~ * 2^-p; the offsets
-// z~ go to one accumulator per 16 channels.  Accumulation is in the rotated
-// domain; H^T is applied once in the merge.
+// Values: a code masked out of its word (all other bits zero) is the exact
+// fp32 subnormal c * 2^(p-149), p its bit position; packed fp32 FMAs with
+// weights p_t * kappa * s~ * 2^(109-p) accumulate p_t * kappa * s~ * c * 2^-40
+// per channel, the offsets z~ going to separate accumulators.  Accumulation
+// is in the rotated domain; H^T is applied once in the merge.
 #include "rq_decode_common.cuh"
 
 namespace rq {
@@ -28,43 +29,56 @@ namespace {
 
 constexpr int kWarps = 8;                      // BF16 kernel: compute warps per CTA
 constexpr int kThreads = (kWarps + 1) * 32;    // + producer warp
-constexpr int kMaxRing = 4;
+constexpr int kMaxRing = 4;                    // BF16 kernel ring
 
 constexpr int kCWarps = 4;                     // compressed kernel: warps per CTA
 constexpr int kCThreads = kCWarps * 32;
-constexpr int kCChunk = 64;                    // tokens per stage
+constexpr int kCMaxRing = 8;                   // compressed kernel ring
 constexpr int kCMinCtas = 5;                   // register target: CTAs per SM
-constexpr size_t kCRingBudget = 40 * 1024;     // stage ring per CTA (several CTAs per SM)
+constexpr size_t kCRingBudget = 43 * 1024;     // stage ring per CTA (5 CTAs per SM)
 constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, up to 1024 splits
 
+// Compile-time layout of one stage: for side K then V, component c occupies
+// RPS = 2 consecutive records (64 tokens, one copy); a record is
+// [codes[32][wpr] | meta[32][gpr] | alpha[32]].
 template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
 struct Spec {
-  static constexpr int D = D_, NC = NC_, TC = kCChunk;
+  static constexpr int D = D_, NC = NC_, RPS = 2, TC = kBlock * RPS;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
   __host__ __device__ static constexpr int wpr(int c) { return D_ * bits(c) / 32; }
   __host__ __device__ static constexpr int gpr(int c) { return D_ / group(c); }
-  __host__ __device__ static constexpr uint32_t comp_bytes(int c) {
-    return TC * (wpr(c) * 4 + gpr(c) * 4 + (has_alpha(c) ? 2 : 0));
+  __host__ __device__ static constexpr uint32_t rec_bytes(int c) {
+    return kBlock * (wpr(c) * 4 + gpr(c) * 4 + (has_alpha(c) ? 2 : 0));
   }
+  __host__ __device__ static constexpr uint32_t comp_bytes(int c) { return RPS * rec_bytes(c); }
   __host__ __device__ static constexpr uint32_t side_bytes() {
     uint32_t s = 0;
     for (int c = 0; c < NC_; ++c) s += comp_bytes(c);
     return s;
   }
   __host__ __device__ static constexpr uint32_t stage_bytes() { return 2 * side_bytes(); }
-  __host__ __device__ static constexpr uint32_t codes_off(int side, int c) {
+  __host__ __device__ static constexpr uint32_t comp_off(int side, int c) {
     uint32_t o = side * side_bytes();
     for (int k = 0; k < c; ++k) o += comp_bytes(k);
     return o;
   }
-  __host__ __device__ static constexpr uint32_t meta_off(int side, int c) {
-    return codes_off(side, c) + TC * wpr(c) * 4;
+  // Record of component c (side) holding stage token j.
+  __device__ static const unsigned char* rec(const unsigned char* st, int side, int c, int j) {
+    return st + comp_off(side, c) + (RPS == 1 ? 0 : (j / kBlock) * rec_bytes(c));
   }
-  __host__ __device__ static constexpr uint32_t alpha_off(int side, int c) {
-    return meta_off(side, c) + TC * gpr(c) * 4;
-  }
+};
+
+// Offsets inside a record of a component with these parameters.
+template <int D, int BITS, int G>
+struct RecGeom {
+  enum : uint32_t {
+    WPR = D * BITS / 32,
+    GPR = D / G,
+    META = kBlock * WPR * 4,
+    ALPHA = META + kBlock * GPR * 4,
+  };
 };
 
 // Fixed-point rotated query of one lane's 32 channels as int8 limb bytes in
@@ -130,13 +144,13 @@ __device__ __forceinline__ void build_limbs(const float* qrow, float inv_sigma, 
     }
 }
 
-// q~ . D(c) over one lane's 32 channels of token j of a component, in sigma
-// units: sum over group parts of s~ * (q~ . codes) + z~ * (sum q~).
+// q~ . D(c) over one lane's 32 channels of record token jl of a component,
+// in sigma units: sum over group parts of s~ * (q~ . codes) + z~ * (sum q~).
 template <int D, int BITS, int G>
-__device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned char* meta, int j,
-                                      int slice, const QLimbs& ql) {
-  constexpr int WPR = D * BITS / 32, GPR = D / G;
-  const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + j * WPR + slice * BITS;
+__device__ __forceinline__ float kdot(const unsigned char* rec, int jl, int slice,
+                                      const QLimbs& ql) {
+  using RG = RecGeom<D, BITS, G>;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * RG::WPR + slice * BITS;
   int ah[2] = {0, 0}, al[2] = {0, 0};   // per 16-channel block
   if constexpr (BITS == 4) {
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
@@ -163,7 +177,7 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
         al[k] = __dp4a(ql.l[k][s], x, al[k]);
       }
   }
-  const uint32_t* mr = reinterpret_cast<const uint32_t*>(meta) + j * GPR;
+  const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + RG::META) + jl * RG::GPR;
   float s0, z0;
   if constexpr (G >= 32) {
     unpack_meta(mr[(slice * 32) / G], s0, z0);
@@ -179,85 +193,91 @@ __device__ __forceinline__ float kdot(const unsigned char* codes, const unsigned
   }
 }
 
-// Value path.  A code masked out of its word with the rest of the register
-// (and so the exponent field) zero is the exact fp32 subnormal c * 2^(p-149),
-// p its bit position (p + bits <= 23).  One FFMA with the fp32 weight
-// w_p = p_t * kappa * s~ * 2^(kPosBias - p) adds p_t * kappa * s~ * c * 2^-40
-// to the channel's accumulator: one mask and one FMA per code, fp32 weights.
-constexpr int kPosBias = 109;                        // 2^(109 - p) <= 2^109 stays finite
-constexpr float kValueUnscale = 1099511627776.0f;    // 2^(149 - kPosBias) = 2^40
-constexpr float kWeightMax = 262144.0f;              // 2^18: weights above this are flagged
+// Value accumulators of one lane: channel pairs (2i, 2i+1) of its 32-channel
+// slice as packed fp32 (acc[i]); z~ terms per 16-channel half (cst[0], cst[1])
+// and for groups spanning the whole slice (cst[2]).
+struct VAcc {
+  float2 acc[16];
+  float cst[3];
+};
 
-__device__ __forceinline__ float pow2_bias(int pos) {
-  return __uint_as_float(static_cast<uint32_t>(127 + kPosBias - pos) << 23);
+constexpr int kPosBias = 109;                        // weights w * 2^(109 - p), p <= 14
+constexpr float kValueUnscale = 1099511627776.0f;    // 2^(149 - kPosBias) = 2^40
+
+__device__ __forceinline__ float pow2i(int e) {
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
 }
 
-// acc += w * D(c) over one lane's 32 channels of token j (codes part; the z~
-// offsets go to cst per 16-channel half).  pk = p_t * kappa.
+__device__ __forceinline__ float2 masked_pair(uint32_t w, uint32_t ma, uint32_t mb) {
+  return make_float2(__uint_as_float(w & ma), __uint_as_float(w & mb));
+}
+
+// acc += pk * D(c) over one lane's 32 channels of record token jl (codes
+// part; the z~ offsets go to cst).  A channel pair shares a word, and the
+// code positions (pa, pb) of the pair fix its weight pair
+// {w 2^(109-pa), w 2^(109-pb)}, w = pk * s~:
+//   b = 2: word k holds channels 16k + 2i, +1 at bits 4i, 4i+2 (i < 4), and
+//          channels 16k + 8 + 2i, +1 at the same bits of word >> 16;
+//   b = 4: word 2k + hh holds channels 16k + 2hh, +1 at bits 0, 4 and
+//          16k + 4 + 2hh, +1 at bits 8, 12; word >> 16 gives channels + 8.
 template <int D, int BITS, int G>
-__device__ __forceinline__ void vacc(const unsigned char* codes, const unsigned char* meta, int j,
-                                     int slice, float pk, float (&acc)[32], float (&cst)[2],
-                                     uint32_t& range_err) {
-  constexpr int WPR = D * BITS / 32, GPR = D / G;
-  const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + j * WPR + slice * BITS;
-  const uint32_t* mr = reinterpret_cast<const uint32_t*>(meta) + j * GPR;
+__device__ __forceinline__ void vacc(const unsigned char* rec, int jl, int slice, float pk,
+                                     VAcc& va) {
+  using RG = RecGeom<D, BITS, G>;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * RG::WPR + slice * BITS;
+  const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + RG::META) + jl * RG::GPR;
+  constexpr int NW = G >= 32 ? 1 : 2;   // weights per lane (16-channel halves for g = 16)
   float sc[2], zc[2];
-  if constexpr (G >= 32) {
+  if constexpr (NW == 1) {
     unpack_meta(mr[(slice * 32) / G], sc[0], zc[0]);
-    sc[1] = sc[0];
-    zc[1] = zc[0];
+    va.cst[2] = fmaf(pk, zc[0], va.cst[2]);
   } else {
     const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
     unpack_meta(mw.x, sc[0], zc[0]);
     unpack_meta(mw.y, sc[1], zc[1]);
+    va.cst[0] = fmaf(pk, zc[0], va.cst[0]);
+    va.cst[1] = fmaf(pk, zc[1], va.cst[1]);
   }
-  constexpr int NPOS = BITS == 2 ? 8 : 4;   // positions 0,2,..,14 or 0,4,8,12 (after >>16)
-  constexpr int NW = G >= 32 ? 1 : 2;       // distinct weights per lane
-  float ws[2][NPOS];
+  constexpr int NP = BITS == 2 ? 4 : 2;   // distinct weight pairs
+  float2 wp[NW][NP];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    cst[h] = fmaf(pk, zc[h], cst[h]);
-    if (h >= NW) continue;
-    float w = pk * sc[h];
-    if (!(fabsf(w) <= kWeightMax)) {
-      range_err = 1u;
-      w = 0.0f;
+  for (int h = 0; h < NW; ++h) {
+    const float w = pk * sc[h];
+    const float2 ww = make_float2(w, w);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int pa = BITS == 2 ? 4 * i : 8 * i;
+      const int pb = pa + BITS;
+      wp[h][i] = __fmul2_rn(ww, make_float2(pow2i(kPosBias - pa), pow2i(kPosBias - pb)));
     }
-#pragma unroll
-    for (int q = 0; q < NPOS; ++q) ws[h][q] = w * pow2_bias(q * BITS);
   }
   if constexpr (BITS == 4) {
-    // word 2k + hh, nibble n: channel 16k + 4(n>>1) + 2hh + (n&1); nibbles
-    // 4..7 are read from word >> 16 at the positions of nibbles 0..3.
     const uint4 v = *reinterpret_cast<const uint4*>(cw);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
       const int k = k4 >> 1, hh = k4 & 1;
       const uint32_t w16 = w[k4] >> 16;
-      const float* wq = ws[NW == 1 ? 0 : k];
-#pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        const uint32_t m = 0xFu << (4 * n);
-        const int ch = 16 * k + 4 * (n >> 1) + 2 * hh + (n & 1);
-        acc[ch] = fmaf(wq[n], __uint_as_float(w[k4] & m), acc[ch]);
-        acc[ch + 8] = fmaf(wq[n], __uint_as_float(w16 & m), acc[ch + 8]);
-      }
+      const float2* wq = wp[NW == 1 ? 0 : k];
+      float2* a = va.acc + 8 * k + hh;
+      a[0] = __ffma2_rn(wq[0], masked_pair(w[k4], 0xFu, 0xF0u), a[0]);
+      a[2] = __ffma2_rn(wq[1], masked_pair(w[k4], 0xF00u, 0xF000u), a[2]);
+      a[4] = __ffma2_rn(wq[0], masked_pair(w16, 0xFu, 0xF0u), a[4]);
+      a[6] = __ffma2_rn(wq[1], masked_pair(w16, 0xF00u, 0xF000u), a[6]);
     }
   } else {
-    // word k: field f (channel 16k + f) at bits 2f; fields 8..15 are read from
-    // word >> 16 at the positions of fields 0..7.
     const uint2 v = *reinterpret_cast<const uint2*>(cw);
     const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const uint32_t w16 = w[k] >> 16;
-      const float* wq = ws[NW == 1 ? 0 : k];
+      const float2* wq = wp[NW == 1 ? 0 : k];
 #pragma unroll
-      for (int f = 0; f < 8; ++f) {
-        const uint32_t m = 3u << (2 * f);
-        acc[16 * k + f] = fmaf(wq[f], __uint_as_float(w[k] & m), acc[16 * k + f]);
-        acc[16 * k + 8 + f] = fmaf(wq[f], __uint_as_float(w16 & m), acc[16 * k + 8 + f]);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t ma = 3u << (4 * i), mb = 3u << (4 * i + 2);
+        va.acc[8 * k + i] = __ffma2_rn(wq[i], masked_pair(w[k], ma, mb), va.acc[8 * k + i]);
+        va.acc[8 * k + 4 + i] =
+            __ffma2_rn(wq[i], masked_pair(w16, ma, mb), va.acc[8 * k + 4 + i]);
       }
     }
   }
@@ -268,33 +288,54 @@ template <class SP, int C = 0>
 __device__ __forceinline__ void score_comps(const unsigned char* st, int j, int slice,
                                             const QLimbs& ql, float& part, float& kap) {
   if constexpr (C < SP::NC) {
-    const float d = kdot<SP::D, SP::bits(C), SP::group(C)>(st + SP::codes_off(0, C),
-                                                           st + SP::meta_off(0, C), j, slice, ql);
+    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
+    const unsigned char* rec = SP::rec(st, 0, C, j);
+    const int jl = SP::RPS == 1 ? j : j % kBlock;
+    const float d = kdot<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, ql);
     part = fmaf(kap, d, part);
     if constexpr (SP::has_alpha(C))
-      kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(st + SP::alpha_off(0, C))[j]);
+      kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
     score_comps<SP, C + 1>(st, j, slice, ql, part, kap);
   }
 }
 
 template <class SP, int C = 0>
 __device__ __forceinline__ void value_comps(const unsigned char* st, int j, int slice, float kap,
-                                            float (&acc)[32], float (&cst)[2],
-                                            uint32_t& range_err) {
+                                            VAcc& va) {
   if constexpr (C < SP::NC) {
-    vacc<SP::D, SP::bits(C), SP::group(C)>(st + SP::codes_off(1, C), st + SP::meta_off(1, C), j,
-                                           slice, kap, acc, cst, range_err);
+    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
+    const unsigned char* rec = SP::rec(st, 1, C, j);
+    const int jl = SP::RPS == 1 ? j : j % kBlock;
+    vacc<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, kap, va);
     if constexpr (SP::has_alpha(C))
-      kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(st + SP::alpha_off(1, C))[j]);
-    value_comps<SP, C + 1>(st, j, slice, kap, acc, cst, range_err);
+      kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
+    value_comps<SP, C + 1>(st, j, slice, kap, va);
   }
 }
 
-// Final value of the accumulators: undo the weight and subnormal scales and
-// add the z~ terms of each 16-channel half.
-__device__ __forceinline__ void finish_values(float (&acc)[32], const float (&cst)[2]) {
+__device__ __forceinline__ void rescale(VAcc& va, float f) {
+  const float2 ff = make_float2(f, f);
 #pragma unroll
-  for (int ch = 0; ch < 32; ++ch) acc[ch] = fmaf(acc[ch], kValueUnscale, cst[ch / 16]);
+  for (int i = 0; i < 16; ++i) va.acc[i] = __fmul2_rn(va.acc[i], ff);
+  va.cst[0] *= f;
+  va.cst[1] *= f;
+  va.cst[2] *= f;
+}
+
+// Final per-channel values: undo the 2^-40 code scale and add the z~ terms.
+// A weight past the scaled range (p_t * kappa * s~ >= 2^19) leaves an
+// infinity or NaN here and is reported.
+__device__ __forceinline__ void finish_values(const VAcc& va, float (&acc)[32],
+                                              uint32_t& range_err) {
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float c = va.cst[i / 8] + va.cst[2];
+    acc[2 * i] = fmaf(va.acc[i].x, kValueUnscale, c);
+    acc[2 * i + 1] = fmaf(va.acc[i].y, kValueUnscale, c);
+    finite = finite && isfinite(acc[2 * i]) && isfinite(acc[2 * i + 1]);
+  }
+  if (!finite) range_err = 1u;
 }
 
 // Token range of this CTA's split.
@@ -354,8 +395,8 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   constexpr int NSLOT = kCWarps * TPW;
   static_assert(TT >= 1 && TT * TPC == TC, "chunk must be a multiple of the tokens per pass");
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t full_bar[kMaxRing];
-  __shared__ uint32_t s_release[kMaxRing];
+  __shared__ uint64_t full_bar[kCMaxRing];
+  __shared__ uint32_t s_release[kCMaxRing];
   __shared__ float svec[D];
   __shared__ float sred[kCThreads / 32];
   __shared__ volatile int s_abort;
@@ -367,9 +408,11 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   const int S = p.stages;
   const int n = seq_len_of(p.seq_lens, bhi / p.heads, p.max_seq_len, p.err);
   const Range R = split_range(n, split, p.chunks_per_split, TC);
-  static_assert(TC == kBlock, "a decode stage is one storage record per component");
 
-  // Copies of chunk i into stage s (one lane): one record per component.
+  // Copies of chunk i into stage s (one lane): RPS consecutive records per
+  // component and side, one copy each.  Splits start at multiples of TC
+  // tokens and rows hold a multiple of 64 tokens, so a stage never leaves
+  // its row.
   auto issue = [&](int i, int s) {
     const int t0 = R.t_begin + i * TC;
     fence_proxy_async_smem();
@@ -380,7 +423,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       const Comp* cs = side == 0 ? p.k : p.v;
 #pragma unroll
       for (int c = 0; c < NC; ++c)
-        bulk_copy_g2s(st + SP::codes_off(side, c), comp_record(cs[c], bhi, p.nblk, t0),
+        bulk_copy_g2s(st + SP::comp_off(side, c), comp_record(cs[c], bhi, p.nblk, t0),
                       SP::comp_bytes(c), &full_bar[s]);
     }
   };
@@ -427,16 +470,16 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   QLimbs ql;
   build_limbs(qv, 1.0f / sigma, ql);
   __syncthreads();   // barrier initialisation is visible to every warp
-  float acc[32];
+  VAcc va;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-  float cst[2] = {0.0f, 0.0f};
-  uint32_t range_err = 0u;
+  for (int i = 0; i < 16; ++i) va.acc[i] = make_float2(0.0f, 0.0f);
+  va.cst[0] = va.cst[1] = va.cst[2] = 0.0f;
   float m = kNegInf, l = 0.0f;
 
+  int s = 0;
+  uint32_t phase = 0u;
   for (int i = 0; i < R.nchunks; ++i) {
-    const int s = i % S;
-    if (!mbar_wait(&full_bar[s], (i / S) & 1, p.err)) s_abort = 1;
+    if (!mbar_wait(&full_bar[s], phase, p.err)) s_abort = 1;
     if (s_abort) break;
     const unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
     const int nt = min(TC, R.t_end - (R.t_begin + i * TC));
@@ -456,10 +499,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
     if (mc > m) {
       const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
       l *= f;
-      cst[0] *= f;
-      cst[1] *= f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) acc[k] *= f;
+      rescale(va, f);
       m = mc;
     }
 #pragma unroll
@@ -468,7 +508,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       if (sc[tt] == kNegInf) continue;
       const float pt = fast_exp2(sc[tt] - m);
       l += pt;
-      value_comps<SP>(st, j, slice, pt, acc, cst, range_err);
+      value_comps<SP>(st, j, slice, pt, va);
     }
     // Release the stage; the last warp to do so refills it.
     __syncwarp();
@@ -481,9 +521,15 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
         atomicAdd(&s_issued, 1);
       }
     }
+    if (++s == S) {
+      s = 0;
+      phase ^= 1u;
+    }
   }
-  finish_values(acc, cst);
-  if (range_err) atomicOr(p.err, kErrRange);
+  float acc[32];
+  uint32_t range_err = 0u;
+  finish_values(va, acc, range_err);
+  if (range_err && !s_abort) atomicOr(p.err, kErrRange);
   if (s_abort) {
     m = kNegInf;
     l = 0.0f;
@@ -678,6 +724,7 @@ size_t dyn_bytes(int stages) {
 struct FastEntry {
   int D, NC, RB, RG, AB, AG;
   uint32_t stage_bytes;
+  int chunk;
   cudaError_t (*launch)(const DecodeParams&, cudaStream_t);
   cudaError_t (*occupancy)(int stages, int* occ);
 };
@@ -698,6 +745,7 @@ cudaError_t occ_spec(int stages, int* occ) {
 
 #define RQ_FAST(D, NC, RB, RG, AB, AG)                                                        \
   FastEntry{D,  NC, RB, RG, AB, AG, Spec<D, NC, RB, RG, AB, AG>::stage_bytes(),              \
+            Spec<D, NC, RB, RG, AB, AG>::TC,                                                 \
             &launch_spec<Spec<D, NC, RB, RG, AB, AG>>, &occ_spec<Spec<D, NC, RB, RG, AB, AG>>}
 
 const FastEntry kFast[] = {
@@ -719,10 +767,10 @@ const FastEntry* find_fast(const DecodeParams& p, int D) {
     if (f.D != D || f.NC != NC) continue;
     bool ok = p.k[NC - 1].bits == f.AB && p.k[NC - 1].group == f.AG;
     for (int c = 0; c + 1 < NC; ++c) ok = ok && p.k[c].bits == f.RB && p.k[c].group == f.RG;
-    // a stage is exactly one record per component and side
+    // a stage is exactly RPS records per component and side
     uint32_t rec = 0;
     for (int c = 0; c < NC; ++c) rec += p.k[c].rec_bytes + p.v[c].rec_bytes;
-    ok = ok && rec == f.stage_bytes;
+    ok = ok && rec * (f.chunk / kBlock) == f.stage_bytes;
     if (ok) return &f;
   }
   return nullptr;
@@ -744,19 +792,17 @@ cudaError_t launch_bf16_t(const DecodeBf16Params& p, cudaStream_t s) {
 
 // ---- host interface (rq_internal.cuh) ----
 
-bool fast_decode_plan(const DecodeParams& p, int D, size_t ring_budget, int max_stages,
-                      int* stages, int* ctas_per_sm) {
+bool fast_decode_plan(const DecodeParams& p, int D, int* stages, int* chunk, int* ctas_per_sm) {
   const FastEntry* f = find_fast(p, D);
   if (f == nullptr) return false;
-  (void)ring_budget;
   int s = static_cast<int>(kCRingBudget / f->stage_bytes);
-  if (s > max_stages) s = max_stages;
-  if (s > kMaxRing) s = kMaxRing;
+  if (s > kCMaxRing) s = kCMaxRing;
   if (s < 2) s = 2;
   if (static_cast<size_t>(s) * f->stage_bytes > 220 * 1024) return false;
   int occ = 0;
   if (f->occupancy(s, &occ) != cudaSuccess || occ < 1) return false;
   *stages = s;
+  *chunk = f->chunk;
   *ctas_per_sm = occ;
   return true;
 }
@@ -771,7 +817,6 @@ uint32_t bf16_stage_bytes(int D) {
   return D == 64 ? 2u * bf16_tc<64>() * 64 * 2 : 2u * bf16_tc<128>() * 128 * 2;
 }
 int bf16_chunk(int D) { return D == 64 ? bf16_tc<64>() : bf16_tc<128>(); }
-int fast_chunk() { return kCChunk; }
 
 cudaError_t bf16_occupancy(int D, int stages, int* occ) {
   const size_t ring = static_cast<size_t>(stages) * bf16_stage_bytes(D);

@@ -17,9 +17,9 @@ namespace rq {
 // Device-side error bits recorded in the decode workspace.
 constexpr uint32_t kErrSeqLen = 1u;    // a seq_lens entry was outside [0, max_seq_len]
 constexpr uint32_t kErrTimeout = 2u;   // a bounded mbarrier wait ran out
-constexpr uint32_t kErrRange = 4u;     // a value weight left the f16 range (group scale too large)
+constexpr uint32_t kErrRange = 4u;     // a value weight left the scaled-accumulator range
 
-// Tokens per pipeline stage of the decode kernels.
+// Tokens per pipeline stage of the generic decode kernel (two records).
 constexpr int kChunk = 64;
 constexpr int kDecodeThreads = 128;
 
@@ -28,7 +28,7 @@ constexpr int kDecodeThreads = 128;
 // ---------------------------------------------------------------------------
 
 // One packed component (anchor or one residual loop) of one side, stored as
-// 64-token records [codes[64][D*bits/32] | meta[64][D/group] | alpha[64]].
+// 32-token records [codes[32][D*bits/32] | meta[32][D/group] | alpha[32]].
 struct Comp {
   unsigned char* base;     // record of (row 0, block 0)
   uint32_t rec_bytes;      // bytes per record
@@ -38,6 +38,10 @@ struct Comp {
 };
 
 constexpr int kBlock = RQ_BLOCK_TOKENS;
+// Rows hold a multiple of 64 tokens, so a 64-token stage aligned to 64 never
+// leaves its row.
+constexpr int kRowTokens = 64;
+static_assert(kChunk % kBlock == 0 && kRowTokens % kChunk == 0, "stages are whole records");
 
 // Record holding token t of row `row` (nblk = records per row).
 __host__ __device__ inline unsigned char* comp_record(const Comp& c, int64_t row, int64_t nblk,
@@ -99,6 +103,7 @@ struct DecodeParams {
   uint32_t* counters;      // [B*H]
   uint32_t* err;           // [1]
   int32_t splits;
+  int32_t chunk;           // tokens per pipeline stage (whole records)
   int32_t chunks_per_split;
   int32_t stages;
   uint32_t stage_bytes;
@@ -135,11 +140,9 @@ cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s);
 // generic compressed decode (any chain of bits / groups), chunk kChunk
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t s);
-// warp-specialised decode for compiled layouts, chunk fast_chunk()
-bool fast_decode_plan(const DecodeParams& p, int D, size_t ring_budget, int max_stages,
-                      int* stages, int* ctas_per_sm);
+// decode for compiled layouts: stages, tokens per stage and resident CTAs
+bool fast_decode_plan(const DecodeParams& p, int D, int* stages, int* chunk, int* ctas_per_sm);
 cudaError_t launch_decode_fast(const DecodeParams& p, int D, cudaStream_t s);
-int fast_chunk();
 // uncompressed bf16 decode, chunk bf16_chunk(D)
 cudaError_t launch_decode_bf16(const DecodeBf16Params& p, int D,
                                cudaStream_t s);

@@ -79,7 +79,7 @@ extern "C" rq_status rq_decode_attention_noalloc(const rq_cache* c, int32_t laye
   if (partials_off + per_split > kNoAllocScratchBytes) return RQ_ERR_WORKSPACE;
   const int fit = static_cast<int>((kNoAllocScratchBytes - partials_off) / per_split);
   if (p.splits > fit) {
-    const int chunks = (max_seq_len + kBlock - 1) / kBlock;
+    const int chunks = (max_seq_len + p.chunk - 1) / p.chunk;
     int cps = (chunks + fit - 1) / fit;
     if (cps < 1) cps = 1;
     p.chunks_per_split = cps;

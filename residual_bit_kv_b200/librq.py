@@ -13,7 +13,7 @@ import os
 from typing import Optional, Sequence
 
 RQ_MAX_LOOPS = 32
-RQ_BLOCK_TOKENS = 64
+RQ_BLOCK_TOKENS = 32
 RQ_POLICY_LAST_LOOP = 0
 RQ_POLICY_NEXT_LOOP = 1
 

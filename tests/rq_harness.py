@@ -86,7 +86,7 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
                   bsel: Optional[Sequence[int]] = None,
                   hsel: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
-    """Packed arrays of one component, unblocked from the 64-token records into
+    """Packed arrays of one component, unblocked from the storage records into
     numpy [B, H, token_stride, ...] arrays (or [len(bsel), len(hsel), ...] for
     a selection, copying only those rows off the device)."""
     c = gc.cache
