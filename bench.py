@@ -24,6 +24,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -69,31 +70,77 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs:
+    NVML every 10 ms from a thread (the device found by PCI bus id), else
+    nvidia-smi every 200 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int):
+        self.dev = device_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.stop = None
+        self.samples = []   # (sm_mhz, reasons bitmask)
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devid = getattr(props, "pci_device_id", 0)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devid:02x}.0")
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.stop = threading.Event()
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                             int(reasons(h))))
+                    except Exception:
+                        pass
+                    time.sleep(0.01)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+        except Exception:
+            self._start_smi()
+        time.sleep(0.05)
+        return self
+
+    def _start_smi(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         time.sleep(0.3)
-        return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -102,6 +149,14 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.thread is not None:
+            if not self.samples:
+                return None
+            reasons = sorted(n for n, bit in self.REASON_BITS.items()
+                             if any(r & bit for _, r in self.samples))
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                    "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(self.samples), "source": "nvml 10 ms"}
         if self.path is None or not os.path.exists(self.path):
             return None
         sm, mx, reasons = [], [], set()
@@ -123,7 +178,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi 200 ms"}
 
 
 def file_sha(path):
@@ -326,48 +381,53 @@ def timed(fn, steps, warmup, stream, dist=None):
 
 # --------------------------------------------------------- oracle (CPU) legs --
 
-def oracle_decode_sample(w, pairs, loops):
-    """Times the oracle's decode of `pairs` (b, h) units for `loops` of layer 0:
+def oracle_decode_sample(w, pairs, loops, budget_s=None):
+    """Times the oracle's decode of (b, h) units for `loops` of layer 0:
     reconstruction of every past row in fp64 and exact softmax attention.
-    Encoding the sample cache is set-up, not timed."""
+    Pairs are taken in order until `budget_s` seconds of timed work (all of
+    them if None).  Encoding a pair's cache is set-up, not timed."""
     import oracle
     T = w.tokens
     D = w.head_dim
-    encs = {}
-    for side in (0, 1):
-        cs = synth.key_channel_scale(w, 0) if side == 0 else None
-        xl = []
-        for loop in range(w.loops):
-            rows = [synth.bits_of(synth.kv(w, 0, side, loop, [b], [h], 0, T, "cpu", cs)).reshape(-1, D)
-                    for b, h in pairs]
-            xl.append(np.concatenate(rows))
-        encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
     q = synth.bits_of(torch.stack([synth.query(w, 0, l) for l in range(w.loops)]))
     kc = {l: synth.bits_of(synth.current_token(w, 0, 0, l)) for l in loops}
     vc = {l: synth.bits_of(synth.current_token(w, 0, 1, l)) for l in loops}
-    t0 = time.perf_counter()
-    units = 0
-    for loop in loops:
-        kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(len(pairs), T, D)
-        vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(len(pairs), T, D)
-        for i, (b, h) in enumerate(pairs):
-            oracle.attention(oracle.bf16_bits_to_f64(q[loop, b, h]), kh[i], vh[i],
+    secs, units = 0.0, 0
+    for b, h in pairs:
+        encs = {}
+        for side in (0, 1):
+            cs = synth.key_channel_scale(w, 0) if side == 0 else None
+            xl = [synth.bits_of(synth.kv(w, 0, side, loop, [b], [h], 0, T, "cpu", cs)).reshape(-1, D)
+                  for loop in range(w.loops)]
+            encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
+        t0 = time.perf_counter()
+        for loop in loops:
+            kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(T, D)
+            vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(T, D)
+            oracle.attention(oracle.bf16_bits_to_f64(q[loop, b, h]), kh, vh,
                              oracle.bf16_bits_to_f64(kc[loop][b, h]),
                              oracle.bf16_bits_to_f64(vc[loop][b, h]), 1.0 / np.sqrt(D))
             units += 1
-    return time.perf_counter() - t0, units
+        secs += time.perf_counter() - t0
+        if budget_s is not None and secs >= budget_s:
+            break
+    return secs, units
+
+
+CPU_BASELINE_SECONDS = 10.0
 
 
 def cpu_baseline(w):
-    """Oracle decode on a bounded sample: 2 (batch, head) units x 4 loops of
-    layer 0 at the full 16k context, scaled to the step's 24*4*B*H units."""
-    pairs = [(0, 0), (w.batch - 1, w.heads - 1)]
-    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)))
+    """Oracle decode on a bounded sample: (batch, head) units x 4 loops of
+    layer 0 at the full 16k context until about 10 s of timed CPU work,
+    scaled to the step's 24*4*B*H units."""
+    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(w.batch * w.heads)]
+    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)), CPU_BASELINE_SECONDS)
     step_units = w.layers * w.loops * w.batch * w.heads
     step_s = secs / units * step_units
     return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens} "
-                      f"({secs:.1f} s), scaled to {step_units} units per step"}
+                      f"({secs:.1f} s timed), scaled to {step_units} units per step"}
 
 
 def run_reference(args, rank):

@@ -89,61 +89,6 @@ struct QLimbs {
   float sq[2];   // sum of q~ over channels 0-15 / 16-31
 };
 
-// Unnormalised Hadamard butterflies over a row held by P = D/32 lanes, lane
-// `slice` holding channels 32*slice .. 32*slice+31 (stages h = 1..16 inside
-// the lane, then across lanes by xor-shuffles).
-template <int D>
-__device__ __forceinline__ void fwht_lanes(float (&z)[32], int slice) {
-#pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 2 * h) {
-#pragma unroll
-      for (int j = i; j < i + h; ++j) {
-        const float a = z[j], b = z[j + h];
-        z[j] = a + b;
-        z[j + h] = a - b;
-      }
-    }
-  }
-#pragma unroll
-  for (int hl = 1; hl < D / 32; hl <<= 1) {
-    const bool upper = (slice & hl) != 0;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const float o = __shfl_xor_sync(0xffffffffu, z[k], hl);
-      z[k] = upper ? o - z[k] : z[k] + o;
-    }
-  }
-}
-
-__device__ __forceinline__ int pack_bytes(int a, int b, int c, int d) {
-  return (a & 0xFF) | ((b & 0xFF) << 8) | ((c & 0xFF) << 16) | (d << 24);
-}
-
-__device__ __forceinline__ void build_limbs(const float* qrow, float inv_sigma, QLimbs& ql) {
-  int hi[32], lo[32];
-  float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int qt = __float2int_rn(qrow[i] * inv_sigma);   // |qt| <= 32639
-    const int h = (qt + 128) >> 8;
-    hi[i] = h;
-    lo[i] = qt - 256 * h;
-    if (i < 16) s0 += static_cast<float>(qt); else s1 += static_cast<float>(qt);
-  }
-  ql.sq[0] = s0;
-  ql.sq[1] = s1;
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int b = 16 * k + s;
-      ql.h[k][s] = pack_bytes(hi[b], hi[b + 4], hi[b + 8], hi[b + 12]);
-      ql.l[k][s] = pack_bytes(lo[b], lo[b + 4], lo[b + 8], lo[b + 12]);
-    }
-}
-
 // q~ . D(c) over one lane's 32 channels of record token jl of a component,
 // in sigma units: sum over group parts of s~ * (q~ . codes) + z~ * (sum q~).
 template <int D, int BITS, int G>
@@ -439,37 +384,52 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
     for (int i = 0; i < first; ++i) issue(i, i);
     s_issued = first;
   }
-  // q' = H q * softmax scale * log2 e, rotated in registers by the P lanes of
-  // each token slot (every slot holds the same query), then its fixed-point
-  // scale from max |q'|.
-  float qv[32];
+  // q' = H q * softmax scale * log2 e, one channel per thread (every split
+  // of a row forms the same q'), its fixed-point scale sigma from max |q'|,
+  // and the int8 limbs stored in the quad order each lane reads: channel
+  // 32*sl + 16k + s + 4u goes to word 8*sl + 4k + s, byte u.
+  __shared__ __align__(16) int s_limb[2][D / 4];
+  __shared__ float s_sq[D / 16];
+  __shared__ float s_amax[kCWarps];
+  if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
+  __syncthreads();
+  smem_fwht<D>(svec);
+  const float qscale = p.rot_scale * p.scale_log2;
+  const float qv = t < D ? svec[t] * qscale : 0.0f;
+  float amax = fabsf(qv);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (lane == 0) s_amax[warp] = amax;
+  __syncthreads();
+  amax = s_amax[0];
+#pragma unroll
+  for (int w = 1; w < kCWarps; ++w) amax = fmaxf(amax, s_amax[w]);
+  const float sigma = amax > 0.0f ? amax / 32639.0f : 1.0f;
   {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + static_cast<size_t>(bhi) * D + slice * 32);
+    const int qt = __float2int_rn(qv * (1.0f / sigma));   // |qt| <= 32639
+    const int hi = (qt + 128) >> 8;
+    float qs = static_cast<float>(qt);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = src[i];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qv[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
-        qv[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-      }
+    for (int off = 8; off >= 1; off >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, off);
+    if (t < D) {
+      const int c = t & 31;
+      const int byte = (t >> 5) * 32 + ((c >> 4) * 4 + (c & 3)) * 4 + ((c >> 2) & 3);
+      reinterpret_cast<signed char*>(s_limb[0])[byte] = static_cast<signed char>(hi);
+      reinterpret_cast<signed char*>(s_limb[1])[byte] = static_cast<signed char>(qt - 256 * hi);
+      if ((c & 15) == 0) s_sq[t >> 4] = qs;
     }
   }
-  fwht_lanes<D>(qv, slice);
-  const float qscale = p.rot_scale * p.scale_log2;
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    qv[i] *= qscale;
-    amax = fmaxf(amax, fabsf(qv[i]));
-  }
-#pragma unroll
-  for (int off = P / 2; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float sigma = amax > 0.0f ? amax / 32639.0f : 1.0f;
+  __syncthreads();
   QLimbs ql;
-  build_limbs(qv, 1.0f / sigma, ql);
-  __syncthreads();   // barrier initialisation is visible to every warp
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      ql.h[k][q4] = s_limb[0][slice * 8 + k * 4 + q4];
+      ql.l[k][q4] = s_limb[1][slice * 8 + k * 4 + q4];
+    }
+  ql.sq[0] = s_sq[slice * 2];
+  ql.sq[1] = s_sq[slice * 2 + 1];
   VAcc va;
 #pragma unroll
   for (int i = 0; i < 16; ++i) va.acc[i] = make_float2(0.0f, 0.0f);
