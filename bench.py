@@ -50,13 +50,30 @@ def dist_env():
     return ws, rank, local
 
 
-def init_dist(ws):
+def init_dist(ws, backend="nccl"):
+    """One process per GPU (torchrun env); None for a single process."""
     if ws <= 1:
         return None
     import datetime
     import torch.distributed as dist
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return dist
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's value (each rank calls this at the same
+    point); the value itself for a single process."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world_size: int, batch: int, ms_per_step: float) -> float:
+    """Whole-job decode throughput: every rank decodes its own batch per step
+    (weak scaling), the step time being the slowest rank's."""
+    return world_size * batch * 1e3 / ms_per_step
 
 
 def peaks():
@@ -370,11 +387,8 @@ def timed(fn, steps, warmup, stream, dist=None):
         fn()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, "cuda")
     if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
 
@@ -520,11 +534,7 @@ def main():
             eng.step(stream, ev)
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     clocks = clk.summary()
     dec_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
     dec_bytes = args.steps * w.layers * sum(decode_call_bytes(w, l, w.tokens) for l in range(w.loops))
@@ -592,7 +602,7 @@ def main():
         cpu = cpu_baseline(w)
 
     if rank == 0:
-        value = ws * w.batch * 1e3 / ms
+        value = job_tokens_per_s(ws, w.batch, ms)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -606,7 +616,7 @@ def main():
             "decode_per_loop": per_loop,
             "decode_splits_loop0": splits0,
             "decode_hbm_frac_of_8tbs": achieved / 8000.0,
-            "e2e": {"value": ws * w.batch * 1e3 / e2e_ms, "unit": "tokens/s",
+            "e2e": {"value": job_tokens_per_s(ws, w.batch, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,
