@@ -303,13 +303,21 @@ class Engine:
                     self.bf16[(layer, side, loop)] = buf
                 del xs
             torch.cuda.synchronize(device)
-        # step inputs: per (layer, loop) query and the current token's K/V
+        # step inputs: per (layer, loop) query, and the current token's K/V of
+        # every loop of a layer stacked [L, B, H, D] (the append's input)
         self.q, self.kc, self.vc = {}, {}, {}
+        self.kc_layer, self.vc_layer = [], []
         for layer in range(w.layers):
+            kcl = torch.stack([synth.current_token(w, layer, 0, loop, device)
+                               for loop in range(w.loops)]).contiguous()
+            vcl = torch.stack([synth.current_token(w, layer, 1, loop, device)
+                               for loop in range(w.loops)]).contiguous()
+            self.kc_layer.append(kcl)
+            self.vc_layer.append(vcl)
             for loop in range(w.loops):
                 self.q[(layer, loop)] = synth.query(w, layer, loop, device).contiguous()
-                self.kc[(layer, loop)] = synth.current_token(w, layer, 0, loop, device).contiguous()
-                self.vc[(layer, loop)] = synth.current_token(w, layer, 1, loop, device).contiguous()
+                self.kc[(layer, loop)] = kcl[loop]
+                self.vc[(layer, loop)] = vcl[loop]
         self.seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
         self.out = torch.empty(w.layers, w.loops, w.batch, w.heads, w.head_dim,
                                dtype=torch.float32, device=device)
@@ -322,15 +330,17 @@ class Engine:
 
     def launches_per_step(self):
         w = self.w
-        return w.layers * w.loops + w.layers * w.loops * 2
+        return w.layers * w.loops + w.layers
 
-    def step(self, stream, ev=None, q=None, kc=None, vc=None):
-        """One decode step.  ev: optional list collecting (start, end) event
-        pairs around each decode-attention launch."""
+    def step(self, stream, ev=None, q=None, kc_layer=None, vc_layer=None):
+        """One decode step: the decode attention of every (layer, loop), then
+        per layer one launch that quantises and appends the new token of every
+        loop, K and V.  ev: optional list collecting (start, end) event pairs
+        around each decode-attention launch."""
         L, w, T = self.L, self.w, self.w.tokens
         q = q or self.q
-        kc = kc or self.kc
-        vc = vc or self.vc
+        kcl = kc_layer or self.kc_layer
+        vcl = vc_layer or self.vc_layer
         for layer in range(w.layers):
             for loop in range(w.loops):
                 if ev is not None:
@@ -338,18 +348,13 @@ class Engine:
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record(stream)
                 L.rq_decode_attention(self.cache, layer, loop, q[(layer, loop)], self.seq, T,
-                                      kc[(layer, loop)], vc[(layer, loop)], 0.0,
+                                      kcl[layer][loop], vcl[layer][loop], 0.0,
                                       self.out[layer, loop], self.ws, self.ws_bytes, stream)
                 if ev is not None:
                     e1.record(stream)
                     ev.append((e0, e1, loop))
             # after the final loop: quantise and append the new token (position T)
-            for side, cur in ((0, kc), (1, vc)):
-                A = w.loops - 1
-                L.rq_quantize_anchor(self.cache, layer, side, cur[(layer, A)], T, 1, stream)
-                for loop in range(w.loops - 2, -1, -1):
-                    L.rq_quantize_append_residual(self.cache, layer, side, loop,
-                                                  cur[(layer, loop)], T, 1, stream)
+            L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1, stream)
 
     def bf16_step(self, stream, ev=None, nlayers_buf=4):
         L, w, T = self.L, self.w, self.w.tokens
@@ -519,23 +524,22 @@ def main():
     w = eng.w
     stream = torch.cuda.current_stream(dev)
 
-    # ---- main timed region: the decode step, per-launch events on the decode kernel
+    # ---- the decode step launched eagerly, with CUDA events around every
+    # decode-attention launch (the roofline's kernel times)
     ev = []
     for _ in range(args.warmup):
         eng.step(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    with ClockSampler(local) as clk:
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            eng.step(stream, ev)
-        e1.record(stream)
-        torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
-    clocks = clk.summary()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        eng.step(stream, ev)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     dec_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
     dec_bytes = args.steps * w.layers * sum(decode_call_bytes(w, l, w.tokens) for l in range(w.loops))
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
@@ -545,28 +549,57 @@ def main():
         per_loop[str(l)] = {"us": t_l * 1e3,
                             "gbs": decode_call_bytes(w, l, w.tokens) / (t_l * 1e-3) / 1e9}
     hbm, hbm_kind = peaks()
-    n_launch_dec = args.steps * w.layers * w.loops
     traffic = profile_traffic(DECODE_SOURCES, "decode_kernel_ouro_16k.md")
+
+    # ---- main timed region: the same step captured once as a CUDA graph
+    # (the launch sequence of one step: no host work or launch gaps between
+    # kernels) and replayed
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        eng.step(cap)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=cap):
+        eng.step(cap)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    clocks = clk.summary()
 
     # ---- end to end: host buffers, H2D of the step's inputs, D2H of the outputs
     pin = {k: v.cpu().pin_memory() for k, v in eng.q.items()}
-    pkc = {k: v.cpu().pin_memory() for k, v in eng.kc.items()}
-    pvc = {k: v.cpu().pin_memory() for k, v in eng.vc.items()}
+    pkc = [t.cpu().pin_memory() for t in eng.kc_layer]
+    pvc = [t.cpu().pin_memory() for t in eng.vc_layer]
     hout = torch.empty(eng.out.shape, dtype=torch.float32).pin_memory()
     dq = {k: torch.empty_like(v) for k, v in eng.q.items()}
-    dkc = {k: torch.empty_like(v) for k, v in eng.kc.items()}
-    dvc = {k: torch.empty_like(v) for k, v in eng.vc.items()}
+    dkc = [torch.empty_like(t) for t in eng.kc_layer]
+    dvc = [torch.empty_like(t) for t in eng.vc_layer]
 
     def e2e_step():
         for k in pin:
             dq[k].copy_(pin[k], non_blocking=True)
-            dkc[k].copy_(pkc[k], non_blocking=True)
-            dvc[k].copy_(pvc[k], non_blocking=True)
+        for i in range(len(pkc)):
+            dkc[i].copy_(pkc[i], non_blocking=True)
+            dvc[i].copy_(pvc[i], non_blocking=True)
         eng.step(stream, None, dq, dkc, dvc)
         hout.copy_(eng.out, non_blocking=True)
 
     e2e_ms = timed(e2e_step, args.steps, args.warmup, stream, dist)
-    h2d = sum(v.numel() * 2 for v in pin.values()) * 3
+    h2d = (sum(v.numel() for v in pin.values()) + sum(t.numel() for t in pkc) +
+           sum(t.numel() for t in pvc)) * 2
     d2h = hout.numel() * 4
 
     # ---- BF16 baseline kernel on identical K/V (4 distinct layer buffers cycled)
@@ -614,10 +647,15 @@ def main():
                          "kernel": "decode_fast_kernel (all loops of the step)", "peak_kind": hbm_kind,
                          "bytes_per_step": dec_bytes / args.steps},
             "decode_per_loop": per_loop,
+            "step_launch": {"timed": f"one CUDA graph per step ({w.layers * w.loops} decode + "
+                                     f"{w.layers} append launches)",
+                            "eager_ms_per_step": eager_ms,
+                            "eager_tokens_per_s": job_tokens_per_s(ws, w.batch, eager_ms)},
             "decode_splits_loop0": splits0,
             "decode_hbm_frac_of_8tbs": achieved / 8000.0,
             "e2e": {"value": job_tokens_per_s(ws, w.batch, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "path": "public API per call (eager), inputs from pinned host memory"},
             "gpu_launches": launches,
             "clocks": clocks,
             "bf16_baseline": bf16,

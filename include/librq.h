@@ -156,6 +156,20 @@ rq_status rq_quantize_append_residual(const rq_cache* cache, int32_t layer,
                                       int32_t kv, int32_t loop, const void* x,
                                       int32_t t0, int32_t n, void* stream);
 
+/* Quantise-and-append of every loop of `layer` at token positions
+ * [t0, t0 + n), K and V, in one launch [RQ §3.2, §3.4, §4.2 Decode: the new
+ * token's loops are stored after the final loop]: the anchor (loop L-1) and
+ * every residual loop against it (LAST_LOOP) or against the chain Z^_{r+1}
+ * (NEXT_LOOP, loops L-2 down to 0).  Stores exactly the bytes of
+ * rq_quantize_anchor followed by rq_quantize_append_residual for each loop in
+ * the policy's order; the anchor is not re-read from the cache.
+ *   xk, xv  bf16 [num_loops][batch][kv_heads][n][head_dim], contiguous,
+ *           16-byte aligned; either may be NULL to skip that side (not both).
+ * n = 0 is a no-op.  t0 + n > max_tokens -> RQ_ERR_CAPACITY. */
+rq_status rq_quantize_append_loops(const rq_cache* cache, int32_t layer,
+                                   const void* xk, const void* xv, int32_t t0,
+                                   int32_t n, void* stream);
+
 /* Reconstructs X^ of loop `loop` at positions [t0, t0 + n) in the original
  * (unrotated) domain into out (fp32, [batch][kv_heads][n][head_dim]).
  * For tests and export; not on the decode path [RQ App. G.2]. */

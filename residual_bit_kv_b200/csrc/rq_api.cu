@@ -286,6 +286,32 @@ rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t 
       launch_quantize(p, l.head_dim, l.bits[loop], l.group[loop], as_stream(stream)));
 }
 
+rq_status rq_quantize_append_loops(const rq_cache* c, int32_t layer, const void* xk,
+                                   const void* xv, int32_t t0, int32_t n, void* stream) {
+  rq_status st = check_cache(c, layer, 0);
+  if (st != RQ_OK) return st;
+  if ((st = check_range(c, t0, n)) != RQ_OK) return st;
+  if (xk == nullptr && xv == nullptr) return RQ_ERR_INVALID_ARG;
+  if ((xk != nullptr && !aligned(xk, 16)) || (xv != nullptr && !aligned(xv, 16)))
+    return RQ_ERR_INVALID_ARG;
+  if (n == 0) return RQ_OK;
+  const rq_layout& l = c->layout;
+  QuantLoopsParams p;
+  memset(&p, 0, sizeof(p));
+  p.x[0] = static_cast<const uint16_t*>(xk);
+  p.x[1] = static_cast<const uint16_t*>(xv);
+  p.bh = l.batch * l.kv_heads;
+  p.n = n;
+  p.nloops = l.num_loops;
+  p.chained = l.policy == RQ_POLICY_NEXT_LOOP ? 1 : 0;
+  p.t0 = t0;
+  p.nblk = c->token_stride / kBlock;
+  for (int kv = 0; kv < 2; ++kv)
+    for (int r = 0; r < l.num_loops; ++r) p.dst[kv][r] = comp_of(c, layer, kv, r);
+  p.rot_scale = rot_scale_of(l.head_dim);
+  return cuda_status(launch_quantize_loops(p, l.head_dim, as_stream(stream)));
+}
+
 rq_status rq_dequantize(const rq_cache* c, int32_t layer, int32_t kv, int32_t loop, int32_t t0,
                         int32_t n, float* out, void* stream) {
   rq_status st = check_cache(c, layer, kv);

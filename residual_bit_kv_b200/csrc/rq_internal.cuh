@@ -74,6 +74,16 @@ struct QuantParams {
   float rot_scale;         // fp32(1/sqrt(D))
 };
 
+// Every loop of one (layer, token range), both sides, in one launch.
+struct QuantLoopsParams {
+  const uint16_t* x[2];    // bf16 [L][B*H][n][D] per side (K, V); nullptr skips the side
+  int32_t bh, n, nloops;
+  int32_t chained;         // 1: reference of loop r is Z^_{r+1} (Next-loop)
+  int64_t t0, nblk;
+  Comp dst[2][RQ_MAX_LOOPS];
+  float rot_scale;
+};
+
 struct DequantParams {
   int32_t bh, n, t0;
   int64_t nblk;
@@ -138,6 +148,7 @@ struct DecodeBf16Params {
 cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
                             cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s);
+cudaError_t launch_quantize_loops(const QuantLoopsParams& p, int D, cudaStream_t s);
 // generic compressed decode (any chain of bits / groups), chunk kChunk
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t s);
 // decode for compiled layouts: stages, tokens per stage and resident CTAs

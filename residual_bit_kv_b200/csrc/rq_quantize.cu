@@ -109,11 +109,13 @@ __device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t ro
   }
 }
 
-// Affine quantisation [RQ §2.1] of one lane's 32 values and the packed store.
+// Affine quantisation [RQ §2.1] of one lane's 32 values and the packed store;
+// if `levels` is given it receives the stored levels fma(s~, code, z~) (what
+// a reader of the record reconstructs).
 template <int D, int BITS, int G>
 __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
                                                bool active, uint32_t* codes_row,
-                                               uint32_t* meta_row) {
+                                               uint32_t* meta_row, float* levels = nullptr) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   constexpr int GL = G < 32 ? G : 32;    // group part held by this lane
   constexpr int NG = 32 / GL;            // group parts per lane
@@ -154,6 +156,7 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
       // leaves that integer in the low mantissa bits.
       const uint32_t code = __float_as_uint(__fadd_rn(u, 12582912.0f)) & QMAX;
       words[slice_word<BITS>(ch)] |= code << slice_shift<BITS>(ch);
+      if (levels != nullptr) levels[ch] = __fmaf_rn(st, static_cast<float>(code), zt);
     }
   }
   if (!active) return;
@@ -172,6 +175,56 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
   }
 }
 
+// Row of bf16 x -> fp32 -> Z = H x (normalised) in one lane's 32 registers.
+template <int D>
+__device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, int slice,
+                                            float rot_scale, float (&z)[32]) {
+  if (active) {
+    const uint4* src = reinterpret_cast<const uint4*>(xrow + slice * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = src[i];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        z[i * 8 + 2 * j] = __uint_as_float(w[j] << 16);
+        z[i * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) z[k] = 0.0f;
+  }
+  fwht_row<D>(z, slice);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) z[k] = __fmul_rn(z[k], rot_scale);
+}
+
+// Least-squares coefficient of z against the reference over the row
+// [RQ §3.2 scaling coefficient, App. G.1]: alpha~ = bf16(<z, ref> / <ref, ref>)
+// (0 for a zero reference); z becomes the residual fma(-alpha~, ref, z).
+template <int D>
+__device__ __forceinline__ __nv_bfloat16 ls_residual(float (&z)[32], const float (&ref)[32]) {
+  constexpr int P = D / 32;
+  float dzr = 0.0f, drr = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    dzr = __fmaf_rn(z[k], ref[k], dzr);
+    drr = __fmaf_rn(ref[k], ref[k], drr);
+  }
+#pragma unroll
+  for (int off = P / 2; off >= 1; off >>= 1) {
+    dzr = __fadd_rn(dzr, __shfl_xor_sync(0xffffffffu, dzr, off));
+    drr = __fadd_rn(drr, __shfl_xor_sync(0xffffffffu, drr, off));
+  }
+  const float a = (drr > 0.0f) ? __fdiv_rn(dzr, drr) : 0.0f;
+  const __nv_bfloat16 ab = __float2bfloat16_rn(a);
+  const float at = __bfloat162float(ab);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) z[k] = __fmaf_rn(-at, ref[k], z[k]);
+  return ab;
+}
+
 template <int D, int BITS, int G>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_kernel(const __grid_constant__ QuantParams p) {
@@ -187,25 +240,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int64_t row = base + lane / P;
     const bool active = row < total;
     float z[32];
-    if (active) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + row * D + slice * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = src[i];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          z[i * 8 + 2 * j] = __uint_as_float(w[j] << 16);
-          z[i * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = 0.0f;
-    }
-    fwht_row<D>(z, slice);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) z[k] = __fmul_rn(z[k], p.rot_scale);
+    load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, z);
 
     const int64_t bhi = active ? row / p.n : 0;
     const int64_t t = p.t0 + (active ? row % p.n : 0);
@@ -220,22 +255,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
         for (int k = 0; k < 32; ++k) ref[k] = 0.0f;
       }
-      float dzr = 0.0f, drr = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        dzr = __fmaf_rn(z[k], ref[k], dzr);
-        drr = __fmaf_rn(ref[k], ref[k], drr);
-      }
-#pragma unroll
-      for (int off = P / 2; off >= 1; off >>= 1) {
-        dzr = __fadd_rn(dzr, __shfl_xor_sync(0xffffffffu, dzr, off));
-        drr = __fadd_rn(drr, __shfl_xor_sync(0xffffffffu, drr, off));
-      }
-      const float a = (drr > 0.0f) ? __fdiv_rn(dzr, drr) : 0.0f;
-      const __nv_bfloat16 ab = __float2bfloat16_rn(a);
-      const float at = __bfloat162float(ab);
-#pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = __fmaf_rn(-at, ref[k], z[k]);
+      const __nv_bfloat16 ab = ls_residual<D>(z, ref);
       if (active && slice == 0)
         *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock)) =
             __bfloat16_as_ushort(ab);
@@ -244,6 +264,86 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int i = static_cast<int>(t % kBlock);
     quantize_store<D, BITS, G>(z, slice, active, rec_codes(rec, D, BITS, i),
                                rec_meta(rec, D, BITS, G, i));
+  }
+}
+
+// Quantisation of one component at token t (run-time bits / group): codes,
+// metadata and (if `levels`) the stored levels of this lane's 32 channels.
+template <int D>
+__device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_t nblk, int64_t t,
+                                              const float (&z)[32], int slice, bool active,
+                                              float* levels) {
+  unsigned char* rec = comp_record(c, row, nblk, t);
+  const int i = static_cast<int>(t % kBlock);
+  uint32_t* cw = rec_codes(rec, D, c.bits, i);
+  uint32_t* mw = rec_meta(rec, D, c.bits, c.group, i);
+  const int key = c.bits * 1000 + c.group;
+  switch (key) {
+    case 2016: quantize_store<D, 2, 16>(z, slice, active, cw, mw, levels); break;
+    case 2032: quantize_store<D, 2, 32>(z, slice, active, cw, mw, levels); break;
+    case 2064: quantize_store<D, 2, 64>(z, slice, active, cw, mw, levels); break;
+    case 4016: quantize_store<D, 4, 16>(z, slice, active, cw, mw, levels); break;
+    case 4032: quantize_store<D, 4, 32>(z, slice, active, cw, mw, levels); break;
+    case 4064: quantize_store<D, 4, 64>(z, slice, active, cw, mw, levels); break;
+    default:
+      if constexpr (D >= 128) {
+        if (key == 2128) quantize_store<D, 2, 128>(z, slice, active, cw, mw, levels);
+        else if (key == 4128) quantize_store<D, 4, 128>(z, slice, active, cw, mw, levels);
+      }
+      break;
+  }
+}
+
+// Every loop of a (layer, token range) for one side (blockIdx.y): the anchor
+// is quantised first and its stored levels stay in registers as the
+// reference; each residual loop then takes its LS coefficient, residual and
+// quantisation against it [RQ §3.2, §3.4, App. G.1].  Under the Next-loop
+// policy the loops run from L-2 down to 0 and the reference becomes
+// Z^_r = fma(alpha~_r, Z^_{r+1}, D(c_r)) after loop r.  The anchor is read
+// once and never re-read from the cache; the arithmetic (and so every
+// stored bit) is that of the per-loop kernels.
+template <int D>
+__global__ void __launch_bounds__(kQuantThreads, 2)
+    quantize_loops_kernel(const __grid_constant__ QuantLoopsParams p) {
+  constexpr int P = D / 32;
+  constexpr int RPW = 32 / P;
+  const int side = blockIdx.y;
+  const uint16_t* xs = p.x[side];
+  if (xs == nullptr) return;
+  const int lane = threadIdx.x & 31;
+  const int slice = lane % P;
+  const int64_t total = static_cast<int64_t>(p.bh) * p.n;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kQuantThreads / 32);
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) +
+                       (threadIdx.x >> 5);
+  const int a = p.nloops - 1;
+  for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
+    const int64_t row = base + lane / P;
+    const bool active = row < total;
+    const int64_t r_in = active ? row : 0;
+    const int64_t bhi = active ? row / p.n : 0;
+    const int64_t t = p.t0 + (active ? row % p.n : 0);
+    float ref[32], z[32];
+    load_rotate<D>(xs + (static_cast<int64_t>(a) * total + r_in) * D, active, slice, p.rot_scale,
+                   z);
+    quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, z, slice, active, ref);
+    for (int k = 0; k < a; ++k) {
+      const int r = p.chained ? a - 1 - k : k;
+      const Comp& c = p.dst[side][r];
+      load_rotate<D>(xs + (static_cast<int64_t>(r) * total + r_in) * D, active, slice,
+                     p.rot_scale, z);
+      const __nv_bfloat16 ab = ls_residual<D>(z, ref);
+      if (active && slice == 0)
+        *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
+                   static_cast<int>(t % kBlock)) = __bfloat16_as_ushort(ab);
+      float lv[32];
+      quantize_comp<D>(c, bhi, p.nblk, t, z, slice, active, lv);
+      if (p.chained) {
+        const float at = __bfloat162float(ab);
+#pragma unroll
+        for (int ch = 0; ch < 32; ++ch) ref[ch] = __fmaf_rn(at, ref[ch], lv[ch]);
+      }
+    }
   }
 }
 
@@ -324,6 +424,19 @@ cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
   if (D == 64) return launch_q_bits<64>(p, bits, group, s);
   if (D == 128) return launch_q_bits<128>(p, bits, group, s);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quantize_loops(const QuantLoopsParams& p, int D, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(p.bh) * p.n;
+  if (rows == 0) return cudaSuccess;
+  const dim3 grid(quant_grid(rows, D), 2);
+  if (D == 64)
+    quantize_loops_kernel<64><<<grid, kQuantThreads, 0, s>>>(p);
+  else if (D == 128)
+    quantize_loops_kernel<128><<<grid, kQuantThreads, 0, s>>>(p);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s) {

@@ -34,6 +34,7 @@ SYMBOLS = (
     "rq_dequantize", "rq_decode_workspace_bytes", "rq_decode_workspace_init",
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
     "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
+    "rq_quantize_append_loops",
 )
 
 
@@ -90,6 +91,7 @@ def load() -> ctypes.CDLL:
         "rq_cache_bind": ([LP, _P, _P, CP], ctypes.c_int),
         "rq_quantize_anchor": ([CP, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_residual": ([CP, _I32, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
+        "rq_quantize_append_loops": ([CP, _I32, _P, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_dequantize": ([CP, _I32, _I32, _I32, _I32, _I32, _P, _P], ctypes.c_int),
         "rq_decode_workspace_bytes": ([LP, _I32], _U64),
         "rq_decode_workspace_init": ([_P, _U64, _P], ctypes.c_int),
@@ -187,6 +189,15 @@ def rq_quantize_append_residual(cache: rq_cache, layer: int, kv: int, loop: int,
                                 n: int, stream=None) -> None:
     _check(load().rq_quantize_append_residual(ctypes.byref(cache), layer, kv, loop, _ptr(x), t0,
                                               n, _stream(stream)), "rq_quantize_append_residual")
+
+
+def rq_quantize_append_loops(cache: rq_cache, layer: int, xk, xv, t0: int, n: int,
+                             stream=None) -> None:
+    """xk, xv: bf16 [num_loops, batch, kv_heads, n, head_dim] device tensors (or None)."""
+    _check(load().rq_quantize_append_loops(ctypes.byref(cache), layer,
+                                           None if xk is None else _ptr(xk),
+                                           None if xv is None else _ptr(xv), t0, n,
+                                           _stream(stream)), "rq_quantize_append_loops")
 
 
 def rq_dequantize(cache: rq_cache, layer: int, kv: int, loop: int, t0: int, n: int, out,

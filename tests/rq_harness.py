@@ -47,11 +47,13 @@ class GpuCache:
 
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
                     keep_inputs: bool = True, tokens: Optional[int] = None,
-                    max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None
-                    ) -> GpuCache:
+                    max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
+                    fused: bool = False) -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
-    the C ABI in the order the policy requires.  append_chunks splits the
-    token range into consecutive appends (e.g. prefill then single tokens)."""
+    the C ABI in the order the policy requires (fused: every loop and both
+    sides of a chunk in one rq_quantize_append_loops call).  append_chunks
+    splits the token range into consecutive appends (e.g. prefill then
+    single tokens)."""
     T = w.tokens if tokens is None else tokens
     lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens)
     nbytes = L.rq_cache_bytes(lay)
@@ -63,6 +65,20 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
     bounds = [0] + list(np.cumsum(append_chunks)) if append_chunks else [0, T]
     assert bounds[-1] == T
     for layer in layers:
+        if fused:
+            xs = {(side, loop): synth.kv_full(w, layer, side, loop, 0, T, device="cuda", chunk_b=4)
+                  for side in SIDES for loop in range(w.loops)}
+            for a, b in zip(bounds[:-1], bounds[1:]):
+                if b == a:
+                    continue
+                xk, xv = (torch.stack([xs[(side, loop)][:, :, a:b] for loop in range(w.loops)])
+                          .contiguous() for side in SIDES)
+                L.rq_quantize_append_loops(cache, layer, xk, xv, a, b - a)
+            if keep_inputs:
+                for (side, loop), x in xs.items():
+                    inputs[(layer, side, loop)] = x
+            del xs
+            continue
         for side in SIDES:
             xs = {loop: synth.kv_full(w, layer, side, loop, 0, T, device="cuda", chunk_b=4)
                   for loop in range(w.loops)}

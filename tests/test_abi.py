@@ -97,6 +97,14 @@ def test_host_checks_reject_before_launch(L):
     with pytest.raises(L.RQError) as e:
         L.rq_quantize_append_residual(cache, 0, 0, 3, 1 << 12, 0, 2, stream=0)   # 3 is the anchor
     assert e.value.status == L.RQ_ERR_INVALID_ARG
+    for args, status in [((0, None, None, 0, 2), L.RQ_ERR_INVALID_ARG),      # no side
+                         ((0, 1 << 12, None, 90, 20), L.RQ_ERR_CAPACITY),
+                         ((1, 1 << 12, 1 << 13, 0, 2), L.RQ_ERR_INVALID_ARG),  # layer
+                         ((0, None, (1 << 12) + 8, 0, 2), L.RQ_ERR_INVALID_ARG),
+                         ((0, 1 << 12, None, -3, 2), L.RQ_ERR_INVALID_ARG)]:
+        with pytest.raises(L.RQError) as e:
+            L.rq_quantize_append_loops(cache, *args, stream=0)
+        assert e.value.status == status, args
     with pytest.raises(L.RQError) as e:
         L.rq_decode_attention(cache, 0, 0, 256, 256, 101, 256, 256, 0.0, 256, 256, 1 << 30,
                               stream=0)

@@ -133,3 +133,56 @@ def test_dequantize_matches_oracle(cuda_dev):
                 ref = ref[:, :, 25:125]
                 err = np.max(np.abs(out.cpu().numpy() - ref))
                 assert err <= 2e-6 * np.max(np.abs(ref)) + 1e-7, (policy, side, loop, err)
+
+
+# ---- every loop of a layer, both sides, in one launch (rq_quantize_append_loops)
+
+@pytest.mark.parametrize("bits,group,policy", [
+    ((2, 2, 2, 4), (32, 32, 32, 32), "last"),
+    ((4, 2, 2, 4), (32, 32, 32, 32), "last"),
+    ((2, 2, 2, 4), (16, 16, 16, 32), "last"),
+    ((2, 2, 4, 4), (64, 64, 16, 16), "next"),
+    ((2, 2, 2, 4), (128, 32, 64, 128), "next"),
+])
+def test_fused_loops_bit_exact(cuda_dev, bits, group, policy):
+    """One launch per chunk stores the bits of the per-loop path: codes,
+    metadata and LS coefficients of every loop against the oracle."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=203, bits=bits, group=group)
+    gc = build_gpu_cache(w, policy=policy, fused=True)
+    _check_all(gc)
+
+
+def test_fused_loops_head_dim_64_deep_chain(cuda_dev):
+    w = synth.WORKLOADS["huginn_deep"].replace(batch=1, heads=3, tokens=77, head_dim=64, loops=5,
+                                               bits=(2, 2, 4, 2, 4), group=(32, 16, 64, 64, 32),
+                                               sigma=(0.4, 0.3, 0.2, 0.1))
+    gc = build_gpu_cache(w, policy="next", fused=True)
+    _check_all(gc)
+
+
+def test_fused_single_token_appends(cuda_dev):
+    """Prefill then single-token appends of every loop (the decode step's
+    append) through the fused entry point."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=2, tokens=133)
+    gc = build_gpu_cache(w, append_chunks=[128, 1, 1, 3], fused=True)
+    _check_all(gc)
+
+
+def test_fused_one_side_leaves_the_other(cuda_dev):
+    """xv = NULL appends K only: K matches the oracle over the longer sequence
+    and the V cache bytes are untouched."""
+    import residual_bit_kv_b200.librq as L
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=2, tokens=64)
+    gc = build_gpu_cache(w, fused=True, max_tokens=128)
+    before = gc.vbuf.clone()
+    xk = torch.stack([synth.kv_full(w, 0, synth.SIDE_K, l, 64, 66, device="cuda")
+                      for l in range(w.loops)]).contiguous()
+    L.rq_quantize_append_loops(gc.cache, 0, xk, None, 64, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(before, gc.vbuf)
+    w66 = w.replace(tokens=66)
+    encs, _ = oracle_encode(w66, 0, synth.SIDE_K, [0], [0, 1], 0, 66, "last")
+    for loop in range(w.loops):
+        g = gpu_component(gc, 0, synth.SIDE_K, loop)
+        g = {k: (None if v is None else v[:, :, :66]) for k, v in g.items()}
+        assert_component_equal(g, encs[loop], None, f"K loop {loop}")
