@@ -264,6 +264,16 @@ def quant_call_bytes(w, loop, n):
     return rows * (2 * D + out + ref)
 
 
+def quant_loops_bytes(w, n):
+    """Algorithmic bytes of one fused call (every loop, one side) over n tokens:
+    the bf16 input of every loop and the packed output; nothing is re-read."""
+    rows = w.batch * w.heads * n
+    D = w.head_dim
+    A = w.loops - 1
+    return rows * sum(2 * D + D * w.bits[l] // 8 + (D // w.group[l]) * 4 + (2 if l != A else 0)
+                      for l in range(w.loops))
+
+
 # --------------------------------------------------------------- rq engine --
 
 class Engine:
@@ -759,6 +769,13 @@ def bench_quantize(dev, stream, args, hbm):
     ms = timed(one, args.steps, args.warmup, stream)
     one(True)
     torch.cuda.synchronize()
+    # every loop of both sides in one launch (rq_quantize_append_loops)
+    xk = torch.stack([xs[(0, l)] for l in range(w.loops)]).contiguous()
+    xv = torch.stack([xs[(1, l)] for l in range(w.loops)]).contiguous()
+    del xs
+    fused_ms = timed(lambda: L.rq_quantize_append_loops(cache, 0, xk, xv, 0, T, stream),
+                     args.steps, args.warmup, stream)
+    fused_bytes = 2 * quant_loops_bytes(w, T)
     inp = 2 * w.loops * w.batch * w.heads * T * w.head_dim * 2
     req = 2 * sum(quant_call_bytes(w, l, T) for l in range(w.loops))
     kern_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
@@ -770,7 +787,11 @@ def bench_quantize(dev, stream, args, hbm):
             "required_gbs": req / (kern_ms * 1e-3) / 1e9,
             "frac_of_hbm": req / (kern_ms * 1e-3) / 1e9 / hbm,
             "residual_kernel_gbs": res_bytes / (res_ms * 1e-3) / 1e9,
-            "residual_codes_per_pass": 2 * (w.loops - 1) * w.batch * w.heads * T * w.head_dim}
+            "residual_codes_per_pass": 2 * (w.loops - 1) * w.batch * w.heads * T * w.head_dim,
+            "fused": {"ms_per_pass": fused_ms, "bytes_per_pass": fused_bytes,
+                      "gbs": fused_bytes / (fused_ms * 1e-3) / 1e9,
+                      "frac_of_hbm": fused_bytes / (fused_ms * 1e-3) / 1e9 / hbm,
+                      "note": "every loop, K and V, one launch; the anchor is not re-read"}}
 
 
 if __name__ == "__main__":

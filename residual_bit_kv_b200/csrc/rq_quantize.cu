@@ -6,7 +6,10 @@
 //
 // Thread mapping: a row (one token of one head, D channels) is owned by
 // P = D/32 consecutive lanes; lane `slice` of the row holds channels
-// [32*slice, 32*slice + 32) in registers.  The Hadamard transform runs its
+// [32*slice, 32*slice + 32) in registers as 16 packed fp32 pairs
+// v[k] = (channel k, channel k + 16) of the slice, so that the butterflies,
+// the scaling, the residual and the quantisation run as packed fp32
+// operations (each element of a pair rounded exactly as its scalar op).  The Hadamard transform runs its
 // first five butterfly stages inside the lane and the remaining log2(P)
 // stages across lanes with xor-shuffles; group min/max and the two dot
 // products of the LS coefficient are lane-serial followed by xor-shuffle
@@ -24,39 +27,90 @@ namespace rq {
 namespace {
 
 constexpr int kQuantThreads = 256;
+constexpr float kRoundMagic = 12582912.0f;       // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 
-// Normalised-free Sylvester-Hadamard butterflies over one row held as
-// P x 32 registers (lane `slice` holds channels 32*slice .. 32*slice+31).
+// Channel k of a slice held as pairs v[k mod 16].(x if k < 16 else y).
+__device__ __forceinline__ float ch_of(const float2 (&v)[16], int k) {
+  return k < 16 ? v[k].x : v[k - 16].y;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);   // RN(a - b)
+}
+
+// Normalisation-free Sylvester-Hadamard butterflies over one row (stages
+// h = 1, 2, ..., D/2 in order): h = 1..8 pair-wise on v, h = 16 inside each
+// pair, h >= 32 across lanes by xor shuffles.
 template <int D>
-__device__ __forceinline__ void fwht_row(float (&z)[32], int slice) {
+__device__ __forceinline__ void fwht_row(float2 (&v)[16], int slice) {
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
+  for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2 * h) {
-#pragma unroll
-      for (int j = i; j < i + h; ++j) {
-        const float a = z[j], b = z[j + h];
-        z[j] = __fadd_rn(a, b);
-        z[j + h] = __fsub_rn(a, b);
-      }
+    for (int i = 0; i < 16; ++i) {
+      if (i & h) continue;
+      const float2 a = v[i], b = v[i + h];
+      v[i] = __fadd2_rn(a, b);
+      v[i + h] = sub2(a, b);
     }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float a = v[k].x, b = v[k].y;
+    v[k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
 #pragma unroll
   for (int hl = 1; hl < D / 32; hl <<= 1) {
-    const bool upper = (slice & hl) != 0;   // this lane holds the "a - b" half
+    // this lane holds the "a - b" half when (slice & hl): RN(s * mine + other)
+    const float sg = (slice & hl) ? -1.0f : 1.0f;
+    const float2 s2 = make_float2(sg, sg);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const float o = __shfl_xor_sync(0xffffffffu, z[k], hl);
-      z[k] = upper ? __fsub_rn(o, z[k]) : __fadd_rn(z[k], o);
+    for (int k = 0; k < 16; ++k) {
+      const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[k].x, hl),
+                                   __shfl_xor_sync(0xffffffffu, v[k].y, hl));
+      v[k] = __ffma2_rn(v[k], s2, o);
     }
   }
+}
+
+// Row of bf16 x -> fp32 -> Z = H x (normalised) in one lane's 16 pairs.
+template <int D>
+__device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, int slice,
+                                            float rot_scale, float2 (&v)[16]) {
+  if (active) {
+    const uint4* src = reinterpret_cast<const uint4*>(xrow + slice * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = src[i];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c0 = i * 8 + 2 * j;   // channels c0, c0 + 1
+        const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+        if (c0 < 16) {
+          v[c0].x = lo;
+          v[c0 + 1].x = hi;
+        } else {
+          v[c0 - 16].y = lo;
+          v[c0 - 15].y = hi;
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = make_float2(0.0f, 0.0f);
+  }
+  fwht_row<D>(v, slice);
+  const float2 rs = make_float2(rot_scale, rot_scale);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fmul2_rn(v[k], rs);
 }
 
 // Stored levels fma(s~, code, z~) of one lane's 32 channels of a component
 // at token t of row `row`.
 template <int BITS>
 __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t row, int64_t nblk, int64_t t,
-                                            int slice, int D, float (&o)[32]) {
+                                            int slice, int D, float2 (&o)[16]) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   unsigned char* rec = comp_record(c, row, nblk, t);
   const int i = static_cast<int>(t % kBlock);
@@ -73,20 +127,20 @@ __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t row, int64_t 
     mw0 = m[slice * 2];
     mw1 = m[slice * 2 + 1];
   }
-  const float s0 = __half2float(__ushort_as_half((unsigned short)(mw0 & 0xFFFFu)));
-  const float z0 = __half2float(__ushort_as_half((unsigned short)(mw0 >> 16)));
-  const float s1 = __half2float(__ushort_as_half((unsigned short)(mw1 & 0xFFFFu)));
-  const float z1 = __half2float(__ushort_as_half((unsigned short)(mw1 >> 16)));
+  const float2 s2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 & 0xFFFFu))),
+                                __half2float(__ushort_as_half((unsigned short)(mw1 & 0xFFFFu))));
+  const float2 z2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 >> 16))),
+                                __half2float(__ushort_as_half((unsigned short)(mw1 >> 16))));
 #pragma unroll
-  for (int ch = 0; ch < 32; ++ch) {
-    const uint32_t code = (words[slice_word<BITS>(ch)] >> slice_shift<BITS>(ch)) & QMAX;
-    const float cf = static_cast<float>(code);
-    o[ch] = (ch < 16) ? __fmaf_rn(s0, cf, z0) : __fmaf_rn(s1, cf, z1);
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t c0 = (words[slice_word<BITS>(k)] >> slice_shift<BITS>(k)) & QMAX;
+    const uint32_t c1 = (words[slice_word<BITS>(k + 16)] >> slice_shift<BITS>(k + 16)) & QMAX;
+    o[k] = __ffma2_rn(s2, make_float2(static_cast<float>(c0), static_cast<float>(c1)), z2);
   }
 }
 
 __device__ __forceinline__ void deq_slice(const Comp& c, int64_t row, int64_t nblk, int64_t t,
-                                          int slice, int D, float (&o)[32]) {
+                                          int slice, int D, float2 (&o)[16]) {
   if (c.bits == 4)
     deq_slice_t<4>(c, row, nblk, t, slice, D, o);
   else
@@ -96,41 +150,63 @@ __device__ __forceinline__ void deq_slice(const Comp& c, int64_t row, int64_t nb
 // Rotated reconstruction of a chain [0 .. n-1] (anchor last) at token t of
 // row `row`: Z = deq(anchor); for k = n-2 .. 0: Z = fma(alpha~_k, Z, deq_k).
 __device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t row, int64_t nblk,
-                                            int64_t t, int slice, int D, float (&zr)[32]) {
+                                            int64_t t, int slice, int D, float2 (&zr)[16]) {
   deq_slice(comps[n - 1], row, nblk, t, slice, D, zr);
   for (int k = n - 2; k >= 0; --k) {
-    float d[32];
+    float2 d[16];
     deq_slice(comps[k], row, nblk, t, slice, D, d);
     const Comp& c = comps[k];
     const float a = bf16_bits_to_f32(
         *rec_alpha(comp_record(c, row, nblk, t), D, c.bits, c.group, static_cast<int>(t % kBlock)));
+    const float2 a2 = make_float2(a, a);
 #pragma unroll
-    for (int ch = 0; ch < 32; ++ch) zr[ch] = __fmaf_rn(a, zr[ch], d[ch]);
+    for (int j = 0; j < 16; ++j) zr[j] = __ffma2_rn(a2, zr[j], d[j]);
   }
+}
+
+// Sum over the channels of one packed word of (kRoundMagicBits << shift),
+// mod 2^32: what packing the rounded floats' bit patterns adds on top of
+// the codes.
+template <int BITS>
+__host__ __device__ constexpr uint32_t magic_pack_offset(int word) {
+  uint32_t o = 0u;
+  for (int ch = 0; ch < 32; ++ch)
+    if (slice_word<BITS>(ch) == word) o += kRoundMagicBits << slice_shift<BITS>(ch);
+  return o;
 }
 
 // Affine quantisation [RQ §2.1] of one lane's 32 values and the packed store;
 // if `levels` is given it receives the stored levels fma(s~, code, z~) (what
-// a reader of the record reconstructs).
+// a reader of the record reconstructs).  Group parts: channels 0-15 (.x)
+// and 16-31 (.y) for g = 16, the whole slice (or several lanes) otherwise.
 template <int D, int BITS, int G>
-__device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
-                                               bool active, uint32_t* codes_row,
-                                               uint32_t* meta_row, float* levels = nullptr) {
+__device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice, bool active,
+                                               uint32_t* codes_row, uint32_t* meta_row,
+                                               float2* levels = nullptr) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
-  constexpr int GL = G < 32 ? G : 32;    // group part held by this lane
-  constexpr int NG = 32 / GL;            // group parts per lane
+  constexpr int NG = G < 32 ? 2 : 1;        // group parts per lane
   constexpr int LPG = G > 32 ? G / 32 : 1;  // lanes sharing a group
-  uint32_t words[BITS];
-#pragma unroll
-  for (int i = 0; i < BITS; ++i) words[i] = 0u;
-  uint32_t metaw[NG];
+  float st[2], zt[2], inv[2];
+  uint32_t metaw[2];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
-    float mn = z[gi * GL], mx = z[gi * GL];
+    float mn, mx;
+    if constexpr (NG == 2) {
+      mn = mx = gi == 0 ? v[0].x : v[0].y;
 #pragma unroll
-    for (int k = 1; k < GL; ++k) {
-      mn = fminf(mn, z[gi * GL + k]);
-      mx = fmaxf(mx, z[gi * GL + k]);
+      for (int k = 1; k < 16; ++k) {
+        const float e = gi == 0 ? v[k].x : v[k].y;
+        mn = fminf(mn, e);
+        mx = fmaxf(mx, e);
+      }
+    } else {
+      mn = fminf(v[0].x, v[0].y);
+      mx = fmaxf(v[0].x, v[0].y);
+#pragma unroll
+      for (int k = 1; k < 16; ++k) {
+        mn = fminf(mn, fminf(v[k].x, v[k].y));
+        mx = fmaxf(mx, fmaxf(v[k].x, v[k].y));
+      }
     }
 #pragma unroll
     for (int off = 1; off < LPG; off <<= 1) {
@@ -142,21 +218,39 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
     const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
     const __half sh = __float2half_rn(s);
     const __half zh = __float2half_rn(mn);
-    const float st = __half2float(sh);
-    const float zt = __half2float(zh);
-    const float inv = (st > 0.0f) ? __fdiv_rn(1.0f, st) : 0.0f;
+    st[gi] = __half2float(sh);
+    zt[gi] = __half2float(zh);
+    inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
     metaw[gi] = static_cast<uint32_t>(__half_as_ushort(sh)) |
                 (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
+  }
+  if constexpr (NG == 1) {
+    st[1] = st[0];
+    zt[1] = zt[0];
+    inv[1] = inv[0];
+  }
+  const float2 nz = make_float2(-zt[0], -zt[1]), iv = make_float2(inv[0], inv[1]);
+  const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+  uint32_t words[BITS];
 #pragma unroll
-    for (int k = 0; k < GL; ++k) {
-      const int ch = gi * GL + k;
-      float u = __fmul_rn(__fsub_rn(z[ch], zt), inv);
-      u = fminf(fmaxf(u, 0.0f), static_cast<float>(QMAX));
-      // u + 1.5*2^23 rounds u to the nearest integer, ties to even, and
-      // leaves that integer in the low mantissa bits.
-      const uint32_t code = __float_as_uint(__fadd_rn(u, 12582912.0f)) & QMAX;
-      words[slice_word<BITS>(ch)] |= code << slice_shift<BITS>(ch);
-      if (levels != nullptr) levels[ch] = __fmaf_rn(st, static_cast<float>(code), zt);
+  for (int i = 0; i < BITS; ++i) words[i] = 0u - magic_pack_offset<BITS>(i);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    // u = (x - z~) * (1/s~), clamped to [0, 2^b - 1]; u + 1.5 * 2^23 rounds it
+    // to the nearest integer (ties to even), held in the low mantissa bits
+    // of a float whose bit pattern is kRoundMagicBits + code.
+    float2 u = __fmul2_rn(__fadd2_rn(v[k], nz), iv);
+    u.x = fminf(fmaxf(u.x, 0.0f), static_cast<float>(QMAX));
+    u.y = fminf(fmaxf(u.y, 0.0f), static_cast<float>(QMAX));
+    const float2 r = __fadd2_rn(u, mg);
+    const uint32_t b0 = __float_as_uint(r.x), b1 = __float_as_uint(r.y);
+    // packing: + (kRoundMagicBits + code) << shift (the offsets were
+    // subtracted up front), as integer multiply-adds
+    words[slice_word<BITS>(k)] += b0 << slice_shift<BITS>(k);
+    words[slice_word<BITS>(k + 16)] += b1 << slice_shift<BITS>(k + 16);
+    if (levels != nullptr) {
+      const float2 cf = __fadd2_rn(r, make_float2(-kRoundMagic, -kRoundMagic));   // exact codes
+      levels[k] = __ffma2_rn(make_float2(st[0], st[1]), cf, make_float2(zt[0], zt[1]));
     }
   }
   if (!active) return;
@@ -175,42 +269,19 @@ __device__ __forceinline__ void quantize_store(const float (&z)[32], int slice,
   }
 }
 
-// Row of bf16 x -> fp32 -> Z = H x (normalised) in one lane's 32 registers.
-template <int D>
-__device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, int slice,
-                                            float rot_scale, float (&z)[32]) {
-  if (active) {
-    const uint4* src = reinterpret_cast<const uint4*>(xrow + slice * 32);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = src[i];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        z[i * 8 + 2 * j] = __uint_as_float(w[j] << 16);
-        z[i * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) z[k] = 0.0f;
-  }
-  fwht_row<D>(z, slice);
-#pragma unroll
-  for (int k = 0; k < 32; ++k) z[k] = __fmul_rn(z[k], rot_scale);
-}
-
 // Least-squares coefficient of z against the reference over the row
 // [RQ §3.2 scaling coefficient, App. G.1]: alpha~ = bf16(<z, ref> / <ref, ref>)
 // (0 for a zero reference); z becomes the residual fma(-alpha~, ref, z).
+// The dots run lane-serially in channel order, then across the row's lanes.
 template <int D>
-__device__ __forceinline__ __nv_bfloat16 ls_residual(float (&z)[32], const float (&ref)[32]) {
+__device__ __forceinline__ __nv_bfloat16 ls_residual(float2 (&v)[16], const float2 (&ref)[16]) {
   constexpr int P = D / 32;
   float dzr = 0.0f, drr = 0.0f;
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
-    dzr = __fmaf_rn(z[k], ref[k], dzr);
-    drr = __fmaf_rn(ref[k], ref[k], drr);
+    const float z = ch_of(v, k), r = ch_of(ref, k);
+    dzr = __fmaf_rn(z, r, dzr);
+    drr = __fmaf_rn(r, r, drr);
   }
 #pragma unroll
   for (int off = P / 2; off >= 1; off >>= 1) {
@@ -220,8 +291,9 @@ __device__ __forceinline__ __nv_bfloat16 ls_residual(float (&z)[32], const float
   const float a = (drr > 0.0f) ? __fdiv_rn(dzr, drr) : 0.0f;
   const __nv_bfloat16 ab = __float2bfloat16_rn(a);
   const float at = __bfloat162float(ab);
+  const float2 na = make_float2(-at, -at);
 #pragma unroll
-  for (int k = 0; k < 32; ++k) z[k] = __fmaf_rn(-at, ref[k], z[k]);
+  for (int k = 0; k < 16; ++k) v[k] = __ffma2_rn(na, ref[k], v[k]);
   return ab;
 }
 
@@ -239,8 +311,8 @@ __global__ void __launch_bounds__(kQuantThreads)
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    float z[32];
-    load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, z);
+    float2 v[16];
+    load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
 
     const int64_t bhi = active ? row / p.n : 0;
     const int64_t t = p.t0 + (active ? row % p.n : 0);
@@ -248,21 +320,21 @@ __global__ void __launch_bounds__(kQuantThreads)
     if (p.dst.has_alpha) {
       // Least-squares coefficient against the reconstructed reference
       // [RQ §3.2 scaling coefficient, App. G.1], then the residual.
-      float ref[32];
+      float2 ref[16];
       if (active) {
         chain_slice(p.ref, p.nref, bhi, p.nblk, t, slice, D, ref);
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) ref[k] = 0.0f;
+        for (int k = 0; k < 16; ++k) ref[k] = make_float2(0.0f, 0.0f);
       }
-      const __nv_bfloat16 ab = ls_residual<D>(z, ref);
+      const __nv_bfloat16 ab = ls_residual<D>(v, ref);
       if (active && slice == 0)
         *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock)) =
             __bfloat16_as_ushort(ab);
     }
     unsigned char* rec = comp_record(p.dst, bhi, p.nblk, t);
     const int i = static_cast<int>(t % kBlock);
-    quantize_store<D, BITS, G>(z, slice, active, rec_codes(rec, D, BITS, i),
+    quantize_store<D, BITS, G>(v, slice, active, rec_codes(rec, D, BITS, i),
                                rec_meta(rec, D, BITS, G, i));
   }
 }
@@ -271,24 +343,24 @@ __global__ void __launch_bounds__(kQuantThreads)
 // metadata and (if `levels`) the stored levels of this lane's 32 channels.
 template <int D>
 __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_t nblk, int64_t t,
-                                              const float (&z)[32], int slice, bool active,
-                                              float* levels) {
+                                              const float2 (&v)[16], int slice, bool active,
+                                              float2* levels) {
   unsigned char* rec = comp_record(c, row, nblk, t);
   const int i = static_cast<int>(t % kBlock);
   uint32_t* cw = rec_codes(rec, D, c.bits, i);
   uint32_t* mw = rec_meta(rec, D, c.bits, c.group, i);
   const int key = c.bits * 1000 + c.group;
   switch (key) {
-    case 2016: quantize_store<D, 2, 16>(z, slice, active, cw, mw, levels); break;
-    case 2032: quantize_store<D, 2, 32>(z, slice, active, cw, mw, levels); break;
-    case 2064: quantize_store<D, 2, 64>(z, slice, active, cw, mw, levels); break;
-    case 4016: quantize_store<D, 4, 16>(z, slice, active, cw, mw, levels); break;
-    case 4032: quantize_store<D, 4, 32>(z, slice, active, cw, mw, levels); break;
-    case 4064: quantize_store<D, 4, 64>(z, slice, active, cw, mw, levels); break;
+    case 2016: quantize_store<D, 2, 16>(v, slice, active, cw, mw, levels); break;
+    case 2032: quantize_store<D, 2, 32>(v, slice, active, cw, mw, levels); break;
+    case 2064: quantize_store<D, 2, 64>(v, slice, active, cw, mw, levels); break;
+    case 4016: quantize_store<D, 4, 16>(v, slice, active, cw, mw, levels); break;
+    case 4032: quantize_store<D, 4, 32>(v, slice, active, cw, mw, levels); break;
+    case 4064: quantize_store<D, 4, 64>(v, slice, active, cw, mw, levels); break;
     default:
       if constexpr (D >= 128) {
-        if (key == 2128) quantize_store<D, 2, 128>(z, slice, active, cw, mw, levels);
-        else if (key == 4128) quantize_store<D, 4, 128>(z, slice, active, cw, mw, levels);
+        if (key == 2128) quantize_store<D, 2, 128>(v, slice, active, cw, mw, levels);
+        else if (key == 4128) quantize_store<D, 4, 128>(v, slice, active, cw, mw, levels);
       }
       break;
   }
@@ -323,25 +395,26 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     const int64_t r_in = active ? row : 0;
     const int64_t bhi = active ? row / p.n : 0;
     const int64_t t = p.t0 + (active ? row % p.n : 0);
-    float ref[32], z[32];
+    float2 ref[16], v[16];
     load_rotate<D>(xs + (static_cast<int64_t>(a) * total + r_in) * D, active, slice, p.rot_scale,
-                   z);
-    quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, z, slice, active, ref);
+                   v);
+    quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, v, slice, active, ref);
     for (int k = 0; k < a; ++k) {
       const int r = p.chained ? a - 1 - k : k;
       const Comp& c = p.dst[side][r];
       load_rotate<D>(xs + (static_cast<int64_t>(r) * total + r_in) * D, active, slice,
-                     p.rot_scale, z);
-      const __nv_bfloat16 ab = ls_residual<D>(z, ref);
+                     p.rot_scale, v);
+      const __nv_bfloat16 ab = ls_residual<D>(v, ref);
       if (active && slice == 0)
         *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
                    static_cast<int>(t % kBlock)) = __bfloat16_as_ushort(ab);
-      float lv[32];
-      quantize_comp<D>(c, bhi, p.nblk, t, z, slice, active, lv);
+      float2 lv[16];
+      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, lv);
       if (p.chained) {
         const float at = __bfloat162float(ab);
+        const float2 a2 = make_float2(at, at);
 #pragma unroll
-        for (int ch = 0; ch < 32; ++ch) ref[ch] = __fmaf_rn(at, ref[ch], lv[ch]);
+        for (int j = 0; j < 16; ++j) ref[j] = __ffma2_rn(a2, ref[j], lv[j]);
       }
     }
   }
@@ -361,21 +434,22 @@ __global__ void __launch_bounds__(kQuantThreads)
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    float z[32];
+    float2 v[16];
     if (active) {
-      chain_slice(p.comp, p.ncomp, row / p.n, p.nblk, p.t0 + row % p.n, slice, D, z);
+      chain_slice(p.comp, p.ncomp, row / p.n, p.nblk, p.t0 + row % p.n, slice, D, v);
     } else {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = 0.0f;
+      for (int k = 0; k < 16; ++k) v[k] = make_float2(0.0f, 0.0f);
     }
     // X^ = H^T Z^ = H Z^ (the normalised Sylvester matrix is symmetric).
-    fwht_row<D>(z, slice);
+    fwht_row<D>(v, slice);
     if (active) {
+      const float rs = p.rot_scale;
       float4* dst = reinterpret_cast<float4*>(p.out + row * D + slice * 32);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        dst[i] = make_float4(z[4 * i] * p.rot_scale, z[4 * i + 1] * p.rot_scale,
-                             z[4 * i + 2] * p.rot_scale, z[4 * i + 3] * p.rot_scale);
+        dst[i] = make_float4(ch_of(v, 4 * i) * rs, ch_of(v, 4 * i + 1) * rs,
+                             ch_of(v, 4 * i + 2) * rs, ch_of(v, 4 * i + 3) * rs);
     }
   }
 }
