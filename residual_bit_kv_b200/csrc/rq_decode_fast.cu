@@ -22,10 +22,21 @@
 // weights p_t * kappa * s~ * 2^(109-p) accumulate p_t * kappa * s~ * c * 2^-40
 // per channel, the offsets z~ going to separate accumulators.  Accumulation
 // is in the rotated domain; H^T is applied once in the merge.
+#include <type_traits>
+
 #include "rq_decode_common.cuh"
 
 namespace rq {
 namespace {
+
+// Shared-memory atomic add returning the old value (one lane; no warp
+// aggregation).
+__device__ __forceinline__ uint32_t atom_add_shared(uint32_t* a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(a)), "r"(v)
+               : "memory");
+  return old;
+}
 
 constexpr int kWarps = 8;                      // BF16 kernel: compute warps per CTA
 constexpr int kThreads = (kWarps + 1) * 32;    // + producer warp
@@ -229,32 +240,63 @@ __device__ __forceinline__ void vacc(const unsigned char* rec, int jl, int slice
 }
 
 // Components of a chain, unrolled at compile time: [own residual, ..., anchor].
-template <class SP, int C = 0>
-__device__ __forceinline__ void score_comps(const unsigned char* st, int j, int slice,
+// Components of a chain, unrolled at compile time: [own residual, ..., anchor].
+// REC is the stage record (compile-time), jl the token inside it.
+template <class SP, int REC, int C = 0>
+__device__ __forceinline__ void score_comps(const unsigned char* st, int rl, int jl, int slice,
                                             const QLimbs& ql, float& part, float& kap) {
   if constexpr (C < SP::NC) {
     using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
-    const unsigned char* rec = SP::rec(st, 0, C, j);
-    const int jl = SP::RPS == 1 ? j : j % kBlock;
+    const unsigned char* rec = st + SP::comp_off(0, C) + (REC + rl) * SP::rec_bytes(C);
     const float d = kdot<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, ql);
     part = fmaf(kap, d, part);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
-    score_comps<SP, C + 1>(st, j, slice, ql, part, kap);
+    score_comps<SP, REC, C + 1>(st, rl, jl, slice, ql, part, kap);
   }
 }
 
-template <class SP, int C = 0>
-__device__ __forceinline__ void value_comps(const unsigned char* st, int j, int slice, float kap,
-                                            VAcc& va) {
+template <class SP, int REC, int C = 0>
+__device__ __forceinline__ void value_comps(const unsigned char* st, int rl, int jl, int slice,
+                                            float kap, VAcc& va) {
   if constexpr (C < SP::NC) {
     using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
-    const unsigned char* rec = SP::rec(st, 1, C, j);
-    const int jl = SP::RPS == 1 ? j : j % kBlock;
+    const unsigned char* rec = st + SP::comp_off(1, C) + (REC + rl) * SP::rec_bytes(C);
     vacc<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, kap, va);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
-    value_comps<SP, C + 1>(st, j, slice, kap, va);
+    value_comps<SP, REC, C + 1>(st, rl, jl, slice, kap, va);
+  }
+}
+
+// The TT tokens of one chunk held by this thread.  Token tt of the thread is
+// stage token tt * TPC + jr: record tt * TPC / 32 + rl (rl = jr / 32, zero
+// when a CTA pass is one record), row jl = jr % 32.  MASK: the chunk may end
+// before TC tokens (nt < TC); full chunks skip the per-token tests.
+template <class SP, int TT, int TPC, int P, bool MASK, int TTI = 0>
+__device__ __forceinline__ void chunk_scores(const unsigned char* st, int jr, int rl, int jl,
+                                             int slice, const QLimbs& ql, float sigma, int nt,
+                                             float (&sc)[TT]) {
+  if constexpr (TTI < TT) {
+    float part = 0.0f, kap = 1.0f;
+    score_comps<SP, TTI * TPC / kBlock>(st, rl, jl, slice, ql, part, kap);
+#pragma unroll
+    for (int off = P / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    sc[TTI] = (!MASK || TTI * TPC + jr < nt) ? part * sigma : kNegInf;
+    chunk_scores<SP, TT, TPC, P, MASK, TTI + 1>(st, jr, rl, jl, slice, ql, sigma, nt, sc);
+  }
+}
+
+template <class SP, int TT, int TPC, bool MASK, int TTI = 0>
+__device__ __forceinline__ void chunk_values(const unsigned char* st, int rl, int jl, int slice,
+                                             const float (&sc)[TT], float m, float& l, VAcc& va) {
+  if constexpr (TTI < TT) {
+    if (!MASK || sc[TTI] != kNegInf) {
+      const float pt = fast_exp2(sc[TTI] - m);
+      l += pt;
+      value_comps<SP, TTI * TPC / kBlock>(st, rl, jl, slice, pt, va);
+    }
+    chunk_values<SP, TT, TPC, MASK, TTI + 1>(st, rl, jl, slice, sc, m, l, va);
   }
 }
 
@@ -436,23 +478,14 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   va.cst[0] = va.cst[1] = va.cst[2] = 0.0f;
   float m = kNegInf, l = 0.0f;
 
-  int s = 0;
-  uint32_t phase = 0u;
-  for (int i = 0; i < R.nchunks; ++i) {
-    if (!mbar_wait(&full_bar[s], phase, p.err)) s_abort = 1;
-    if (s_abort) break;
-    const unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
-    const int nt = min(TC, R.t_end - (R.t_begin + i * TC));
+  // This thread's tokens: jr inside a CTA pass of TPC tokens.
+  const int jr = warp * TPW + tw;
+  const int rl = TPC == kBlock ? 0 : jr / kBlock;
+  const int jl = jr % kBlock;
+  auto chunk = [&](const unsigned char* st, auto mask_tag, int nt) {
+    constexpr bool MASK = decltype(mask_tag)::value;
     float sc[TT];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const int j = tt * TPC + warp * TPW + tw;
-      float part = 0.0f, kap = 1.0f;
-      score_comps<SP>(st, j, slice, ql, part, kap);
-#pragma unroll
-      for (int off = P / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      sc[tt] = (j < nt) ? part * sigma : kNegInf;
-    }
+    chunk_scores<SP, TT, TPC, P, MASK>(st, jr, rl, jl, slice, ql, sigma, nt, sc);
     float mc = sc[0];
 #pragma unroll
     for (int tt = 1; tt < TT; ++tt) mc = fmaxf(mc, sc[tt]);
@@ -462,23 +495,30 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
       rescale(va, f);
       m = mc;
     }
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const int j = tt * TPC + warp * TPW + tw;
-      if (sc[tt] == kNegInf) continue;
-      const float pt = fast_exp2(sc[tt] - m);
-      l += pt;
-      value_comps<SP>(st, j, slice, pt, va);
+    chunk_values<SP, TT, TPC, MASK>(st, rl, jl, slice, sc, m, l, va);
+  };
+  int s = 0;
+  uint32_t phase = 0u;
+  for (int i = 0; i < R.nchunks; ++i) {
+    if (!mbar_wait(&full_bar[s], phase, p.err)) {
+      s_abort = 1;   // this warp stops; the others stop at their own timeout
+      break;
     }
+    const unsigned char* st = smem + static_cast<size_t>(s) * SP::stage_bytes();
+    const int nt = R.t_end - (R.t_begin + i * TC);
+    if (nt >= TC)
+      chunk(st, std::integral_constant<bool, false>{}, TC);
+    else
+      chunk(st, std::integral_constant<bool, true>{}, nt);
     // Release the stage; the last warp to do so refills it.
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
-      const uint32_t r = atomicAdd(&s_release[s], 1u);
+      const uint32_t r = atom_add_shared(&s_release[s], 1u);
       if (r % kCWarps == kCWarps - 1 && i + S < R.nchunks && !s_abort) {
         __threadfence_block();
         issue(i + S, s);
-        atomicAdd(&s_issued, 1);
+        atom_add_shared(reinterpret_cast<uint32_t*>(&s_issued), 1u);
       }
     }
     if (++s == S) {
@@ -489,15 +529,16 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   float acc[32];
   uint32_t range_err = 0u;
   finish_values(va, acc, range_err);
-  if (range_err && !s_abort) atomicOr(p.err, kErrRange);
-  if (s_abort) {
+  __syncthreads();   // every warp has left the loop: s_abort is settled
+  const bool aborted = s_abort != 0;
+  if (range_err && !aborted) atomicOr(p.err, kErrRange);
+  if (aborted) {
     m = kNegInf;
     l = 0.0f;
 #pragma unroll
     for (int k = 0; k < 32; ++k) acc[k] = 0.0f;
+    if (t == 0) drain(s_issued, S, full_bar, p.err);
   }
-  __syncthreads();
-  if (s_abort && t == 0) drain(s_issued, S, full_bar, p.err);
   __syncthreads();
   finish_split<D, kCThreads, NSLOT, true>(m, l, acc, slice, warp * TPW + tw,
                                           reinterpret_cast<float*>(smem), bhi, split, p.splits,
