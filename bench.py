@@ -410,33 +410,51 @@ def timed(fn, steps, warmup, stream, dist=None):
 
 # --------------------------------------------------------- oracle (CPU) legs --
 
-def oracle_decode_sample(w, pairs, loops, budget_s=None):
-    """Times the oracle's decode of (b, h) units for `loops` of layer 0:
-    reconstruction of every past row in fp64 and exact softmax attention.
-    Pairs are taken in order until `budget_s` seconds of timed work (all of
-    them if None).  Encoding a pair's cache is set-up, not timed."""
+def oracle_prepare(w, b, h):
+    """Set-up of one (batch, head) unit of layer 0 for the oracle: the unit's
+    K/V rows of every loop generated and encoded (not timed)."""
     import oracle
-    T = w.tokens
-    D = w.head_dim
+    T, D = w.tokens, w.head_dim
+    encs = {}
+    for side in (0, 1):
+        cs = synth.key_channel_scale(w, 0) if side == 0 else None
+        xl = [synth.bits_of(synth.kv(w, 0, side, loop, [b], [h], 0, T, "cpu", cs)).reshape(-1, D)
+              for loop in range(w.loops)]
+        encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
+    return encs
+
+
+def oracle_run(w, b, h, encs, loops, q, kc, vc):
+    """The oracle's decode of one unit for `loops`: reconstruction of every
+    past row in fp64 and exact softmax attention (the timed work)."""
+    import oracle
+    T, D = w.tokens, w.head_dim
+    for loop in loops:
+        kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(T, D)
+        vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(T, D)
+        oracle.attention(oracle.bf16_bits_to_f64(q[loop, b, h]), kh, vh,
+                         oracle.bf16_bits_to_f64(kc[loop][b, h]),
+                         oracle.bf16_bits_to_f64(vc[loop][b, h]), 1.0 / np.sqrt(D))
+    return len(loops)
+
+
+def step_inputs_cpu(w, loops):
     q = synth.bits_of(torch.stack([synth.query(w, 0, l) for l in range(w.loops)]))
     kc = {l: synth.bits_of(synth.current_token(w, 0, 0, l)) for l in loops}
     vc = {l: synth.bits_of(synth.current_token(w, 0, 1, l)) for l in loops}
+    return q, kc, vc
+
+
+def oracle_decode_sample(w, pairs, loops, budget_s=None):
+    """Times the oracle's decode of (b, h) units for `loops` of layer 0.
+    Pairs are taken in order until `budget_s` seconds of timed work (all of
+    them if None).  Encoding a pair's cache is set-up, not timed."""
+    q, kc, vc = step_inputs_cpu(w, loops)
     secs, units = 0.0, 0
     for b, h in pairs:
-        encs = {}
-        for side in (0, 1):
-            cs = synth.key_channel_scale(w, 0) if side == 0 else None
-            xl = [synth.bits_of(synth.kv(w, 0, side, loop, [b], [h], 0, T, "cpu", cs)).reshape(-1, D)
-                  for loop in range(w.loops)]
-            encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
+        encs = oracle_prepare(w, b, h)
         t0 = time.perf_counter()
-        for loop in loops:
-            kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(T, D)
-            vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(T, D)
-            oracle.attention(oracle.bf16_bits_to_f64(q[loop, b, h]), kh, vh,
-                             oracle.bf16_bits_to_f64(kc[loop][b, h]),
-                             oracle.bf16_bits_to_f64(vc[loop][b, h]), 1.0 / np.sqrt(D))
-            units += 1
+        units += oracle_run(w, b, h, encs, loops, q, kc, vc)
         secs += time.perf_counter() - t0
         if budget_s is not None and secs >= budget_s:
             break
@@ -444,6 +462,57 @@ def oracle_decode_sample(w, pairs, loops, budget_s=None):
 
 
 CPU_BASELINE_SECONDS = 10.0
+CPU_POOL_MAX_WORKERS = 64
+
+
+def _pool_worker(args):
+    """One oracle process: set-up (generation and encoding) untimed, then a
+    barrier, then the timed decode of its units.  Returns its timed window."""
+    name, (b, h), loops, barrier = args
+    w = synth.WORKLOADS[name]
+    q, kc, vc = step_inputs_cpu(w, loops)
+    encs = oracle_prepare(w, b, h)
+    oracle_run(w, b, h, encs, loops, q, kc, vc)   # warm: library load, page-in
+    barrier.wait()
+    t0 = time.perf_counter()
+    units = oracle_run(w, b, h, encs, loops, q, kc, vc)
+    t1 = time.perf_counter()
+    return t0, t1, units
+
+
+def cpu_baseline_all_cores(w):
+    """The same oracle decode run as independent processes over (batch, head)
+    units on every host core (capped at CPU_POOL_MAX_WORKERS), each unit
+    single-threaded; throughput = units / wall time of the timed windows."""
+    import multiprocessing as mp
+    ncpu = os.cpu_count() or 1
+    workers = max(1, min(ncpu, CPU_POOL_MAX_WORKERS))
+    ctx = mp.get_context("spawn")
+    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(workers)]
+    with ctx.Manager() as man:
+        barrier = man.Barrier(workers)
+        with ctx.Pool(workers) as pool:
+            res = pool.map(_pool_worker,
+                           [(w.name, pr, list(range(w.loops)), barrier) for pr in pairs])
+    t0 = min(r[0] for r in res)
+    t1 = max(r[1] for r in res)
+    units = sum(r[2] for r in res)
+    step_units = w.layers * w.loops * w.batch * w.heads
+    step_s = (t1 - t0) / units * step_units
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": workers, "nproc": ncpu,
+            "cpu_model": model, "kind": "oracle",
+            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens}, one "
+                      f"(batch,head) per process ({t1 - t0:.1f} s wall), scaled to {step_units} "
+                      f"units per step"}
 
 
 def cpu_baseline(w):
@@ -640,9 +709,10 @@ def main():
         torch.cuda.empty_cache()
         ablation = bench_ablation(dev, stream, args, hbm)
 
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         cpu = cpu_baseline(w)
+        cpu_all = cpu_baseline_all_cores(w)
 
     if rank == 0:
         value = job_tokens_per_s(ws, w.batch, ms)
@@ -672,6 +742,7 @@ def main():
             "quantize": quant,
             "ablation_shared_vs_chained": ablation,
             "cpu_baseline": cpu,
+            "cpu_baseline_all_cores": cpu_all,
         }
         print(json.dumps(line))
     if dist is not None:

@@ -90,3 +90,50 @@ def test_huginn_deep_full_size(cuda_dev, policy):
     _sampled_decode_close(gc, 0, bsel, hsel, policy, loops=[0, 3, 6, 7])
     del gc
     torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_ouro_16k_layer0_every_unit(cuda_dev):
+    """16k decode workload, layer 0 in full: every stored code and scale of both
+    sides, and the decode output of every (batch, head) for all four loops, in
+    the launch configuration the benchmark times (capacity T+16, T past tokens)."""
+    w = synth.WORKLOADS["ouro_16k"]
+    T, D = w.tokens, w.head_dim
+    gc = build_gpu_cache(w, layers=(0,), keep_inputs=True, max_tokens=T + 16)
+    ws = Workspace(gc.layout, T)
+    outs = {}
+    for loop in range(w.loops):
+        out, status = gpu_decode(gc, 0, loop, [T] * w.batch, T, ws)
+        assert status == L.RQ_OK
+        outs[loop] = out
+    hsel = list(range(w.heads))
+    q = synth.bits_of(torch.stack([synth.query(w, 0, l) for l in range(w.loops)]))
+    kc = [synth.bits_of(synth.current_token(w, 0, synth.SIDE_K, l)) for l in range(w.loops)]
+    vc = [synth.bits_of(synth.current_token(w, 0, synth.SIDE_V, l)) for l in range(w.loops)]
+    units = 0
+    for b0 in range(0, w.batch, 4):
+        bsel = list(range(b0, b0 + 4))
+        encs = {}
+        for side in SIDES:
+            xl = [synth.bits_of(gc.inputs[(0, side, l)][bsel].cpu()).reshape(-1, D)
+                  for l in range(w.loops)]
+            encs[side] = oracle.encode_side(np.stack(xl), w.bits, w.group)
+            del xl
+            for loop in range(w.loops):
+                g = gpu_component(gc, 0, side, loop, bsel, hsel)
+                g = {k: (None if v is None else v[:, :, :T]) for k, v in g.items()}
+                assert_component_equal(g, encs[side][loop], None,
+                                       f"rows {b0}.. side {side} loop {loop}")
+        bi, hi = np.ix_(bsel, hsel)
+        for loop in range(w.loops):
+            kh = oracle.reconstruct(encs[0], loop, w.bits, w.group).reshape(len(bsel), w.heads, T, D)
+            vh = oracle.reconstruct(encs[1], loop, w.bits, w.group).reshape(len(bsel), w.heads, T, D)
+            ref = oracle.decode_attention(kh, vh, q[loop][bi, hi], [T] * len(bsel),
+                                          kc[loop][bi, hi], vc[loop][bi, hi])
+            del kh, vh
+            got = outs[loop][np.ix_(bsel, hsel)]
+            err = float(np.max(np.abs(got - ref)))
+            assert err <= attn_tolerance(ref), (b0, loop, err, attn_tolerance(ref))
+            units += len(bsel) * w.heads
+        del encs
+    assert units == w.batch * w.heads * w.loops
