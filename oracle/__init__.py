@@ -34,8 +34,38 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "rqo.c")
 _LIB_PATH = os.path.join(_HERE, "librqo.so")
 
-POLICY_LAST = "last"   # shared anchor at the final loop [RQ §3.2]
-POLICY_NEXT = "next"   # chain toward the final loop [RQ §5.2 "Next-loop"]
+POLICY_LAST = "last"           # shared anchor at the final loop [RQ §3.2 Last-loop]
+POLICY_NEXT = "next"           # chain toward the final loop [RQ §5.2 Next-loop]
+POLICY_FIRST = "first"         # shared anchor at the first loop [RQ §3.2 First-loop]
+POLICY_PREVIOUS = "previous"   # chain toward the first loop [RQ §3.1, §3.2 Previous-loop]
+POLICIES = (POLICY_LAST, POLICY_NEXT, POLICY_FIRST, POLICY_PREVIOUS)
+
+
+def anchor_loop(L: int, policy: str) -> int:
+    """Index of the anchor loop: the final loop for Last-/Next-loop, the first
+    for First-/Previous-loop [RQ §3.2, App. D]."""
+    return L - 1 if policy in (POLICY_LAST, POLICY_NEXT) else 0
+
+
+def is_chained(policy: str) -> bool:
+    return policy in (POLICY_NEXT, POLICY_PREVIOUS)
+
+
+def reference_loop(L: int, r: int, policy: str) -> int:
+    """The loop whose reconstruction loop r references [RQ §3.2, App. D]:
+    the anchor (shared policies), r + 1 (Next-loop) or r - 1 (Previous-loop)."""
+    if policy == POLICY_NEXT:
+        return r + 1
+    if policy == POLICY_PREVIOUS:
+        return r - 1
+    return anchor_loop(L, policy)
+
+
+def encode_order(L: int, policy: str) -> List[int]:
+    """Residual loops in an order where every reference is encoded first:
+    away from the anchor."""
+    a = anchor_loop(L, policy)
+    return list(range(a - 1, -1, -1)) if a == L - 1 else list(range(1, L))
 
 GCC_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
              "-fPIC", "-shared"]
@@ -78,10 +108,10 @@ def lib() -> ctypes.CDLL:
             "rqo_dot_f32": ([_P, _P, _I], _F),
             "rqo_quantize": ([_P, _I, _I, _I, _P, _P, _P], None),
             "rqo_encode_anchor": ([_P, _I, _I, _I, _P, _P, _P], None),
-            "rqo_encode_residual_rot": ([_P, _P, _I, _I, _I, _P, _P, _P, _P], None),
-            "rqo_encode_residual": ([_P, _P, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_residual_rot": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_residual": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P], None),
             "rqo_encode_anchor_rows": ([_P, _I64, _I, _I, _I, _P, _P, _P], None),
-            "rqo_encode_residual_rows": ([_P, _P, _I64, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_residual_rows": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P], None),
             "rqo_dequant_codes_f64": ([_P, _P, _I, _I, _I, _P], None),
             "rqo_dequant_rows_f64": ([_P, _P, _I64, _I, _I, _I, _P], None),
             "rqo_attention_f64": ([_P, _P, _P, _I64, _P, _P, _I, _D, _P], None),
@@ -163,7 +193,8 @@ def quantize(z: np.ndarray, bits: int, group: int):
     return words, meta, deq
 
 
-def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int):
+def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int,
+                        unit_alpha: bool = False):
     """Residual encoder on an already-rotated fp32 row: (words, meta, alpha_bits, zhat)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
     ref = np.ascontiguousarray(ref, dtype=np.float32)
@@ -172,8 +203,8 @@ def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int):
     meta = np.zeros(D // group, np.uint32)
     alpha = np.zeros(1, np.uint16)
     zhat = np.zeros(D, np.float32)
-    lib().rqo_encode_residual_rot(_ptr(z), _ptr(ref), D, bits, group, _ptr(words),
-                                  _ptr(meta), _ptr(alpha), _ptr(zhat))
+    lib().rqo_encode_residual_rot(_ptr(z), _ptr(ref), D, bits, group, int(unit_alpha),
+                                  _ptr(words), _ptr(meta), _ptr(alpha), _ptr(zhat))
     return words, meta, int(alpha[0]), zhat
 
 
@@ -210,17 +241,21 @@ def meta_scale_zero(meta: np.ndarray):
 # --------------------------------------------------------------------------
 
 def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
-                policy: str = POLICY_LAST) -> List[Dict[str, np.ndarray]]:
+                policy: str = POLICY_LAST, unit_alpha: bool = False
+                ) -> List[Dict[str, np.ndarray]]:
     """Encode every loop of one (layer, K|V) side.
 
-    x: uint16 [L, N, D].  Returns per loop l a dict with 'codes', 'meta',
-    'alpha' (None for the anchor) and 'zhat' (fp32 reconstructed rotated row,
-    the value a chained predecessor references).
+    x: uint16 [L, N, D].  The anchor loop (anchor_loop) is quantised directly;
+    every other loop r stores the LS coefficient against its reference's
+    reconstruction (alpha = 1 if unit_alpha) and its quantised residual.
+    Returns per loop l a dict with 'codes', 'meta', 'alpha' (None for the
+    anchor) and 'zhat' (fp32 reconstructed rotated row, the value a chained
+    neighbour references).
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     L, N, D = x.shape
     out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
-    a = L - 1
+    a = anchor_loop(L, policy)
     enc = {"codes": np.zeros((N, D * bits[a] // 32), np.uint32),
            "meta": np.zeros((N, D // group[a]), np.uint32),
            "alpha": None,
@@ -228,15 +263,14 @@ def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
     lib().rqo_encode_anchor_rows(_ptr(x[a]), N, D, bits[a], group[a], _ptr(enc["codes"]),
                                  _ptr(enc["meta"]), _ptr(enc["zhat"]))
     out[a] = enc
-    order = range(L - 2, -1, -1)
-    for r in order:
-        ref = out[a]["zhat"] if policy == POLICY_LAST else out[r + 1]["zhat"]
+    for r in encode_order(L, policy):
+        ref = out[reference_loop(L, r, policy)]["zhat"]
         enc = {"codes": np.zeros((N, D * bits[r] // 32), np.uint32),
                "meta": np.zeros((N, D // group[r]), np.uint32),
                "alpha": np.zeros(N, np.uint16),
                "zhat": np.zeros((N, D), np.float32)}
         lib().rqo_encode_residual_rows(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D,
-                                       bits[r], group[r], _ptr(enc["codes"]),
+                                       bits[r], group[r], int(unit_alpha), _ptr(enc["codes"]),
                                        _ptr(enc["meta"]), _ptr(enc["alpha"]),
                                        _ptr(enc["zhat"]))
         out[r] = enc
@@ -254,20 +288,19 @@ def _levels_f64(enc: Dict[str, np.ndarray], bits: int, group: int, D: int) -> np
 def reconstruct_rotated(encs: List[Dict[str, np.ndarray]], loop: int, bits: Sequence[int],
                         group: Sequence[int], policy: str = POLICY_LAST) -> np.ndarray:
     """fp64 rotated reconstruction Z^_loop [RQ App. G.2]:
-    Z^_anchor = A; Z^_r = alpha~_r * Z^_ref + D(c_r), ref = anchor (Last-loop)
-    or Z^_{r+1} (Next-loop chain)."""
+    Z^_anchor = A; Z^_r = alpha~_r * Z^_ref + D(c_r), ref the anchor (shared
+    policies) or the neighbour toward the anchor (chained policies), so a
+    chained loop is rebuilt from the anchor outwards."""
     L = len(encs)
-    D = encs[L - 1]["zhat"].shape[1]
-    a = L - 1
-    zA = _levels_f64(encs[a], bits[a], group[a], D)
+    a = anchor_loop(L, policy)
+    D = encs[a]["zhat"].shape[1]
+    z = _levels_f64(encs[a], bits[a], group[a], D)
     if loop == a:
-        return zA
-    if policy == POLICY_LAST:
-        al = encs[loop]["alpha"].astype(np.uint32) << 16
-        al = al.view(np.float32).astype(np.float64)[:, None]
-        return al * zA + _levels_f64(encs[loop], bits[loop], group[loop], D)
-    z = zA
-    for r in range(a - 1, loop - 1, -1):
+        return z
+    path = [loop]
+    while reference_loop(L, path[-1], policy) != a:
+        path.append(reference_loop(L, path[-1], policy))
+    for r in reversed(path):
         al = (encs[r]["alpha"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         z = al[:, None] * z + _levels_f64(encs[r], bits[r], group[r], D)
     return z

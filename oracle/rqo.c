@@ -202,12 +202,18 @@ void rqo_encode_anchor(const uint16_t* x, int D, int bits, int group,
 }
 
 void rqo_encode_residual_rot(const float* z, const float* ref, int D, int bits,
-                             int group, uint32_t* words, uint32_t* meta,
-                             uint16_t* alpha, float* zhat) {
-  /* Least-squares scale of the reference: alpha = <X_r, R>/||R||^2. */
-  const float d_zr = rqo_dot_f32(z, ref, D);
-  const float d_rr = rqo_dot_f32(ref, ref, D);
-  const float a = (d_rr > 0.0f) ? d_zr / d_rr : 0.0f;
+                             int group, int unit_alpha, uint32_t* words,
+                             uint32_t* meta, uint16_t* alpha, float* zhat) {
+  /* Least-squares scale of the reference: alpha = <X_r, R>/||R||^2 [RQ §3.2
+   * scaling coefficient]; alpha = 1 without LS scaling (the plain
+   * inter-loop difference of the Previous-loop description, and the "w/o LS
+   * scaling" columns of [RQ Table 3]). */
+  float a = 1.0f;
+  if (!unit_alpha) {
+    const float d_zr = rqo_dot_f32(z, ref, D);
+    const float d_rr = rqo_dot_f32(ref, ref, D);
+    a = (d_rr > 0.0f) ? d_zr / d_rr : 0.0f;
+  }
   const uint16_t ab = rqo_f32_to_bf16(a);
   const float at = rqo_bf16_to_f32(ab);
   *alpha = ab;
@@ -222,12 +228,13 @@ void rqo_encode_residual_rot(const float* z, const float* ref, int D, int bits,
 }
 
 void rqo_encode_residual(const uint16_t* x, const float* ref, int D, int bits,
-                         int group, uint32_t* words, uint32_t* meta,
-                         uint16_t* alpha, float* zhat) {
+                         int group, int unit_alpha, uint32_t* words,
+                         uint32_t* meta, uint16_t* alpha, float* zhat) {
   float z[256];
   for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[i]);
   rqo_fwht_f32(z, D);
-  rqo_encode_residual_rot(z, ref, D, bits, group, words, meta, alpha, zhat);
+  rqo_encode_residual_rot(z, ref, D, bits, group, unit_alpha, words, meta, alpha,
+                          zhat);
 }
 
 void rqo_encode_anchor_rows(const uint16_t* x, int64_t n, int D, int bits,
@@ -240,12 +247,13 @@ void rqo_encode_anchor_rows(const uint16_t* x, int64_t n, int D, int bits,
 }
 
 void rqo_encode_residual_rows(const uint16_t* x, const float* ref, int64_t n,
-                              int D, int bits, int group, uint32_t* words,
-                              uint32_t* meta, uint16_t* alpha, float* zhat) {
+                              int D, int bits, int group, int unit_alpha,
+                              uint32_t* words, uint32_t* meta, uint16_t* alpha,
+                              float* zhat) {
   const int W = D * bits / 32, G = D / group;
   for (int64_t r = 0; r < n; ++r)
-    rqo_encode_residual(x + r * D, ref + r * D, D, bits, group, words + r * W,
-                        meta + r * G, alpha + r, zhat + r * D);
+    rqo_encode_residual(x + r * D, ref + r * D, D, bits, group, unit_alpha,
+                        words + r * W, meta + r * G, alpha + r, zhat + r * D);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -316,11 +324,13 @@ double rqo_effective_bits(int L, const int* bits, const int* group, int D,
 }
 
 int64_t rqo_component_reads(int L, int chained) {
-  /* Loops are 0..L-1 with the anchor at L-1 (Last-loop / Next-loop).  The
-   * anchor loop reads one component.  Under the shared anchor every other
-   * loop reads the anchor and its own residual; under the chain, loop r
-   * reads its residual, every residual between it and the anchor, and the
-   * anchor. */
+  /* One decode step over loops 0..L-1 [RQ §3.2, App. D].  The anchor loop
+   * reads one component.  Under a shared anchor (First-loop, Last-loop)
+   * every other loop reads the anchor and its own residual; under a chain
+   * (Previous-loop, Next-loop) loop r reads its residual, every residual
+   * between it and the anchor, and the anchor: 1 + its distance from the
+   * anchor.  The count does not depend on which end holds the anchor, so
+   * it is written for the anchor at L-1. */
   int64_t total = 0;
   for (int r = 0; r < L; ++r) {
     if (r == L - 1)

@@ -86,21 +86,22 @@ void rqo_encode_anchor(const uint16_t* x, int D, int bits, int group,
  * E = fma(-alpha~, ref, z); E quantised with (bits, group);
  * zhat = fma(alpha~, ref, deq(E)) is the reconstructed rotated row. */
 void rqo_encode_residual_rot(const float* z, const float* ref, int D, int bits,
-                             int group, uint32_t* words, uint32_t* meta,
-                             uint16_t* alpha, float* zhat);
+                             int group, int unit_alpha, uint32_t* words,
+                             uint32_t* meta, uint16_t* alpha, float* zhat);
 
 /* Same, from a bf16 row x (rotated here with rqo_fwht_f32). */
 void rqo_encode_residual(const uint16_t* x, const float* ref, int D, int bits,
-                         int group, uint32_t* words, uint32_t* meta,
-                         uint16_t* alpha, float* zhat);
+                         int group, int unit_alpha, uint32_t* words,
+                         uint32_t* meta, uint16_t* alpha, float* zhat);
 
 /* Row-batched forms of the two encoders: n rows, row-major. */
 void rqo_encode_anchor_rows(const uint16_t* x, int64_t n, int D, int bits,
                             int group, uint32_t* words, uint32_t* meta,
                             float* zhat);
 void rqo_encode_residual_rows(const uint16_t* x, const float* ref, int64_t n,
-                              int D, int bits, int group, uint32_t* words,
-                              uint32_t* meta, uint16_t* alpha, float* zhat);
+                              int D, int bits, int group, int unit_alpha,
+                              uint32_t* words, uint32_t* meta, uint16_t* alpha,
+                              float* zhat);
 
 /* fp64 value of the stored levels of one packed row: s~ * c + z~. */
 void rqo_dequant_codes_f64(const uint32_t* words, const uint32_t* meta, int D,

@@ -413,3 +413,90 @@ def test_component_reads_match_pages():
     for L in range(1, 40):
         assert oracle.component_reads(L, True) == L * (L + 1) // 2
         assert oracle.component_reads(L, False) == 2 * L - 1
+
+
+# ------------------------------------------- First-loop / Previous-loop [RQ §3.2]
+
+def _synthetic_loops(w, side, T=24):
+    import residual_bit_kv_b200.synth as synth
+    return np.stack([synth.bits_of(synth.kv(w, 0, side, l, [0], [0], 0, T)).reshape(-1, w.head_dim)
+                     for l in range(w.loops)])
+
+
+@pytest.mark.parametrize("pol,mirror", [("first", "last"), ("previous", "next")])
+def test_first_and_previous_mirror_last_and_next(oracle_mod, pol, mirror):
+    """First-loop (Previous-loop) is Last-loop (Next-loop) with the loop order
+    reversed: the anchor moves to loop 0 and the references point down the
+    loop index instead of up [RQ §3.2, App. D].  Encoding the reversed loops
+    under the mirrored policy stores identical bits, and reconstructs
+    identically."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["huginn_deep"].replace(loops=5, bits=(4, 2, 2, 4, 2),
+                                               group=(32, 64, 16, 32, 64),
+                                               sigma=(0.4, 0.3, 0.2, 0.1))
+    x = _synthetic_loops(w, synth.SIDE_K)
+    L = w.loops
+    e = oracle_mod.encode_side(x, w.bits, w.group, pol)
+    m = oracle_mod.encode_side(x[::-1], w.bits[::-1], w.group[::-1], mirror)
+    assert oracle_mod.anchor_loop(L, pol) == 0 and e[0]["alpha"] is None
+    for r in range(L):
+        for k in ("codes", "meta", "alpha"):
+            if e[r][k] is None:
+                assert m[L - 1 - r][k] is None
+            else:
+                np.testing.assert_array_equal(e[r][k], m[L - 1 - r][k])
+        np.testing.assert_array_equal(
+            oracle_mod.reconstruct_rotated(e, r, w.bits, w.group, pol),
+            oracle_mod.reconstruct_rotated(m, L - 1 - r, w.bits[::-1], w.group[::-1], mirror))
+
+
+def test_previous_loop_chain_is_the_recursion(oracle_mod):
+    """Previous-loop: loop r is rebuilt from loop r-1's reconstruction,
+    Z^_r = alpha~_r Z^_{r-1} + D(c_r), down to the first-loop anchor."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"]
+    x = _synthetic_loops(w, synth.SIDE_V)
+    e = oracle_mod.encode_side(x, w.bits[::-1], w.group[::-1], "previous")
+    bits, group = w.bits[::-1], w.group[::-1]
+    for r in range(1, w.loops):
+        zr = oracle_mod.reconstruct_rotated(e, r, bits, group, "previous")
+        zp = oracle_mod.reconstruct_rotated(e, r - 1, bits, group, "previous")
+        lv = oracle_mod._levels_f64(e[r], bits[r], group[r], w.head_dim)
+        a = oracle_mod.bf16_bits_to_f64(e[r]["alpha"])[:, None]
+        np.testing.assert_allclose(zr, a * zp + lv, rtol=0, atol=1e-12)
+
+
+def test_unit_alpha_residual_closed_form(oracle_mod):
+    """Without LS scaling alpha = 1 [RQ §3.1-§3.2]: a loop equal to twice the
+    anchor, whose rotation hits the INT4 levels exactly (integers 0..15 with
+    s~ = 1, z~ = 0), leaves the residual E = 2Z - Z = Z; INT2 then takes
+    s~ = 15/3 = 5, z~ = 0 and codes rint(Z/5), and the loop is rebuilt as
+    Z + 5 rint(Z/5).  LS scaling instead finds alpha = 2 and a zero residual."""
+    D = 64
+    rng = np.random.default_rng(7)
+    Z = rng.integers(0, 16, size=D).astype(np.float64)
+    Z[0], Z[1], Z[32], Z[33] = 0, 15, 0, 15            # every group spans [0, 15]
+    H = scipy.linalg.hadamard(D).astype(np.float64) / np.sqrt(D)
+    xa = H @ Z                                          # exact multiples of 1/8
+    assert np.all(xa * 8 == np.round(xa * 8)) and np.max(np.abs(xa)) < 64
+    xa_b = torch.tensor(xa, dtype=torch.float32).to(torch.bfloat16)
+    assert np.array_equal(xa_b.float().numpy().astype(np.float64), xa)
+    xb = synth_bits(xa_b)
+    x = np.stack([synth_bits(xa_b * 2), xb])[:, None, :]   # loop 0 = 2 x anchor, loop 1 = anchor
+    bits, group = (2, 4), (32, 32)
+    unit = oracle_mod.encode_side(x, bits, group, "last", unit_alpha=True)
+    ls = oracle_mod.encode_side(x, bits, group, "last")
+    assert np.all(unit[0]["alpha"] == 0x3F80)           # bf16(1.0)
+    assert np.all(ls[0]["alpha"] == 0x4000)             # bf16(2.0)
+    assert np.all(ls[0]["codes"] == 0) and np.all(ls[0]["meta"] == 0)
+    codes = oracle_mod.unpack_codes(unit[0]["codes"], 2, D).reshape(D)
+    np.testing.assert_array_equal(codes, np.round(Z / 5))
+    s, z = oracle_mod.meta_scale_zero(unit[0]["meta"])
+    np.testing.assert_array_equal(s.reshape(-1), [5.0, 5.0])
+    np.testing.assert_array_equal(z.reshape(-1), [0.0, 0.0])
+    rec = oracle_mod.reconstruct_rotated(unit, 0, bits, group, "last").reshape(D)
+    np.testing.assert_array_equal(rec, Z + 5 * np.round(Z / 5))
+
+
+def synth_bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
