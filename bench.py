@@ -234,12 +234,23 @@ def profile_traffic(files, profile_name: str):
 
 # ----------------------------------------------------------- byte accounting --
 
+def policy_chain(L, loop, policy):
+    """Loops read to rebuild `loop`: itself, then its references up to the
+    anchor (loop L-1 for Last-/Next-loop, loop 0 for First-/Previous-loop)."""
+    A = L - 1 if policy in ("last", "next") else 0
+    comps = [loop]
+    r = loop
+    while r != A:
+        r = A if policy in ("last", "first") else (r + 1 if policy == "next" else r - 1)
+        comps.append(r)
+    return comps, A
+
+
 def component_bytes_per_row(w, loop, policy="last"):
     """Packed bytes of one (token, head) row of every component loop `loop`
     reads, for one side (codes + fp16 scale/offset + bf16 LS coefficient)."""
     D = w.head_dim
-    A = w.loops - 1
-    comps = [A] if loop == A else ([loop, A] if policy == "last" else list(range(loop, w.loops)))
+    comps, A = policy_chain(w.loops, loop, policy)
     tot = 0
     for r in comps:
         tot += D * w.bits[r] // 8 + (D // w.group[r]) * 4 + (2 if r != A else 0)
@@ -751,57 +762,84 @@ def main():
     return 0
 
 
-def bench_ablation(dev, stream, args, hbm):
-    """Deep-recurrence workload (8 loops, batch 32, 40 heads, 8192 tokens, g 64),
-    one layer: decode of all 8 loops under the shared final-loop anchor and under
-    the chained Next-loop reference (loop r reads the anchor and every residual
-    r..6), to measure the read-traffic gap [RQ §3.2, §5.2, App. D]."""
+POLICY_NAMES = ("last", "next", "first", "previous")
+
+
+def policy_decode_step(w, policy, dev, stream, args):
+    """One layer of workload w stored under `policy`: the time of a decode
+    step over every loop (one call per loop) and its algorithmic bytes."""
     import residual_bit_kv_b200.librq as L
+    T = w.tokens
+    code = {"last": L.RQ_POLICY_LAST_LOOP, "next": L.RQ_POLICY_NEXT_LOOP,
+            "first": L.RQ_POLICY_FIRST_LOOP, "previous": L.RQ_POLICY_PREVIOUS_LOOP}[policy]
+    lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T + 16, w.bits, w.group, code)
+    nb = L.rq_cache_bytes(lay)
+    kb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    vb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    cache = L.rq_cache_bind(lay, kb, vb)
+    for side in (0, 1):
+        xs = torch.stack([synth.kv_full(w, 0, side, loop, 0, T, device=dev, chunk_b=2)
+                          for loop in range(w.loops)])
+        L.rq_quantize_append_loops(cache, 0, xs if side == 0 else None,
+                                   xs if side == 1 else None, 0, T, stream)
+        torch.cuda.synchronize()
+        del xs
+    q = [synth.query(w, 0, l, dev).contiguous() for l in range(w.loops)]
+    kc = [synth.current_token(w, 0, 0, l, dev).contiguous() for l in range(w.loops)]
+    vc = [synth.current_token(w, 0, 1, l, dev).contiguous() for l in range(w.loops)]
+    seq = torch.full((w.batch,), T, dtype=torch.int32, device=dev)
+    o = torch.empty(w.batch, w.heads, w.head_dim, dtype=torch.float32, device=dev)
+    wsb = L.rq_decode_workspace_bytes(lay, T)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    L.rq_decode_workspace_init(ws, wsb, stream)
+
+    def step():
+        for loop in range(w.loops):
+            L.rq_decode_attention(cache, 0, loop, q[loop], seq, T, kc[loop], vc[loop], 0.0, o,
+                                  ws, wsb, stream)
+
+    ms = timed(step, args.steps, args.warmup, stream)
+    byt = sum(decode_call_bytes(w, l, T, policy) for l in range(w.loops))
+    reads = sum(len(policy_chain(w.loops, l, policy)[0]) for l in range(w.loops))
+    del kb, vb, ws
+    torch.cuda.empty_cache()
+    return ms, byt, reads
+
+
+def bench_ablation(dev, stream, args, hbm):
+    """Reference-policy ablation [RQ §3.2, §5.2, App. D]: decode steps of one
+    layer under the shared anchors (Last-/First-loop) and the chains
+    (Next-/Previous-loop).  (1) the deep-recurrence workload (8 loops, batch
+    32, 40 heads, 8192 tokens, g 64): shared final-loop anchor vs the Next-loop
+    chain; (2) one layer of the 16k-context Ouro-like workload (4 loops, batch
+    16, 16 heads, 16384 tokens, g 32) under all four policies, the higher
+    precision on the anchor loop ([2,2,2,4] for Last/Next, [4,2,2,2] for
+    First/Previous, as in the pages' policy comparison)."""
     w = synth.WORKLOADS["huginn_deep"]
     T = w.tokens
     out = {"workload": f"{w.name}: 1 layer x {w.loops} loops, batch {w.batch}, {w.heads} heads, "
                        f"{T} past tokens, bits {list(w.bits)}, group {w.group[0]}"}
-    for policy, name in ((L.RQ_POLICY_LAST_LOOP, "shared"), (L.RQ_POLICY_NEXT_LOOP, "chained")):
-        lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T + 16, w.bits, w.group,
-                            policy)
-        nb = L.rq_cache_bytes(lay)
-        kb = torch.empty(nb, dtype=torch.uint8, device=dev)
-        vb = torch.empty(nb, dtype=torch.uint8, device=dev)
-        cache = L.rq_cache_bind(lay, kb, vb)
-        for side in (0, 1):
-            for loop in [w.loops - 1] + list(range(w.loops - 2, -1, -1)):
-                x = synth.kv_full(w, 0, side, loop, 0, T, device=dev, chunk_b=2)
-                if loop == w.loops - 1:
-                    L.rq_quantize_anchor(cache, 0, side, x, 0, T, stream)
-                else:
-                    L.rq_quantize_append_residual(cache, 0, side, loop, x, 0, T, stream)
-                del x
-        q = [synth.query(w, 0, l, dev).contiguous() for l in range(w.loops)]
-        kc = [synth.current_token(w, 0, 0, l, dev).contiguous() for l in range(w.loops)]
-        vc = [synth.current_token(w, 0, 1, l, dev).contiguous() for l in range(w.loops)]
-        seq = torch.full((w.batch,), T, dtype=torch.int32, device=dev)
-        o = torch.empty(w.batch, w.heads, w.head_dim, dtype=torch.float32, device=dev)
-        wsb = L.rq_decode_workspace_bytes(lay, T)
-        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-        L.rq_decode_workspace_init(ws, wsb, stream)
-
-        def step():
-            for loop in range(w.loops):
-                L.rq_decode_attention(cache, 0, loop, q[loop], seq, T, kc[loop], vc[loop], 0.0, o,
-                                      ws, wsb, stream)
-
-        ms = timed(step, args.steps, args.warmup, stream)
-        pol = "last" if policy == L.RQ_POLICY_LAST_LOOP else "next"
-        byt = sum(decode_call_bytes(w, l, T, pol) for l in range(w.loops))
+    for policy, name in (("last", "shared"), ("next", "chained")):
+        ms, byt, reads = policy_decode_step(w, policy, dev, stream, args)
         out[name] = {"ms_per_step": ms, "bytes_per_step": byt,
                      "gbs": byt / (ms * 1e-3) / 1e9, "frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
-                     "component_reads": w.loops * 2 - 1 if name == "shared"
-                     else w.loops * (w.loops + 1) // 2}
-        del kb, vb, ws
-        torch.cuda.empty_cache()
+                     "component_reads": reads}
     out["speedup_shared_over_chained"] = out["chained"]["ms_per_step"] / out["shared"]["ms_per_step"]
     out["bytes_ratio_chained_over_shared"] = (out["chained"]["bytes_per_step"] /
                                               out["shared"]["bytes_per_step"])
+    wo = synth.WORKLOADS["ouro_16k"].replace(layers=1, bits=(2, 2, 2, 4))
+    pol = {"workload": f"{wo.name}: 1 layer x {wo.loops} loops, batch {wo.batch}, {wo.heads} "
+                       f"heads, {wo.tokens} past tokens, group {wo.group[0]}"}
+    for policy in POLICY_NAMES:
+        bits = tuple(wo.bits) if policy in ("last", "next") else tuple(wo.bits)[::-1]
+        wp = wo.replace(bits=bits)
+        ms, byt, reads = policy_decode_step(wp, policy, dev, stream, args)
+        pol[policy] = {"bits": list(bits), "ms_per_step": ms, "bytes_per_step": byt,
+                       "gbs": byt / (ms * 1e-3) / 1e9, "component_reads": reads}
+    pol["throughput_last_over_previous"] = pol["previous"]["ms_per_step"] / pol["last"]["ms_per_step"]
+    pol["throughput_first_over_previous"] = (pol["previous"]["ms_per_step"] /
+                                             pol["first"]["ms_per_step"])
+    out["policies_ouro_16k_layer"] = pol
     return out
 
 

@@ -5,14 +5,18 @@
  * Citations: [RQ §x] = "ResidualQuant: KV Cache Quantization for Looped
  * Transformers with 2-Bit Residuals" (paperpeel.com/paper/2610.10381).
  *
- * What is stored [RQ §3.2 Last-loop policy, §3.3, §3.4, App. G.2]:
+ * What is stored [RQ §3.2, §3.3, §3.4, App. D, App. G.2]:
  *   For every past token and KV head of loop r, with Z = H x the normalised
  *   Sylvester-Hadamard rotation of the bf16 row x:
- *     anchor (final loop L-1):  A = deq(Q_bL(Z_{L-1}))
- *     residual loop r < L-1:    alpha_r = <Z_r, R>/<R, R>, alpha~ = bf16(alpha_r),
+ *     anchor loop a:            A = deq(Q_ba(Z_a))
+ *     every other loop r:       alpha_r = <Z_r, R>/<R, R> (1 with
+ *                               RQ_FLAG_UNIT_ALPHA), alpha~ = bf16(alpha_r),
  *                               codes of Q_br(Z_r - alpha~ R)
- *   where R = A (RQ_POLICY_LAST_LOOP, shared anchor) or R = Z^_{r+1}
- *   (RQ_POLICY_NEXT_LOOP, the chained "Next-loop" reference [RQ §5.2]).
+ *   where the policy fixes a and R [RQ §3.2 reference KV, §5.2]:
+ *     RQ_POLICY_LAST_LOOP      a = L-1, R = A (shared final-loop anchor)
+ *     RQ_POLICY_NEXT_LOOP      a = L-1, R = Z^_{r+1} (chain toward the anchor)
+ *     RQ_POLICY_FIRST_LOOP     a = 0,   R = A (shared first-loop anchor)
+ *     RQ_POLICY_PREVIOUS_LOOP  a = 0,   R = Z^_{r-1} (chain toward the anchor)
  *   Q_b is group-wise affine quantisation [RQ §2.1]: per group of g
  *   consecutive channels, s = (max - min)/(2^b - 1), s~ = fp16(s),
  *   z~ = fp16(min), code = rint_even(clamp((z - z~) * (1/s~), 0, 2^b - 1)).
@@ -35,7 +39,8 @@
  *   [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v, word
  *   2u + ((v>>1)&1), bits [4*(2*(v>>2) + (v&1)), +4).  Little-endian words.
  *   Effective bits per element of loop r: bits[r] + 32/group[r]
- *   (+ 16/head_dim for a residual loop).
+ *   (+ 16/head_dim for a residual loop).  Components are laid out anchor
+ *   first, then the other loops in increasing index (comp_off).
  *
  * Conventions for every entry point:
  *   - All pointers except rq_layout / rq_cache arguments are DEVICE pointers
@@ -75,19 +80,27 @@ typedef enum rq_status {
   RQ_ERR_WORKSPACE = 6      /* workspace too small                            */
 } rq_status;
 
-/* Reference policy [RQ §3.2, §5.2]. */
+/* Reference policy [RQ §3.2, §5.2, App. D]. */
 typedef enum rq_policy {
-  RQ_POLICY_LAST_LOOP = 0,  /* every loop r < L-1 references the final-loop anchor */
-  RQ_POLICY_NEXT_LOOP = 1   /* loop r references loop r+1 (chain to the anchor)    */
+  RQ_POLICY_LAST_LOOP = 0,     /* anchor L-1; every loop references the anchor  */
+  RQ_POLICY_NEXT_LOOP = 1,     /* anchor L-1; loop r references loop r+1        */
+  RQ_POLICY_FIRST_LOOP = 2,    /* anchor 0; every loop references the anchor    */
+  RQ_POLICY_PREVIOUS_LOOP = 3  /* anchor 0; loop r references loop r-1          */
 } rq_policy;
+
+/* rq_layout.flags */
+#define RQ_FLAG_UNIT_ALPHA 1   /* alpha_r = 1: plain differences, no LS scaling
+                                  [RQ §3.1-§3.2, Table 3 "w/o LS scaling"] */
 
 /* Shape and precision of a compressed KV cache.
  *   num_layers  >= 1
- *   num_loops   L in [1, RQ_MAX_LOOPS]; loop L-1 (0-based) is the anchor
+ *   num_loops   L in [1, RQ_MAX_LOOPS]; the anchor is loop L-1 (Last-/Next-
+ *               loop) or loop 0 (First-/Previous-loop)
  *   batch, kv_heads >= 1
  *   head_dim    D in {64, 128}
  *   max_tokens  token capacity per (batch, head), >= 1
  *   policy      rq_policy
+ *   flags       0 or RQ_FLAG_UNIT_ALPHA
  *   bits[r]     2 or 4
  *   group[r]    g in {16, 32, 64, 128}, g divides D, g * bits[r] >= 32
  */
@@ -99,7 +112,7 @@ typedef struct rq_layout {
   int32_t head_dim;
   int32_t max_tokens;
   int32_t policy;
-  int32_t reserved;            /* must be 0 */
+  int32_t flags;               /* RQ_FLAG_* */
   int32_t bits[RQ_MAX_LOOPS];
   int32_t group[RQ_MAX_LOOPS];
 } rq_layout;
@@ -138,29 +151,31 @@ uint64_t rq_layer_bytes(const rq_layout* layout);
 rq_status rq_cache_bind(const rq_layout* layout, void* k_base, void* v_base,
                         rq_cache* out);
 
-/* Quantise-and-append the final-loop anchor [RQ §3.2, §3.4, §4.2 Prefill /
- * Decode]: rows x (bf16, [batch][kv_heads][n][head_dim], contiguous) of
- * loop L-1 are rotated, affine-quantised with bits[L-1] / group[L-1] and
- * stored at token positions [t0, t0 + n) of `layer`, side kv (0 = K, 1 = V).
+/* Quantise-and-append the anchor loop a (L-1, or 0 under First-/Previous-
+ * loop) [RQ §3.2, §3.4, §4.2 Prefill / Decode]: rows x (bf16,
+ * [batch][kv_heads][n][head_dim], contiguous) of loop a are rotated,
+ * affine-quantised with bits[a] / group[a] and stored at token positions
+ * [t0, t0 + n) of `layer`, side kv (0 = K, 1 = V).
  * n = 0 is a no-op.  t0 + n > max_tokens -> RQ_ERR_CAPACITY. */
 rq_status rq_quantize_anchor(const rq_cache* cache, int32_t layer, int32_t kv,
                              const void* x, int32_t t0, int32_t n,
                              void* stream);
 
-/* Quantise-and-append residual loop `loop` (0 <= loop < L-1) [RQ §3.2
- * scaling coefficient, §3.3, App. G.1]: alpha, residual, rotation, affine
- * quantisation and bit-packing of rows x (same layout as above).
+/* Quantise-and-append residual loop `loop` (any loop but the anchor) [RQ
+ * §3.2 scaling coefficient, §3.3, App. G.1]: alpha, residual, rotation,
+ * affine quantisation and bit-packing of rows x (same layout as above).
  * Stream-ordered precondition: the reference rows [t0, t0 + n) are stored
- * already -- the anchor (LAST_LOOP) or loops loop+1 .. L-1 (NEXT_LOOP). */
+ * already -- the anchor (LAST_LOOP, FIRST_LOOP), loops loop+1 .. L-1
+ * (NEXT_LOOP) or loops 0 .. loop-1 (PREVIOUS_LOOP). */
 rq_status rq_quantize_append_residual(const rq_cache* cache, int32_t layer,
                                       int32_t kv, int32_t loop, const void* x,
                                       int32_t t0, int32_t n, void* stream);
 
 /* Quantise-and-append of every loop of `layer` at token positions
  * [t0, t0 + n), K and V, in one launch [RQ §3.2, §3.4, §4.2 Decode: the new
- * token's loops are stored after the final loop]: the anchor (loop L-1) and
- * every residual loop against it (LAST_LOOP) or against the chain Z^_{r+1}
- * (NEXT_LOOP, loops L-2 down to 0).  Stores exactly the bytes of
+ * token's loops are stored after the final loop]: the anchor and every other
+ * loop against its reference (the anchor, or the chain Z^_{r+1} / Z^_{r-1}
+ * processed away from the anchor).  Stores exactly the bytes of
  * rq_quantize_anchor followed by rq_quantize_append_residual for each loop in
  * the policy's order; the anchor is not re-read from the cache.
  *   xk, xv  bf16 [num_loops][batch][kv_heads][n][head_dim], contiguous,
@@ -190,7 +205,8 @@ rq_status rq_decode_workspace_init(void* workspace, uint64_t ws_bytes,
 /* Compressed decode attention of loop `loop` for one query token per
  * (batch, head) [RQ §4.1, §4.2 Decode, App. G.2]:
  *   past keys/values t < seq_lens[b] are rebuilt on the fly from the packed
- *   cache (anchor + the loop's residual; the whole chain under NEXT_LOOP),
+ *   cache (anchor + the loop's residual; the whole chain under NEXT_LOOP and
+ *   PREVIOUS_LOOP),
  *   scores use the rotated query (Hq) . Z^_K, values are accumulated in the
  *   rotated domain and rotated back once; the current token's own k_cur /
  *   v_cur (bf16, unrotated, [batch][kv_heads][head_dim]) are merged with the

@@ -26,6 +26,25 @@ inline rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : 
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
+// Anchor loop of a layout: the final loop (Last-/Next-loop) or the first
+// (First-/Previous-loop) [RQ §3.2, App. D].
+inline int anchor_of(const rq_layout* l) {
+  return (l->policy == RQ_POLICY_FIRST_LOOP || l->policy == RQ_POLICY_PREVIOUS_LOOP)
+             ? 0
+             : l->num_loops - 1;
+}
+
+inline bool chained_of(const rq_layout* l) {
+  return l->policy == RQ_POLICY_NEXT_LOOP || l->policy == RQ_POLICY_PREVIOUS_LOOP;
+}
+
+// The loop that loop r references (r != anchor).
+inline int reference_of(const rq_layout* l, int r) {
+  if (l->policy == RQ_POLICY_NEXT_LOOP) return r + 1;
+  if (l->policy == RQ_POLICY_PREVIOUS_LOOP) return r - 1;
+  return anchor_of(l);
+}
+
 inline int64_t token_stride_of(const rq_layout* l) {
   return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), kRowTokens));
 }
@@ -33,19 +52,20 @@ inline int64_t token_stride_of(const rq_layout* l) {
 inline uint32_t record_bytes(const rq_layout* l, int r) {
   const int D = l->head_dim;
   const uint32_t per_token = (D * l->bits[r] / 32) * 4 + (D / l->group[r]) * 4 +
-                             (r != l->num_loops - 1 ? 2 : 0);
+                             (r != anchor_of(l) ? 2 : 0);
   return kBlock * per_token;   // a multiple of 64 bytes
 }
 
 // Byte offset of every component's first record inside one (layer, side);
-// returns the layer bytes.  Anchor (loop L-1) first, then loops 0 .. L-2.
+// returns the layer bytes.  Anchor first, then the other loops ascending.
 uint64_t layout_offsets(const rq_layout* l, uint64_t* comp_off, uint32_t* rec_bytes) {
   const uint64_t records = static_cast<uint64_t>(l->batch) * l->kv_heads *
                            (token_stride_of(l) / kBlock);
   const int L = l->num_loops;
   uint64_t off = 0;
+  const int a = anchor_of(l);
   for (int k = 0; k < L; ++k) {
-    const int r = (k == 0) ? L - 1 : k - 1;
+    const int r = (k == 0) ? a : (k - 1 < a ? k - 1 : k);
     comp_off[r] = off;
     rec_bytes[r] = record_bytes(l, r);
     off = align_up(off + records * rec_bytes[r], kAlign);
@@ -130,22 +150,21 @@ Comp comp_of(const rq_cache* c, int layer, int kv, int r) {
   k.rec_bytes = c->rec_bytes[r];
   k.bits = c->layout.bits[r];
   k.group = c->layout.group[r];
-  k.has_alpha = (r != c->layout.num_loops - 1) ? 1 : 0;
+  k.has_alpha = (r != anchor_of(&c->layout)) ? 1 : 0;
   return k;
 }
 
 // Reference chain used to reconstruct loop `loop`: [loop, ..., anchor]
-// (LAST_LOOP: [loop, anchor]; the anchor loop alone is [anchor]).
+// (shared anchor: [loop, anchor]; the anchor loop alone is [anchor]).
 int chain_of(const rq_cache* c, int layer, int kv, int loop, Comp* out) {
-  const int L = c->layout.num_loops;
+  const rq_layout* l = &c->layout;
+  const int a = anchor_of(l);
   int n = 0;
-  if (loop == L - 1) {
-    out[n++] = comp_of(c, layer, kv, L - 1);
-  } else if (c->layout.policy == RQ_POLICY_LAST_LOOP) {
-    out[n++] = comp_of(c, layer, kv, loop);
-    out[n++] = comp_of(c, layer, kv, L - 1);
-  } else {
-    for (int r = loop; r < L; ++r) out[n++] = comp_of(c, layer, kv, r);
+  int r = loop;
+  out[n++] = comp_of(c, layer, kv, r);
+  while (r != a) {
+    r = reference_of(l, r);
+    out[n++] = comp_of(c, layer, kv, r);
   }
   return n;
 }
@@ -196,8 +215,9 @@ rq_status rq_layout_validate(const rq_layout* l) {
   if (l == nullptr) return RQ_ERR_INVALID_ARG;
   if (l->num_layers < 1 || l->num_loops < 1 || l->num_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
   if (l->batch < 1 || l->kv_heads < 1 || l->max_tokens < 1) return RQ_ERR_INVALID_ARG;
-  if (l->policy != RQ_POLICY_LAST_LOOP && l->policy != RQ_POLICY_NEXT_LOOP) return RQ_ERR_INVALID_ARG;
-  if (l->reserved != 0) return RQ_ERR_INVALID_ARG;
+  if (l->policy < RQ_POLICY_LAST_LOOP || l->policy > RQ_POLICY_PREVIOUS_LOOP)
+    return RQ_ERR_INVALID_ARG;
+  if ((l->flags & ~RQ_FLAG_UNIT_ALPHA) != 0) return RQ_ERR_INVALID_ARG;
   if (!is_pow2(l->head_dim) || l->head_dim < 32 || l->head_dim > 256) return RQ_ERR_INVALID_ARG;
   if (l->head_dim != 64 && l->head_dim != 128) return RQ_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(l->batch) * l->kv_heads > 65535) return RQ_ERR_UNSUPPORTED;
@@ -245,7 +265,7 @@ rq_status rq_quantize_anchor(const rq_cache* c, int32_t layer, int32_t kv, const
   if (n == 0) return RQ_OK;
   if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
   const rq_layout& l = c->layout;
-  const int a = l.num_loops - 1;
+  const int a = anchor_of(&l);
   QuantParams p;
   memset(&p, 0, sizeof(p));
   p.x = static_cast<const uint16_t*>(x);
@@ -264,7 +284,7 @@ rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t 
   rq_status st = check_cache(c, layer, kv);
   if (st != RQ_OK) return st;
   const rq_layout& l = c->layout;
-  if (loop < 0 || loop >= l.num_loops - 1) return RQ_ERR_INVALID_ARG;
+  if (loop < 0 || loop >= l.num_loops || loop == anchor_of(&l)) return RQ_ERR_INVALID_ARG;
   if ((st = check_range(c, t0, n)) != RQ_OK) return st;
   if (n == 0) return RQ_OK;
   if (x == nullptr || !aligned(x, 16)) return RQ_ERR_INVALID_ARG;
@@ -276,11 +296,12 @@ rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t 
   p.t0 = t0;
   p.nblk = c->token_stride / kBlock;
   p.dst = comp_of(c, layer, kv, loop);
-  // Reference: the anchor (Last-loop) or the chain loop+1 .. anchor (Next-loop).
+  // Reference: the anchor (shared policies) or the chain toward it.
   Comp chain[RQ_MAX_LOOPS];
   const int len = chain_of(c, layer, kv, loop, chain);   // [loop, ref...]
   p.nref = len - 1;
   for (int i = 1; i < len; ++i) p.ref[i - 1] = chain[i];
+  p.unit_alpha = (l.flags & RQ_FLAG_UNIT_ALPHA) ? 1 : 0;
   p.rot_scale = rot_scale_of(l.head_dim);
   return cuda_status(
       launch_quantize(p, l.head_dim, l.bits[loop], l.group[loop], as_stream(stream)));
@@ -303,7 +324,14 @@ rq_status rq_quantize_append_loops(const rq_cache* c, int32_t layer, const void*
   p.bh = l.batch * l.kv_heads;
   p.n = n;
   p.nloops = l.num_loops;
-  p.chained = l.policy == RQ_POLICY_NEXT_LOOP ? 1 : 0;
+  p.anchor = anchor_of(&l);
+  p.chained = chained_of(&l) ? 1 : 0;
+  p.unit_alpha = (l.flags & RQ_FLAG_UNIT_ALPHA) ? 1 : 0;
+  // residual loops away from the anchor, so every reference is stored first
+  for (int k = 0, r = 0; r < l.num_loops; ++r) {
+    const int rr = p.anchor == 0 ? r : l.num_loops - 1 - r;
+    if (rr != p.anchor) p.order[k++] = rr;
+  }
   p.t0 = t0;
   p.nblk = c->token_stride / kBlock;
   for (int kv = 0; kv < 2; ++kv)
@@ -407,8 +435,9 @@ int32_t rq_decode_splits(const rq_layout* l, int32_t max_seq_len) {
     return 0;
   DecodeParams p;
   int D = 0;
-  // loop 0 is the most expensive loop to decode (longest chain)
-  if (fill_decode_params(&c, 0, 0, max_seq_len, &p, &D) != RQ_OK) return 0;
+  // the loop farthest from the anchor is the most expensive to decode
+  const int far = anchor_of(l) == 0 ? l->num_loops - 1 : 0;
+  if (fill_decode_params(&c, 0, far, max_seq_len, &p, &D) != RQ_OK) return 0;
   return p.splits;
 }
 

@@ -61,14 +61,16 @@ __host__ __device__ inline uint16_t* rec_alpha(unsigned char* rec, int D, int bi
 }
 
 struct QuantParams {
+  int32_t unit_alpha;      // 1: alpha = 1 (no LS scaling)
   const uint16_t* x;       // bf16 [B*H][n][D]
   int32_t bh;              // B*H
   int32_t n;
   int32_t t0;
   int64_t nblk;            // records per row
   Comp dst;                // destination component
-  // Reference chain, nearest first: for LAST_LOOP one entry (the anchor);
-  // for NEXT_LOOP loops loop+1 .. L-1 (the anchor last).
+  // Reference chain, nearest first: for a shared anchor one entry (the
+  // anchor); for a chain the neighbour toward the anchor first, the anchor
+  // last.
   int32_t nref;
   Comp ref[RQ_MAX_LOOPS];
   float rot_scale;         // fp32(1/sqrt(D))
@@ -78,7 +80,10 @@ struct QuantParams {
 struct QuantLoopsParams {
   const uint16_t* x[2];    // bf16 [L][B*H][n][D] per side (K, V); nullptr skips the side
   int32_t bh, n, nloops;
-  int32_t chained;         // 1: reference of loop r is Z^_{r+1} (Next-loop)
+  int32_t anchor;          // anchor loop
+  int32_t order[RQ_MAX_LOOPS];   // the other loops, away from the anchor
+  int32_t chained;         // 1: loop order[k] references order[k-1] (the anchor for k = 0)
+  int32_t unit_alpha;      // 1: alpha = 1 (no LS scaling)
   int64_t t0, nblk;
   Comp dst[2][RQ_MAX_LOOPS];
   float rot_scale;

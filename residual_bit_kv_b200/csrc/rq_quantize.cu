@@ -271,24 +271,29 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
 
 // Least-squares coefficient of z against the reference over the row
 // [RQ §3.2 scaling coefficient, App. G.1]: alpha~ = bf16(<z, ref> / <ref, ref>)
-// (0 for a zero reference); z becomes the residual fma(-alpha~, ref, z).
-// The dots run lane-serially in channel order, then across the row's lanes.
+// (0 for a zero reference; 1 without LS scaling); z becomes the residual
+// fma(-alpha~, ref, z).  The dots run lane-serially in channel order, then
+// across the row's lanes.
 template <int D>
-__device__ __forceinline__ __nv_bfloat16 ls_residual(float2 (&v)[16], const float2 (&ref)[16]) {
+__device__ __forceinline__ __nv_bfloat16 ls_residual(float2 (&v)[16], const float2 (&ref)[16],
+                                                     bool unit_alpha) {
   constexpr int P = D / 32;
-  float dzr = 0.0f, drr = 0.0f;
+  float a = 1.0f;
+  if (!unit_alpha) {
+    float dzr = 0.0f, drr = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const float z = ch_of(v, k), r = ch_of(ref, k);
-    dzr = __fmaf_rn(z, r, dzr);
-    drr = __fmaf_rn(r, r, drr);
-  }
+    for (int k = 0; k < 32; ++k) {
+      const float z = ch_of(v, k), r = ch_of(ref, k);
+      dzr = __fmaf_rn(z, r, dzr);
+      drr = __fmaf_rn(r, r, drr);
+    }
 #pragma unroll
-  for (int off = P / 2; off >= 1; off >>= 1) {
-    dzr = __fadd_rn(dzr, __shfl_xor_sync(0xffffffffu, dzr, off));
-    drr = __fadd_rn(drr, __shfl_xor_sync(0xffffffffu, drr, off));
+    for (int off = P / 2; off >= 1; off >>= 1) {
+      dzr = __fadd_rn(dzr, __shfl_xor_sync(0xffffffffu, dzr, off));
+      drr = __fadd_rn(drr, __shfl_xor_sync(0xffffffffu, drr, off));
+    }
+    a = (drr > 0.0f) ? __fdiv_rn(dzr, drr) : 0.0f;
   }
-  const float a = (drr > 0.0f) ? __fdiv_rn(dzr, drr) : 0.0f;
   const __nv_bfloat16 ab = __float2bfloat16_rn(a);
   const float at = __bfloat162float(ab);
   const float2 na = make_float2(-at, -at);
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
         for (int k = 0; k < 16; ++k) ref[k] = make_float2(0.0f, 0.0f);
       }
-      const __nv_bfloat16 ab = ls_residual<D>(v, ref);
+      const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
         *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock)) =
             __bfloat16_as_ushort(ab);
@@ -368,10 +373,10 @@ __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_
 
 // Every loop of a (layer, token range) for one side (blockIdx.y): the anchor
 // is quantised first and its stored levels stay in registers as the
-// reference; each residual loop then takes its LS coefficient, residual and
-// quantisation against it [RQ §3.2, §3.4, App. G.1].  Under the Next-loop
-// policy the loops run from L-2 down to 0 and the reference becomes
-// Z^_r = fma(alpha~_r, Z^_{r+1}, D(c_r)) after loop r.  The anchor is read
+// reference; each other loop then takes its LS coefficient, residual and
+// quantisation against it [RQ §3.2, §3.4, App. G.1].  Loops run away from
+// the anchor (p.order); under a chained policy the reference becomes
+// Z^_r = fma(alpha~_r, Z^_ref, D(c_r)) after loop r.  The anchor is read
 // once and never re-read from the cache; the arithmetic (and so every
 // stored bit) is that of the per-loop kernels.
 template <int D>
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kQuantThreads / 32);
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) +
                        (threadIdx.x >> 5);
-  const int a = p.nloops - 1;
+  const int a = p.anchor;
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
@@ -399,12 +404,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     load_rotate<D>(xs + (static_cast<int64_t>(a) * total + r_in) * D, active, slice, p.rot_scale,
                    v);
     quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, v, slice, active, ref);
-    for (int k = 0; k < a; ++k) {
-      const int r = p.chained ? a - 1 - k : k;
+    for (int k = 0; k + 1 < p.nloops; ++k) {
+      const int r = p.order[k];
       const Comp& c = p.dst[side][r];
       load_rotate<D>(xs + (static_cast<int64_t>(r) * total + r_in) * D, active, slice,
                      p.rot_scale, v);
-      const __nv_bfloat16 ab = ls_residual<D>(v, ref);
+      const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
         *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
                    static_cast<int>(t % kBlock)) = __bfloat16_as_ushort(ab);

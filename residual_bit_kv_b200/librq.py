@@ -16,6 +16,9 @@ RQ_MAX_LOOPS = 32
 RQ_BLOCK_TOKENS = 32
 RQ_POLICY_LAST_LOOP = 0
 RQ_POLICY_NEXT_LOOP = 1
+RQ_POLICY_FIRST_LOOP = 2
+RQ_POLICY_PREVIOUS_LOOP = 3
+RQ_FLAG_UNIT_ALPHA = 1
 
 RQ_OK = 0
 RQ_ERR_INVALID_ARG = 1
@@ -43,7 +46,7 @@ class rq_layout(ctypes.Structure):
         ("num_layers", ctypes.c_int32), ("num_loops", ctypes.c_int32),
         ("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("max_tokens", ctypes.c_int32),
-        ("policy", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("policy", ctypes.c_int32), ("flags", ctypes.c_int32),
         ("bits", ctypes.c_int32 * RQ_MAX_LOOPS), ("group", ctypes.c_int32 * RQ_MAX_LOOPS),
     ]
 
@@ -140,10 +143,10 @@ def _check(status: int, what: str) -> None:
 
 def make_layout(num_layers: int, num_loops: int, batch: int, kv_heads: int, head_dim: int,
                 max_tokens: int, bits: Sequence[int], group: Sequence[int],
-                policy: int = RQ_POLICY_LAST_LOOP) -> rq_layout:
+                policy: int = RQ_POLICY_LAST_LOOP, flags: int = 0) -> rq_layout:
     lay = rq_layout()
     lay.num_layers, lay.num_loops, lay.batch, lay.kv_heads = num_layers, num_loops, batch, kv_heads
-    lay.head_dim, lay.max_tokens, lay.policy, lay.reserved = head_dim, max_tokens, policy, 0
+    lay.head_dim, lay.max_tokens, lay.policy, lay.flags = head_dim, max_tokens, policy, flags
     for r in range(min(num_loops, RQ_MAX_LOOPS, len(bits), len(group))):
         lay.bits[r] = int(bits[r])
         lay.group[r] = int(group[r])

@@ -19,19 +19,25 @@ import residual_bit_kv_b200.synth as synth
 SIDES = (synth.SIDE_K, synth.SIDE_V)
 
 
+POLICY_CODES = {"last": L.RQ_POLICY_LAST_LOOP, "next": L.RQ_POLICY_NEXT_LOOP,
+                "first": L.RQ_POLICY_FIRST_LOOP, "previous": L.RQ_POLICY_PREVIOUS_LOOP}
+
+
 def policy_code(policy: str) -> int:
-    return L.RQ_POLICY_LAST_LOOP if policy == "last" else L.RQ_POLICY_NEXT_LOOP
+    return POLICY_CODES[policy]
 
 
 def layout_of(w: synth.Workload, policy: str = "last", layers: Optional[int] = None,
-              max_tokens: Optional[int] = None) -> L.rq_layout:
+              max_tokens: Optional[int] = None, unit_alpha: bool = False) -> L.rq_layout:
     return L.make_layout(layers or w.layers, w.loops, w.batch, w.heads, w.head_dim,
-                         max_tokens or (w.tokens + 1), w.bits, w.group, policy_code(policy))
+                         max_tokens or (w.tokens + 1), w.bits, w.group, policy_code(policy),
+                         L.RQ_FLAG_UNIT_ALPHA if unit_alpha else 0)
 
 
 def append_order(w: synth.Workload, policy: str) -> List[int]:
-    """Anchor first, then residual loops (descending, as the chain requires)."""
-    return [w.loops - 1] + list(range(w.loops - 2, -1, -1))
+    """Anchor first, then the other loops away from it (as a chain requires)."""
+    a = oracle.anchor_loop(w.loops, policy)
+    return [a] + oracle.encode_order(w.loops, policy)
 
 
 @dataclasses.dataclass
@@ -43,19 +49,20 @@ class GpuCache:
     kbuf: torch.Tensor
     vbuf: torch.Tensor
     inputs: Dict  # (layer, side, loop) -> bf16 [B, H, T, D] cuda tensor (if kept)
+    unit_alpha: bool = False
 
 
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
                     keep_inputs: bool = True, tokens: Optional[int] = None,
                     max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
-                    fused: bool = False) -> GpuCache:
+                    fused: bool = False, unit_alpha: bool = False) -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
     the C ABI in the order the policy requires (fused: every loop and both
     sides of a chunk in one rq_quantize_append_loops call).  append_chunks
     splits the token range into consecutive appends (e.g. prefill then
     single tokens)."""
     T = w.tokens if tokens is None else tokens
-    lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens)
+    lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens, unit_alpha=unit_alpha)
     nbytes = L.rq_cache_bytes(lay)
     assert nbytes > 0
     kbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
@@ -87,7 +94,7 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     continue
                 for loop in append_order(w, policy):
                     x = xs[loop][:, :, a:b].contiguous()
-                    if loop == w.loops - 1:
+                    if loop == oracle.anchor_loop(w.loops, policy):
                         L.rq_quantize_anchor(cache, layer, side, x, a, b - a)
                     else:
                         L.rq_quantize_append_residual(cache, layer, side, loop, x, a, b - a)
@@ -96,7 +103,7 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     inputs[(layer, side, loop)] = x
             del xs
     torch.cuda.synchronize()
-    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs)
+    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha)
 
 
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
@@ -125,7 +132,7 @@ def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
     codes = recs[:, : blk * W * 4].copy().view(np.uint32).reshape(*shp, W)
     meta = recs[:, blk * W * 4: blk * (W + G) * 4].copy().view(np.uint32).reshape(*shp, G)
     out = {"codes": codes, "meta": meta, "alpha": None}
-    if loop != w.loops - 1:
+    if loop != oracle.anchor_loop(w.loops, gc.policy):
         a0 = blk * (W + G) * 4
         out["alpha"] = recs[:, a0: a0 + blk * 2].copy().view(np.uint16).reshape(*shp)
     return out
@@ -133,7 +140,7 @@ def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
 
 def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
                   hsel: Sequence[int], t0: int, t1: int, policy: str = "last",
-                  x_loops: Optional[List[np.ndarray]] = None):
+                  x_loops: Optional[List[np.ndarray]] = None, unit_alpha: bool = False):
     """Oracle encodings of the selected rows.  Returns (encs, x) where
     x is uint16 [L, nb*nh*(t1-t0), D]."""
     if x_loops is None:
@@ -141,7 +148,7 @@ def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
         x_loops = [synth.bits_of(synth.kv(w, layer, side, loop, bsel, hsel, t0, t1, "cpu", cs))
                    .reshape(-1, w.head_dim) for loop in range(w.loops)]
     x = np.stack(x_loops)
-    return oracle.encode_side(x, w.bits, w.group, policy), x
+    return oracle.encode_side(x, w.bits, w.group, policy, unit_alpha), x
 
 
 def assert_component_equal(gpu: Dict[str, np.ndarray], enc: Dict[str, np.ndarray], shape,
@@ -189,7 +196,8 @@ def gpu_decode(gc: GpuCache, layer: int, loop: int, seq_lens: Sequence[int], max
 
 def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
                   hsel: Sequence[int], seq_lens: Sequence[int], policy: str = "last",
-                  inputs: Optional[Dict] = None, scale: Optional[float] = None) -> np.ndarray:
+                  inputs: Optional[Dict] = None, scale: Optional[float] = None,
+                  unit_alpha: bool = False) -> np.ndarray:
     """fp64 oracle decode for the selected (b, h): [len(bsel), len(hsel), D]."""
     T = max(int(seq_lens[b]) for b in bsel)
     D = w.head_dim
@@ -200,7 +208,7 @@ def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
         if inputs is not None:
             xl = [synth.bits_of(inputs[(layer, side, l)][list(bsel)][:, list(hsel), :T].cpu())
                   .reshape(-1, D) for l in range(w.loops)]
-        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl)
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl, unit_alpha)
         rec[side] = oracle.reconstruct(encs, loop, w.bits, w.group, policy).reshape(
             len(bsel), len(hsel), T, D)
     q = synth.bits_of(synth.query(w, layer, loop)).reshape(w.batch, w.heads, D)

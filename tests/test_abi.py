@@ -54,7 +54,32 @@ def test_layout_validation(L):
     lay = _lay(L)
     lay.policy = 7
     assert L.rq_layout_validate(lay) == L.RQ_ERR_INVALID_ARG
+    for pol in (L.RQ_POLICY_LAST_LOOP, L.RQ_POLICY_NEXT_LOOP, L.RQ_POLICY_FIRST_LOOP,
+                L.RQ_POLICY_PREVIOUS_LOOP):
+        assert L.rq_layout_validate(_lay(L, policy=pol)) == L.RQ_OK
+        assert L.rq_layout_validate(_lay(L, policy=pol, flags=L.RQ_FLAG_UNIT_ALPHA)) == L.RQ_OK
+    assert L.rq_layout_validate(_lay(L, flags=2)) == L.RQ_ERR_INVALID_ARG
     assert L.rq_cache_bytes(_lay(L, batch=0)) == 0
+
+
+def test_anchor_position_follows_the_policy(L):
+    """The anchor component (no LS coefficient, laid out first) is loop L-1
+    under Last-/Next-loop and loop 0 under First-/Previous-loop; the layer
+    size is the same (bits mirrored)."""
+    bits, group = (2, 2, 2, 4), (32, 16, 32, 64)
+    last = L.rq_cache_bind(_lay(L, bits=bits, group=group), 1 << 20, 1 << 30)
+    first = L.rq_cache_bind(_lay(L, bits=bits[::-1], group=group[::-1],
+                                 policy=L.RQ_POLICY_FIRST_LOOP), 1 << 20, 1 << 30)
+    assert last.layer_bytes == first.layer_bytes
+    assert last.comp_off[3] == 0 and first.comp_off[0] == 0
+    rec = lambda c, r: c.rec_bytes[r]
+    for r in range(4):
+        assert rec(last, r) == rec(first, 3 - r)
+    # the anchor record carries no alpha: 32 tokens x (codes + meta) only
+    assert rec(first, 0) == 32 * (128 * 4 // 8 + (128 // 64) * 4)
+    assert rec(first, 1) == 32 * (128 * 2 // 8 + (128 // 32) * 4 + 2)
+    # with the loops ascending after the anchor
+    assert first.comp_off[1] < first.comp_off[2] < first.comp_off[3]
 
 
 @pytest.mark.parametrize("bits,group", [((2, 2, 2, 4), (32,) * 4), ((4, 2, 2, 4), (32,) * 4),

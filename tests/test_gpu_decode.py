@@ -22,7 +22,8 @@ def _check_decode(gc, seq_lens, max_seq_len, loops=None, layer=0, bsel=None, hse
     for loop in loops:
         out, status = gpu_decode(gc, layer, loop, seq_lens, max_seq_len, ws)
         assert status == L.RQ_OK
-        ref = oracle_decode(w, layer, loop, bsel, hsel, seq_lens, gc.policy, gc.inputs or None)
+        ref = oracle_decode(w, layer, loop, bsel, hsel, seq_lens, gc.policy, gc.inputs or None,
+                            unit_alpha=gc.unit_alpha)
         got = out[np.ix_(bsel, hsel)]
         err = np.max(np.abs(got - ref))
         assert err <= attn_tolerance(ref), (loop, err, attn_tolerance(ref))
@@ -34,7 +35,7 @@ def test_tiny_reference_decode(cuda_dev):
     _check_decode(gc, [256], 256)
 
 
-@pytest.mark.parametrize("policy", ["last", "next"])
+@pytest.mark.parametrize("policy", ["last", "next", "first", "previous"])
 def test_ragged_lengths(cuda_dev, policy):
     """Ragged past lengths (0, a partial chunk, several chunks, full) in one batch."""
     w = synth.WORKLOADS["ouro_layer"].replace(batch=4, heads=3, tokens=777)
@@ -51,9 +52,19 @@ def test_mixed_precision_and_groups(cuda_dev):
 
 def test_deep_chain_head_dim_64(cuda_dev):
     w = synth.WORKLOADS["huginn_deep"].replace(batch=2, heads=2, tokens=300, head_dim=64)
-    for policy in ("last", "next"):
+    for policy in ("last", "next", "first", "previous"):
         gc = build_gpu_cache(w, policy=policy)
         _check_decode(gc, [300, 129], 300, loops=[0, 3, 6, 7])
+
+
+@pytest.mark.parametrize("policy", ["last", "previous"])
+def test_unit_alpha_decode(cuda_dev, policy):
+    """alpha = 1 (no LS scaling, [RQ Table 3]): plain inter-loop differences."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=300,
+                                              bits=(4, 2, 2, 2) if policy == "previous"
+                                              else (2, 2, 2, 4))
+    gc = build_gpu_cache(w, policy=policy, unit_alpha=True)
+    _check_decode(gc, [300, 77], 300)
 
 
 def test_no_past_tokens_returns_current_value(cuda_dev):

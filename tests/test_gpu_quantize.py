@@ -22,7 +22,7 @@ def _check_all(gc, layer=0, tokens=None, bsel=None, hsel=None, from_gpu_inputs=T
         if from_gpu_inputs:
             xl = [synth.bits_of(gc.inputs[(layer, side, l)][bsel][:, hsel].cpu()).reshape(-1, w.head_dim)
                   for l in range(w.loops)]
-        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, gc.policy, xl)
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, gc.policy, xl, gc.unit_alpha)
         for loop in range(w.loops):
             g = gpu_component(gc, layer, side, loop, bsel, hsel)
             gsel = {k: (None if v is None else v[:, :, :T]) for k, v in g.items()}
@@ -54,6 +54,8 @@ def test_tiny_reference_bit_exact(cuda_dev):
     ((2, 2, 4, 4), (64, 64, 16, 16), "last"),
     ((2, 2, 2, 4), (128, 32, 64, 128), "next"),
     ((2, 4, 2, 4), (32, 32, 32, 64), "next"),
+    ((4, 2, 2, 2), (32, 32, 32, 32), "first"),
+    ((4, 2, 4, 2), (32, 16, 64, 128), "previous"),
 ])
 def test_ragged_shapes_bit_exact(cuda_dev, bits, group, policy):
     """Several warps, a ragged row tail and every bit-width / group size."""
@@ -143,6 +145,8 @@ def test_dequantize_matches_oracle(cuda_dev):
     ((2, 2, 2, 4), (16, 16, 16, 32), "last"),
     ((2, 2, 4, 4), (64, 64, 16, 16), "next"),
     ((2, 2, 2, 4), (128, 32, 64, 128), "next"),
+    ((4, 2, 2, 2), (32, 32, 32, 32), "first"),
+    ((4, 2, 4, 2), (32, 16, 64, 128), "previous"),
 ])
 def test_fused_loops_bit_exact(cuda_dev, bits, group, policy):
     """One launch per chunk stores the bits of the per-loop path: codes,
@@ -186,3 +190,28 @@ def test_fused_one_side_leaves_the_other(cuda_dev):
         g = gpu_component(gc, 0, synth.SIDE_K, loop)
         g = {k: (None if v is None else v[:, :, :66]) for k, v in g.items()}
         assert_component_equal(g, encs[loop], None, f"K loop {loop}")
+
+
+@pytest.mark.parametrize("policy,fused", [("last", False), ("next", True), ("first", True),
+                                          ("previous", False)])
+def test_unit_alpha_bit_exact(cuda_dev, policy, fused):
+    """alpha = 1 (RQ_FLAG_UNIT_ALPHA): plain differences against the reference,
+    every alpha stored as bf16(1.0), both append paths."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=97)
+    gc = build_gpu_cache(w, policy=policy, fused=fused, unit_alpha=True)
+    _check_all(gc)
+    a = oracle.anchor_loop(w.loops, policy)
+    for loop in range(w.loops):
+        if loop != a:
+            al = gpu_component(gc, 0, 0, loop)["alpha"][:, :, :w.tokens]
+            assert np.all(al == 0x3F80)
+
+
+def test_first_loop_deep_head_dim_64_bit_exact(cuda_dev):
+    w = synth.WORKLOADS["huginn_deep"].replace(batch=1, heads=3, tokens=77, head_dim=64, loops=5,
+                                               bits=(4, 2, 2, 4, 2), group=(32, 16, 64, 64, 32),
+                                               sigma=(0.4, 0.3, 0.2, 0.1))
+    for policy in ("first", "previous"):
+        for fused in (False, True):
+            gc = build_gpu_cache(w, policy=policy, fused=fused)
+            _check_all(gc)
