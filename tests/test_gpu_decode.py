@@ -128,3 +128,14 @@ def test_bf16_decode_matches_oracle(cuda_dev):
     ref = oracle.decode_attention(kf, vf, synth.bits_of(q), seq, synth.bits_of(kc), synth.bits_of(vc))
     got = out.cpu().numpy()
     assert np.max(np.abs(got - ref)) <= attn_tolerance(ref)
+
+
+def test_maximum_loop_count_chain_decode(cuda_dev):
+    """32 loops under the Next-loop chain: loop 0 reads 32 components (the
+    layout-generic decode kernel); every loop within tolerance."""
+    bits = tuple([2] * 31 + [4])
+    w = synth.WORKLOADS["huginn_deep"].replace(loops=32, batch=1, heads=2, tokens=200, head_dim=64,
+                                               bits=bits, group=tuple([32] * 32),
+                                               sigma=tuple(np.linspace(0.4, 0.1, 31)))
+    gc = build_gpu_cache(w, policy="next")
+    _check_decode(gc, [200], 200, loops=[0, 1, 15, 30, 31])

@@ -215,3 +215,108 @@ def test_first_loop_deep_head_dim_64_bit_exact(cuda_dev):
         for fused in (False, True):
             gc = build_gpu_cache(w, policy=policy, fused=fused)
             _check_all(gc)
+
+
+# ---- degenerate rows and extreme magnitudes, through the C ABI on given rows
+
+def _encode_given_rows(x_loops, bits, group, policy="last"):
+    """x_loops: uint16 numpy [L, N, D] bf16 bits.  Quantises them through the
+    C ABI (per-loop and fused paths) as batch 1, N heads, 1 token, and returns
+    (gpu components of both paths, oracle encodings)."""
+    import residual_bit_kv_b200.librq as L
+    from rq_harness import policy_code
+    Lp, N, D = x_loops.shape
+    lay = L.make_layout(1, Lp, 1, N, D, 64, bits, group, policy_code(policy))
+    nb = L.rq_cache_bytes(lay)
+    out = []
+    for fused in (False, True):
+        kb = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        vb = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        cache = L.rq_cache_bind(lay, kb, vb)
+        xs = torch.from_numpy(x_loops.astype(np.int16)).view(torch.bfloat16).cuda()
+        if fused:
+            L.rq_quantize_append_loops(cache, 0, xs.contiguous(), None, 0, 1)
+        else:
+            a = oracle.anchor_loop(Lp, policy)
+            for loop in [a] + oracle.encode_order(Lp, policy):
+                x = xs[loop].contiguous()
+                if loop == a:
+                    L.rq_quantize_anchor(cache, 0, 0, x, 0, 1)
+                else:
+                    L.rq_quantize_append_residual(cache, 0, 0, loop, x, 0, 1)
+        torch.cuda.synchronize()
+        w = synth.WORKLOADS["tiny"].replace(loops=Lp, batch=1, heads=N, head_dim=D, tokens=1,
+                                           bits=tuple(bits), group=tuple(group))
+        from rq_harness import GpuCache
+        gc = GpuCache(w, policy, lay, cache, kb, vb, {})
+        out.append([{k: (None if v is None else v[:, :, :1]) for k, v in
+                     gpu_component(gc, 0, 0, loop).items()} for loop in range(Lp)])
+    return out, oracle.encode_side(x_loops, bits, group, policy)
+
+
+def _bf16_bits(a):
+    return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy() \
+        .view(np.uint16)
+
+
+def test_degenerate_rows_bit_exact(cuda_dev):
+    """Zero rows, constant rows (every group range 0: s~ = 0, codes 0),
+    a single non-zero channel, and loops equal to the anchor (zero residual)."""
+    D = 128
+    rows = np.zeros((6, D), np.float32)
+    rows[1] = 3.25                                   # constant row
+    rows[2, 17] = -7.0                               # one non-zero channel
+    rows[3] = np.linspace(-1, 1, D)
+    rows[4] = -0.0                                   # negative zero
+    rows[5, ::2] = 1e-30                             # subnormal after rotation
+    anchor = _bf16_bits(rows)
+    loops = np.stack([anchor, _bf16_bits(rows * 0.5), _bf16_bits(np.zeros_like(rows)), anchor])
+    for policy in ("last", "next"):
+        (per_loop, fused), encs = _encode_given_rows(loops, (2, 2, 2, 4), (32, 16, 64, 32), policy)
+        for got in (per_loop, fused):
+            for r in range(4):
+                assert_component_equal(got[r], encs[r], None, f"{policy} loop {r}")
+
+
+def test_extreme_magnitudes_bit_exact(cuda_dev):
+    """Large magnitudes with tiny ranges (the fp16 offset's rounding exceeds
+    a quantisation step, so the clamps decide codes), spikes near the fp16
+    limit after rotation, and very small values: bit-exact on both sides.
+    Inputs stay where the fp16 scale and offset are finite; beyond that the
+    method produces NaN metadata, whose bit pattern the pages do not fix."""
+    D = 64
+    rng = np.random.default_rng(3)
+    rows = rng.standard_normal((8, D)).astype(np.float32)
+    rows[0] *= 2000.0
+    rows[1] = 5e3 + 1e-2 * rows[1]                   # range far below the offset's ulp
+    rows[2, :5] = 7999.0
+    rows[3] *= 1e-6
+    rows[4, 0] = 8000.0
+    rows[5] = 1000.0 + np.arange(D, dtype=np.float32)
+    rows[6, 10] = -8000.0
+    anchor = _bf16_bits(rows)
+    loops = np.stack([_bf16_bits(rows[::-1].copy()), anchor])
+    for bits in ((2, 4), (4, 2)):
+        (per_loop, fused), encs = _encode_given_rows(loops, bits, (32, 64), "last")
+        for r in range(2):
+            m = encs[r]["meta"]
+            assert not np.any(((m & 0x7C00) == 0x7C00) & ((m & 0x3FF) != 0))
+            assert not np.any((((m >> 16) & 0x7C00) == 0x7C00) & (((m >> 16) & 0x3FF) != 0))
+        for got in (per_loop, fused):
+            for r in range(2):
+                assert_component_equal(got[r], encs[r], None, f"bits {bits} loop {r}")
+
+
+def test_maximum_loop_count_chain(cuda_dev):
+    """RQ_MAX_LOOPS = 32 loops under the Next-loop chain (loop 0 is rebuilt from
+    32 components): every code bit-exact, both append paths."""
+    import residual_bit_kv_b200.librq as L
+    bits = tuple([2] * 31 + [4])
+    group = tuple([32] * 32)
+    w = synth.WORKLOADS["huginn_deep"].replace(loops=32, batch=1, heads=2, tokens=40, head_dim=64,
+                                               bits=bits, group=group,
+                                               sigma=tuple(np.linspace(0.4, 0.1, 31)))
+    assert w.loops == L.RQ_MAX_LOOPS
+    for fused in (False, True):
+        gc = build_gpu_cache(w, policy="next", fused=fused)
+        _check_all(gc)
