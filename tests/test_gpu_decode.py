@@ -139,3 +139,16 @@ def test_maximum_loop_count_chain_decode(cuda_dev):
                                                sigma=tuple(np.linspace(0.4, 0.1, 31)))
     gc = build_gpu_cache(w, policy="next")
     _check_decode(gc, [200], 200, loops=[0, 1, 15, 30, 31])
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 777, 4096, 16384, 65536])
+@pytest.mark.parametrize("batch,heads", [(1, 1), (2, 3), (16, 16), (64, 40)])
+def test_split_plan_invariants(cuda_dev, T, batch, heads):
+    """The split count of a decode call: at least one, no more than the
+    workspace holds (one per 64-token chunk), and never an empty split."""
+    lay = L.make_layout(1, 4, batch, heads, 128, T, (2, 2, 2, 4), (32,) * 4)
+    s = L.rq_decode_splits(lay, T)
+    chunks = (T + 63) // 64
+    assert 1 <= s <= max(1, chunks)
+    cps = -(-chunks // s)
+    assert -(-chunks // cps) == s
