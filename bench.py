@@ -477,34 +477,37 @@ CPU_POOL_MAX_WORKERS = 64
 
 
 def _pool_worker(args):
-    """One oracle process: set-up (generation and encoding) untimed, then a
-    barrier, then the timed decode of its units.  Returns its timed window."""
-    name, (b, h), loops, barrier = args
+    """One oracle process: set-up (generation and encoding of its units)
+    untimed, then a barrier, then the timed decode of its units for every
+    loop.  Returns its timed window."""
+    name, pairs, loops, barrier = args
     w = synth.WORKLOADS[name]
     q, kc, vc = step_inputs_cpu(w, loops)
-    encs = oracle_prepare(w, b, h)
-    oracle_run(w, b, h, encs, loops, q, kc, vc)   # warm: library load, page-in
+    prep = [(b, h, oracle_prepare(w, b, h)) for b, h in pairs]
+    b0, h0, e0 = prep[0]
+    oracle_run(w, b0, h0, e0, loops[:1], q, kc, vc)   # warm: library load, page-in
     barrier.wait()
     t0 = time.perf_counter()
-    units = oracle_run(w, b, h, encs, loops, q, kc, vc)
+    units = sum(oracle_run(w, b, h, e, loops, q, kc, vc) for b, h, e in prep)
     t1 = time.perf_counter()
     return t0, t1, units
 
 
 def cpu_baseline_all_cores(w):
-    """The same oracle decode run as independent processes over (batch, head)
-    units on every host core (capped at CPU_POOL_MAX_WORKERS), each unit
-    single-threaded; throughput = units / wall time of the timed windows."""
+    """The oracle's decode of the whole of layer 0 (every (batch, head) unit,
+    every loop) as independent processes on every host core (capped at
+    CPU_POOL_MAX_WORKERS), each unit single-threaded; throughput = units /
+    wall time of the timed windows."""
     import multiprocessing as mp
     ncpu = os.cpu_count() or 1
-    workers = max(1, min(ncpu, CPU_POOL_MAX_WORKERS))
+    pairs = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    workers = max(1, min(ncpu, CPU_POOL_MAX_WORKERS, len(pairs)))
     ctx = mp.get_context("spawn")
-    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(workers)]
     with ctx.Manager() as man:
         barrier = man.Barrier(workers)
         with ctx.Pool(workers) as pool:
-            res = pool.map(_pool_worker,
-                           [(w.name, pr, list(range(w.loops)), barrier) for pr in pairs])
+            res = pool.map(_pool_worker, [(w.name, pairs[i::workers], list(range(w.loops)),
+                                           barrier) for i in range(workers)])
     t0 = min(r[0] for r in res)
     t1 = max(r[1] for r in res)
     units = sum(r[2] for r in res)
@@ -521,22 +524,10 @@ def cpu_baseline_all_cores(w):
         pass
     return {"value": w.batch / step_s, "unit": "tokens/s", "cores": workers, "nproc": ncpu,
             "cpu_model": model, "kind": "oracle",
-            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens}, one "
-                      f"(batch,head) per process ({t1 - t0:.1f} s wall), scaled to {step_units} "
-                      f"units per step"}
-
-
-def cpu_baseline(w):
-    """Oracle decode on a bounded sample: (batch, head) units x 4 loops of
-    layer 0 at the full 16k context until about 10 s of timed CPU work,
-    scaled to the step's 24*4*B*H units."""
-    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(w.batch * w.heads)]
-    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)), CPU_BASELINE_SECONDS)
-    step_units = w.layers * w.loops * w.batch * w.heads
-    step_s = secs / units * step_units
-    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens} "
-                      f"({secs:.1f} s timed), scaled to {step_units} units per step"}
+            "ms_per_call": (t1 - t0) / w.loops * 1e3,
+            "sample": f"all of layer 0: {units} (batch,head,loop) decode units at T={w.tokens} "
+                      f"({t1 - t0:.1f} s wall on {workers} processes; one call = one loop of "
+                      f"the layer), scaled to {step_units} units per step"}
 
 
 def run_reference(args, rank):
