@@ -530,6 +530,19 @@ def cpu_baseline_all_cores(w):
                       f"the layer), scaled to {step_units} units per step"}
 
 
+def cpu_baseline(w):
+    """Oracle decode on a bounded sample: (batch, head) units x 4 loops of
+    layer 0 at the full 16k context until about 10 s of timed CPU work,
+    scaled to the step's 24*4*B*H units."""
+    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(w.batch * w.heads)]
+    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)), CPU_BASELINE_SECONDS)
+    step_units = w.layers * w.loops * w.batch * w.heads
+    step_s = secs / units * step_units
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens} "
+                      f"({secs:.1f} s timed), scaled to {step_units} units per step"}
+
+
 def run_reference(args, rank):
     if rank != 0:
         return 0
