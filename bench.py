@@ -477,37 +477,39 @@ CPU_POOL_MAX_WORKERS = 64
 
 
 def _pool_worker(args):
-    """One oracle process: set-up (generation and encoding of its units)
-    untimed, then a barrier, then the timed decode of its units for every
-    loop.  Returns its timed window."""
-    name, pairs, loops, barrier = args
+    """One oracle process (one torch thread): set-up (generation and encoding
+    of its unit) untimed, then a barrier, then the timed decode of its unit
+    for every loop.  Returns its timed window."""
+    name, (b, h), loops, barrier = args
+    torch.set_num_threads(1)
     w = synth.WORKLOADS[name]
     q, kc, vc = step_inputs_cpu(w, loops)
-    prep = [(b, h, oracle_prepare(w, b, h)) for b, h in pairs]
-    b0, h0, e0 = prep[0]
-    oracle_run(w, b0, h0, e0, loops[:1], q, kc, vc)   # warm: library load, page-in
+    encs = oracle_prepare(w, b, h)
+    oracle_run(w, b, h, encs, loops[:1], q, kc, vc)   # warm: library load, page-in
     barrier.wait()
     t0 = time.perf_counter()
-    units = sum(oracle_run(w, b, h, e, loops, q, kc, vc) for b, h, e in prep)
+    units = oracle_run(w, b, h, encs, loops, q, kc, vc)
     t1 = time.perf_counter()
     return t0, t1, units
 
 
 def cpu_baseline_all_cores(w):
-    """The oracle's decode of the whole of layer 0 (every (batch, head) unit,
-    every loop) as independent processes on every host core (capped at
-    CPU_POOL_MAX_WORKERS), each unit single-threaded; throughput = units /
-    wall time of the timed windows."""
+    """The oracle's decode as independent processes on every host core
+    (capped at CPU_POOL_MAX_WORKERS): one (batch, head) unit of layer 0 per
+    process, every loop, each unit single-threaded; throughput = units / wall
+    time of the timed windows.  (The whole layer would take several minutes of
+    set-up on the host, outside the benchmark's time budget; this is a
+    bounded sample of it.)"""
     import multiprocessing as mp
     ncpu = os.cpu_count() or 1
-    pairs = [(b, h) for b in range(w.batch) for h in range(w.heads)]
-    workers = max(1, min(ncpu, CPU_POOL_MAX_WORKERS, len(pairs)))
+    workers = max(1, min(ncpu, CPU_POOL_MAX_WORKERS, w.batch * w.heads))
+    pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(workers)]
     ctx = mp.get_context("spawn")
     with ctx.Manager() as man:
         barrier = man.Barrier(workers)
         with ctx.Pool(workers) as pool:
-            res = pool.map(_pool_worker, [(w.name, pairs[i::workers], list(range(w.loops)),
-                                           barrier) for i in range(workers)])
+            res = pool.map(_pool_worker, [(w.name, pr, list(range(w.loops)), barrier)
+                                          for pr in pairs])
     t0 = min(r[0] for r in res)
     t1 = max(r[1] for r in res)
     units = sum(r[2] for r in res)
@@ -522,12 +524,13 @@ def cpu_baseline_all_cores(w):
                     break
     except OSError:
         pass
+    call_units = w.batch * w.heads   # one decode call = one loop of one layer
     return {"value": w.batch / step_s, "unit": "tokens/s", "cores": workers, "nproc": ncpu,
             "cpu_model": model, "kind": "oracle",
-            "ms_per_call": (t1 - t0) / w.loops * 1e3,
-            "sample": f"all of layer 0: {units} (batch,head,loop) decode units at T={w.tokens} "
-                      f"({t1 - t0:.1f} s wall on {workers} processes; one call = one loop of "
-                      f"the layer), scaled to {step_units} units per step"}
+            "ms_per_call": (t1 - t0) / units * call_units * 1e3,
+            "sample": f"{units} (batch,head,loop) decode units of layer 0 at T={w.tokens}, one "
+                      f"(batch,head) per process ({t1 - t0:.1f} s wall on {workers} processes), "
+                      f"scaled to {step_units} units per step ({call_units} per call)"}
 
 
 def cpu_baseline(w):

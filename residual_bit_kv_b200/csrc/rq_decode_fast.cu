@@ -547,12 +547,6 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
 }
 
 // ---------------------------------------------------------------- BF16 --
-//
-// Uncompressed baseline on the same split-K engine: a producer warp streams
-// the bf16 K and V rows of a split through an S-stage ring (full / empty
-// mbarriers, bulk copies of TC rows); 8 compute warps score with packed fp32
-// FMAs against the unrotated query, run the same online softmax and
-// accumulate V; partials merge as in the compressed kernel (no rotation).
 
 template <int D>
 __host__ __device__ constexpr int bf16_tc() { return D == 64 ? 128 : 64; }

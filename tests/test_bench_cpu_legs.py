@@ -29,7 +29,7 @@ def test_cpu_baseline_single_core(monkeypatch):
     assert "decode units of layer 0" in r["sample"]
 
 
-def test_cpu_baseline_all_cores_covers_the_layer(monkeypatch):
+def test_cpu_baseline_all_cores(monkeypatch):
     import bench
     monkeypatch.setattr(bench, "CPU_POOL_MAX_WORKERS", 2)
     import residual_bit_kv_b200.synth as synth
@@ -37,7 +37,7 @@ def test_cpu_baseline_all_cores_covers_the_layer(monkeypatch):
     r = bench.cpu_baseline_all_cores(w)
     assert r["kind"] == "oracle" and 1 <= r["cores"] <= 2 and r["nproc"] >= 1
     assert r["value"] > 0 and r["ms_per_call"] > 0
-    assert f"{w.batch * w.heads * w.loops} (batch,head,loop)" in r["sample"]
+    assert f"{r['cores'] * w.loops} (batch,head,loop)" in r["sample"]
 
 
 def test_reference_arm_prints_one_line():
