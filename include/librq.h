@@ -126,7 +126,7 @@ typedef struct rq_cache {
   uint64_t layer_bytes;
   int64_t token_stride;              /* max_tokens rounded up to 64 */
   uint64_t comp_off[RQ_MAX_LOOPS];   /* first record of loop r (256-B aligned) */
-  uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 64-token record of loop r */
+  uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 32-token record of loop r */
 } rq_cache;
 
 /* ABI version of the loaded library (RQ_ABI_VERSION at build time). */
