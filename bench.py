@@ -472,7 +472,7 @@ def oracle_decode_sample(w, pairs, loops, budget_s=None):
     return secs, units
 
 
-CPU_BASELINE_SECONDS = 10.0
+CPU_SAMPLE_SECONDS = 10.0
 CPU_POOL_MAX_WORKERS = 64
 
 
@@ -538,7 +538,7 @@ def cpu_baseline(w):
     layer 0 at the full 16k context until about 10 s of timed CPU work,
     scaled to the step's 24*4*B*H units."""
     pairs = [(i % w.batch, (5 * i) % w.heads) for i in range(w.batch * w.heads)]
-    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)), CPU_BASELINE_SECONDS)
+    secs, units = oracle_decode_sample(w, pairs, list(range(w.loops)), CPU_SAMPLE_SECONDS)
     step_units = w.layers * w.loops * w.batch * w.heads
     step_s = secs / units * step_units
     return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",

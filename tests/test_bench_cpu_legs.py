@@ -21,7 +21,7 @@ def _small():
 
 def test_cpu_baseline_single_core(monkeypatch):
     import bench
-    monkeypatch.setattr(bench, "CPU_BASELINE_SECONDS", 0.01)
+    monkeypatch.setattr(bench, "CPU_SAMPLE_SECONDS", 0.01)
     w = _small()
     r = bench.cpu_baseline(w)
     assert r["kind"] == "oracle" and r["cores"] == 1 and r["unit"] == "tokens/s"
