@@ -15,6 +15,8 @@ Array conventions (all C-contiguous):
          that nesting order), channel d.  Loop L-1 is the final-loop anchor.
   codes  uint32 [N, D*bits/32]; meta uint32 [N, D/group] (fp16 scale in the
          low half, fp16 offset in the high half); alpha uint16 [N] (bf16).
+  quantize_m8: the 16-bit-metadata variant, meta uint16 [D/group] (scale
+         byte, offset byte); see rqo.h.
 
 Parity unpinned: nothing here is pinned against learned rotations, real
 model KV, or the pages' accuracy / NMSE / throughput numbers; the pins are
@@ -118,6 +120,9 @@ def lib() -> ctypes.CDLL:
             "rqo_effective_bits": ([_I, _P, _P, _I, _I, _I], _D),
             "rqo_component_reads": ([_I, _I], _I64),
             "rqo_code_pos": ([_I, _I, _P, _P], None),
+            "rqo_m8_scale_encode": ([_F], ctypes.c_uint8),
+            "rqo_m8_scale_decode": ([ctypes.c_uint8], _F),
+            "rqo_quantize_m8": ([_P, _I, _I, _I, _P, _P, _P], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(h, name)
@@ -190,6 +195,30 @@ def quantize(z: np.ndarray, bits: int, group: int):
     meta = np.zeros(D // group, np.uint32)
     deq = np.zeros(D, np.float32)
     lib().rqo_quantize(_ptr(z), D, bits, group, _ptr(words), _ptr(meta), _ptr(deq))
+    return words, meta, deq
+
+
+M8_BIAS = 18   # exponent bias of the 16-bit-metadata scale byte (rqo.h)
+
+
+def m8_scale_encode(s: float) -> int:
+    """Scale byte (unsigned e5m3) of the 16-bit-metadata variant."""
+    return int(lib().rqo_m8_scale_encode(float(s)))
+
+
+def m8_scale_decode(b: int) -> float:
+    return float(lib().rqo_m8_scale_decode(int(b)))
+
+
+def quantize_m8(z: np.ndarray, bits: int, group: int):
+    """Affine-quantise one rotated fp32 row with 16-bit metadata per group:
+    (words, meta uint16 [D/group] = scale byte | offset byte << 8, deq)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    D = z.shape[-1]
+    words = np.zeros(D * bits // 32, np.uint32)
+    meta = np.zeros(D // group, np.uint16)
+    deq = np.zeros(D, np.float32)
+    lib().rqo_quantize_m8(_ptr(z), D, bits, group, _ptr(words), _ptr(meta), _ptr(deq))
     return words, meta, deq
 
 

@@ -190,6 +190,81 @@ void rqo_quantize(const float* z, int D, int bits, int group, uint32_t* words,
 }
 
 /* ------------------------------------------------------------------------ */
+/* 16-bit metadata variant [RQ §5.1, App. A.3: 16 bits of scale and offset  */
+/* per group]                                                              */
+/* ------------------------------------------------------------------------ */
+
+uint8_t rqo_m8_scale_encode(float s) {
+  if (!(s > 0.0f)) return 0u;                       /* zero, negative, NaN */
+  uint32_t b;
+  memcpy(&b, &s, sizeof(b));
+  int E = (int)((b >> 23) & 0xFFu);
+  if (E == 0xFF) return 0xFFu;                      /* infinity: the largest */
+  if (E == 0) return 0x08u;                         /* fp32 subnormal: the smallest */
+  uint32_t m = (b & 0x7FFFFFu) >> 20;               /* top 3 mantissa bits */
+  const uint32_t rem = b & 0xFFFFFu;                /* the 20 bits dropped */
+  if (rem > 0x80000u || (rem == 0x80000u && (m & 1u))) ++m;
+  if (m == 8u) {
+    m = 0u;
+    ++E;
+  }
+  const int Eb = E - 127 + RQO_M8_BIAS;
+  if (Eb < 1) return 0x08u;
+  if (Eb > 31) return 0xFFu;
+  return (uint8_t)(((uint32_t)Eb << 3) | m);
+}
+
+float rqo_m8_scale_decode(uint8_t b) {
+  const int Eb = b >> 3, m = b & 7;
+  if (Eb == 0) return 0.0f;
+  return ldexpf(1.0f + (float)m / 8.0f, Eb - RQO_M8_BIAS);
+}
+
+void rqo_quantize_m8(const float* z, int D, int bits, int group, uint32_t* words,
+                     uint16_t* meta, float* deq) {
+  const int qmax = (1 << bits) - 1;
+  for (int w = 0; w < D * bits / 32; ++w) words[w] = 0u;
+
+  for (int g0 = 0, j = 0; g0 < D; g0 += group, ++j) {
+    float mn = z[g0], mx = z[g0];
+    for (int i = g0 + 1; i < g0 + group; ++i) {
+      if (z[i] < mn) mn = z[i];
+      if (z[i] > mx) mx = z[i];
+    }
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
+
+    /* Scale: the range over the code steps, at least |mn| / 15.875 so that
+     * the offset fits its byte; rounded to the scale byte. */
+    const float s0 = (mx - mn) / (float)qmax;
+    const float s1 = fabsf(mn) / 15.875f;
+    const uint8_t sb = rqo_m8_scale_encode(s0 > s1 ? s0 : s1);
+    const float st = rqo_m8_scale_decode(sb);
+
+    /* Offset: the largest multiple of s~/8 not above mn (clamped). */
+    int zq = 0;
+    if (st > 0.0f) {
+      const float t = floorf((8.0f * mn) / st);
+      zq = t < -128.0f ? -128 : (t > 127.0f ? 127 : (int)t);
+    }
+    const float zt = (float)zq * st * 0.125f;
+    const float inv = (st > 0.0f) ? 1.0f / st : 0.0f;
+    meta[j] = (uint16_t)((uint32_t)sb | (((uint32_t)zq & 0xFFu) << 8));
+
+    for (int i = g0; i < g0 + group; ++i) {
+      float u = (z[i] - zt) * inv;
+      if (u < 0.0f) u = 0.0f;
+      if (u > (float)qmax) u = (float)qmax;
+      const uint32_t code = (uint32_t)rintf(u);
+      int wi, bit;
+      rqo_code_pos(i, bits, &wi, &bit);
+      words[wi] |= code << bit;
+      deq[i] = fmaf(st, (float)code, zt);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Anchor and residual encoders [RQ §3.2, §3.3, §3.4, App. G.1, App. G.2]    */
 /* ------------------------------------------------------------------------ */
 

@@ -73,6 +73,28 @@ void rqo_code_pos(int i, int bits, int* word, int* shift);
 void rqo_quantize(const float* z, int D, int bits, int group,
                   uint32_t* words, uint32_t* meta, float* deq);
 
+/* 16-bit metadata per group (scale byte + offset byte), the storage the
+ * pages count for scales and offsets (16 bits per group [RQ §5.1, App. A.3];
+ * the pages do not give the format, this one is the library's choice):
+ *   scale byte: unsigned e5m3, b = 8 E + m; E = 0 encodes a zero scale,
+ *     else s~ = (1 + m/8) * 2^(E - RQO_M8_BIAS), E in 1..31, m in 0..7.
+ *   rqo_m8_scale_encode rounds a finite s >= 0 to the nearest such value
+ *     (ties to even m), sends s below the smallest positive value to the
+ *     smallest and above the largest to the largest; s <= 0 or NaN -> 0. */
+#define RQO_M8_BIAS 18
+uint8_t rqo_m8_scale_encode(float s);
+float   rqo_m8_scale_decode(uint8_t b);
+
+/* Group-wise affine quantisation with 16-bit metadata: per group, mn, mx
+ * (+0 for zeros); s0 = (mx - mn)/(2^b - 1); s1 = |mn| / 15.875;
+ * s~ = decode(encode(max(s0, s1))) (s1 keeps the offset inside the offset
+ * byte's range); offset byte zq = clamp(floor((8 mn) / s~), -128, 127)
+ * (0 if s~ == 0), z~ = zq * s~ / 8 (exact); codes and levels as in
+ * rqo_quantize: inv = 1/s~ (0 if s~ == 0), c = rint(clamp((z - z~) * inv)),
+ * deq = fma(s~, c, z~).  meta[j] = scale byte | (offset byte << 8). */
+void rqo_quantize_m8(const float* z, int D, int bits, int group,
+                     uint32_t* words, uint16_t* meta, float* deq);
+
 /* Anchor of the final loop [RQ §3.2 Last-loop policy, §3.4, App. G.2]:
  * Z = H x (x bf16), quantised with the anchor's bits and group.
  * zhat receives the dequantised rotated anchor A (fp32). */

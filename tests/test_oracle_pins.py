@@ -500,3 +500,132 @@ def test_unit_alpha_residual_closed_form(oracle_mod):
 
 def synth_bits(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------- 16-bit metadata per group --
+# The pages count 16 bits of scale and offset per group [RQ §5.1, App. A.3]
+# without fixing a format; the variant here is a scale byte (unsigned e5m3)
+# and an offset byte (a multiple of scale/8).
+
+def _m8_value(b):
+    """The scale byte's value from its definition, in exact fp64."""
+    E, m = b >> 3, b & 7
+    return 0.0 if E == 0 else (1 + m / 8) * 2.0 ** (E - 18)
+
+
+def test_m8_scale_byte_table_and_round_trip(oracle_mod):
+    assert oracle_mod.M8_BIAS == 18
+    for b in range(256):
+        v = oracle_mod.m8_scale_decode(b)
+        assert v == _m8_value(b), b
+        if b >> 3:
+            assert oracle_mod.m8_scale_encode(v) == b, b
+    assert oracle_mod.m8_scale_encode(0.0) == 0 and oracle_mod.m8_scale_encode(-1.0) == 0
+    assert oracle_mod.m8_scale_encode(float("nan")) == 0
+
+
+def test_m8_scale_is_nearest_brute_force(oracle_mod):
+    """Every positive input goes to the nearest representable value (ties to
+    the even m), below the range to the smallest, above it to the largest."""
+    vals = np.array([_m8_value(b) for b in range(8, 256)])
+    rng = np.random.default_rng(11)
+    s = np.float32(2.0) ** rng.uniform(-20, 15, 3000).astype(np.float32)
+    # exact midpoints between neighbours (ties)
+    mids = ((vals[:-1] + vals[1:]) / 2)
+    mids = mids[np.float32(mids) == mids].astype(np.float32)
+    for x in np.concatenate([s, mids]):
+        x = float(x)
+        b = oracle_mod.m8_scale_encode(x)
+        got = _m8_value(b)
+        if x < vals[0]:
+            assert b == 0x08
+            continue
+        if x > vals[-1]:
+            assert b == 0xFF
+            continue
+        d = np.abs(vals - x)
+        best = d.min()
+        assert abs(got - x) == best, (x, got)
+        if (d == best).sum() == 2:      # a tie: the even mantissa wins
+            assert (b & 7) % 2 == 0, (x, b)
+
+
+def test_m8_ramp_uses_all_four_levels(oracle_mod):
+    """Scale 1 and offset -1.5 are exact in the bytes: the INT2 ramp
+    -1.5, -0.5, 0.5, 1.5 gets codes 0..3 and dequantises exactly."""
+    z = np.array([-1.5, -0.5, 0.5, 1.5] * 8, np.float32)
+    words, meta, deq = oracle_mod.quantize_m8(z, 2, 32)
+    np.testing.assert_array_equal(oracle_mod.unpack_codes(words, 2, 32), np.tile(np.arange(4), 8))
+    assert meta[0] & 0xFF == oracle_mod.m8_scale_encode(1.0)
+    assert np.int8(np.uint8(meta[0] >> 8)) == -12
+    np.testing.assert_array_equal(deq, z)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 16), (2, 32), (2, 64), (4, 32), (4, 128)])
+def test_m8_codes_are_nearest_level_brute_force(oracle_mod, bits, group):
+    """Metadata from its definition; every code the nearest level of the
+    grid z~ + k s~ (clamped), away from half-way ties; z~ <= mn < z~ + s~/8
+    while the offset byte is not saturated."""
+    rng = np.random.default_rng(bits * 1000 + group)
+    qmax = (1 << bits) - 1
+    checked = 0
+    for trial in range(40):
+        z = (rng.standard_normal(128) * rng.uniform(0.01, 5) +
+             rng.uniform(-1, 1) * (trial % 3)).astype(np.float32)
+        words, meta, deq = oracle_mod.quantize_m8(z, bits, group)
+        codes = oracle_mod.unpack_codes(words, bits, 128).astype(np.int64)
+        for gi in range(128 // group):
+            sl = slice(gi * group, (gi + 1) * group)
+            zg = z[sl]
+            mn, mx = np.float32(zg.min()), np.float32(zg.max())
+            s0 = np.float32(np.float32(mx - mn) / np.float32(qmax))
+            s1 = np.float32(np.float32(abs(mn)) / np.float32(15.875))
+            sb = int(meta[gi]) & 0xFF
+            zq = int(np.int8(np.uint8(int(meta[gi]) >> 8)))
+            assert sb == oracle_mod.m8_scale_encode(float(max(s0, s1)))
+            s = _m8_value(sb)
+            o = zq * s / 8
+            t = np.floor(np.float32(np.float32(8) * mn) / np.float32(s))
+            if -128 <= t <= 127:
+                assert zq == t and o <= mn < o + s / 8
+            levels = o + s * np.arange(qmax + 1)
+            best = np.argmin(np.abs(zg[:, None].astype(np.float64) - levels[None, :]), axis=1)
+            u = (zg.astype(np.float64) - o) / s
+            ok = _tie_distance(np.clip(u, 0, qmax)) > 1e-4
+            np.testing.assert_array_equal(codes[sl][ok], best[ok])
+            checked += ok.sum()
+            np.testing.assert_array_equal(deq[sl], np.float32(levels[codes[sl]]))
+    assert checked > 1000
+
+
+def test_m8_constant_group_keeps_its_value(oracle_mod):
+    """A constant nonzero group (zero range) is still reproduced: the scale
+    becomes |c| / 15.875 (rounded) and the level nearest to c is within half
+    a step; a zero group stays exactly zero."""
+    for c in (3.0, -0.7, 1e-3, -250.0):
+        z = np.full(32, c, np.float32)
+        words, meta, deq = oracle_mod.quantize_m8(z, 2, 32)
+        s = _m8_value(int(meta[0]) & 0xFF)
+        assert 0 < s <= abs(c) / 15.875 * (1 + 1 / 16) + 1e-12
+        assert np.all(np.abs(deq - c) <= s / 2 + 1e-6 * abs(c))
+    words, meta, deq = oracle_mod.quantize_m8(np.zeros(32, np.float32), 2, 32)
+    assert meta[0] == 0 and not deq.any() and not words.any()
+
+
+def test_m8_error_close_to_fp16_metadata(oracle_mod):
+    """Design check on rotated synthetic rows: halving the metadata costs at
+    most 10% (INT2) / 15% (INT4) more squared error than fp16 scale + fp16
+    offset, and the offset byte never saturates on this data."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"]
+    x = synth.kv_full(w, 0, 0, 1, 0, 32, device="cpu").float().numpy().reshape(-1, 128)[:512]
+    Z = oracle_mod.fwht_f32(x.astype(np.float32))
+    for bits, lim in ((2, 1.10), (4, 1.15)):
+        e16 = e8 = 0.0
+        for row in Z:
+            e16 += float(((oracle_mod.quantize(row, bits, 32)[2] - row) ** 2).sum())
+            words, meta, deq = oracle_mod.quantize_m8(row, bits, 32)
+            e8 += float(((deq - row) ** 2).sum())
+            zq = (meta >> 8).astype(np.uint8).view(np.int8)
+            assert np.all((zq > -128) & (zq < 127))
+        assert e8 <= lim * e16, (bits, e8 / e16)
