@@ -123,6 +123,11 @@ def lib() -> ctypes.CDLL:
             "rqo_m8_scale_encode": ([_F], ctypes.c_uint8),
             "rqo_m8_scale_decode": ([ctypes.c_uint8], _F),
             "rqo_quantize_m8": ([_P, _I, _I, _I, _P, _P, _P], None),
+            "rqo_encode_anchor_rows_m8": ([_P, _I64, _I, _I, _I, _P, _P, _P], None),
+            "rqo_encode_residual_rot_m8": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P], None),
+            "rqo_encode_residual_rows_m8": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P],
+                                            None),
+            "rqo_dequant_rows_m8_f64": ([_P, _P, _I64, _I, _I, _I, _P], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(h, name)
@@ -237,6 +242,21 @@ def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int,
     return words, meta, int(alpha[0]), zhat
 
 
+def encode_residual_rot_m8(z: np.ndarray, ref: np.ndarray, bits: int, group: int,
+                           unit_alpha: bool = False):
+    """encode_residual_rot with 16-bit metadata: (words, meta uint16, alpha_bits, zhat)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    ref = np.ascontiguousarray(ref, dtype=np.float32)
+    D = z.shape[-1]
+    words = np.zeros(D * bits // 32, np.uint32)
+    meta = np.zeros(D // group, np.uint16)
+    alpha = np.zeros(1, np.uint16)
+    zhat = np.zeros(D, np.float32)
+    lib().rqo_encode_residual_rot_m8(_ptr(z), _ptr(ref), D, bits, group, int(unit_alpha),
+                                     _ptr(words), _ptr(meta), _ptr(alpha), _ptr(zhat))
+    return words, meta, int(alpha[0]), zhat
+
+
 @functools.lru_cache(maxsize=None)
 def code_positions(bits: int, D: int):
     """(word, shift) of every channel of a packed row (rqo_code_pos)."""
@@ -270,7 +290,7 @@ def meta_scale_zero(meta: np.ndarray):
 # --------------------------------------------------------------------------
 
 def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
-                policy: str = POLICY_LAST, unit_alpha: bool = False
+                policy: str = POLICY_LAST, unit_alpha: bool = False, meta16: bool = False
                 ) -> List[Dict[str, np.ndarray]]:
     """Encode every loop of one (layer, K|V) side.
 
@@ -279,38 +299,43 @@ def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
     reconstruction (alpha = 1 if unit_alpha) and its quantised residual.
     Returns per loop l a dict with 'codes', 'meta', 'alpha' (None for the
     anchor) and 'zhat' (fp32 reconstructed rotated row, the value a chained
-    neighbour references).
+    neighbour references).  meta16: 16-bit metadata per group (uint16 meta,
+    rqo_quantize_m8) instead of fp16 scale + fp16 offset (uint32 meta).
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     L, N, D = x.shape
+    mdt = np.uint16 if meta16 else np.uint32
+    enc_anchor = lib().rqo_encode_anchor_rows_m8 if meta16 else lib().rqo_encode_anchor_rows
+    enc_resid = lib().rqo_encode_residual_rows_m8 if meta16 else lib().rqo_encode_residual_rows
     out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
     a = anchor_loop(L, policy)
     enc = {"codes": np.zeros((N, D * bits[a] // 32), np.uint32),
-           "meta": np.zeros((N, D // group[a]), np.uint32),
+           "meta": np.zeros((N, D // group[a]), mdt),
            "alpha": None,
            "zhat": np.zeros((N, D), np.float32)}
-    lib().rqo_encode_anchor_rows(_ptr(x[a]), N, D, bits[a], group[a], _ptr(enc["codes"]),
-                                 _ptr(enc["meta"]), _ptr(enc["zhat"]))
+    enc_anchor(_ptr(x[a]), N, D, bits[a], group[a], _ptr(enc["codes"]), _ptr(enc["meta"]),
+               _ptr(enc["zhat"]))
     out[a] = enc
     for r in encode_order(L, policy):
         ref = out[reference_loop(L, r, policy)]["zhat"]
         enc = {"codes": np.zeros((N, D * bits[r] // 32), np.uint32),
-               "meta": np.zeros((N, D // group[r]), np.uint32),
+               "meta": np.zeros((N, D // group[r]), mdt),
                "alpha": np.zeros(N, np.uint16),
                "zhat": np.zeros((N, D), np.float32)}
-        lib().rqo_encode_residual_rows(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D,
-                                       bits[r], group[r], int(unit_alpha), _ptr(enc["codes"]),
-                                       _ptr(enc["meta"]), _ptr(enc["alpha"]),
-                                       _ptr(enc["zhat"]))
+        enc_resid(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D, bits[r], group[r],
+                  int(unit_alpha), _ptr(enc["codes"]), _ptr(enc["meta"]), _ptr(enc["alpha"]),
+                  _ptr(enc["zhat"]))
         out[r] = enc
     return out  # type: ignore[return-value]
 
 
 def _levels_f64(enc: Dict[str, np.ndarray], bits: int, group: int, D: int) -> np.ndarray:
+    """fp64 stored levels of a component (either metadata form, by its dtype)."""
     N = enc["codes"].shape[0]
     out = np.zeros((N, D), np.float64)
-    lib().rqo_dequant_rows_f64(_ptr(enc["codes"]), _ptr(enc["meta"]), N, D, bits, group,
-                               _ptr(out))
+    fn = lib().rqo_dequant_rows_m8_f64 if enc["meta"].dtype == np.uint16 else \
+        lib().rqo_dequant_rows_f64
+    fn(_ptr(enc["codes"]), _ptr(enc["meta"]), N, D, bits, group, _ptr(out))
     return out
 
 

@@ -357,6 +357,70 @@ void rqo_dequant_rows_f64(const uint32_t* words, const uint32_t* meta,
                           out + r * D);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Encoders and levels with 16-bit metadata                                  */
+/* ------------------------------------------------------------------------ */
+
+void rqo_encode_anchor_rows_m8(const uint16_t* x, int64_t n, int D, int bits,
+                               int group, uint32_t* words, uint16_t* meta,
+                               float* zhat) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r) {
+    float z[256];
+    for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[r * D + i]);
+    rqo_fwht_f32(z, D);
+    rqo_quantize_m8(z, D, bits, group, words + r * W, meta + r * G, zhat + r * D);
+  }
+}
+
+void rqo_encode_residual_rot_m8(const float* z, const float* ref, int D, int bits,
+                                int group, int unit_alpha, uint32_t* words,
+                                uint16_t* meta, uint16_t* alpha, float* zhat) {
+  float a = 1.0f;
+  if (!unit_alpha) {
+    const float d_zr = rqo_dot_f32(z, ref, D);
+    const float d_rr = rqo_dot_f32(ref, ref, D);
+    a = (d_rr > 0.0f) ? d_zr / d_rr : 0.0f;
+  }
+  const uint16_t ab = rqo_f32_to_bf16(a);
+  const float at = rqo_bf16_to_f32(ab);
+  *alpha = ab;
+  float e[256], deq[256];
+  for (int i = 0; i < D; ++i) e[i] = fmaf(-at, ref[i], z[i]);
+  rqo_quantize_m8(e, D, bits, group, words, meta, deq);
+  for (int i = 0; i < D; ++i) zhat[i] = fmaf(at, ref[i], deq[i]);
+}
+
+void rqo_encode_residual_rows_m8(const uint16_t* x, const float* ref, int64_t n,
+                                 int D, int bits, int group, int unit_alpha,
+                                 uint32_t* words, uint16_t* meta,
+                                 uint16_t* alpha, float* zhat) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r) {
+    float z[256];
+    for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[r * D + i]);
+    rqo_fwht_f32(z, D);
+    rqo_encode_residual_rot_m8(z, ref + r * D, D, bits, group, unit_alpha,
+                               words + r * W, meta + r * G, alpha + r, zhat + r * D);
+  }
+}
+
+void rqo_dequant_rows_m8_f64(const uint32_t* words, const uint16_t* meta,
+                             int64_t n, int D, int bits, int group, double* out) {
+  const int W = D * bits / 32, G = D / group;
+  const uint32_t qmax = (1u << bits) - 1u;
+  for (int64_t r = 0; r < n; ++r)
+    for (int i = 0; i < D; ++i) {
+      int wi, sh;
+      rqo_code_pos(i, bits, &wi, &sh);
+      const uint32_t code = (words[r * W + wi] >> sh) & qmax;
+      const uint16_t m = meta[r * G + i / group];
+      const double st = rqo_m8_scale_decode((uint8_t)(m & 0xFFu));
+      const double zt = (double)(int8_t)(uint8_t)(m >> 8) * st * 0.125;
+      out[r * D + i] = st * (double)code + zt;
+    }
+}
+
 void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
                        int64_t T, const double* kcur, const double* vcur, int D,
                        double scale, double* out) {

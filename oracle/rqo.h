@@ -131,6 +131,22 @@ void rqo_dequant_codes_f64(const uint32_t* words, const uint32_t* meta, int D,
 void rqo_dequant_rows_f64(const uint32_t* words, const uint32_t* meta,
                           int64_t n, int D, int bits, int group, double* out);
 
+/* The encoders, the row forms and the level reconstruction with 16-bit
+ * metadata (rqo_quantize_m8 in place of rqo_quantize; meta uint16 per
+ * group); every other step as in the functions above. */
+void rqo_encode_anchor_rows_m8(const uint16_t* x, int64_t n, int D, int bits,
+                               int group, uint32_t* words, uint16_t* meta,
+                               float* zhat);
+void rqo_encode_residual_rot_m8(const float* z, const float* ref, int D, int bits,
+                                int group, int unit_alpha, uint32_t* words,
+                                uint16_t* meta, uint16_t* alpha, float* zhat);
+void rqo_encode_residual_rows_m8(const uint16_t* x, const float* ref, int64_t n,
+                                 int D, int bits, int group, int unit_alpha,
+                                 uint32_t* words, uint16_t* meta,
+                                 uint16_t* alpha, float* zhat);
+void rqo_dequant_rows_m8_f64(const uint32_t* words, const uint16_t* meta,
+                             int64_t n, int D, int bits, int group, double* out);
+
 /* Softmax attention of one query against T rows, fp64 [RQ §4.1, §4.2,
  * App. G.1]: s_t = scale * q.k_t for t < T, plus the current token
  * s_cur = scale * q.k_cur; p = softmax(s); out = sum_t p_t v_t + p_cur v_cur.

@@ -629,3 +629,61 @@ def test_m8_error_close_to_fp16_metadata(oracle_mod):
             zq = (meta >> 8).astype(np.uint8).view(np.int8)
             assert np.all((zq > -128) & (zq < 127))
         assert e8 <= lim * e16, (bits, e8 / e16)
+
+
+def test_m8_levels_follow_the_byte_definitions(oracle_mod):
+    """The fp64 levels of 16-bit-metadata rows are s~ c + zq s~ / 8 with s~
+    read off the scale byte's definition, and match the quantiser's fp32
+    levels to one fp32 rounding."""
+    rng = np.random.default_rng(21)
+    for bits, group in ((2, 32), (4, 32), (2, 16), (4, 64)):
+        z = (rng.standard_normal((6, 128)) * 2).astype(np.float32)
+        rows = [oracle_mod.quantize_m8(r, bits, group) for r in z]
+        enc = {"codes": np.stack([r[0] for r in rows]), "meta": np.stack([r[1] for r in rows])}
+        lv = oracle_mod._levels_f64(enc, bits, group, 128)
+        codes = oracle_mod.unpack_codes(enc["codes"], bits, 128).astype(np.float64)
+        for n in range(6):
+            for i in range(128):
+                m = int(enc["meta"][n, i // group])
+                s = _m8_value(m & 0xFF)
+                zq = int(np.int8(np.uint8(m >> 8)))
+                assert lv[n, i] == s * codes[n, i] + zq * s / 8
+            np.testing.assert_allclose(rows[n][2], lv[n], rtol=2 ** -24, atol=0)
+
+
+@pytest.mark.parametrize("c", [1.0, 0.5, -0.25, 4.0])
+def test_m8_scaled_reference_gives_alpha_c_and_zero_residual(oracle_mod, c):
+    """With 16-bit metadata too, X_r = c R^ gives alpha = c, a zero residual
+    (all-zero codes and metadata) and Z^_r = X_r [RQ §3.2, App. G.1]."""
+    rng = np.random.default_rng(7)
+    _, _, A = oracle_mod.quantize_m8(rng.standard_normal(128).astype(np.float32), 4, 32)
+    z = (np.float32(c) * A).astype(np.float32)
+    words, meta, ab, zhat = oracle_mod.encode_residual_rot_m8(z, A, 2, 32)
+    assert oracle_mod.bf16_bits_to_f32(ab) == c
+    assert not words.any() and not meta.any()
+    np.testing.assert_array_equal(zhat, z)
+
+
+def test_m8_side_encoding_invariants(oracle_mod):
+    """encode_side with 16-bit metadata: Last-loop and Next-loop agree next to
+    the anchor; every kept reference row equals the fp64 reconstruction from
+    the stored data to fp32 rounding; the reconstruction error stays within
+    10% of the fp16-metadata encoding's."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=2, tokens=64)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_K, l, [0], [0, 1], 0, 64)).reshape(-1, 128)
+                  for l in range(w.loops)])
+    es = oracle_mod.encode_side(x, w.bits, w.group, "last", meta16=True)
+    ec = oracle_mod.encode_side(x, w.bits, w.group, "next", meta16=True)
+    r = w.loops - 2
+    for k in ("codes", "meta", "alpha"):
+        np.testing.assert_array_equal(es[r][k], ec[r][k])
+    assert es[0]["meta"].dtype == np.uint16
+    e16 = oracle_mod.encode_side(x, w.bits, w.group, "last")
+    xr = oracle_mod.fwht_f64(oracle_mod.bf16_bits_to_f64(x))
+    for loop in range(w.loops):
+        z = oracle_mod.reconstruct_rotated(es, loop, w.bits, w.group)
+        np.testing.assert_allclose(es[loop]["zhat"], z, rtol=2e-6, atol=2e-6)
+        err8 = float(((z - xr[loop]) ** 2).sum())
+        err16 = float(((oracle_mod.reconstruct_rotated(e16, loop, w.bits, w.group) - xr[loop]) ** 2).sum())
+        assert err8 <= 1.10 * err16, (loop, err8 / err16)
