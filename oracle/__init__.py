@@ -128,6 +128,10 @@ def lib() -> ctypes.CDLL:
             "rqo_encode_residual_rows_m8": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P],
                                             None),
             "rqo_dequant_rows_m8_f64": ([_P, _P, _I64, _I, _I, _I, _P], None),
+            "rqo_encode_residual_rot_ex": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P],
+                                           None),
+            "rqo_encode_residual_rows_ex": ([_P, _P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P,
+                                             _P], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(h, name)
@@ -257,6 +261,25 @@ def encode_residual_rot_m8(z: np.ndarray, ref: np.ndarray, bits: int, group: int
     return words, meta, int(alpha[0]), zhat
 
 
+def encode_residual_rot_ex(z: np.ndarray, ref: np.ndarray, mu: Optional[np.ndarray],
+                           bits: int, group: int, unit_alpha: bool = False,
+                           meta16: bool = False):
+    """Residual encoder with a fixed mean (None: no mean) and either metadata
+    form: (words, meta, alpha_bits, zhat)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    ref = np.ascontiguousarray(ref, dtype=np.float32)
+    D = z.shape[-1]
+    words = np.zeros(D * bits // 32, np.uint32)
+    meta = np.zeros(D // group, np.uint16 if meta16 else np.uint32)
+    alpha = np.zeros(1, np.uint16)
+    zhat = np.zeros(D, np.float32)
+    m = None if mu is None else np.ascontiguousarray(mu, dtype=np.float32)
+    lib().rqo_encode_residual_rot_ex(_ptr(z), _ptr(ref), None if m is None else _ptr(m), D, bits,
+                                     group, int(unit_alpha), int(meta16), _ptr(words),
+                                     _ptr(meta), _ptr(alpha), _ptr(zhat))
+    return words, meta, int(alpha[0]), zhat
+
+
 @functools.lru_cache(maxsize=None)
 def code_positions(bits: int, D: int):
     """(word, shift) of every channel of a packed row (rqo_code_pos)."""
@@ -290,8 +313,8 @@ def meta_scale_zero(meta: np.ndarray):
 # --------------------------------------------------------------------------
 
 def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
-                policy: str = POLICY_LAST, unit_alpha: bool = False, meta16: bool = False
-                ) -> List[Dict[str, np.ndarray]]:
+                policy: str = POLICY_LAST, unit_alpha: bool = False, meta16: bool = False,
+                mu: Optional[np.ndarray] = None) -> List[Dict[str, np.ndarray]]:
     """Encode every loop of one (layer, K|V) side.
 
     x: uint16 [L, N, D].  The anchor loop (anchor_loop) is quantised directly;
@@ -301,6 +324,8 @@ def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
     anchor) and 'zhat' (fp32 reconstructed rotated row, the value a chained
     neighbour references).  meta16: 16-bit metadata per group (uint16 meta,
     rqo_quantize_m8) instead of fp16 scale + fp16 offset (uint32 meta).
+    mu: optional fp32 [L, N, D] fixed means of the residual loops in the
+    rotated domain [RQ App. G.2] (the anchor's entry is not used).
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     L, N, D = x.shape
@@ -322,9 +347,16 @@ def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
                "meta": np.zeros((N, D // group[r]), mdt),
                "alpha": np.zeros(N, np.uint16),
                "zhat": np.zeros((N, D), np.float32)}
-        enc_resid(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D, bits[r], group[r],
-                  int(unit_alpha), _ptr(enc["codes"]), _ptr(enc["meta"]), _ptr(enc["alpha"]),
-                  _ptr(enc["zhat"]))
+        if mu is None:
+            enc_resid(_ptr(x[r]), _ptr(np.ascontiguousarray(ref)), N, D, bits[r], group[r],
+                      int(unit_alpha), _ptr(enc["codes"]), _ptr(enc["meta"]),
+                      _ptr(enc["alpha"]), _ptr(enc["zhat"]))
+        else:
+            m = np.ascontiguousarray(mu[r], dtype=np.float32)
+            lib().rqo_encode_residual_rows_ex(
+                _ptr(x[r]), _ptr(np.ascontiguousarray(ref)), _ptr(m), N, D, bits[r], group[r],
+                int(unit_alpha), int(meta16), _ptr(enc["codes"]), _ptr(enc["meta"]),
+                _ptr(enc["alpha"]), _ptr(enc["zhat"]))
         out[r] = enc
     return out  # type: ignore[return-value]
 
@@ -340,11 +372,13 @@ def _levels_f64(enc: Dict[str, np.ndarray], bits: int, group: int, D: int) -> np
 
 
 def reconstruct_rotated(encs: List[Dict[str, np.ndarray]], loop: int, bits: Sequence[int],
-                        group: Sequence[int], policy: str = POLICY_LAST) -> np.ndarray:
+                        group: Sequence[int], policy: str = POLICY_LAST,
+                        mu: Optional[np.ndarray] = None) -> np.ndarray:
     """fp64 rotated reconstruction Z^_loop [RQ App. G.2]:
-    Z^_anchor = A; Z^_r = alpha~_r * Z^_ref + D(c_r), ref the anchor (shared
-    policies) or the neighbour toward the anchor (chained policies), so a
-    chained loop is rebuilt from the anchor outwards."""
+    Z^_anchor = A; Z^_r = alpha~_r * Z^_ref + D(c_r) (+ mu_r, the fixed mean,
+    when mu [L, N, D] is given), ref the anchor (shared policies) or the
+    neighbour toward the anchor (chained policies), so a chained loop is
+    rebuilt from the anchor outwards."""
     L = len(encs)
     a = anchor_loop(L, policy)
     D = encs[a]["zhat"].shape[1]
@@ -357,12 +391,14 @@ def reconstruct_rotated(encs: List[Dict[str, np.ndarray]], loop: int, bits: Sequ
     for r in reversed(path):
         al = (encs[r]["alpha"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         z = al[:, None] * z + _levels_f64(encs[r], bits[r], group[r], D)
+        if mu is not None:
+            z = z + np.asarray(mu[r], np.float64)
     return z
 
 
-def reconstruct(encs, loop, bits, group, policy=POLICY_LAST) -> np.ndarray:
+def reconstruct(encs, loop, bits, group, policy=POLICY_LAST, mu=None) -> np.ndarray:
     """fp64 reconstruction in the original domain: X^ = H^T Z^ (H symmetric)."""
-    return fwht_f64(reconstruct_rotated(encs, loop, bits, group, policy))
+    return fwht_f64(reconstruct_rotated(encs, loop, bits, group, policy, mu))
 
 
 def attention(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, kcur: np.ndarray,

@@ -421,6 +421,54 @@ void rqo_dequant_rows_m8_f64(const uint32_t* words, const uint16_t* meta,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Residual encoder with a fixed mean [RQ App. G.2]                          */
+/* ------------------------------------------------------------------------ */
+
+void rqo_encode_residual_rot_ex(const float* z, const float* ref, const float* mu,
+                                int D, int bits, int group, int unit_alpha,
+                                int meta16, uint32_t* words, void* meta,
+                                uint16_t* alpha, float* zhat) {
+  float zc[256], e[256], deq[256];
+  for (int i = 0; i < D; ++i) zc[i] = mu ? z[i] - mu[i] : z[i];
+  float a = 1.0f;
+  if (!unit_alpha) {
+    const float d_zr = rqo_dot_f32(zc, ref, D);
+    const float d_rr = rqo_dot_f32(ref, ref, D);
+    a = (d_rr > 0.0f) ? d_zr / d_rr : 0.0f;
+  }
+  const uint16_t ab = rqo_f32_to_bf16(a);
+  const float at = rqo_bf16_to_f32(ab);
+  *alpha = ab;
+  for (int i = 0; i < D; ++i) e[i] = fmaf(-at, ref[i], zc[i]);
+  if (meta16)
+    rqo_quantize_m8(e, D, bits, group, words, (uint16_t*)meta, deq);
+  else
+    rqo_quantize(e, D, bits, group, words, (uint32_t*)meta, deq);
+  for (int i = 0; i < D; ++i) {
+    const float r = fmaf(at, ref[i], deq[i]);
+    zhat[i] = mu ? r + mu[i] : r;
+  }
+}
+
+void rqo_encode_residual_rows_ex(const uint16_t* x, const float* ref,
+                                 const float* mu, int64_t n, int D, int bits,
+                                 int group, int unit_alpha, int meta16,
+                                 uint32_t* words, void* meta, uint16_t* alpha,
+                                 float* zhat) {
+  const int W = D * bits / 32, G = D / group;
+  const size_t mb = meta16 ? 2 : 4;
+  for (int64_t r = 0; r < n; ++r) {
+    float z[256];
+    for (int i = 0; i < D; ++i) z[i] = rqo_bf16_to_f32(x[r * D + i]);
+    rqo_fwht_f32(z, D);
+    rqo_encode_residual_rot_ex(z, ref + r * D, mu ? mu + r * D : NULL, D, bits, group,
+                               unit_alpha, meta16, words + r * W,
+                               (unsigned char*)meta + (size_t)(r * G) * mb, alpha + r,
+                               zhat + r * D);
+  }
+}
+
 void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
                        int64_t T, const double* kcur, const double* vcur, int D,
                        double scale, double* out) {

@@ -147,6 +147,22 @@ void rqo_encode_residual_rows_m8(const uint16_t* x, const float* ref, int64_t n,
 void rqo_dequant_rows_m8_f64(const uint32_t* words, const uint16_t* meta,
                              int64_t n, int D, int bits, int group, double* out);
 
+/* Residual encoder with a fixed mean [RQ App. G.2: Z^_r = alpha_r A +
+ * D(c_r) + mu_r] and either metadata form: zc = z - mu (mu NULL: no mean);
+ * alpha = <zc, ref>/<ref, ref> (1 with unit_alpha); E = fma(-alpha~, ref, zc)
+ * quantised with rqo_quantize (meta uint32) or rqo_quantize_m8 (meta16:
+ * meta uint16); zhat = fma(alpha~, ref, deq(E)) + mu.  Row forms take x
+ * (bf16, rotated here), ref and mu as n rows of D. */
+void rqo_encode_residual_rot_ex(const float* z, const float* ref, const float* mu,
+                                int D, int bits, int group, int unit_alpha,
+                                int meta16, uint32_t* words, void* meta,
+                                uint16_t* alpha, float* zhat);
+void rqo_encode_residual_rows_ex(const uint16_t* x, const float* ref,
+                                 const float* mu, int64_t n, int D, int bits,
+                                 int group, int unit_alpha, int meta16,
+                                 uint32_t* words, void* meta, uint16_t* alpha,
+                                 float* zhat);
+
 /* Softmax attention of one query against T rows, fp64 [RQ §4.1, §4.2,
  * App. G.1]: s_t = scale * q.k_t for t < T, plus the current token
  * s_cur = scale * q.k_cur; p = softmax(s); out = sum_t p_t v_t + p_cur v_cur.

@@ -687,3 +687,61 @@ def test_m8_side_encoding_invariants(oracle_mod):
         err8 = float(((z - xr[loop]) ** 2).sum())
         err16 = float(((oracle_mod.reconstruct_rotated(e16, loop, w.bits, w.group) - xr[loop]) ** 2).sum())
         assert err8 <= 1.10 * err16, (loop, err8 / err16)
+
+
+# ------------------------------------------------------ fixed mean mu_r --
+# Z^_r = alpha_r A + D(c_r) + mu_r [RQ App. G.2]; the mean is a fixed
+# per-loop vector in the rotated domain (not stored per token).
+
+@pytest.mark.parametrize("meta16", [False, True])
+@pytest.mark.parametrize("policy", ["last", "next", "first", "previous"])
+def test_zero_mean_is_the_plain_encoder(oracle_mod, policy, meta16):
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=2, tokens=32)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_V, l, [0], [0, 1], 0, 32)).reshape(-1, 128)
+                  for l in range(w.loops)])
+    e0 = oracle_mod.encode_side(x, w.bits, w.group, policy, meta16=meta16)
+    em = oracle_mod.encode_side(x, w.bits, w.group, policy, meta16=meta16,
+                                mu=np.zeros((w.loops,) + x.shape[1:], np.float32))
+    for a, b in zip(e0, em):
+        for k in ("codes", "meta", "alpha"):
+            if a[k] is None:
+                assert b[k] is None
+            else:
+                np.testing.assert_array_equal(a[k], b[k])
+        np.testing.assert_array_equal(a["zhat"], b["zhat"])
+
+
+@pytest.mark.parametrize("meta16", [False, True])
+def test_mean_shift_invariance_on_an_exact_grid(oracle_mod, meta16):
+    """With every sum exact (values on a 2^-10 grid), encoding z + mu with
+    mean mu stores exactly what encoding z without a mean stores, and its
+    reconstruction is the mean-free one plus mu."""
+    rng = np.random.default_rng(31)
+    A = _anchor_row(oracle_mod, 5)
+    for trial in range(20):
+        z = (np.round(rng.standard_normal(128) * 512) / 1024).astype(np.float32)
+        mu = (np.round(rng.uniform(-1, 1, 128) * 1024) / 1024).astype(np.float32)
+        w0, m0, a0, zh0 = oracle_mod.encode_residual_rot_ex(z, A, None, 2, 32, meta16=meta16)
+        w1, m1, a1, zh1 = oracle_mod.encode_residual_rot_ex(z + mu, A, mu, 2, 32, meta16=meta16)
+        assert a0 == a1
+        np.testing.assert_array_equal(w0, w1)
+        np.testing.assert_array_equal(m0, m1)
+        np.testing.assert_array_equal(zh1, (zh0 + mu).astype(np.float32))
+
+
+@pytest.mark.parametrize("policy", ["last", "next", "previous"])
+def test_mean_reconstruction_matches_the_kept_rows(oracle_mod, policy):
+    """The fp32 rows the encoder keeps equal the fp64 reconstruction
+    alpha~ Z^_ref + D(c) + mu from the stored data (fp32 rounding)."""
+    import residual_bit_kv_b200.synth as synth
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=1, heads=1, tokens=64)
+    x = np.stack([synth.bits_of(synth.kv(w, 0, synth.SIDE_K, l, [0], [0], 0, 64)).reshape(-1, 128)
+                  for l in range(w.loops)])
+    rng = np.random.default_rng(32)
+    mu = np.broadcast_to(rng.standard_normal((w.loops, 1, 128)).astype(np.float32),
+                         (w.loops,) + x.shape[1:]).copy()
+    encs = oracle_mod.encode_side(x, w.bits, w.group, policy, mu=mu)
+    for r in range(w.loops):
+        z = oracle_mod.reconstruct_rotated(encs, r, w.bits, w.group, policy, mu=mu)
+        np.testing.assert_allclose(encs[r]["zhat"], z, rtol=2e-6, atol=2e-6)
