@@ -146,6 +146,19 @@ def _ptr(a: np.ndarray) -> int:
     return a.ctypes.data
 
 
+MAX_D = 256   # the C row functions keep rows of up to 256 channels on the stack
+
+
+def _check_dim(D: int) -> int:
+    """Head dimension accepted by the C row functions: a power of two in
+    [32, 256] (the FWHT needs a power of two; rows live in 256-entry stack
+    buffers).  Anything else raises before the C code runs."""
+    D = int(D)
+    if D < 32 or D > MAX_D or D & (D - 1):
+        raise ValueError(f"oracle: head_dim {D} is not a power of two in [32, {MAX_D}]")
+    return D
+
+
 # --------------------------------------------------------------------------
 # Scalar / row-level entry points (used by the pins)
 # --------------------------------------------------------------------------
@@ -173,7 +186,7 @@ def rot_scale(D: int) -> float:
 def fwht_f32(z: np.ndarray) -> np.ndarray:
     """Normalised Hadamard transform of each row of z (fp32, canonical order)."""
     z = np.array(z, dtype=np.float32, order="C", copy=True)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     flat = z.reshape(-1, D)
     for r in range(flat.shape[0]):
         row = np.ascontiguousarray(flat[r])
@@ -184,7 +197,7 @@ def fwht_f32(z: np.ndarray) -> np.ndarray:
 
 def fwht_f64(z: np.ndarray) -> np.ndarray:
     z = np.array(z, dtype=np.float64, order="C", copy=True)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     n = z.size // D
     lib().rqo_fwht_rows_f64(_ptr(z), n, D)
     return z
@@ -199,7 +212,7 @@ def dot_f32(a: np.ndarray, b: np.ndarray) -> float:
 def quantize(z: np.ndarray, bits: int, group: int):
     """Affine-quantise one rotated fp32 row: (words, meta, deq)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     words = np.zeros(D * bits // 32, np.uint32)
     meta = np.zeros(D // group, np.uint32)
     deq = np.zeros(D, np.float32)
@@ -223,7 +236,7 @@ def quantize_m8(z: np.ndarray, bits: int, group: int):
     """Affine-quantise one rotated fp32 row with 16-bit metadata per group:
     (words, meta uint16 [D/group] = scale byte | offset byte << 8, deq)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     words = np.zeros(D * bits // 32, np.uint32)
     meta = np.zeros(D // group, np.uint16)
     deq = np.zeros(D, np.float32)
@@ -236,7 +249,7 @@ def encode_residual_rot(z: np.ndarray, ref: np.ndarray, bits: int, group: int,
     """Residual encoder on an already-rotated fp32 row: (words, meta, alpha_bits, zhat)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
     ref = np.ascontiguousarray(ref, dtype=np.float32)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     words = np.zeros(D * bits // 32, np.uint32)
     meta = np.zeros(D // group, np.uint32)
     alpha = np.zeros(1, np.uint16)
@@ -251,7 +264,7 @@ def encode_residual_rot_m8(z: np.ndarray, ref: np.ndarray, bits: int, group: int
     """encode_residual_rot with 16-bit metadata: (words, meta uint16, alpha_bits, zhat)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
     ref = np.ascontiguousarray(ref, dtype=np.float32)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     words = np.zeros(D * bits // 32, np.uint32)
     meta = np.zeros(D // group, np.uint16)
     alpha = np.zeros(1, np.uint16)
@@ -268,7 +281,7 @@ def encode_residual_rot_ex(z: np.ndarray, ref: np.ndarray, mu: Optional[np.ndarr
     form: (words, meta, alpha_bits, zhat)."""
     z = np.ascontiguousarray(z, dtype=np.float32)
     ref = np.ascontiguousarray(ref, dtype=np.float32)
-    D = z.shape[-1]
+    D = _check_dim(z.shape[-1])
     words = np.zeros(D * bits // 32, np.uint32)
     meta = np.zeros(D // group, np.uint16 if meta16 else np.uint32)
     alpha = np.zeros(1, np.uint16)
@@ -329,6 +342,7 @@ def encode_side(x: np.ndarray, bits: Sequence[int], group: Sequence[int],
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     L, N, D = x.shape
+    _check_dim(D)
     mdt = np.uint16 if meta16 else np.uint32
     enc_anchor = lib().rqo_encode_anchor_rows_m8 if meta16 else lib().rqo_encode_anchor_rows
     enc_resid = lib().rqo_encode_residual_rows_m8 if meta16 else lib().rqo_encode_residual_rows

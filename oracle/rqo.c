@@ -238,13 +238,21 @@ void rqo_quantize_m8(const float* z, int D, int bits, int group, uint32_t* words
      * the offset fits its byte; rounded to the scale byte. */
     const float s0 = (mx - mn) / (float)qmax;
     const float s1 = fabsf(mn) / 15.875f;
-    const uint8_t sb = rqo_m8_scale_encode(s0 > s1 ? s0 : s1);
-    const float st = rqo_m8_scale_decode(sb);
+    uint8_t sb = rqo_m8_scale_encode(s0 > s1 ? s0 : s1);
+    float st = rqo_m8_scale_decode(sb);
 
-    /* Offset: the largest multiple of s~/8 not above mn (clamped). */
+    /* Offset: the largest multiple of s~/8 not above mn.  When the nearest
+     * scale rounded down far enough that this multiple leaves the offset
+     * byte, the scale byte goes up one step (one step always suffices); the
+     * clamp is left only for the largest scale byte. */
     int zq = 0;
     if (st > 0.0f) {
-      const float t = floorf((8.0f * mn) / st);
+      float t = floorf((8.0f * mn) / st);
+      if ((t < -128.0f || t > 127.0f) && sb < 0xFFu) {
+        sb = (uint8_t)(sb + 1u);
+        st = rqo_m8_scale_decode(sb);
+        t = floorf((8.0f * mn) / st);
+      }
       zq = t < -128.0f ? -128 : (t > 127.0f ? 127 : (int)t);
     }
     const float zt = (float)zq * st * 0.125f;

@@ -15,6 +15,10 @@
  * documented order, so the GPU path can be held to bit-exact agreement.
  * Reconstruction and attention are computed in fp64.
  *
+ * Row length: D is a power of two in [32, 256] everywhere (the row
+ * functions keep rows in 256-entry stack buffers); the Python wrapper
+ * rejects any other D before calling in.
+ *
  * Packed formats (the storage contract both sides implement independently):
  *   codes : b = 2: channel i of a row lives in 32-bit word i/16, bits
  *           [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v,
@@ -87,11 +91,17 @@ float   rqo_m8_scale_decode(uint8_t b);
 
 /* Group-wise affine quantisation with 16-bit metadata: per group, mn, mx
  * (+0 for zeros); s0 = (mx - mn)/(2^b - 1); s1 = |mn| / 15.875;
- * s~ = decode(encode(max(s0, s1))) (s1 keeps the offset inside the offset
- * byte's range); offset byte zq = clamp(floor((8 mn) / s~), -128, 127)
- * (0 if s~ == 0), z~ = zq * s~ / 8 (exact); codes and levels as in
+ * s~ = decode(encode(max(s0, s1))) (s1 keeps the offset near the offset
+ * byte's range); t = floor((8 mn) / s~); if t is outside [-128, 127] the
+ * scale byte is raised by one (next larger value) and t recomputed; offset
+ * byte zq = clamp(t, -128, 127) (0 if s~ == 0; the clamp only acts at the
+ * largest scale byte), z~ = zq * s~ / 8 (exact); codes and levels as in
  * rqo_quantize: inv = 1/s~ (0 if s~ == 0), c = rint(clamp((z - z~) * inv)),
- * deq = fma(s~, c, z~).  meta[j] = scale byte | (offset byte << 8). */
+ * deq = fma(s~, c, z~).  meta[j] = scale byte | (offset byte << 8).
+ * Error bound (scales inside the byte's range): s~ is within 1/17 below the
+ * range scale and z~ within s~/8 below mn, so every value is within
+ * max(1/2, (2^b - 1)/16 + 1/8) * s~ of its level (plus fp32 rounding):
+ * half a step for INT2, 1.0625 steps at the top of an INT4 group. */
 void rqo_quantize_m8(const float* z, int D, int bits, int group,
                      uint32_t* words, uint16_t* meta, float* deq);
 

@@ -106,6 +106,16 @@ def test_fwht_involution_exact_d64(oracle_mod):
     np.testing.assert_array_equal(oracle_mod.fwht_f32(e0), np.full(64, 0.125, np.float32))
 
 
+def test_row_length_outside_the_buffers_is_refused(oracle_mod):
+    """The C row functions hold rows of at most 256 channels: longer or
+    non-power-of-two rows raise before any C code runs."""
+    for D in (512, 96, 16):
+        with pytest.raises(ValueError):
+            oracle_mod.quantize(np.zeros(D, np.float32), 2, 16)
+        with pytest.raises(ValueError):
+            oracle_mod.encode_side(np.zeros((2, 1, D), np.uint16), (2, 4), (16, 16))
+
+
 def test_rot_scale_is_rounded_inverse_sqrt(oracle_mod):
     for D in (32, 64, 128, 256):
         assert oracle_mod.rot_scale(D) == float(np.float32(1.0 / np.sqrt(np.float64(D))))
@@ -305,6 +315,49 @@ def test_chained_equals_shared_next_to_anchor(oracle_mod):
     lv = oracle_mod._levels_f64(ec[0], w.bits[0], w.group[0], 128)
     a0 = oracle_mod.bf16_bits_to_f64(ec[0]["alpha"])[:, None]
     np.testing.assert_allclose(z0, a0 * z1 + lv, rtol=0, atol=1e-12)
+
+
+def _exact_multiple_chain(mults):
+    """Three loops on an exact grid at D = 64 (fp32(1/sqrt(64)) = 1/8 exactly):
+    x = a (e_0 + e_1) rotates to Z = a/8 on even channels and 0 on odd ones,
+    so an INT4 anchor with a = 60 spans the levels 0 .. 15 with scale 1 and
+    offset 0 and is stored exactly.  Loop l is x scaled by mults[l]; every
+    product stays bf16-exact."""
+    D = 64
+    x = np.zeros((3, 1, D), np.float32)
+    for l, m in enumerate(mults):
+        x[l, 0, 0] = x[l, 0, 1] = 60.0 * m
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal((bits.astype(np.uint32) << 16).view(np.float32), x)
+    return bits
+
+
+@pytest.mark.parametrize("policy,mults,alphas", [
+    # Next-loop: anchor = loop 2; loop 1 = 3 x loop 2, loop 0 = 2 x loop 1
+    ("next", (6.0, 3.0, 1.0), {1: 3.0, 0: 2.0}),
+    # Previous-loop (the mirror): anchor = loop 0; loop 1 = 3 x loop 0, loop 2 = 2 x loop 1
+    ("previous", (1.0, 3.0, 6.0), {1: 3.0, 2: 2.0}),
+])
+def test_chain_references_on_an_exact_grid(oracle_mod, policy, mults, alphas):
+    """Closed form of the reference chain [RQ §3.2, App. D]: with every loop an
+    exact multiple of its neighbour toward the anchor, each stored LS
+    coefficient is the ratio to that neighbour (3, then 2), every residual is
+    exactly zero and the reconstruction reproduces each loop exactly.  A chain
+    that referenced the anchor, or the loop two steps away, would store 6 for
+    the far loop instead of 2."""
+    bits, group = (4, 2, 4), (32, 32, 32)
+    if policy == "previous":
+        bits = (4, 2, 2)
+    encs = oracle_mod.encode_side(_exact_multiple_chain(mults), bits, group, policy)
+    anchor = oracle_mod.anchor_loop(3, policy)
+    z_anchor = np.zeros(64)
+    z_anchor[0::2] = 15.0
+    for r, a in alphas.items():
+        assert oracle_mod.bf16_bits_to_f32(int(encs[r]["alpha"][0])) == a
+        assert not encs[r]["codes"].any() and not encs[r]["meta"].any()
+    for r in range(3):
+        z = oracle_mod.reconstruct_rotated(encs, r, bits, group, policy)
+        np.testing.assert_array_equal(z[0], mults[r] / mults[anchor] * z_anchor)
 
 
 def test_encoder_reference_row_matches_reconstruction(oracle_mod):
@@ -600,13 +653,14 @@ def test_m8_codes_are_nearest_level_brute_force(oracle_mod, bits, group):
 
 def test_m8_constant_group_keeps_its_value(oracle_mod):
     """A constant nonzero group (zero range) is still reproduced: the scale
-    becomes |c| / 15.875 (rounded) and the level nearest to c is within half
-    a step; a zero group stays exactly zero."""
+    becomes |c| / 15.875 (rounded to nearest, or one step up where the
+    offset byte would otherwise saturate) and the level nearest to c is
+    within half a step; a zero group stays exactly zero."""
     for c in (3.0, -0.7, 1e-3, -250.0):
         z = np.full(32, c, np.float32)
         words, meta, deq = oracle_mod.quantize_m8(z, 2, 32)
         s = _m8_value(int(meta[0]) & 0xFF)
-        assert 0 < s <= abs(c) / 15.875 * (1 + 1 / 16) + 1e-12
+        assert abs(c) / 15.875 * (1 - 1 / 17) <= s <= abs(c) / 15.875 * (1 + 1 / 16) * (1 + 1 / 8)
         assert np.all(np.abs(deq - c) <= s / 2 + 1e-6 * abs(c))
     words, meta, deq = oracle_mod.quantize_m8(np.zeros(32, np.float32), 2, 32)
     assert meta[0] == 0 and not deq.any() and not words.any()
@@ -629,6 +683,50 @@ def test_m8_error_close_to_fp16_metadata(oracle_mod):
             zq = (meta >> 8).astype(np.uint8).view(np.int8)
             assert np.all((zq > -128) & (zq < 127))
         assert e8 <= lim * e16, (bits, e8 / e16)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_m8_error_bound_and_offset_range(oracle_mod, bits):
+    """Worst case of the 16-bit-metadata quantiser: every value lies within
+    max(1/2, (2^b - 1)/16 + 1/8) steps s~ of its level (s~ at most 1/17
+    below the range scale, z~ at most s~/8 below the minimum), and the
+    offset byte never saturates while the scale is inside the byte's range.
+    Rows: normal, shifted, one-sided narrow groups (offset far from zero)
+    and rows whose range scale sits just below a rounding midpoint."""
+    qmax = (1 << bits) - 1
+    bound = max(0.5, qmax / 16 + 1 / 8)
+    rng = np.random.default_rng(40 + bits)
+    rows = [rng.standard_normal(128) * 2.0,
+            rng.standard_normal(128) * 0.3 + 5.0,
+            rng.uniform(20.0, 20.5, 128),
+            -rng.uniform(7.0, 7.2, 128)]
+    for k in range(40):
+        # range scale (1 + 1/16)(1 - eps) 2^e rounds down to 2^e; minimum just
+        # below a multiple of s~/8 above zero
+        e = int(rng.integers(-6, 4))
+        s0 = (1 + 1 / 16) * (1 - 2.0 ** -20) * 2.0 ** e
+        mn = (int(rng.integers(0, 40)) + 0.999) * 2.0 ** e / 8
+        g = np.full(32, mn)
+        g[1] = mn + qmax * s0
+        g[2:] = mn + rng.uniform(0, qmax * s0, 30)
+        rows.append(np.tile(g, 4))
+    worst = 0.0
+    for z in rows:
+        z = z.astype(np.float32)
+        for group in (16, 32, 64, 128):
+            words, meta, deq = oracle_mod.quantize_m8(z, bits, group)
+            for j in range(128 // group):
+                s = _m8_value(int(meta[j]) & 0xFF)
+                zq = int(np.int8(np.uint8(int(meta[j]) >> 8)))
+                assert -128 < zq < 127 or (int(meta[j]) & 0xFF) == 0xFF
+                err = np.max(np.abs(deq[j * group:(j + 1) * group].astype(np.float64) -
+                                    z[j * group:(j + 1) * group]))
+                assert err <= bound * s * (1 + 2 ** -20) + 1e-6 * np.max(np.abs(z)), (group, err / s)
+                worst = max(worst, err / s)
+    if bits == 4:
+        assert worst > 1.0   # the INT4 bound is reached: more than one step at a group's top
+    else:
+        assert worst <= 0.5 + 1e-6
 
 
 def test_m8_levels_follow_the_byte_definitions(oracle_mod):
