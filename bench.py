@@ -70,6 +70,14 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
+def rank_share(w, rank: int, world: int):
+    """This rank's rows of the job: the job decodes a global batch of
+    world * w.batch sequences and rank r takes rows [r*B/N, (r+1)*B/N), so
+    per-GPU work stays fixed as N grows (weak scaling) and every rank's
+    inputs are rows of one workload, not a re-seeded copy."""
+    return synth.partition(w.replace(batch=w.batch * world), rank, world)
+
+
 def job_tokens_per_s(world_size: int, batch: int, ms_per_step: float) -> float:
     """Whole-job decode throughput: every rank decodes its own batch per step
     (weak scaling), the step time being the slowest rank's."""
@@ -290,10 +298,10 @@ def quant_loops_bytes(w, n):
 class Engine:
     """Resident packed caches of every layer plus the step's inputs."""
 
-    def __init__(self, w, device, seed_offset=0, keep_bf16_layers=0):
+    def __init__(self, w, device, keep_bf16_layers=0):
         import residual_bit_kv_b200.librq as L
         self.L = L
-        self.w = w = w.replace(seed=w.seed + seed_offset)
+        self.w = w
         self.dev = device
         T = w.tokens
         self.lay = L.make_layout(w.layers, w.loops, w.batch, w.heads, w.head_dim, T + 16,
@@ -566,7 +574,10 @@ def run_reference(args, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based generator)",
-        "config": config_of(w),
+        "config": config_of(w, max(1, args.gpus)),
+        "extrapolated": ("ms_per_step is not a measured step: each timed sample decodes one "
+                         "(batch, head) unit of loop 0 and the median time per unit is scaled "
+                         f"to the {step_units} units of one step"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": "per step: 1 (batch,head) unit of loop 0, layer 0 at T=16384, "
                                    f"scaled to {step_units} units"},
@@ -576,13 +587,16 @@ def run_reference(args, rank):
     return 0
 
 
-def config_of(w):
-    return {"workload": f"{w.name}: {w.layers} layers x {w.loops} loops, batch {w.batch}, "
+def config_of(w, world=1):
+    par = ("one GPU" if world == 1 else
+           f"batch partition over {world} GPUs: rank r decodes batch rows "
+           f"[{w.batch}r, {w.batch}r+{w.batch}) of one global batch; no collective on the path")
+    return {"workload": f"{w.name}: {w.layers} layers x {w.loops} loops, batch {w.batch} per GPU, "
                         f"{w.heads} KV heads, head_dim {w.head_dim}, {w.tokens} past tokens, "
                         f"bits {list(w.bits)}, group {w.group[0]}, Last-loop anchor",
-            "global_batch": w.batch, "seq_len": w.tokens,
+            "global_batch": w.batch * world, "seq_len": w.tokens,
             "l2": "inputs larger than L2: every decode call streams >= 0.67 GB of packed KV",
-            "parallelism": "replicated workload per GPU (batch/head units independent)"}
+            "parallelism": par}
 
 
 # --------------------------------------------------------------------- main --
@@ -617,7 +631,7 @@ def main():
     if args.batch:
         w = w.replace(batch=args.batch)
     nbuf = 0 if args.no_bf16 else 4
-    eng = Engine(w, dev, seed_offset=1000 * rank, keep_bf16_layers=nbuf)
+    eng = Engine(rank_share(w, rank, ws), dev, keep_bf16_layers=nbuf)
     w = eng.w
     stream = torch.cuda.current_stream(dev)
 
@@ -739,7 +753,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded counter-based generator; Ouro-like looped KV)",
-            "config": config_of(w),
+            "config": config_of(w, ws),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
                          "kernel": "decode_fast_kernel (all loops of the step)", "peak_kind": hbm_kind,

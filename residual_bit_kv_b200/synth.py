@@ -106,6 +106,7 @@ class Workload:
     layers: int = 1
     key_scale_std: float = 0.5
     recipe: str = "default"    # "default" or "tiny"
+    batch0: int = 0            # global index of batch row 0 (a slice of a larger batch)
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -140,12 +141,25 @@ def key_channel_scale(w: Workload, layer: int) -> torch.Tensor:
 
 
 def _row_index(w: Workload, b: torch.Tensor, h: torch.Tensor, t: torch.Tensor) -> torch.Tensor:
+    b = b + w.batch0
     return (b[:, None, None] * w.heads + h[None, :, None]) * T_SPACE + t[None, None, :]
+
+
+def partition(w: Workload, rank: int, world: int) -> Workload:
+    """Rank `rank`'s share of w's batch when `world` ranks split it: rows
+    [rank*B/world, (rank+1)*B/world) (B = w.batch), as a workload whose values
+    are exactly those rows of w (the generator indexes global rows)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank outside the world")
+    lo = rank * w.batch // world
+    hi = (rank + 1) * w.batch // world
+    return w.replace(batch0=w.batch0 + lo, batch=hi - lo)
 
 
 def kv(w: Workload, layer: int, side: int, loop: int, b: Sequence[int], h: Sequence[int],
        t0: int, t1: int, device="cpu", cscale: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """bf16 [len(b), len(h), t1-t0, D] states of `loop` for the selected rows."""
+    """bf16 [len(b), len(h), t1-t0, D] states of `loop` for the selected rows
+    (b: batch rows of w, 0 .. w.batch-1)."""
     dev = torch.device(device)
     bt = torch.as_tensor(list(b), dtype=torch.int64, device=dev)
     ht = torch.as_tensor(list(h), dtype=torch.int64, device=dev)
@@ -182,6 +196,7 @@ def query(w: Workload, layer: int, loop: int, device="cpu") -> torch.Tensor:
     """bf16 [B, H, D] query of one decode step for `loop`."""
     dev = torch.device(device)
     idx = torch.arange(w.batch * w.heads * w.head_dim, dtype=torch.int64, device=dev)
+    idx = idx + w.batch0 * w.heads * w.head_dim
     n = normal_t(stream_key(w.seed, layer, SIDE_K, loop, KIND_Q), idx).to(torch.float32)
     return n.reshape(w.batch, w.heads, w.head_dim).to(torch.bfloat16)
 
@@ -215,7 +230,7 @@ def seq_lens_ragged(w: Workload, min_frac: float = 0.5) -> list:
     """Deterministic ragged past lengths in [min_frac*T, T] (sequence 0 gets T)."""
     out = []
     key = stream_key(w.seed, 0, 0, 0, 15)
-    for b in range(w.batch):
+    for b in range(w.batch0, w.batch0 + w.batch):
         u = (hash_py(key, b) >> 40) / float(1 << 24)
         n = w.tokens if b == 0 else int(math.floor(w.tokens * (min_frac + (1 - min_frac) * u)))
         out.append(max(0, min(w.tokens, n)))

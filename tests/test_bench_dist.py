@@ -56,6 +56,55 @@ def test_two_rank_max_and_job_throughput(tmp_path):
         assert d["value"] == pytest.approx(world * 16 * 1e3 / 17.5)
 
 
+def _partition_rank_main(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port),
+                       "RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    import numpy as np
+    import bench
+    import residual_bit_kv_b200.synth as synth
+    from rq_harness import oracle_decode
+    ws, r, _ = bench.dist_env()
+    dist = bench.init_dist(ws, backend="gloo")
+    try:
+        per_rank = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=2, tokens=40)
+        mine = bench.rank_share(per_rank, r, ws)
+        lens = synth.seq_lens_ragged(mine)
+        outs = [oracle_decode(mine, 0, loop, range(mine.batch), range(mine.heads), lens)
+                for loop in range(mine.loops)]
+        gathered = [None] * ws
+        dist.all_gather_object(gathered, (mine.batch0, mine.batch, np.stack(outs)))
+        if r == 0:
+            np.save(os.path.join(out_dir, "gathered.npy"),
+                    np.concatenate([g[2] for g in sorted(gathered, key=lambda g: g[0])], axis=1))
+            with open(os.path.join(out_dir, "slices.json"), "w") as f:
+                json.dump([[g[0], g[1]] for g in gathered], f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_batch_partition_matches_one_rank(tmp_path):
+    """Multi-GPU runs split one global batch: rank r takes batch rows
+    [rB/N, (r+1)B/N) of a workload of N times the per-rank batch.  Two gloo
+    ranks each decode their rows with the oracle; their outputs, put side by
+    side, equal the one-process oracle decode of the whole batch."""
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numpy as np
+    import residual_bit_kv_b200.synth as synth
+    from rq_harness import oracle_decode
+    world = 2
+    mp.start_processes(_partition_rank_main, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    assert json.load(open(tmp_path / "slices.json")) == [[0, 2], [2, 2]]
+    whole = synth.WORKLOADS["ouro_layer"].replace(batch=4, heads=2, tokens=40)
+    lens = synth.seq_lens_ragged(whole)
+    want = np.stack([oracle_decode(whole, 0, loop, range(4), range(2), lens)
+                     for loop in range(whole.loops)])
+    np.testing.assert_array_equal(np.load(tmp_path / "gathered.npy"), want)
+
+
 def test_single_process_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench

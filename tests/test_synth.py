@@ -49,3 +49,24 @@ def test_loops_are_correlated_with_the_anchor():
         xr = synth.kv_full(w, 0, synth.SIDE_V, r, 0, 256).float()
         resid = (xr - xa * (xr * xa).sum(-1, keepdim=True) / (xa * xa).sum(-1, keepdim=True))
         assert abs(resid.std().item() - sig) < 0.05 * sig + 0.01
+
+
+def test_batch_partition_reproduces_the_global_rows():
+    """A rank's share of a batch generates exactly those rows of the global
+    workload: states, queries, current tokens and ragged lengths."""
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=5, heads=2, tokens=24)
+    full_k = synth.kv_full(w, 0, synth.SIDE_K, 1, 0, 24)
+    full_q = synth.query(w, 0, 2)
+    full_c = synth.current_token(w, 0, synth.SIDE_V, 0)
+    full_l = synth.seq_lens_ragged(w)
+    rows = []
+    for r in range(3):
+        p = synth.partition(w, r, 3)
+        lo = r * 5 // 3
+        assert p.batch0 == lo and p.batch == (r + 1) * 5 // 3 - lo
+        rows += list(range(lo, lo + p.batch))
+        assert torch.equal(synth.kv_full(p, 0, synth.SIDE_K, 1, 0, 24), full_k[lo:lo + p.batch])
+        assert torch.equal(synth.query(p, 0, 2), full_q[lo:lo + p.batch])
+        assert torch.equal(synth.current_token(p, 0, synth.SIDE_V, 0), full_c[lo:lo + p.batch])
+        assert synth.seq_lens_ragged(p) == full_l[lo:lo + p.batch]
+    assert rows == list(range(5))
