@@ -55,12 +55,14 @@ class GpuCache:
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
                     keep_inputs: bool = True, tokens: Optional[int] = None,
                     max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
-                    fused: bool = False, unit_alpha: bool = False) -> GpuCache:
+                    fused: bool = False, unit_alpha: bool = False,
+                    gen_device: str = "cuda") -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
     the C ABI in the order the policy requires (fused: every loop and both
     sides of a chunk in one rq_quantize_append_loops call).  append_chunks
     splits the token range into consecutive appends (e.g. prefill then
-    single tokens)."""
+    single tokens).  gen_device "cpu" draws the inputs on the host and copies
+    them over (no generator kernels on the GPU)."""
     T = w.tokens if tokens is None else tokens
     lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens, unit_alpha=unit_alpha)
     nbytes = L.rq_cache_bytes(lay)
@@ -73,7 +75,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
     assert bounds[-1] == T
     for layer in layers:
         if fused:
-            xs = {(side, loop): synth.kv_full(w, layer, side, loop, 0, T, device="cuda", chunk_b=4)
+            xs = {(side, loop): synth.kv_full(w, layer, side, loop, 0, T, device=gen_device,
+                                              chunk_b=4).to("cuda")
                   for side in SIDES for loop in range(w.loops)}
             for a, b in zip(bounds[:-1], bounds[1:]):
                 if b == a:
@@ -87,7 +90,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
             del xs
             continue
         for side in SIDES:
-            xs = {loop: synth.kv_full(w, layer, side, loop, 0, T, device="cuda", chunk_b=4)
+            xs = {loop: synth.kv_full(w, layer, side, loop, 0, T, device=gen_device,
+                                      chunk_b=4).to("cuda")
                   for loop in range(w.loops)}
             for a, b in zip(bounds[:-1], bounds[1:]):
                 if b == a:
@@ -166,10 +170,11 @@ def assert_component_equal(gpu: Dict[str, np.ndarray], enc: Dict[str, np.ndarray
 
 
 def decode_inputs(w: synth.Workload, layer: int, loop: int, device="cuda"):
+    """q, k_cur, v_cur of one decode call on the GPU, drawn on `device`."""
     q = synth.query(w, layer, loop, device)
     kc = synth.current_token(w, layer, synth.SIDE_K, loop, device)
     vc = synth.current_token(w, layer, synth.SIDE_V, loop, device)
-    return q.contiguous(), kc.contiguous(), vc.contiguous()
+    return tuple(t.contiguous().to("cuda") for t in (q, kc, vc))
 
 
 class Workspace:
@@ -181,9 +186,9 @@ class Workspace:
 
 
 def gpu_decode(gc: GpuCache, layer: int, loop: int, seq_lens: Sequence[int], max_seq_len: int,
-               ws: Optional[Workspace] = None, scale: float = 0.0):
+               ws: Optional[Workspace] = None, scale: float = 0.0, gen_device: str = "cuda"):
     w = gc.w
-    q, kc, vc = decode_inputs(w, layer, loop)
+    q, kc, vc = decode_inputs(w, layer, loop, gen_device)
     sl = torch.tensor(list(seq_lens), dtype=torch.int32, device="cuda")
     out = torch.empty(w.batch, w.heads, w.head_dim, dtype=torch.float32, device="cuda")
     ws = ws or Workspace(gc.layout, max_seq_len)
