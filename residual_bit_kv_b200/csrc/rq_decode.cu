@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
 template <int D>
 size_t scratch_bytes() {
-  return (Geom<D>::NSLOT * D + 2 * Geom<D>::NSLOT) * sizeof(float);
+  return (Geom<D>::NSLOT * red_pitch<D>() + 2 * Geom<D>::NSLOT) * sizeof(float);
 }
 
 template <typename K>

@@ -60,8 +60,17 @@ __device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int ma
 // `slot` for channels [32*slice, 32*slice+32).  The slots are reduced into one
 // partial (m, l, acc[D]) in the workspace; the last CTA of the (batch, head)
 // then merges every split with the current token and writes the output,
-// applying H^T once when ROT.  `scratch` holds max(NSLOT*D + 2*NSLOT,
-// 3*splits) floats.
+// applying H^T once when ROT.  `scratch` holds max(NSLOT*red_pitch<D>() +
+// 2*NSLOT, 3*splits) floats.
+//
+// The slot reduction buffer keeps each slice's 32 channels in a block of 36
+// floats (a slot is D/32 blocks): the 16-byte stores of the lanes of one
+// quarter-warp (consecutive slices and slots) then fall in distinct bank
+// groups.
+constexpr int kRedSliceFloats = 36;
+template <int D>
+__host__ __device__ constexpr int red_pitch() { return (D / 32) * kRedSliceFloats; }
+
 template <int D, int NT, int NSLOT, bool ROT>
 __device__ __forceinline__ void finish_split(float m, float l, const float (&acc)[32], int slice,
                                              int slot, float* scratch, int bhi, int split,
@@ -70,8 +79,9 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
                                              const uint16_t* vcur, float scale_log2,
                                              float rot_scale, float* out, float* svec,
                                              float* sred) {
-  float* red = scratch;                 // [NSLOT][D]
-  float* mred = red + NSLOT * D;        // [NSLOT]
+  constexpr int RP = red_pitch<D>();
+  float* red = scratch;                 // [NSLOT][D/32][36]
+  float* mred = red + NSLOT * RP;       // [NSLOT]
   float* lred = mred + NSLOT;           // [NSLOT]
   const int t = threadIdx.x;
   if (slot >= 0 && slice == 0) {
@@ -83,7 +93,7 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
   for (int s = 0; s < NSLOT; ++s) M = fmaxf(M, mred[s]);
   if (slot >= 0) {
     const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - M);
-    float4* dst = reinterpret_cast<float4*>(red + slot * D + slice * 32);
+    float4* dst = reinterpret_cast<float4*>(red + slot * RP + slice * kRedSliceFloats);
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       dst[i] = make_float4(acc[4 * i] * f, acc[4 * i + 1] * f, acc[4 * i + 2] * f,
@@ -93,7 +103,8 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
   float* part = partials + (static_cast<size_t>(bhi) * splits + split) * (D + 2);
   if (t < D) {
     float sum = 0.0f;
-    for (int s = 0; s < NSLOT; ++s) sum += red[s * D + t];
+    const float* col = red + (t >> 5) * kRedSliceFloats + (t & 31);
+    for (int s = 0; s < NSLOT; ++s) sum += col[s * RP];
     part[2 + t] = sum;
   }
   if (t == 0) {
@@ -103,14 +114,20 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
     part[0] = M;
     part[1] = L;
   }
-  // Publish the partial, then count this split in (no waiting on other CTAs).
-  __threadfence();
+  // Publish the partial, then count this split in (no waiting on other CTAs):
+  // the CTA barrier orders every thread's partial writes before thread 0's
+  // acquire-release add, which makes them visible with it (and, for the last
+  // CTA, makes every other split's partial visible to it).
   __syncthreads();
   __shared__ uint32_t s_last;
-  if (t == 0) s_last = (atomicAdd(counters + bhi, 1u) == static_cast<uint32_t>(splits - 1));
+  if (t == 0) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(old) : "l"(counters + bhi) : "memory");
+    s_last = (old == static_cast<uint32_t>(splits - 1));
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
 
   // ---- last CTA of this (batch, head): merge ----
   // Current token score q.k_cur, original domain [RQ §3.2, §4.2].

@@ -707,10 +707,10 @@ cudaError_t prep(K kernel, size_t dyn, int* occ, int threads = kThreads) {
   return e;
 }
 
-// merge scratch of a kernel with `warps` compute warps: NSLOT*(D+2) floats
+// merge scratch of a kernel with `warps` compute warps: NSLOT*(pitch+2) floats
 template <int D>
 constexpr size_t scratch_floats(int warps = kWarps) {
-  return static_cast<size_t>(warps * (32 / (D / 32))) * (D + 2);
+  return static_cast<size_t>(warps * (32 / (D / 32))) * (red_pitch<D>() + 2);
 }
 
 template <class SP>
