@@ -251,6 +251,14 @@ rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads,
  * re-initialise the workspace). */
 rq_status rq_workspace_error(void* workspace, uint64_t ws_bytes, void* stream);
 
+/* Self-test of the device-side failure path (for tests): one CTA waits on an
+ * mbarrier phase that nothing completes, with a limit of limit_ms of device
+ * time (1..1000), records the timeout in the workspace's error word and
+ * returns; rq_workspace_error then reports RQ_ERR_TIMEOUT and the context
+ * stays usable.  workspace as for rq_decode_attention. */
+rq_status rq_selftest_wait_timeout(void* workspace, uint64_t ws_bytes, int32_t limit_ms,
+                                   void* stream);
+
 /* Number of split-K partitions rq_decode_attention uses for this shape on
  * the current device (for tests and benchmarks). */
 int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);

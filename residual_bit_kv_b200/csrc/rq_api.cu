@@ -426,6 +426,16 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
   return RQ_OK;
 }
 
+rq_status rq_selftest_wait_timeout(void* workspace, uint64_t ws_bytes, int32_t limit_ms,
+                                   void* stream) {
+  if (workspace == nullptr || !aligned(workspace, kAlign) || ws_bytes < kAlign)
+    return RQ_ERR_INVALID_ARG;
+  if (limit_ms < 1 || limit_ms > 1000) return RQ_ERR_INVALID_ARG;
+  uint32_t* err = static_cast<uint32_t*>(workspace);   // the error word (offset 0)
+  return cuda_status(launch_selftest_wait(err, static_cast<uint64_t>(limit_ms) * 1000000ull,
+                                          as_stream(stream)));
+}
+
 int32_t rq_decode_splits(const rq_layout* l, int32_t max_seq_len) {
   if (rq_layout_validate(l) != RQ_OK || max_seq_len < 0) return 0;
   // Shape-only: a cache bound to dummy (aligned, never dereferenced) bases.

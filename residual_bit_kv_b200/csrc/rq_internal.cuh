@@ -150,6 +150,8 @@ struct DecodeBf16Params {
 // Host-side launchers (defined in the .cu files)
 // ---------------------------------------------------------------------------
 
+// Self-test: one CTA waits `limit_ns` on an mbarrier phase nothing completes.
+cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
                             cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s);
@@ -241,13 +243,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on a phase of an mbarrier: gives up after ~2^22 polls (well
-// over a second with the back-off), records kErrTimeout and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint32_t* err) {
-  for (uint32_t it = 0; it < (1u << 22); ++it) {
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on a phase of an mbarrier: gives up once `limit_ns` of device
+// time have passed (checked every 64 polls), or after 2^26 polls whatever the
+// clock says, records kErrTimeout and returns false.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0; it < (1u << 26); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (it == 0) t0 = global_ns();   // the clock is read only once a wait is needed
     if (it > 16) __nanosleep(256);
+    if ((it & 63u) == 63u && global_ns() - t0 > limit_ns) break;
   }
   atomicOr(err, kErrTimeout);
   return false;

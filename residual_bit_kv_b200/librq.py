@@ -37,7 +37,7 @@ SYMBOLS = (
     "rq_dequantize", "rq_decode_workspace_bytes", "rq_decode_workspace_init",
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
     "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
-    "rq_quantize_append_loops",
+    "rq_quantize_append_loops", "rq_selftest_wait_timeout",
 )
 
 
@@ -104,6 +104,7 @@ def load() -> ctypes.CDLL:
         "rq_decode_attention_bf16": ([_I32, _I32, _I32, _P, _P, _P, _I64, _P, _I32, _P, _P, _F,
                                       _P, _P, _U64, _P], ctypes.c_int),
         "rq_workspace_error": ([_P, _U64, _P], ctypes.c_int),
+        "rq_selftest_wait_timeout": ([_P, ctypes.c_uint64, ctypes.c_int32, _P], ctypes.c_int),
         "rq_decode_splits": ([LP, _I32], _I32),
         "rq_decode_attention_noalloc": ([CP, _I32, _I32, _P, _P, _I32, _P, _P, _F, _P, _P],
                                         ctypes.c_int),
@@ -242,6 +243,11 @@ def rq_decode_attention_bf16(batch: int, heads: int, head_dim: int, q, k, v, tok
 
 def rq_workspace_error(workspace, ws_bytes: int, stream=None) -> int:
     return int(load().rq_workspace_error(_ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def rq_selftest_wait_timeout(workspace, ws_bytes: int, limit_ms: int, stream=None) -> None:
+    _check(load().rq_selftest_wait_timeout(_ptr(workspace), ws_bytes, limit_ms, _stream(stream)),
+           "rq_selftest_wait_timeout")
 
 
 def rq_decode_splits(layout: rq_layout, max_seq_len: int) -> int:

@@ -145,6 +145,11 @@ def test_host_checks_reject_before_launch(L):
         L.rq_decode_attention_bf16(1, 1, 96, 256, 256, 256, 10, 256, 10, 256, 256, 0.0, 256, 256,
                                    1 << 20, stream=0)
     assert e.value.status == L.RQ_ERR_UNSUPPORTED
+    for args in [(256, 1 << 20, 0), (256, 1 << 20, 1001), (256 + 4, 1 << 20, 5), (0, 1 << 20, 5),
+                 (256, 8, 5)]:
+        with pytest.raises(L.RQError) as e:
+            L.rq_selftest_wait_timeout(*args, stream=0)
+        assert e.value.status == L.RQ_ERR_INVALID_ARG, args
 
 
 def test_no_cpu_fallback_in_product():
