@@ -254,22 +254,24 @@ def policy_chain(L, loop, policy):
     return comps, A
 
 
-def component_bytes_per_row(w, loop, policy="last"):
+def component_bytes_per_row(w, loop, policy="last", meta_bytes=4):
     """Packed bytes of one (token, head) row of every component loop `loop`
-    reads, for one side (codes + fp16 scale/offset + bf16 LS coefficient)."""
+    reads, for one side (codes + metadata (fp16 scale/offset: 4 bytes per
+    group; 16-bit metadata: 2) + bf16 LS coefficient)."""
     D = w.head_dim
     comps, A = policy_chain(w.loops, loop, policy)
     tot = 0
     for r in comps:
-        tot += D * w.bits[r] // 8 + (D // w.group[r]) * 4 + (2 if r != A else 0)
+        tot += D * w.bits[r] // 8 + (D // w.group[r]) * meta_bytes + (2 if r != A else 0)
     return tot
 
 
-def decode_call_bytes(w, loop, seq_len, policy="last"):
+def decode_call_bytes(w, loop, seq_len, policy="last", meta_bytes=4):
     """Algorithmic bytes of one decode call: packed K and V of every past
     token, plus q, k_cur, v_cur (bf16) and the fp32 output."""
     bh = w.batch * w.heads
-    return bh * (2 * seq_len * component_bytes_per_row(w, loop, policy) + w.head_dim * (2 * 3 + 4))
+    return bh * (2 * seq_len * component_bytes_per_row(w, loop, policy, meta_bytes) +
+                 w.head_dim * (2 * 3 + 4))
 
 
 def quant_call_bytes(w, loop, n):
@@ -786,14 +788,16 @@ def main():
 POLICY_NAMES = ("last", "next", "first", "previous")
 
 
-def policy_decode_step(w, policy, dev, stream, args):
-    """One layer of workload w stored under `policy`: the time of a decode
-    step over every loop (one call per loop) and its algorithmic bytes."""
+def policy_decode_step(w, policy, dev, stream, args, meta16=False):
+    """One layer of workload w stored under `policy` (16-bit metadata per
+    group if meta16): the time of a decode step over every loop (one call
+    per loop) and its algorithmic bytes."""
     import residual_bit_kv_b200.librq as L
     T = w.tokens
     code = {"last": L.RQ_POLICY_LAST_LOOP, "next": L.RQ_POLICY_NEXT_LOOP,
             "first": L.RQ_POLICY_FIRST_LOOP, "previous": L.RQ_POLICY_PREVIOUS_LOOP}[policy]
-    lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T + 16, w.bits, w.group, code)
+    lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T + 16, w.bits, w.group, code,
+                        L.RQ_FLAG_META16 if meta16 else 0)
     nb = L.rq_cache_bytes(lay)
     kb = torch.empty(nb, dtype=torch.uint8, device=dev)
     vb = torch.empty(nb, dtype=torch.uint8, device=dev)
@@ -820,7 +824,8 @@ def policy_decode_step(w, policy, dev, stream, args):
                                   ws, wsb, stream)
 
     ms = timed(step, args.steps, args.warmup, stream)
-    byt = sum(decode_call_bytes(w, l, T, policy) for l in range(w.loops))
+    byt = sum(decode_call_bytes(w, l, T, policy, meta_bytes=2 if meta16 else 4)
+              for l in range(w.loops))
     reads = sum(len(policy_chain(w.loops, l, policy)[0]) for l in range(w.loops))
     del kb, vb, ws
     torch.cuda.empty_cache()
@@ -861,6 +866,25 @@ def bench_ablation(dev, stream, args, hbm):
     pol["throughput_first_over_previous"] = (pol["previous"]["ms_per_step"] /
                                              pol["first"]["ms_per_step"])
     out["policies_ouro_16k_layer"] = pol
+    # 16-bit metadata per group (the pages' accounting) on the same layer
+    wm = synth.WORKLOADS["ouro_16k"].replace(layers=1)
+    m16 = {"workload": f"{wm.name}: 1 layer x {wm.loops} loops, batch {wm.batch}, {wm.heads} "
+                       f"heads, {wm.tokens} past tokens, bits {list(wm.bits)}, group {wm.group[0]}"}
+    for name, flag in (("meta32", False), ("meta16", True)):
+        ms, byt, _ = policy_decode_step(wm, "last", dev, stream, args, meta16=flag)
+        mb = 2 if flag else 4
+        m16[name] = {"ms_per_step": ms, "bytes_per_step": byt, "gbs": byt / (ms * 1e-3) / 1e9,
+                     "frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
+                     "tokens_per_s_layer": wm.batch / (ms * 1e-3),
+                     "bytes_per_token_head_per_loop": [
+                         2 * component_bytes_per_row(wm, l, "last", mb) for l in range(wm.loops)],
+                     "bits_per_element": [
+                         8 * (component_bytes_per_row(wm, l, "last", mb) -
+                              (component_bytes_per_row(wm, wm.loops - 1, "last", mb)
+                               if l != wm.loops - 1 else 0)) / wm.head_dim
+                         for l in range(wm.loops)]}
+    m16["speedup_meta16_over_meta32"] = m16["meta32"]["ms_per_step"] / m16["meta16"]["ms_per_step"]
+    out["metadata16_ouro_16k_layer"] = m16
     return out
 
 

@@ -31,14 +31,20 @@
  *   A record holds, contiguously:
  *     codes  uint32 [32][head_dim * bits[r] / 32]
  *     meta   uint32 [32][head_dim / group[r]]; low half fp16 scale s~,
- *            high half fp16 offset z~
+ *            high half fp16 offset z~ (with RQ_FLAG_META16: uint16
+ *            [32][head_dim / group[r]], scale byte | offset byte << 8, where
+ *            s~ = (1 + m/8) 2^(E - 18) for the byte 8E + m, E = 0 meaning 0;
+ *            s~ is the nearest such value to max((max - min)/(2^b - 1),
+ *            |min|/15.875) (below the range: the smallest; above: the
+ *            largest) and zq = clamp(floor(8 min / s~), -128, 127))
  *     alpha  bf16   [32]             (residual loops only)
  *   so a decode stage of one component (one or two records) is one
  *   contiguous copy.
  *   Code order inside a token's row: b = 2: channel i in word i/16, bits
  *   [2*(i%16), +2).  b = 4: in blocks of 16 channels, i = 16u + v, word
  *   2u + ((v>>1)&1), bits [4*(2*(v>>2) + (v&1)), +4).  Little-endian words.
- *   Effective bits per element of loop r: bits[r] + 32/group[r]
+ *   Effective bits per element of loop r: bits[r] + 32/group[r] (16/group[r]
+ *   with RQ_FLAG_META16)
  *   (+ 16/head_dim for a residual loop).  Components are laid out anchor
  *   first, then the other loops in increasing index (comp_off).
  *
@@ -91,6 +97,10 @@ typedef enum rq_policy {
 /* rq_layout.flags */
 #define RQ_FLAG_UNIT_ALPHA 1   /* alpha_r = 1: plain differences, no LS scaling
                                   [RQ §3.1-§3.2, Table 3 "w/o LS scaling"] */
+#define RQ_FLAG_META16 2       /* 16 bits of metadata per group [RQ §5.1,
+                                  App. A.3]: meta uint16 = scale byte (unsigned
+                                  e5m3, bias 18, 0 = zero scale) | offset byte
+                                  (int8 zq, z~ = zq * s~ / 8) << 8; see below */
 
 /* Shape and precision of a compressed KV cache.
  *   num_layers  >= 1
@@ -100,7 +110,7 @@ typedef enum rq_policy {
  *   head_dim    D in {64, 128}
  *   max_tokens  token capacity per (batch, head), >= 1
  *   policy      rq_policy
- *   flags       0 or RQ_FLAG_UNIT_ALPHA
+ *   flags       0 or RQ_FLAG_UNIT_ALPHA | RQ_FLAG_META16
  *   bits[r]     2 or 4
  *   group[r]    g in {16, 32, 64, 128}, g divides D, g * bits[r] >= 32
  */

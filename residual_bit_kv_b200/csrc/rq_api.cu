@@ -49,9 +49,11 @@ inline int64_t token_stride_of(const rq_layout* l) {
   return static_cast<int64_t>(align_up(static_cast<uint64_t>(l->max_tokens), kRowTokens));
 }
 
+inline int meta_bytes_of(const rq_layout* l) { return (l->flags & RQ_FLAG_META16) ? 2 : 4; }
+
 inline uint32_t record_bytes(const rq_layout* l, int r) {
   const int D = l->head_dim;
-  const uint32_t per_token = (D * l->bits[r] / 32) * 4 + (D / l->group[r]) * 4 +
+  const uint32_t per_token = (D * l->bits[r] / 32) * 4 + (D / l->group[r]) * meta_bytes_of(l) +
                              (r != anchor_of(l) ? 2 : 0);
   return kBlock * per_token;   // a multiple of 64 bytes
 }
@@ -151,6 +153,7 @@ Comp comp_of(const rq_cache* c, int layer, int kv, int r) {
   k.bits = c->layout.bits[r];
   k.group = c->layout.group[r];
   k.has_alpha = (r != anchor_of(&c->layout)) ? 1 : 0;
+  k.meta16 = (c->layout.flags & RQ_FLAG_META16) ? 1 : 0;
   return k;
 }
 
@@ -217,7 +220,7 @@ rq_status rq_layout_validate(const rq_layout* l) {
   if (l->batch < 1 || l->kv_heads < 1 || l->max_tokens < 1) return RQ_ERR_INVALID_ARG;
   if (l->policy < RQ_POLICY_LAST_LOOP || l->policy > RQ_POLICY_PREVIOUS_LOOP)
     return RQ_ERR_INVALID_ARG;
-  if ((l->flags & ~RQ_FLAG_UNIT_ALPHA) != 0) return RQ_ERR_INVALID_ARG;
+  if ((l->flags & ~(RQ_FLAG_UNIT_ALPHA | RQ_FLAG_META16)) != 0) return RQ_ERR_INVALID_ARG;
   if (!is_pow2(l->head_dim) || l->head_dim < 32 || l->head_dim > 256) return RQ_ERR_INVALID_ARG;
   if (l->head_dim != 64 && l->head_dim != 128) return RQ_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(l->batch) * l->kv_heads > 65535) return RQ_ERR_UNSUPPORTED;

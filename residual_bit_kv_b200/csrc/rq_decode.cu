@@ -59,7 +59,7 @@ __host__ __device__ inline void build_stage_map(const DecodeParams& p, int D,
     for (int c = 0; c < p.ncomp; ++c) {
       m.comp[side][c] = off;
       m.meta[side][c] = kBlock * (D * cs[c].bits / 32) * 4;
-      m.alpha[side][c] = m.meta[side][c] + kBlock * (D / cs[c].group) * 4;
+      m.alpha[side][c] = m.meta[side][c] + kBlock * (D / cs[c].group) * (cs[c].meta16 ? 2 : 4);
       off += kRecsPerStage * cs[c].rec_bytes;
     }
   }
@@ -73,12 +73,45 @@ __device__ __forceinline__ const unsigned char* stage_rec(const unsigned char* s
   return st + m.comp[side][c] + (j / kBlock) * cp.rec_bytes;
 }
 
+// Scale and offset of this lane's group parts from one token's metadata row
+// (fp16 pairs, or 16-bit metadata when m16): part 0 = channels 0-15 (the whole
+// slice for g >= 32), part 1 = channels 16-31.
+__device__ __forceinline__ void lane_meta(const unsigned char* mrow, int slice, int gshift,
+                                          bool m16, float& s0, float& z0, float& s1,
+                                          float& z1) {
+  if (m16) {
+    const uint16_t* mr = reinterpret_cast<const uint16_t*>(mrow);
+    uint32_t h0, h1;
+    if (gshift >= 5) {
+      h0 = h1 = mr[(slice * 32) >> gshift];
+    } else {
+      h0 = mr[slice * 2];
+      h1 = mr[slice * 2 + 1];
+    }
+    s0 = m16_scale_value(h0 & 0xFFu);
+    z0 = m16_offset(h0, s0);
+    s1 = m16_scale_value(h1 & 0xFFu);
+    z1 = m16_offset(h1, s1);
+    return;
+  }
+  const uint32_t* mr = reinterpret_cast<const uint32_t*>(mrow);
+  if (gshift >= 5) {
+    unpack_meta(mr[(slice * 32) >> gshift], s0, z0);
+    s1 = s0;
+    z1 = z0;
+  } else {
+    const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
+    unpack_meta(mw.x, s0, z0);
+    unpack_meta(mw.y, s1, z1);
+  }
+}
+
 // q'.D(c) over this lane's 32 channels of one token of one component:
 // s~ * sum q'_i c_i + z~ * sum q'_i per group part.
 template <int BITS>
-__device__ __forceinline__ float comp_dot(const uint32_t* cw, const uint32_t* mrow,
-                                          int slice, int gshift, const float (&q)[32],
-                                          float qsa, float qsb) {
+__device__ __forceinline__ float comp_dot(const uint32_t* cw, const unsigned char* mrow,
+                                          bool m16, int slice, int gshift,
+                                          const float (&q)[32], float qsa, float qsb) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   uint32_t w[BITS];
   if constexpr (BITS == 4) {
@@ -98,21 +131,16 @@ __device__ __forceinline__ float comp_dot(const uint32_t* cw, const uint32_t* mr
       a1 = fmaf(q[ch], code_to_float(c), a1);
   }
   float s0, z0, s1, z1;
-  if (gshift >= 5) {
-    unpack_meta(mrow[(slice * 32) >> gshift], s0, z0);
-    return s0 * (a0 + a1) + z0 * (qsa + qsb);
-  }
-  const uint2 mw = *reinterpret_cast<const uint2*>(mrow + slice * 2);
-  unpack_meta(mw.x, s0, z0);
-  unpack_meta(mw.y, s1, z1);
+  lane_meta(mrow, slice, gshift, m16, s0, z0, s1, z1);
+  if (gshift >= 5) return s0 * (a0 + a1) + z0 * (qsa + qsb);
   return s0 * a0 + z0 * qsa + (s1 * a1 + z1 * qsb);
 }
 
 // acc += pk * D(c) over this lane's 32 channels; the offsets go to cst0/cst1.
 template <int BITS>
-__device__ __forceinline__ void comp_acc(const uint32_t* cw, const uint32_t* mrow,
-                                         int slice, int gshift, float pk, float (&acc)[32],
-                                         float& cst0, float& cst1) {
+__device__ __forceinline__ void comp_acc(const uint32_t* cw, const unsigned char* mrow,
+                                         bool m16, int slice, int gshift, float pk,
+                                         float (&acc)[32], float& cst0, float& cst1) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   uint32_t w[BITS];
   if constexpr (BITS == 4) {
@@ -123,15 +151,7 @@ __device__ __forceinline__ void comp_acc(const uint32_t* cw, const uint32_t* mro
     w[0] = v.x; w[1] = v.y;
   }
   float s0, z0, s1, z1;
-  if (gshift >= 5) {
-    unpack_meta(mrow[(slice * 32) >> gshift], s0, z0);
-    s1 = s0;
-    z1 = z0;
-  } else {
-    const uint2 mw = *reinterpret_cast<const uint2*>(mrow + slice * 2);
-    unpack_meta(mw.x, s0, z0);
-    unpack_meta(mw.y, s1, z1);
-  }
+  lane_meta(mrow, slice, gshift, m16, s0, z0, s1, z1);
   const float w0 = pk * s0, w1 = pk * s1;
   cst0 = fmaf(pk, z0, cst0);
   cst1 = fmaf(pk, z1, cst1);
@@ -239,10 +259,11 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const unsigned char* rec = stage_rec(st, map, p.k[c], 0, c, j);
         const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * (D * bits / 32) +
                              slice * bits;
-        const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + map.meta[0][c]) +
-                             jl * (D / p.k[c].group);
-        const float d = (bits == 4) ? comp_dot<4>(cw, mr, slice, log2_pow2(p.k[c].group), q, qsa, qsb)
-                                    : comp_dot<2>(cw, mr, slice, log2_pow2(p.k[c].group), q, qsa, qsb);
+        const bool m16 = p.k[c].meta16 != 0;
+        const unsigned char* mr = rec + map.meta[0][c] + jl * (D / p.k[c].group) * (m16 ? 2 : 4);
+        const float d = (bits == 4)
+                            ? comp_dot<4>(cw, mr, m16, slice, log2_pow2(p.k[c].group), q, qsa, qsb)
+                            : comp_dot<2>(cw, mr, m16, slice, log2_pow2(p.k[c].group), q, qsa, qsb);
         part = fmaf(kappa, d, part);
         if (c + 1 < p.ncomp)
           kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[0][c])[jl]);
@@ -278,12 +299,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const unsigned char* rec = stage_rec(st, map, p.v[c], 1, c, j);
         const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * (D * bits / 32) +
                              slice * bits;
-        const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + map.meta[1][c]) +
-                             jl * (D / p.v[c].group);
+        const bool m16 = p.v[c].meta16 != 0;
+        const unsigned char* mr = rec + map.meta[1][c] + jl * (D / p.v[c].group) * (m16 ? 2 : 4);
         if (bits == 4)
-          comp_acc<4>(cw, mr, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
+          comp_acc<4>(cw, mr, m16, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
         else
-          comp_acc<2>(cw, mr, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
+          comp_acc<2>(cw, mr, m16, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
         if (c + 1 < p.ncomp)
           kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[1][c])[jl]);
       }

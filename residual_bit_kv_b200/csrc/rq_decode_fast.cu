@@ -52,16 +52,16 @@ constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, u
 // Compile-time layout of one stage: for side K then V, component c occupies
 // RPS = 2 consecutive records (64 tokens, one copy); a record is
 // [codes[32][wpr] | meta[32][gpr] | alpha[32]].
-template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_>
+template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_, int M16_ = 0>
 struct Spec {
-  static constexpr int D = D_, NC = NC_, RPS = 2, TC = kBlock * RPS;
+  static constexpr int D = D_, NC = NC_, RPS = 2, TC = kBlock * RPS, M16 = M16_;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
   __host__ __device__ static constexpr int wpr(int c) { return D_ * bits(c) / 32; }
   __host__ __device__ static constexpr int gpr(int c) { return D_ / group(c); }
   __host__ __device__ static constexpr uint32_t rec_bytes(int c) {
-    return kBlock * (wpr(c) * 4 + gpr(c) * 4 + (has_alpha(c) ? 2 : 0));
+    return kBlock * (wpr(c) * 4 + gpr(c) * (M16_ ? 2 : 4) + (has_alpha(c) ? 2 : 0));
   }
   __host__ __device__ static constexpr uint32_t comp_bytes(int c) { return RPS * rec_bytes(c); }
   __host__ __device__ static constexpr uint32_t side_bytes() {
@@ -81,16 +81,50 @@ struct Spec {
   }
 };
 
-// Offsets inside a record of a component with these parameters.
-template <int D, int BITS, int G>
+// Offsets inside a record of a component with these parameters (M16: 16-bit
+// metadata per group).
+template <int D, int BITS, int G, int M16 = 0>
 struct RecGeom {
   enum : uint32_t {
     WPR = D * BITS / 32,
     GPR = D / G,
     META = kBlock * WPR * 4,
-    ALPHA = META + kBlock * GPR * 4,
+    ALPHA = META + kBlock * GPR * (M16 ? 2 : 4),
   };
 };
+
+// Scale and offset of this lane's group(s) at record token jl: [0] channels
+// 0-15 (or the whole slice when g >= 32), [1] channels 16-31 (g = 16).
+template <int D, int BITS, int G, int M16>
+__device__ __forceinline__ void group_meta(const unsigned char* rec, int jl, int slice,
+                                           float (&s)[2], float (&z)[2]) {
+  using RG = RecGeom<D, BITS, G, M16>;
+  if constexpr (M16) {
+    const uint16_t* mr = reinterpret_cast<const uint16_t*>(rec + RG::META) + jl * RG::GPR;
+    if constexpr (G >= 32) {
+      const uint32_t h = mr[(slice * 32) / G];
+      s[0] = s[1] = m16_scale_value(h & 0xFFu);
+      z[0] = z[1] = m16_offset(h, s[0]);
+    } else {
+      const uint32_t hh = *reinterpret_cast<const uint32_t*>(mr + slice * 2);
+      s[0] = m16_scale_value(hh & 0xFFu);
+      z[0] = m16_offset(hh & 0xFFFFu, s[0]);
+      s[1] = m16_scale_value((hh >> 16) & 0xFFu);
+      z[1] = m16_offset(hh >> 16, s[1]);
+    }
+  } else {
+    const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + RG::META) + jl * RG::GPR;
+    if constexpr (G >= 32) {
+      unpack_meta(mr[(slice * 32) / G], s[0], z[0]);
+      s[1] = s[0];
+      z[1] = z[0];
+    } else {
+      const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
+      unpack_meta(mw.x, s[0], z[0]);
+      unpack_meta(mw.y, s[1], z[1]);
+    }
+  }
+}
 
 // Fixed-point rotated query of one lane's 32 channels as int8 limb bytes in
 // the quad order of the unpacked codes: quad (k, s) holds channels
@@ -102,10 +136,10 @@ struct QLimbs {
 
 // q~ . D(c) over one lane's 32 channels of record token jl of a component,
 // in sigma units: sum over group parts of s~ * (q~ . codes) + z~ * (sum q~).
-template <int D, int BITS, int G>
+template <int D, int BITS, int G, int M16>
 __device__ __forceinline__ float kdot(const unsigned char* rec, int jl, int slice,
                                       const QLimbs& ql) {
-  using RG = RecGeom<D, BITS, G>;
+  using RG = RecGeom<D, BITS, G, M16>;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * RG::WPR + slice * BITS;
   int ah[2] = {0, 0}, al[2] = {0, 0};   // per 16-channel block
   if constexpr (BITS == 4) {
@@ -133,19 +167,14 @@ __device__ __forceinline__ float kdot(const unsigned char* rec, int jl, int slic
         al[k] = __dp4a(ql.l[k][s], x, al[k]);
       }
   }
-  const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + RG::META) + jl * RG::GPR;
-  float s0, z0;
+  float sm[2], zm[2];
+  group_meta<D, BITS, G, M16>(rec, jl, slice, sm, zm);
   if constexpr (G >= 32) {
-    unpack_meta(mr[(slice * 32) / G], s0, z0);
-    return s0 * static_cast<float>((ah[0] + ah[1]) * 256 + (al[0] + al[1])) +
-           z0 * (ql.sq[0] + ql.sq[1]);
+    return sm[0] * static_cast<float>((ah[0] + ah[1]) * 256 + (al[0] + al[1])) +
+           zm[0] * (ql.sq[0] + ql.sq[1]);
   } else {
-    float s1, z1;
-    const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
-    unpack_meta(mw.x, s0, z0);
-    unpack_meta(mw.y, s1, z1);
-    return s0 * static_cast<float>(ah[0] * 256 + al[0]) + z0 * ql.sq[0] +
-           (s1 * static_cast<float>(ah[1] * 256 + al[1]) + z1 * ql.sq[1]);
+    return sm[0] * static_cast<float>(ah[0] * 256 + al[0]) + zm[0] * ql.sq[0] +
+           (sm[1] * static_cast<float>(ah[1] * 256 + al[1]) + zm[1] * ql.sq[1]);
   }
 }
 
@@ -176,21 +205,17 @@ __device__ __forceinline__ float2 masked_pair(uint32_t w, uint32_t ma, uint32_t 
 //          channels 16k + 8 + 2i, +1 at the same bits of word >> 16;
 //   b = 4: word 2k + hh holds channels 16k + 2hh, +1 at bits 0, 4 and
 //          16k + 4 + 2hh, +1 at bits 8, 12; word >> 16 gives channels + 8.
-template <int D, int BITS, int G>
+template <int D, int BITS, int G, int M16>
 __device__ __forceinline__ void vacc(const unsigned char* rec, int jl, int slice, float pk,
                                      VAcc& va) {
-  using RG = RecGeom<D, BITS, G>;
+  using RG = RecGeom<D, BITS, G, M16>;
   const uint32_t* cw = reinterpret_cast<const uint32_t*>(rec) + jl * RG::WPR + slice * BITS;
-  const uint32_t* mr = reinterpret_cast<const uint32_t*>(rec + RG::META) + jl * RG::GPR;
   constexpr int NW = G >= 32 ? 1 : 2;   // weights per lane (16-channel halves for g = 16)
   float sc[2], zc[2];
+  group_meta<D, BITS, G, M16>(rec, jl, slice, sc, zc);
   if constexpr (NW == 1) {
-    unpack_meta(mr[(slice * 32) / G], sc[0], zc[0]);
     va.cst[2] = fmaf(pk, zc[0], va.cst[2]);
   } else {
-    const uint2 mw = *reinterpret_cast<const uint2*>(mr + slice * 2);
-    unpack_meta(mw.x, sc[0], zc[0]);
-    unpack_meta(mw.y, sc[1], zc[1]);
     va.cst[0] = fmaf(pk, zc[0], va.cst[0]);
     va.cst[1] = fmaf(pk, zc[1], va.cst[1]);
   }
@@ -246,9 +271,9 @@ template <class SP, int REC, int C = 0>
 __device__ __forceinline__ void score_comps(const unsigned char* st, int rl, int jl, int slice,
                                             const QLimbs& ql, float& part, float& kap) {
   if constexpr (C < SP::NC) {
-    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
+    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C), SP::M16>;
     const unsigned char* rec = st + SP::comp_off(0, C) + (REC + rl) * SP::rec_bytes(C);
-    const float d = kdot<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, ql);
+    const float d = kdot<SP::D, SP::bits(C), SP::group(C), SP::M16>(rec, jl, slice, ql);
     part = fmaf(kap, d, part);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
@@ -260,9 +285,9 @@ template <class SP, int REC, int C = 0>
 __device__ __forceinline__ void value_comps(const unsigned char* st, int rl, int jl, int slice,
                                             float kap, VAcc& va) {
   if constexpr (C < SP::NC) {
-    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C)>;
+    using RG = RecGeom<SP::D, SP::bits(C), SP::group(C), SP::M16>;
     const unsigned char* rec = st + SP::comp_off(1, C) + (REC + rl) * SP::rec_bytes(C);
-    vacc<SP::D, SP::bits(C), SP::group(C)>(rec, jl, slice, kap, va);
+    vacc<SP::D, SP::bits(C), SP::group(C), SP::M16>(rec, jl, slice, kap, va);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
     value_comps<SP, REC, C + 1>(st, rl, jl, slice, kap, va);
@@ -723,7 +748,7 @@ size_t dyn_bytes(int stages) {
 
 // Host-side description of one compiled layout.
 struct FastEntry {
-  int D, NC, RB, RG, AB, AG;
+  int D, NC, RB, RG, AB, AG, M16;
   uint32_t stage_bytes;
   int chunk;
   cudaError_t (*launch)(const DecodeParams&, cudaStream_t);
@@ -744,10 +769,13 @@ cudaError_t occ_spec(int stages, int* occ) {
   return prep(decode_fast_kernel<SP>, dyn_bytes<SP>(stages), occ, kCThreads);
 }
 
-#define RQ_FAST(D, NC, RB, RG, AB, AG)                                                        \
-  FastEntry{D,  NC, RB, RG, AB, AG, Spec<D, NC, RB, RG, AB, AG>::stage_bytes(),              \
-            Spec<D, NC, RB, RG, AB, AG>::TC,                                                 \
-            &launch_spec<Spec<D, NC, RB, RG, AB, AG>>, &occ_spec<Spec<D, NC, RB, RG, AB, AG>>}
+#define RQ_FAST_M(D, NC, RB, RG, AB, AG, M)                                                    \
+  FastEntry{D,  NC, RB, RG, AB, AG, M, Spec<D, NC, RB, RG, AB, AG, M>::stage_bytes(),        \
+            Spec<D, NC, RB, RG, AB, AG, M>::TC,                                              \
+            &launch_spec<Spec<D, NC, RB, RG, AB, AG, M>>,                                    \
+            &occ_spec<Spec<D, NC, RB, RG, AB, AG, M>>}
+#define RQ_FAST(D, NC, RB, RG, AB, AG) RQ_FAST_M(D, NC, RB, RG, AB, AG, 0)
+#define RQ_FAST16(D, NC, RB, RG, AB, AG) RQ_FAST_M(D, NC, RB, RG, AB, AG, 1)
 
 const FastEntry kFast[] = {
     // anchor loop alone
@@ -760,12 +788,17 @@ const FastEntry kFast[] = {
     RQ_FAST(128, 3, 2, 64, 4, 64), RQ_FAST(128, 4, 2, 64, 4, 64), RQ_FAST(128, 5, 2, 64, 4, 64),
     RQ_FAST(128, 6, 2, 64, 4, 64), RQ_FAST(128, 7, 2, 64, 4, 64), RQ_FAST(128, 8, 2, 64, 4, 64),
     RQ_FAST(128, 3, 2, 32, 4, 32), RQ_FAST(128, 4, 2, 32, 4, 32),
+    // 16-bit metadata: anchor alone, Last-loop pairs, Next-loop chains
+    RQ_FAST16(128, 1, 2, 32, 4, 32), RQ_FAST16(128, 2, 2, 32, 4, 32),
+    RQ_FAST16(128, 2, 4, 32, 4, 32), RQ_FAST16(128, 2, 2, 16, 4, 32),
+    RQ_FAST16(128, 3, 2, 32, 4, 32), RQ_FAST16(128, 4, 2, 32, 4, 32),
+    RQ_FAST16(64, 1, 2, 32, 4, 32), RQ_FAST16(64, 2, 2, 32, 4, 32),
 };
 
 const FastEntry* find_fast(const DecodeParams& p, int D) {
   const int NC = p.ncomp;
   for (const FastEntry& f : kFast) {
-    if (f.D != D || f.NC != NC) continue;
+    if (f.D != D || f.NC != NC || f.M16 != p.k[0].meta16) continue;
     bool ok = p.k[NC - 1].bits == f.AB && p.k[NC - 1].group == f.AG;
     for (int c = 0; c + 1 < NC; ++c) ok = ok && p.k[c].bits == f.RB && p.k[c].group == f.RG;
     // a stage is exactly RPS records per component and side

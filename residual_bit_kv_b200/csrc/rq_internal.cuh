@@ -9,6 +9,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "librq.h"
 
@@ -35,6 +36,7 @@ struct Comp {
   int32_t bits;
   int32_t group;
   int32_t has_alpha;       // 0 for the anchor
+  int32_t meta16;          // 1: 16-bit metadata per group (scale byte | offset byte)
 };
 
 constexpr int kBlock = RQ_BLOCK_TOKENS;
@@ -55,9 +57,57 @@ __host__ __device__ inline uint32_t* rec_meta(unsigned char* rec, int D, int bit
                                               int i) {
   return reinterpret_cast<uint32_t*>(rec) + kBlock * (D * bits / 32) + i * (D / group);
 }
+// 16-bit metadata form: meta16 [32][D/group] after the codes.
+__host__ __device__ inline uint16_t* rec_meta16(unsigned char* rec, int D, int bits, int group,
+                                                int i) {
+  return reinterpret_cast<uint16_t*>(rec + kBlock * 4 * (D * bits / 32)) + i * (D / group);
+}
+// meta_bytes: 4 (fp16 scale | fp16 offset) or 2 (16-bit metadata).
 __host__ __device__ inline uint16_t* rec_alpha(unsigned char* rec, int D, int bits, int group,
-                                               int i) {
-  return reinterpret_cast<uint16_t*>(rec + kBlock * 4 * (D * bits / 32 + D / group)) + i;
+                                               int i, int meta_bytes = 4) {
+  return reinterpret_cast<uint16_t*>(rec + kBlock * (4 * (D * bits / 32) +
+                                                     meta_bytes * (D / group))) + i;
+}
+
+// 16-bit metadata: the scale byte is unsigned e5m3 with this exponent bias
+// (byte 8E + m -> (1 + m/8) 2^(E - bias), E = 0 -> 0).
+constexpr int kM16Bias = 18;
+
+// Scale byte nearest to s > 0 (ties to even m); below the range -> the
+// smallest positive value, above it -> the largest; s <= 0 or NaN -> 0.
+__host__ __device__ inline uint32_t m16_scale_byte(float s) {
+  if (!(s > 0.0f)) return 0u;
+  uint32_t b;
+  memcpy(&b, &s, sizeof(b));
+  int E = static_cast<int>((b >> 23) & 0xFFu);
+  if (E == 0xFF) return 0xFFu;
+  if (E == 0) return 0x08u;
+  uint32_t m = (b & 0x7FFFFFu) >> 20;
+  const uint32_t rem = b & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (m & 1u))) ++m;
+  if (m == 8u) {
+    m = 0u;
+    ++E;
+  }
+  const int Eb = E - 127 + kM16Bias;
+  if (Eb < 1) return 0x08u;
+  if (Eb > 31) return 0xFFu;
+  return (static_cast<uint32_t>(Eb) << 3) | m;
+}
+
+// Offset of a 16-bit metadata word given its scale: zq * s~ / 8 (exact).
+__host__ __device__ inline float m16_offset(uint32_t h, float s) {
+  return static_cast<float>(static_cast<int8_t>(static_cast<uint8_t>(h >> 8))) * s * 0.125f;
+}
+
+// Value of a scale byte (exact: the byte's fields go straight into the
+// exponent and the top mantissa bits).
+__host__ __device__ inline float m16_scale_value(uint32_t byte) {
+  const uint32_t Eb = (byte >> 3) & 31u;
+  const uint32_t bits = Eb == 0u ? 0u : (((Eb + 127u - kM16Bias) << 23) | ((byte & 7u) << 20));
+  float f;
+  memcpy(&f, &bits, sizeof(f));
+  return f;
 }
 
 struct QuantParams {

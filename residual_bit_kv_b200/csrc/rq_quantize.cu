@@ -118,19 +118,34 @@ __device__ __forceinline__ void deq_slice_t(const Comp& c, int64_t row, int64_t 
   uint32_t words[BITS];
 #pragma unroll
   for (int k = 0; k < BITS; ++k) words[k] = w[k];
-  const uint32_t* m = rec_meta(rec, D, BITS, c.group, i);
-  uint32_t mw0, mw1;
-  if (c.group >= 32) {
-    mw0 = m[(slice * 32) / c.group];
-    mw1 = mw0;
-  } else {  // group 16: two groups per lane
-    mw0 = m[slice * 2];
-    mw1 = m[slice * 2 + 1];
+  float2 s2, z2;
+  if (c.meta16) {
+    const uint16_t* m = rec_meta16(rec, D, BITS, c.group, i);
+    uint32_t h0, h1;
+    if (c.group >= 32) {
+      h0 = m[(slice * 32) / c.group];
+      h1 = h0;
+    } else {  // group 16: two groups per lane
+      h0 = m[slice * 2];
+      h1 = m[slice * 2 + 1];
+    }
+    s2 = make_float2(m16_scale_value(h0 & 0xFFu), m16_scale_value(h1 & 0xFFu));
+    z2 = make_float2(m16_offset(h0, s2.x), m16_offset(h1, s2.y));
+  } else {
+    const uint32_t* m = rec_meta(rec, D, BITS, c.group, i);
+    uint32_t mw0, mw1;
+    if (c.group >= 32) {
+      mw0 = m[(slice * 32) / c.group];
+      mw1 = mw0;
+    } else {  // group 16: two groups per lane
+      mw0 = m[slice * 2];
+      mw1 = m[slice * 2 + 1];
+    }
+    s2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 & 0xFFFFu))),
+                     __half2float(__ushort_as_half((unsigned short)(mw1 & 0xFFFFu))));
+    z2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 >> 16))),
+                     __half2float(__ushort_as_half((unsigned short)(mw1 >> 16))));
   }
-  const float2 s2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 & 0xFFFFu))),
-                                __half2float(__ushort_as_half((unsigned short)(mw1 & 0xFFFFu))));
-  const float2 z2 = make_float2(__half2float(__ushort_as_half((unsigned short)(mw0 >> 16))),
-                                __half2float(__ushort_as_half((unsigned short)(mw1 >> 16))));
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const uint32_t c0 = (words[slice_word<BITS>(k)] >> slice_shift<BITS>(k)) & QMAX;
@@ -157,7 +172,8 @@ __device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t ro
     deq_slice(comps[k], row, nblk, t, slice, D, d);
     const Comp& c = comps[k];
     const float a = bf16_bits_to_f32(
-        *rec_alpha(comp_record(c, row, nblk, t), D, c.bits, c.group, static_cast<int>(t % kBlock)));
+        *rec_alpha(comp_record(c, row, nblk, t), D, c.bits, c.group, static_cast<int>(t % kBlock),
+                   c.meta16 ? 2 : 4));
     const float2 a2 = make_float2(a, a);
 #pragma unroll
     for (int j = 0; j < 16; ++j) zr[j] = __ffma2_rn(a2, zr[j], d[j]);
@@ -181,7 +197,8 @@ __host__ __device__ constexpr uint32_t magic_pack_offset(int word) {
 // and 16-31 (.y) for g = 16, the whole slice (or several lanes) otherwise.
 template <int D, int BITS, int G>
 __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice, bool active,
-                                               uint32_t* codes_row, uint32_t* meta_row,
+                                               uint32_t* codes_row, unsigned char* meta_row,
+                                               bool m16,
                                                float2* levels = nullptr) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   constexpr int NG = G < 32 ? 2 : 1;        // group parts per lane
@@ -216,13 +233,34 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     mn = __fadd_rn(mn, 0.0f);   // a zero end of the range is +0
     mx = __fadd_rn(mx, 0.0f);
     const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
-    const __half sh = __float2half_rn(s);
-    const __half zh = __float2half_rn(mn);
-    st[gi] = __half2float(sh);
-    zt[gi] = __half2float(zh);
+    if (m16) {
+      // 16-bit metadata: scale byte nearest to max(s, |mn| / 15.875), offset
+      // byte = floor(8 mn / s~) clamped to int8, z~ = zq s~ / 8 (exact).
+      const float s1 = __fdiv_rn(fabsf(mn), 15.875f);
+      uint32_t sb = m16_scale_byte(s > s1 ? s : s1);
+      st[gi] = m16_scale_value(sb);
+      int zq = 0;
+      if (st[gi] > 0.0f) {
+        float tq = floorf(__fdiv_rn(__fmul_rn(8.0f, mn), st[gi]));
+        // the offset byte would saturate: one scale step up (always enough)
+        if ((tq < -128.0f || tq > 127.0f) && sb < 0xFFu) {
+          ++sb;
+          st[gi] = m16_scale_value(sb);
+          tq = floorf(__fdiv_rn(__fmul_rn(8.0f, mn), st[gi]));
+        }
+        zq = tq < -128.0f ? -128 : (tq > 127.0f ? 127 : static_cast<int>(tq));
+      }
+      zt[gi] = __fmul_rn(__fmul_rn(static_cast<float>(zq), st[gi]), 0.125f);
+      metaw[gi] = sb | ((static_cast<uint32_t>(zq) & 0xFFu) << 8);
+    } else {
+      const __half sh = __float2half_rn(s);
+      const __half zh = __float2half_rn(mn);
+      st[gi] = __half2float(sh);
+      zt[gi] = __half2float(zh);
+      metaw[gi] = static_cast<uint32_t>(__half_as_ushort(sh)) |
+                  (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
+    }
     inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
-    metaw[gi] = static_cast<uint32_t>(__half_as_ushort(sh)) |
-                (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
   }
   if constexpr (NG == 1) {
     st[1] = st[0];
@@ -261,11 +299,22 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     *reinterpret_cast<uint2*>(cw) = make_uint2(words[0], words[1]);
   }
   if constexpr (NG == 2) {
-    *reinterpret_cast<uint2*>(meta_row + slice * 2) = make_uint2(metaw[0], metaw[1]);
+    if (m16)
+      reinterpret_cast<uint32_t*>(meta_row)[slice] = metaw[0] | (metaw[1] << 16);
+    else
+      reinterpret_cast<uint2*>(meta_row)[slice] = make_uint2(metaw[0], metaw[1]);
   } else if constexpr (LPG == 1) {
-    meta_row[slice] = metaw[0];
+    if (m16)
+      reinterpret_cast<uint16_t*>(meta_row)[slice] = static_cast<uint16_t>(metaw[0]);
+    else
+      reinterpret_cast<uint32_t*>(meta_row)[slice] = metaw[0];
   } else {
-    if ((slice % LPG) == 0) meta_row[slice / LPG] = metaw[0];
+    if ((slice % LPG) == 0) {
+      if (m16)
+        reinterpret_cast<uint16_t*>(meta_row)[slice / LPG] = static_cast<uint16_t>(metaw[0]);
+      else
+        reinterpret_cast<uint32_t*>(meta_row)[slice / LPG] = metaw[0];
+    }
   }
 }
 
@@ -334,13 +383,17 @@ __global__ void __launch_bounds__(kQuantThreads)
       }
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
-        *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock)) =
+        *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock),
+                   p.dst.meta16 ? 2 : 4) =
             __bfloat16_as_ushort(ab);
     }
     unsigned char* rec = comp_record(p.dst, bhi, p.nblk, t);
     const int i = static_cast<int>(t % kBlock);
-    quantize_store<D, BITS, G>(v, slice, active, rec_codes(rec, D, BITS, i),
-                               rec_meta(rec, D, BITS, G, i));
+    unsigned char* mrow = p.dst.meta16
+                              ? reinterpret_cast<unsigned char*>(rec_meta16(rec, D, BITS, G, i))
+                              : reinterpret_cast<unsigned char*>(rec_meta(rec, D, BITS, G, i));
+    quantize_store<D, BITS, G>(v, slice, active, rec_codes(rec, D, BITS, i), mrow,
+                               p.dst.meta16 != 0);
   }
 }
 
@@ -353,19 +406,22 @@ __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_
   unsigned char* rec = comp_record(c, row, nblk, t);
   const int i = static_cast<int>(t % kBlock);
   uint32_t* cw = rec_codes(rec, D, c.bits, i);
-  uint32_t* mw = rec_meta(rec, D, c.bits, c.group, i);
+  unsigned char* mw =
+      c.meta16 ? reinterpret_cast<unsigned char*>(rec_meta16(rec, D, c.bits, c.group, i))
+               : reinterpret_cast<unsigned char*>(rec_meta(rec, D, c.bits, c.group, i));
+  const bool m16 = c.meta16 != 0;
   const int key = c.bits * 1000 + c.group;
   switch (key) {
-    case 2016: quantize_store<D, 2, 16>(v, slice, active, cw, mw, levels); break;
-    case 2032: quantize_store<D, 2, 32>(v, slice, active, cw, mw, levels); break;
-    case 2064: quantize_store<D, 2, 64>(v, slice, active, cw, mw, levels); break;
-    case 4016: quantize_store<D, 4, 16>(v, slice, active, cw, mw, levels); break;
-    case 4032: quantize_store<D, 4, 32>(v, slice, active, cw, mw, levels); break;
-    case 4064: quantize_store<D, 4, 64>(v, slice, active, cw, mw, levels); break;
+    case 2016: quantize_store<D, 2, 16>(v, slice, active, cw, mw, m16, levels); break;
+    case 2032: quantize_store<D, 2, 32>(v, slice, active, cw, mw, m16, levels); break;
+    case 2064: quantize_store<D, 2, 64>(v, slice, active, cw, mw, m16, levels); break;
+    case 4016: quantize_store<D, 4, 16>(v, slice, active, cw, mw, m16, levels); break;
+    case 4032: quantize_store<D, 4, 32>(v, slice, active, cw, mw, m16, levels); break;
+    case 4064: quantize_store<D, 4, 64>(v, slice, active, cw, mw, m16, levels); break;
     default:
       if constexpr (D >= 128) {
-        if (key == 2128) quantize_store<D, 2, 128>(v, slice, active, cw, mw, levels);
-        else if (key == 4128) quantize_store<D, 4, 128>(v, slice, active, cw, mw, levels);
+        if (key == 2128) quantize_store<D, 2, 128>(v, slice, active, cw, mw, m16, levels);
+        else if (key == 4128) quantize_store<D, 4, 128>(v, slice, active, cw, mw, m16, levels);
       }
       break;
   }
@@ -412,7 +468,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
         *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
-                   static_cast<int>(t % kBlock)) = __bfloat16_as_ushort(ab);
+                   static_cast<int>(t % kBlock), c.meta16 ? 2 : 4) = __bfloat16_as_ushort(ab);
       float2 lv[16];
       quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, lv);
       if (p.chained) {

@@ -19,6 +19,7 @@ RQ_POLICY_NEXT_LOOP = 1
 RQ_POLICY_FIRST_LOOP = 2
 RQ_POLICY_PREVIOUS_LOOP = 3
 RQ_FLAG_UNIT_ALPHA = 1
+RQ_FLAG_META16 = 2
 
 RQ_OK = 0
 RQ_ERR_INVALID_ARG = 1

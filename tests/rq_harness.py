@@ -28,10 +28,12 @@ def policy_code(policy: str) -> int:
 
 
 def layout_of(w: synth.Workload, policy: str = "last", layers: Optional[int] = None,
-              max_tokens: Optional[int] = None, unit_alpha: bool = False) -> L.rq_layout:
+              max_tokens: Optional[int] = None, unit_alpha: bool = False,
+              meta16: bool = False) -> L.rq_layout:
+    flags = (L.RQ_FLAG_UNIT_ALPHA if unit_alpha else 0) | (L.RQ_FLAG_META16 if meta16 else 0)
     return L.make_layout(layers or w.layers, w.loops, w.batch, w.heads, w.head_dim,
                          max_tokens or (w.tokens + 1), w.bits, w.group, policy_code(policy),
-                         L.RQ_FLAG_UNIT_ALPHA if unit_alpha else 0)
+                         flags)
 
 
 def append_order(w: synth.Workload, policy: str) -> List[int]:
@@ -50,13 +52,14 @@ class GpuCache:
     vbuf: torch.Tensor
     inputs: Dict  # (layer, side, loop) -> bf16 [B, H, T, D] cuda tensor (if kept)
     unit_alpha: bool = False
+    meta16: bool = False
 
 
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
                     keep_inputs: bool = True, tokens: Optional[int] = None,
                     max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
                     fused: bool = False, unit_alpha: bool = False,
-                    gen_device: str = "cuda") -> GpuCache:
+                    gen_device: str = "cuda", meta16: bool = False) -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
     the C ABI in the order the policy requires (fused: every loop and both
     sides of a chunk in one rq_quantize_append_loops call).  append_chunks
@@ -64,7 +67,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
     single tokens).  gen_device "cpu" draws the inputs on the host and copies
     them over (no generator kernels on the GPU)."""
     T = w.tokens if tokens is None else tokens
-    lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens, unit_alpha=unit_alpha)
+    lay = layout_of(w, policy, layers=max(layers) + 1, max_tokens=max_tokens, unit_alpha=unit_alpha,
+                    meta16=meta16)
     nbytes = L.rq_cache_bytes(lay)
     assert nbytes > 0
     kbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
@@ -107,7 +111,7 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     inputs[(layer, side, loop)] = x
             del xs
     torch.cuda.synchronize()
-    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha)
+    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha, meta16)
 
 
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
@@ -133,18 +137,21 @@ def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
     allrec = buf[base: base + w.batch * w.heads * nb * rb].view(w.batch * w.heads, nb * rb)
     recs = allrec[rows].cpu().numpy().reshape(len(rows) * nb, rb)
     shp = (len(bsel), len(hsel), ts)
+    mb = 2 if gc.meta16 else 4
     codes = recs[:, : blk * W * 4].copy().view(np.uint32).reshape(*shp, W)
-    meta = recs[:, blk * W * 4: blk * (W + G) * 4].copy().view(np.uint32).reshape(*shp, G)
+    meta = recs[:, blk * W * 4: blk * (W * 4 + G * mb)].copy().view(
+        np.uint16 if gc.meta16 else np.uint32).reshape(*shp, G)
     out = {"codes": codes, "meta": meta, "alpha": None}
     if loop != oracle.anchor_loop(w.loops, gc.policy):
-        a0 = blk * (W + G) * 4
+        a0 = blk * (W * 4 + G * mb)
         out["alpha"] = recs[:, a0: a0 + blk * 2].copy().view(np.uint16).reshape(*shp)
     return out
 
 
 def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
                   hsel: Sequence[int], t0: int, t1: int, policy: str = "last",
-                  x_loops: Optional[List[np.ndarray]] = None, unit_alpha: bool = False):
+                  x_loops: Optional[List[np.ndarray]] = None, unit_alpha: bool = False,
+                  meta16: bool = False):
     """Oracle encodings of the selected rows.  Returns (encs, x) where
     x is uint16 [L, nb*nh*(t1-t0), D]."""
     if x_loops is None:
@@ -152,7 +159,7 @@ def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
         x_loops = [synth.bits_of(synth.kv(w, layer, side, loop, bsel, hsel, t0, t1, "cpu", cs))
                    .reshape(-1, w.head_dim) for loop in range(w.loops)]
     x = np.stack(x_loops)
-    return oracle.encode_side(x, w.bits, w.group, policy, unit_alpha), x
+    return oracle.encode_side(x, w.bits, w.group, policy, unit_alpha, meta16), x
 
 
 def assert_component_equal(gpu: Dict[str, np.ndarray], enc: Dict[str, np.ndarray], shape,
@@ -202,7 +209,7 @@ def gpu_decode(gc: GpuCache, layer: int, loop: int, seq_lens: Sequence[int], max
 def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
                   hsel: Sequence[int], seq_lens: Sequence[int], policy: str = "last",
                   inputs: Optional[Dict] = None, scale: Optional[float] = None,
-                  unit_alpha: bool = False) -> np.ndarray:
+                  unit_alpha: bool = False, meta16: bool = False) -> np.ndarray:
     """fp64 oracle decode for the selected (b, h): [len(bsel), len(hsel), D]."""
     T = max(int(seq_lens[b]) for b in bsel)
     D = w.head_dim
@@ -213,7 +220,7 @@ def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
         if inputs is not None:
             xl = [synth.bits_of(inputs[(layer, side, l)][list(bsel)][:, list(hsel), :T].cpu())
                   .reshape(-1, D) for l in range(w.loops)]
-        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl, unit_alpha)
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl, unit_alpha, meta16)
         rec[side] = oracle.reconstruct(encs, loop, w.bits, w.group, policy).reshape(
             len(bsel), len(hsel), T, D)
     q = synth.bits_of(synth.query(w, layer, loop)).reshape(w.batch, w.heads, D)

@@ -58,7 +58,8 @@ def test_layout_validation(L):
                 L.RQ_POLICY_PREVIOUS_LOOP):
         assert L.rq_layout_validate(_lay(L, policy=pol)) == L.RQ_OK
         assert L.rq_layout_validate(_lay(L, policy=pol, flags=L.RQ_FLAG_UNIT_ALPHA)) == L.RQ_OK
-    assert L.rq_layout_validate(_lay(L, flags=2)) == L.RQ_ERR_INVALID_ARG
+        assert L.rq_layout_validate(_lay(L, policy=pol, flags=L.RQ_FLAG_META16)) == L.RQ_OK
+    assert L.rq_layout_validate(_lay(L, flags=4)) == L.RQ_ERR_INVALID_ARG
     assert L.rq_cache_bytes(_lay(L, batch=0)) == 0
 
 
@@ -96,6 +97,36 @@ def test_cache_bytes_equal_effective_bits(L, bits, group):
     assert want <= got <= want + 256 * 3 * len(bits)     # only alignment padding on top
     assert L.rq_cache_bytes(_lay(L, num_layers=3, num_loops=len(bits), bits=bits, group=group,
                                  max_tokens=T)) == 3 * got
+
+
+def _golden(name):
+    vals = {}
+    with open(os.path.join(ROOT, "tests", "golden", name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = (x.strip() for x in line.split("="))
+                vals[k] = float(v)
+    return vals
+
+
+@pytest.mark.parametrize("name,bits,group", [
+    ("int2_g32", (2, 2, 2, 2), (32,) * 4), ("int2_g16", (2, 2, 2, 2), (16,) * 4),
+    ("int24_g32", (2, 2, 2, 4), (32,) * 4), ("int24_g16", (2, 2, 2, 4), (16, 16, 16, 32))])
+def test_meta16_cache_bytes_reproduce_the_pages(L, name, bits, group):
+    """With RQ_FLAG_META16 the library's own byte count of a layer gives the
+    residual b_eff the pages print for Ouro-1.4B (L = 4, D = 128):
+    2.6 / 3.1 / 3.1 / 3.5 bits per element [RQ App. A.3, §5.1], and 19.3% of
+    BF16 for INT2/4 at g = 32 [RQ-summary]."""
+    g = _golden("pages_storage.txt")
+    T = 4096
+    lay = _lay(L, num_loops=4, bits=bits, group=group, max_tokens=T, flags=L.RQ_FLAG_META16)
+    elems = 8 * 16 * T * 128 * 4          # batch 8, 16 heads, T tokens, D 128, 4 loops
+    beff = L.rq_layer_bytes(lay) * 8 / elems
+    assert beff == pytest.approx(oracle.effective_bits(bits, group, 128, 16, True), abs=1e-3)
+    assert round(beff, 1) == g[f"beff_residual_{name}"]
+    if name == "int24_g32":
+        assert round(beff / 16, 3) == g["storage_frac_int24_residual_g32"]
 
 
 def test_host_checks_reject_before_launch(L):
