@@ -72,7 +72,7 @@
 extern "C" {
 #endif
 
-#define RQ_ABI_VERSION 1
+#define RQ_ABI_VERSION 2
 #define RQ_MAX_LOOPS 32
 #define RQ_BLOCK_TOKENS 32
 
@@ -137,6 +137,8 @@ typedef struct rq_cache {
   int64_t token_stride;              /* max_tokens rounded up to 64 */
   uint64_t comp_off[RQ_MAX_LOOPS];   /* first record of loop r (256-B aligned) */
   uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 32-token record of loop r */
+  const float* k_means;              /* fixed means (rq_cache_set_means) or NULL */
+  const float* v_means;
 } rq_cache;
 
 /* ABI version of the loaded library (RQ_ABI_VERSION at build time). */
@@ -158,6 +160,18 @@ uint64_t rq_layer_bytes(const rq_layout* layout);
 
 /* Binds device buffers of rq_cache_bytes() each (256-byte aligned) to `out`.
  * The buffers need no initialisation.  Host-only, launches nothing. */
+/* Fixed means of the residual loops [RQ App. G.2]: the reconstruction of a
+ * residual loop r is Z^_r = alpha~_r R + D(c_r) + mu_r, and the encoder
+ * removes mu_r before the LS coefficient (zc = Z_r - mu_r, alpha =
+ * <zc, R>/<R, R>, codes of zc - alpha~ R).  k_means, v_means: device fp32
+ * [num_layers][num_loops][kv_heads][head_dim] in the rotated domain (the
+ * anchor loop's rows are not read), 16-byte aligned, or NULL for no means
+ * (the state after rq_cache_bind).  The cache keeps the pointers; the caller
+ * keeps the buffers alive and unchanged while appends and decodes that use
+ * them are in flight.  Appends and decodes of one cache must see the same
+ * means. */
+rq_status rq_cache_set_means(rq_cache* cache, const float* k_means, const float* v_means);
+
 rq_status rq_cache_bind(const rq_layout* layout, void* k_base, void* v_base,
                         rq_cache* out);
 

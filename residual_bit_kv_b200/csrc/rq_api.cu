@@ -154,6 +154,12 @@ Comp comp_of(const rq_cache* c, int layer, int kv, int r) {
   k.group = c->layout.group[r];
   k.has_alpha = (r != anchor_of(&c->layout)) ? 1 : 0;
   k.meta16 = (c->layout.flags & RQ_FLAG_META16) ? 1 : 0;
+  const float* means = kv ? c->v_means : c->k_means;
+  const rq_layout& l = c->layout;
+  k.mean = (means != nullptr && k.has_alpha)
+               ? means + (static_cast<int64_t>(layer) * l.num_loops + r) * l.kv_heads * l.head_dim
+               : nullptr;
+  k.heads = l.kv_heads;
   return k;
 }
 
@@ -257,6 +263,15 @@ rq_status rq_cache_bind(const rq_layout* l, void* k_base, void* v_base, rq_cache
   out->v_base = v_base;
   out->layer_bytes = layout_offsets(l, out->comp_off, out->rec_bytes);
   out->token_stride = token_stride_of(l);
+  return RQ_OK;
+}
+
+rq_status rq_cache_set_means(rq_cache* c, const float* k_means, const float* v_means) {
+  if (c == nullptr) return RQ_ERR_INVALID_ARG;
+  if ((k_means != nullptr && !aligned(k_means, 16)) || (v_means != nullptr && !aligned(v_means, 16)))
+    return RQ_ERR_INVALID_ARG;
+  c->k_means = k_means;
+  c->v_means = v_means;
   return RQ_OK;
 }
 

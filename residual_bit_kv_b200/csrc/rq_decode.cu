@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   __shared__ float svec[D];
   __shared__ float sred[4];
   __shared__ int s_abort;
+  __shared__ float s_qmu[RQ_MAX_LOOPS][D / 32];   // q'.mu_c per slice (fixed means)
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
@@ -233,6 +234,22 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
   }
 
+  // Fixed means [RQ App. G.2]: q'.mu_c over each 32-channel slice.
+  const int head = bhi % p.heads;
+  {
+    const float sc = p.rot_scale * p.scale_log2;
+    for (int e = t; e < p.ncomp * G::P; e += kDecodeThreads) {
+      const int c = e / G::P, s = e % G::P;
+      float sum = 0.0f;
+      if (p.k[c].mean != nullptr) {
+        const float* mu = p.k[c].mean + static_cast<size_t>(head) * D + s * 32;
+        for (int ch = 0; ch < 32; ++ch) sum = fmaf(svec[s * 32 + ch] * sc, mu[ch], sum);
+      }
+      s_qmu[c][s] = sum;
+    }
+  }
+  __syncthreads();
+
   float m = kNegInf, l = 0.0f;
   float acc[32];
 #pragma unroll
@@ -265,6 +282,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                             ? comp_dot<4>(cw, mr, m16, slice, log2_pow2(p.k[c].group), q, qsa, qsb)
                             : comp_dot<2>(cw, mr, m16, slice, log2_pow2(p.k[c].group), q, qsa, qsb);
         part = fmaf(kappa, d, part);
+        if (p.k[c].mean != nullptr) part = fmaf(kappa, s_qmu[c][slice], part);
         if (c + 1 < p.ncomp)
           kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[0][c])[jl]);
       }
@@ -305,6 +323,11 @@ __global__ void __launch_bounds__(kDecodeThreads)
           comp_acc<4>(cw, mr, m16, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
         else
           comp_acc<2>(cw, mr, m16, slice, log2_pow2(p.v[c].group), kappa, acc, cst0, cst1);
+        if (p.v[c].mean != nullptr) {
+          const float* mu = p.v[c].mean + static_cast<size_t>(head) * D + slice * 32;
+#pragma unroll
+          for (int ch = 0; ch < 32; ++ch) acc[ch] = fmaf(kappa, __ldg(mu + ch), acc[ch]);
+        }
         if (c + 1 < p.ncomp)
           kappa *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + map.alpha[1][c])[jl]);
       }

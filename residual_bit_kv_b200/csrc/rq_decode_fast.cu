@@ -52,9 +52,10 @@ constexpr size_t kMergeScratch = 3 * 1024 * sizeof(float);   // split headers, u
 // Compile-time layout of one stage: for side K then V, component c occupies
 // RPS = 2 consecutive records (64 tokens, one copy); a record is
 // [codes[32][wpr] | meta[32][gpr] | alpha[32]].
-template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_, int M16_ = 0>
+template <int D_, int NC_, int RB_, int RG_, int AB_, int AG_, int M16_ = 0, int MU_ = 0>
 struct Spec {
-  static constexpr int D = D_, NC = NC_, RPS = 2, TC = kBlock * RPS, M16 = M16_;
+  // M16: 16-bit metadata per group; MU: the residual loops carry fixed means [RQ App. G.2]
+  static constexpr int D = D_, NC = NC_, RPS = 2, TC = kBlock * RPS, M16 = M16_, MU = MU_;
   __host__ __device__ static constexpr int bits(int c) { return c == NC_ - 1 ? AB_ : RB_; }
   __host__ __device__ static constexpr int group(int c) { return c == NC_ - 1 ? AG_ : RG_; }
   __host__ __device__ static constexpr bool has_alpha(int c) { return c != NC_ - 1; }
@@ -184,6 +185,7 @@ __device__ __forceinline__ float kdot(const unsigned char* rec, int jl, int slic
 struct VAcc {
   float2 acc[16];
   float cst[3];
+  float mw[8];   // fixed means: sum of p_t * kappa_c per residual component (MU layouts)
 };
 
 constexpr int kPosBias = 109;                        // weights w * 2^(109 - p), p <= 14
@@ -265,19 +267,21 @@ __device__ __forceinline__ void vacc(const unsigned char* rec, int jl, int slice
 }
 
 // Components of a chain, unrolled at compile time: [own residual, ..., anchor].
-// Components of a chain, unrolled at compile time: [own residual, ..., anchor].
 // REC is the stage record (compile-time), jl the token inside it.
 template <class SP, int REC, int C = 0>
 __device__ __forceinline__ void score_comps(const unsigned char* st, int rl, int jl, int slice,
-                                            const QLimbs& ql, float& part, float& kap) {
+                                            const QLimbs& ql, const float* qmu, float& part,
+                                            float& kap) {
   if constexpr (C < SP::NC) {
     using RG = RecGeom<SP::D, SP::bits(C), SP::group(C), SP::M16>;
     const unsigned char* rec = st + SP::comp_off(0, C) + (REC + rl) * SP::rec_bytes(C);
     const float d = kdot<SP::D, SP::bits(C), SP::group(C), SP::M16>(rec, jl, slice, ql);
     part = fmaf(kap, d, part);
+    // the mean's share: kappa * (q~ . mu) over this lane's channels
+    if constexpr (SP::MU && SP::has_alpha(C)) part = fmaf(kap, qmu[C], part);
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
-    score_comps<SP, REC, C + 1>(st, rl, jl, slice, ql, part, kap);
+    score_comps<SP, REC, C + 1>(st, rl, jl, slice, ql, qmu, part, kap);
   }
 }
 
@@ -288,6 +292,7 @@ __device__ __forceinline__ void value_comps(const unsigned char* st, int rl, int
     using RG = RecGeom<SP::D, SP::bits(C), SP::group(C), SP::M16>;
     const unsigned char* rec = st + SP::comp_off(1, C) + (REC + rl) * SP::rec_bytes(C);
     vacc<SP::D, SP::bits(C), SP::group(C), SP::M16>(rec, jl, slice, kap, va);
+    if constexpr (SP::MU && SP::has_alpha(C)) va.mw[C] += kap;
     if constexpr (SP::has_alpha(C))
       kap *= bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(rec + RG::ALPHA)[jl]);
     value_comps<SP, REC, C + 1>(st, rl, jl, slice, kap, va);
@@ -300,15 +305,15 @@ __device__ __forceinline__ void value_comps(const unsigned char* st, int rl, int
 // before TC tokens (nt < TC); full chunks skip the per-token tests.
 template <class SP, int TT, int TPC, int P, bool MASK, int TTI = 0>
 __device__ __forceinline__ void chunk_scores(const unsigned char* st, int jr, int rl, int jl,
-                                             int slice, const QLimbs& ql, float sigma, int nt,
-                                             float (&sc)[TT]) {
+                                             int slice, const QLimbs& ql, const float* qmu,
+                                             float sigma, int nt, float (&sc)[TT]) {
   if constexpr (TTI < TT) {
     float part = 0.0f, kap = 1.0f;
-    score_comps<SP, TTI * TPC / kBlock>(st, rl, jl, slice, ql, part, kap);
+    score_comps<SP, TTI * TPC / kBlock>(st, rl, jl, slice, ql, qmu, part, kap);
 #pragma unroll
     for (int off = P / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     sc[TTI] = (!MASK || TTI * TPC + jr < nt) ? part * sigma : kNegInf;
-    chunk_scores<SP, TT, TPC, P, MASK, TTI + 1>(st, jr, rl, jl, slice, ql, sigma, nt, sc);
+    chunk_scores<SP, TT, TPC, P, MASK, TTI + 1>(st, jr, rl, jl, slice, ql, qmu, sigma, nt, sc);
   }
 }
 
@@ -325,6 +330,7 @@ __device__ __forceinline__ void chunk_values(const unsigned char* st, int rl, in
   }
 }
 
+template <int MU = 0, int NC = 1>
 __device__ __forceinline__ void rescale(VAcc& va, float f) {
   const float2 ff = make_float2(f, f);
 #pragma unroll
@@ -332,6 +338,10 @@ __device__ __forceinline__ void rescale(VAcc& va, float f) {
   va.cst[0] *= f;
   va.cst[1] *= f;
   va.cst[2] *= f;
+  if constexpr (MU) {
+#pragma unroll
+    for (int c = 0; c + 1 < NC; ++c) va.mw[c] *= f;
+  }
 }
 
 // Final per-channel values: undo the 2^-40 code scale and add the z~ terms.
@@ -497,10 +507,32 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
     }
   ql.sq[0] = s_sq[slice * 2];
   ql.sq[1] = s_sq[slice * 2 + 1];
+  // Fixed means [RQ App. G.2]: q~ . mu_c over this lane's 32 channels, per
+  // residual component of the K chain (one warp per slice).
+  float qmu[SP::NC];
+#pragma unroll
+  for (int c = 0; c < SP::NC; ++c) qmu[c] = 0.0f;
+  if constexpr (SP::MU) {
+    __shared__ float s_qmu[SP::NC][kCWarps];
+    const int head = bhi % p.k[0].heads;
+#pragma unroll
+    for (int c = 0; c + 1 < SP::NC; ++c) {
+      const float* mu = p.k[c].mean;
+      float v = (mu != nullptr && t < D) ? (qv * (1.0f / sigma)) * mu[head * D + t] : 0.0f;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) s_qmu[c][warp] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c + 1 < SP::NC; ++c) qmu[c] = s_qmu[c][slice];
+  }
   VAcc va;
 #pragma unroll
   for (int i = 0; i < 16; ++i) va.acc[i] = make_float2(0.0f, 0.0f);
   va.cst[0] = va.cst[1] = va.cst[2] = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) va.mw[c] = 0.0f;
   float m = kNegInf, l = 0.0f;
 
   // This thread's tokens: jr inside a CTA pass of TPC tokens.
@@ -510,14 +542,14 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   auto chunk = [&](const unsigned char* st, auto mask_tag, int nt) {
     constexpr bool MASK = decltype(mask_tag)::value;
     float sc[TT];
-    chunk_scores<SP, TT, TPC, P, MASK>(st, jr, rl, jl, slice, ql, sigma, nt, sc);
+    chunk_scores<SP, TT, TPC, P, MASK>(st, jr, rl, jl, slice, ql, qmu, sigma, nt, sc);
     float mc = sc[0];
 #pragma unroll
     for (int tt = 1; tt < TT; ++tt) mc = fmaxf(mc, sc[tt]);
     if (mc > m) {
       const float f = (m == kNegInf) ? 0.0f : fast_exp2(m - mc);
       l *= f;
-      rescale(va, f);
+      rescale<SP::MU, SP::NC>(va, f);
       m = mc;
     }
     chunk_values<SP, TT, TPC, MASK>(st, rl, jl, slice, sc, m, l, va);
@@ -554,6 +586,24 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   float acc[32];
   uint32_t range_err = 0u;
   finish_values(va, acc, range_err);
+  if constexpr (SP::MU) {
+    // sum_t p_t kappa_c mu_c over this lane's channels
+    const int head = bhi % p.v[0].heads;
+#pragma unroll
+    for (int c = 0; c + 1 < SP::NC; ++c) {
+      const float* mu = p.v[c].mean;
+      if (mu == nullptr) continue;
+      const float4* src = reinterpret_cast<const float4*>(mu + head * D + slice * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 e = src[i];
+        acc[4 * i] = fmaf(va.mw[c], e.x, acc[4 * i]);
+        acc[4 * i + 1] = fmaf(va.mw[c], e.y, acc[4 * i + 1]);
+        acc[4 * i + 2] = fmaf(va.mw[c], e.z, acc[4 * i + 2]);
+        acc[4 * i + 3] = fmaf(va.mw[c], e.w, acc[4 * i + 3]);
+      }
+    }
+  }
   __syncthreads();   // every warp has left the loop: s_abort is settled
   const bool aborted = s_abort != 0;
   if (range_err && !aborted) atomicOr(p.err, kErrRange);
@@ -748,7 +798,7 @@ size_t dyn_bytes(int stages) {
 
 // Host-side description of one compiled layout.
 struct FastEntry {
-  int D, NC, RB, RG, AB, AG, M16;
+  int D, NC, RB, RG, AB, AG, M16, MU;
   uint32_t stage_bytes;
   int chunk;
   cudaError_t (*launch)(const DecodeParams&, cudaStream_t);
@@ -769,13 +819,14 @@ cudaError_t occ_spec(int stages, int* occ) {
   return prep(decode_fast_kernel<SP>, dyn_bytes<SP>(stages), occ, kCThreads);
 }
 
-#define RQ_FAST_M(D, NC, RB, RG, AB, AG, M)                                                    \
-  FastEntry{D,  NC, RB, RG, AB, AG, M, Spec<D, NC, RB, RG, AB, AG, M>::stage_bytes(),        \
-            Spec<D, NC, RB, RG, AB, AG, M>::TC,                                              \
-            &launch_spec<Spec<D, NC, RB, RG, AB, AG, M>>,                                    \
-            &occ_spec<Spec<D, NC, RB, RG, AB, AG, M>>}
-#define RQ_FAST(D, NC, RB, RG, AB, AG) RQ_FAST_M(D, NC, RB, RG, AB, AG, 0)
-#define RQ_FAST16(D, NC, RB, RG, AB, AG) RQ_FAST_M(D, NC, RB, RG, AB, AG, 1)
+#define RQ_FAST_X(D, NC, RB, RG, AB, AG, M, MU)                                                \
+  FastEntry{D,  NC, RB, RG, AB, AG, M, MU, Spec<D, NC, RB, RG, AB, AG, M, MU>::stage_bytes(),  \
+            Spec<D, NC, RB, RG, AB, AG, M, MU>::TC,                                          \
+            &launch_spec<Spec<D, NC, RB, RG, AB, AG, M, MU>>,                                \
+            &occ_spec<Spec<D, NC, RB, RG, AB, AG, M, MU>>}
+#define RQ_FAST(D, NC, RB, RG, AB, AG) RQ_FAST_X(D, NC, RB, RG, AB, AG, 0, 0)
+#define RQ_FAST16(D, NC, RB, RG, AB, AG) RQ_FAST_X(D, NC, RB, RG, AB, AG, 1, 0)
+#define RQ_FAST_MU(D, NC, RB, RG, AB, AG) RQ_FAST_X(D, NC, RB, RG, AB, AG, 0, 1)
 
 const FastEntry kFast[] = {
     // anchor loop alone
@@ -793,12 +844,17 @@ const FastEntry kFast[] = {
     RQ_FAST16(128, 2, 4, 32, 4, 32), RQ_FAST16(128, 2, 2, 16, 4, 32),
     RQ_FAST16(128, 3, 2, 32, 4, 32), RQ_FAST16(128, 4, 2, 32, 4, 32),
     RQ_FAST16(64, 1, 2, 32, 4, 32), RQ_FAST16(64, 2, 2, 32, 4, 32),
+    // residual loops with fixed means: Last-loop pairs and Next-loop chains
+    RQ_FAST_MU(128, 2, 2, 32, 4, 32), RQ_FAST_MU(128, 2, 4, 32, 4, 32),
+    RQ_FAST_MU(128, 3, 2, 32, 4, 32), RQ_FAST_MU(128, 4, 2, 32, 4, 32),
+    RQ_FAST_MU(64, 2, 2, 32, 4, 32),
 };
 
 const FastEntry* find_fast(const DecodeParams& p, int D) {
   const int NC = p.ncomp;
   for (const FastEntry& f : kFast) {
-    if (f.D != D || f.NC != NC || f.M16 != p.k[0].meta16) continue;
+    const int mu = (p.k[0].mean != nullptr || p.v[0].mean != nullptr) ? 1 : 0;
+    if (f.D != D || f.NC != NC || f.M16 != p.k[0].meta16 || f.MU != mu) continue;
     bool ok = p.k[NC - 1].bits == f.AB && p.k[NC - 1].group == f.AG;
     for (int c = 0; c + 1 < NC; ++c) ok = ok && p.k[c].bits == f.RB && p.k[c].group == f.RG;
     // a stage is exactly RPS records per component and side

@@ -37,6 +37,10 @@ struct Comp {
   int32_t group;
   int32_t has_alpha;       // 0 for the anchor
   int32_t meta16;          // 1: 16-bit metadata per group (scale byte | offset byte)
+  // Fixed mean of this residual loop [RQ App. G.2]: fp32 [kv_heads][D] in
+  // the rotated domain (row b*H + h uses row h), or nullptr.
+  const float* mean;
+  int32_t heads;
 };
 
 constexpr int kBlock = RQ_BLOCK_TOKENS;

@@ -162,8 +162,46 @@ __device__ __forceinline__ void deq_slice(const Comp& c, int64_t row, int64_t nb
     deq_slice_t<2>(c, row, nblk, t, slice, D, o);
 }
 
+// This lane's 32 channels of a component's fixed mean (row `row` uses the
+// mean of head row % heads), as pairs (channel k, channel k + 16).
+__device__ __forceinline__ void mean_slice(const Comp& c, int64_t row, int slice, int D,
+                                           float2 (&m)[16]) {
+  const float4* src =
+      reinterpret_cast<const float4*>(c.mean + (row % c.heads) * D + slice * 32);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 q = src[i];
+    const float e[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ch = 4 * i + j;
+      if (ch < 16)
+        m[ch].x = e[j];
+      else
+        m[ch - 16].y = e[j];
+    }
+  }
+}
+
+// v <- v - mean (the encoder's mean removal), v <- v + mean (reconstruction).
+__device__ __forceinline__ void sub_mean(const Comp& c, int64_t row, int slice, int D,
+                                         float2 (&v)[16]) {
+  float2 m[16];
+  mean_slice(c, row, slice, D, m);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fadd2_rn(v[k], make_float2(-m[k].x, -m[k].y));
+}
+__device__ __forceinline__ void add_mean(const Comp& c, int64_t row, int slice, int D,
+                                         float2 (&v)[16]) {
+  float2 m[16];
+  mean_slice(c, row, slice, D, m);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fadd2_rn(v[k], m[k]);
+}
+
 // Rotated reconstruction of a chain [0 .. n-1] (anchor last) at token t of
-// row `row`: Z = deq(anchor); for k = n-2 .. 0: Z = fma(alpha~_k, Z, deq_k).
+// row `row`: Z = deq(anchor); for k = n-2 .. 0: Z = fma(alpha~_k, Z, deq_k)
+// (+ mu_k when the loop has a fixed mean).
 __device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t row, int64_t nblk,
                                             int64_t t, int slice, int D, float2 (&zr)[16]) {
   deq_slice(comps[n - 1], row, nblk, t, slice, D, zr);
@@ -177,6 +215,7 @@ __device__ __forceinline__ void chain_slice(const Comp* comps, int n, int64_t ro
     const float2 a2 = make_float2(a, a);
 #pragma unroll
     for (int j = 0; j < 16; ++j) zr[j] = __ffma2_rn(a2, zr[j], d[j]);
+    if (c.mean != nullptr) add_mean(c, row, slice, D, zr);
   }
 }
 
@@ -191,6 +230,38 @@ __host__ __device__ constexpr uint32_t magic_pack_offset(int word) {
   return o;
 }
 
+// Codes of one lane's 32 values packed into BITS words: u = (x - z~) * (1/s~)
+// (clamped to [0, 2^b - 1] when CLAMP); u + 1.5 * 2^23 rounds it to the
+// nearest integer (ties to even), held in the low mantissa bits of a float
+// whose bit pattern is kRoundMagicBits + code; packing adds that pattern
+// shifted into place (the magic offsets are subtracted up front), one
+// integer multiply-add per code.  LEVELS: `levels` receives fma(s~, code, z~).
+template <int BITS, bool CLAMP, bool LEVELS>
+__device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, float2 iv,
+                                           const float (&st)[2], const float (&zt)[2],
+                                           uint32_t (&words)[BITS], float2* levels) {
+  constexpr uint32_t QMAX = (1u << BITS) - 1u;
+  const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) words[i] = 0u - magic_pack_offset<BITS>(i);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float2 u = __fmul2_rn(__fadd2_rn(v[k], nz), iv);
+    if constexpr (CLAMP) {
+      u.x = fminf(fmaxf(u.x, 0.0f), static_cast<float>(QMAX));
+      u.y = fminf(fmaxf(u.y, 0.0f), static_cast<float>(QMAX));
+    }
+    const float2 r = __fadd2_rn(u, mg);
+    const uint32_t b0 = __float_as_uint(r.x), b1 = __float_as_uint(r.y);
+    words[slice_word<BITS>(k)] += b0 << slice_shift<BITS>(k);
+    words[slice_word<BITS>(k + 16)] += b1 << slice_shift<BITS>(k + 16);
+    if constexpr (LEVELS) {
+      const float2 cf = __fadd2_rn(r, make_float2(-kRoundMagic, -kRoundMagic));   // exact codes
+      levels[k] = __ffma2_rn(make_float2(st[0], st[1]), cf, make_float2(zt[0], zt[1]));
+    }
+  }
+}
+
 // Affine quantisation [RQ §2.1] of one lane's 32 values and the packed store;
 // if `levels` is given it receives the stored levels fma(s~, code, z~) (what
 // a reader of the record reconstructs).  Group parts: channels 0-15 (.x)
@@ -203,7 +274,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   constexpr int NG = G < 32 ? 2 : 1;        // group parts per lane
   constexpr int LPG = G > 32 ? G / 32 : 1;  // lanes sharing a group
-  float st[2], zt[2], inv[2];
+  float st[2], zt[2], inv[2], gmn[2], gmx[2];
   uint32_t metaw[2];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
@@ -232,6 +303,8 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     mn = __fadd_rn(mn, 0.0f);   // a zero end of the range is +0
     mx = __fadd_rn(mx, 0.0f);
+    gmn[gi] = mn;
+    gmx[gi] = mx;
     const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
     if (m16) {
       // 16-bit metadata: scale byte nearest to max(s, |mn| / 15.875), offset
@@ -262,34 +335,34 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
   }
+  // (x - z~) * (1/s~) is monotone in x, so when a group's ends map into
+  // [-1/2, 2^b - 1/2) every element rounds into [0, 2^b - 1] and the clamp
+  // changes nothing; the warp skips it when that holds for all its lanes.
+  bool in_range = true;
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    const float ulo = __fmul_rn(__fsub_rn(gmn[gi], zt[gi]), inv[gi]);
+    const float uhi = __fmul_rn(__fsub_rn(gmx[gi], zt[gi]), inv[gi]);
+    in_range = in_range && ulo >= -0.5f && uhi < static_cast<float>(QMAX) + 0.5f;
+  }
   if constexpr (NG == 1) {
     st[1] = st[0];
     zt[1] = zt[0];
     inv[1] = inv[0];
   }
   const float2 nz = make_float2(-zt[0], -zt[1]), iv = make_float2(inv[0], inv[1]);
-  const float2 mg = make_float2(kRoundMagic, kRoundMagic);
   uint32_t words[BITS];
-#pragma unroll
-  for (int i = 0; i < BITS; ++i) words[i] = 0u - magic_pack_offset<BITS>(i);
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    // u = (x - z~) * (1/s~), clamped to [0, 2^b - 1]; u + 1.5 * 2^23 rounds it
-    // to the nearest integer (ties to even), held in the low mantissa bits
-    // of a float whose bit pattern is kRoundMagicBits + code.
-    float2 u = __fmul2_rn(__fadd2_rn(v[k], nz), iv);
-    u.x = fminf(fmaxf(u.x, 0.0f), static_cast<float>(QMAX));
-    u.y = fminf(fmaxf(u.y, 0.0f), static_cast<float>(QMAX));
-    const float2 r = __fadd2_rn(u, mg);
-    const uint32_t b0 = __float_as_uint(r.x), b1 = __float_as_uint(r.y);
-    // packing: + (kRoundMagicBits + code) << shift (the offsets were
-    // subtracted up front), as integer multiply-adds
-    words[slice_word<BITS>(k)] += b0 << slice_shift<BITS>(k);
-    words[slice_word<BITS>(k + 16)] += b1 << slice_shift<BITS>(k + 16);
-    if (levels != nullptr) {
-      const float2 cf = __fadd2_rn(r, make_float2(-kRoundMagic, -kRoundMagic));   // exact codes
-      levels[k] = __ffma2_rn(make_float2(st[0], st[1]), cf, make_float2(zt[0], zt[1]));
-    }
+  const bool fast = __all_sync(0xffffffffu, in_range);
+  if (levels == nullptr) {
+    if (fast)
+      pack_codes<BITS, false, false>(v, nz, iv, st, zt, words, levels);
+    else
+      pack_codes<BITS, true, false>(v, nz, iv, st, zt, words, levels);
+  } else {
+    if (fast)
+      pack_codes<BITS, false, true>(v, nz, iv, st, zt, words, levels);
+    else
+      pack_codes<BITS, true, true>(v, nz, iv, st, zt, words, levels);
   }
   if (!active) return;
   uint32_t* cw = codes_row + slice * BITS;
@@ -372,8 +445,10 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int64_t t = p.t0 + (active ? row % p.n : 0);
 
     if (p.dst.has_alpha) {
-      // Least-squares coefficient against the reconstructed reference
-      // [RQ §3.2 scaling coefficient, App. G.1], then the residual.
+      // Fixed mean removed first [RQ App. G.2]; least-squares coefficient
+      // against the reconstructed reference [RQ §3.2 scaling coefficient,
+      // App. G.1], then the residual.
+      if (p.dst.mean != nullptr && active) sub_mean(p.dst, bhi, slice, D, v);
       float2 ref[16];
       if (active) {
         chain_slice(p.ref, p.nref, bhi, p.nblk, t, slice, D, ref);
@@ -465,17 +540,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
       const Comp& c = p.dst[side][r];
       load_rotate<D>(xs + (static_cast<int64_t>(r) * total + r_in) * D, active, slice,
                      p.rot_scale, v);
+      if (c.mean != nullptr && active) sub_mean(c, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
         *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
                    static_cast<int>(t % kBlock), c.meta16 ? 2 : 4) = __bfloat16_as_ushort(ab);
-      float2 lv[16];
-      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, lv);
+      float2 lv[16];   // stored levels, the next reference of a chain
+      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, p.chained ? lv : nullptr);
       if (p.chained) {
         const float at = __bfloat162float(ab);
         const float2 a2 = make_float2(at, at);
 #pragma unroll
         for (int j = 0; j < 16; ++j) ref[j] = __ffma2_rn(a2, ref[j], lv[j]);
+        if (c.mean != nullptr && active) add_mean(c, bhi, slice, D, ref);
       }
     }
   }

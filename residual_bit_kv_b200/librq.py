@@ -38,7 +38,7 @@ SYMBOLS = (
     "rq_dequantize", "rq_decode_workspace_bytes", "rq_decode_workspace_init",
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
     "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
-    "rq_quantize_append_loops", "rq_selftest_wait_timeout",
+    "rq_quantize_append_loops", "rq_selftest_wait_timeout", "rq_cache_set_means",
 )
 
 
@@ -58,6 +58,7 @@ class rq_cache(ctypes.Structure):
         ("layer_bytes", ctypes.c_uint64), ("token_stride", ctypes.c_int64),
         ("comp_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
         ("rec_bytes", ctypes.c_uint32 * RQ_MAX_LOOPS),
+        ("k_means", ctypes.c_void_p), ("v_means", ctypes.c_void_p),
     ]
 
 
@@ -93,6 +94,7 @@ def load() -> ctypes.CDLL:
         "rq_cache_bytes": ([LP], _U64),
         "rq_layer_bytes": ([LP], _U64),
         "rq_cache_bind": ([LP, _P, _P, CP], ctypes.c_int),
+        "rq_cache_set_means": ([CP, _P, _P], ctypes.c_int),
         "rq_quantize_anchor": ([CP, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_residual": ([CP, _I32, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_loops": ([CP, _I32, _P, _P, _I32, _I32, _P], ctypes.c_int),
@@ -182,6 +184,15 @@ def rq_cache_bind(layout: rq_layout, k_base, v_base) -> rq_cache:
     _check(load().rq_cache_bind(ctypes.byref(layout), _ptr(k_base), _ptr(v_base), ctypes.byref(c)),
            "rq_cache_bind")
     return c
+
+
+def rq_cache_set_means(cache: rq_cache, k_means, v_means) -> None:
+    """k_means, v_means: fp32 [num_layers, num_loops, kv_heads, head_dim] device
+    tensors (rotated domain) or None."""
+    _check(load().rq_cache_set_means(ctypes.byref(cache),
+                                     None if k_means is None else _ptr(k_means),
+                                     None if v_means is None else _ptr(v_means)),
+           "rq_cache_set_means")
 
 
 def rq_quantize_anchor(cache: rq_cache, layer: int, kv: int, x, t0: int, n: int,

@@ -53,13 +53,15 @@ class GpuCache:
     inputs: Dict  # (layer, side, loop) -> bf16 [B, H, T, D] cuda tensor (if kept)
     unit_alpha: bool = False
     meta16: bool = False
+    means: Optional[Dict] = None   # side -> fp32 [layers, loops, H, D] cuda tensor
 
 
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
                     keep_inputs: bool = True, tokens: Optional[int] = None,
                     max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
                     fused: bool = False, unit_alpha: bool = False,
-                    gen_device: str = "cuda", meta16: bool = False) -> GpuCache:
+                    gen_device: str = "cuda", meta16: bool = False,
+                    means_seed: Optional[int] = None) -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
     the C ABI in the order the policy requires (fused: every loop and both
     sides of a chunk in one rq_quantize_append_loops call).  append_chunks
@@ -74,6 +76,12 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
     kbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     vbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     cache = L.rq_cache_bind(lay, kbuf, vbuf)
+    means = None
+    if means_seed is not None:
+        g = torch.Generator().manual_seed(means_seed)
+        means = {side: (torch.randn(lay.num_layers, w.loops, w.heads, w.head_dim, generator=g) *
+                        0.5).to("cuda") for side in SIDES}
+        L.rq_cache_set_means(cache, means[0], means[1])
     inputs = {}
     bounds = [0] + list(np.cumsum(append_chunks)) if append_chunks else [0, T]
     assert bounds[-1] == T
@@ -111,7 +119,7 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     inputs[(layer, side, loop)] = x
             del xs
     torch.cuda.synchronize()
-    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha, meta16)
+    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha, meta16, means)
 
 
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
@@ -151,15 +159,26 @@ def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,
 def oracle_encode(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
                   hsel: Sequence[int], t0: int, t1: int, policy: str = "last",
                   x_loops: Optional[List[np.ndarray]] = None, unit_alpha: bool = False,
-                  meta16: bool = False):
+                  meta16: bool = False, means: Optional[Dict] = None):
     """Oracle encodings of the selected rows.  Returns (encs, x) where
-    x is uint16 [L, nb*nh*(t1-t0), D]."""
+    x is uint16 [L, nb*nh*(t1-t0), D] (means: the cache's fixed means)."""
     if x_loops is None:
         cs = synth.key_channel_scale(w, layer) if side == synth.SIDE_K else None
         x_loops = [synth.bits_of(synth.kv(w, layer, side, loop, bsel, hsel, t0, t1, "cpu", cs))
                    .reshape(-1, w.head_dim) for loop in range(w.loops)]
     x = np.stack(x_loops)
-    return oracle.encode_side(x, w.bits, w.group, policy, unit_alpha, meta16), x
+    return oracle.encode_side(x, w.bits, w.group, policy, unit_alpha, meta16,
+                              mu=mean_rows(w, layer, side, bsel, hsel, t1 - t0, means)), x
+
+
+def mean_rows(w: synth.Workload, layer: int, side: int, bsel: Sequence[int],
+              hsel: Sequence[int], T: int, means: Optional[Dict]) -> Optional[np.ndarray]:
+    """The fixed means expanded to the oracle's rows (b, h, t): [L, N, D]."""
+    if means is None:
+        return None
+    m = means[side][layer].cpu().numpy().astype(np.float32)   # [L, H, D]
+    rows = [m[:, h] for b in bsel for h in hsel for _ in range(T)]
+    return np.ascontiguousarray(np.stack(rows, axis=1))
 
 
 def assert_component_equal(gpu: Dict[str, np.ndarray], enc: Dict[str, np.ndarray], shape,
@@ -209,7 +228,8 @@ def gpu_decode(gc: GpuCache, layer: int, loop: int, seq_lens: Sequence[int], max
 def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
                   hsel: Sequence[int], seq_lens: Sequence[int], policy: str = "last",
                   inputs: Optional[Dict] = None, scale: Optional[float] = None,
-                  unit_alpha: bool = False, meta16: bool = False) -> np.ndarray:
+                  unit_alpha: bool = False, meta16: bool = False,
+                  means: Optional[Dict] = None) -> np.ndarray:
     """fp64 oracle decode for the selected (b, h): [len(bsel), len(hsel), D]."""
     T = max(int(seq_lens[b]) for b in bsel)
     D = w.head_dim
@@ -220,8 +240,10 @@ def oracle_decode(w: synth.Workload, layer: int, loop: int, bsel: Sequence[int],
         if inputs is not None:
             xl = [synth.bits_of(inputs[(layer, side, l)][list(bsel)][:, list(hsel), :T].cpu())
                   .reshape(-1, D) for l in range(w.loops)]
-        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl, unit_alpha, meta16)
-        rec[side] = oracle.reconstruct(encs, loop, w.bits, w.group, policy).reshape(
+        encs, _ = oracle_encode(w, layer, side, bsel, hsel, 0, T, policy, xl, unit_alpha, meta16,
+                                means)
+        rec[side] = oracle.reconstruct(encs, loop, w.bits, w.group, policy,
+                                       mean_rows(w, layer, side, bsel, hsel, T, means)).reshape(
             len(bsel), len(hsel), T, D)
     q = synth.bits_of(synth.query(w, layer, loop)).reshape(w.batch, w.heads, D)
     kc = synth.bits_of(synth.current_token(w, layer, synth.SIDE_K, loop))

@@ -27,7 +27,7 @@ def test_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(L.SYMBOLS)
-    assert L.rq_abi_version() == 1
+    assert L.rq_abi_version() == 2
 
 
 def test_status_strings(L):
