@@ -240,7 +240,10 @@ rq_status rq_decode_workspace_init(void* workspace, uint64_t ws_bytes,
  *            clamped and flagged (rq_workspace_error -> RQ_ERR_CAPACITY)
  *   max_seq_len  host bound on seq_lens, <= max_tokens (sizes the grid)
  *   softmax_scale  0 selects 1/sqrt(head_dim)
- *   out      fp32 [batch][kv_heads][head_dim]
+ *   out      fp32 [batch][kv_heads][head_dim]; the row of a (batch, head)
+ *            whose decode is not valid (a bounded wait ran out, or a value
+ *            weight left the accumulator range, see rq_workspace_error) is
+ *            written as NaN
  *   workspace  >= rq_decode_workspace_bytes(layout, max_seq_len), zeroed by
  *            rq_decode_workspace_init once; calls sharing a workspace must be
  *            ordered on one stream. */
@@ -270,9 +273,9 @@ rq_status rq_decode_attention_bf16(int32_t batch, int32_t heads,
 /* Reads and clears the device-side error word of a decode workspace
  * (synchronises `stream`).  RQ_OK, RQ_ERR_CAPACITY (a seq_lens entry was out
  * of range), RQ_ERR_UNSUPPORTED (a value weight p_t * kappa * s~ reached
- * 2^19, outside the range of the decode kernel's scaled accumulators; that
- * call's output is not valid) or RQ_ERR_TIMEOUT (a bounded wait ran out;
- * re-initialise the workspace). */
+ * 2^36, outside the range of the decode kernel's scaled accumulators; the
+ * affected output rows are NaN) or RQ_ERR_TIMEOUT (a bounded wait ran out;
+ * the affected output rows are NaN; re-initialise the workspace). */
 rq_status rq_workspace_error(void* workspace, uint64_t ws_bytes, void* stream);
 
 /* Self-test of the device-side failure path (for tests): one CTA waits on an
@@ -304,8 +307,11 @@ int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);
  *   If the split partials of a shape do not fit, fewer splits are used; if
  *   one split per (batch, head) does not fit (batch * kv_heads * (head_dim+2)
  *   * 4 bytes above ~8 MiB) the call returns RQ_ERR_WORKSPACE without
- *   launching.  Device-side conditions (a seq_lens entry out of range is
- *   clamped, as in rq_decode_attention) are not reported by this entry point. */
+ *   launching.  With no workspace there is no error word for the caller to
+ *   read: a (batch, head) whose decode is not valid (a bounded wait ran out,
+ *   or a value weight left the accumulator range) gets a NaN output row, as
+ *   in rq_decode_attention; a seq_lens entry out of range is clamped without
+ *   a report. */
 rq_status rq_decode_attention_noalloc(const rq_cache* cache, int32_t layer,
                                       int32_t loop, const void* q,
                                       const int32_t* seq_lens,

@@ -352,10 +352,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 #pragma unroll
   for (int ch = 0; ch < 32; ++ch) acc[ch] += (ch < 16) ? cst0 : cst1;
-  __syncthreads();
+  const bool aborted = __syncthreads_or(s_abort != 0) != 0;
   finish_split<D, kDecodeThreads, Geom<D>::NSLOT, true>(
       m, l, acc, slice, slot, reinterpret_cast<float*>(smem), bhi, split, p.splits, p.partials,
-      p.counters, p.q, p.kcur, p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred);
+      p.counters, p.q, p.kcur, p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred, aborted);
 }
 
 template <int D>

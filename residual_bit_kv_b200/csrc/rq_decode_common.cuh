@@ -61,7 +61,11 @@ __device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int ma
 // partial (m, l, acc[D]) in the workspace; the last CTA of the (batch, head)
 // then merges every split with the current token and writes the output,
 // applying H^T once when ROT.  `scratch` holds max(NSLOT*red_pitch<D>() +
-// 2*NSLOT, 3*splits) floats.
+// 2*NSLOT, 3*splits) floats.  `bad` (the same for every thread of the CTA)
+// marks a split whose result is not valid (a bounded wait ran out, or a value
+// left the accumulator range): it is counted in the upper half of the
+// (batch, head)'s split counter, and the merging CTA then writes NaN to that
+// (batch, head)'s output row instead of a partial sum.
 //
 // The slot reduction buffer keeps each slice's 32 channels in a block of 36
 // floats (a slot is D/32 blocks): the 16-byte stores of the lanes of one
@@ -78,7 +82,7 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
                                              const uint16_t* q, const uint16_t* kcur,
                                              const uint16_t* vcur, float scale_log2,
                                              float rot_scale, float* out, float* svec,
-                                             float* sred) {
+                                             float* sred, bool bad) {
   constexpr int RP = red_pitch<D>();
   float* red = scratch;                 // [NSLOT][D/32][36]
   float* mred = red + NSLOT * RP;       // [NSLOT]
@@ -119,15 +123,23 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
   // acquire-release add, which makes them visible with it (and, for the last
   // CTA, makes every other split's partial visible to it).
   __syncthreads();
-  __shared__ uint32_t s_last;
+  __shared__ uint32_t s_last, s_bad;
   if (t == 0) {
+    // low 16 bits: splits counted in (splits <= 1024); high 16: bad splits
+    const uint32_t inc = bad ? 0x10001u : 1u;
     uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                 : "=r"(old) : "l"(counters + bhi) : "memory");
-    s_last = (old == static_cast<uint32_t>(splits - 1));
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old) : "l"(counters + bhi), "r"(inc) : "memory");
+    s_last = ((old + inc) & 0xFFFFu) == static_cast<uint32_t>(splits);
+    s_bad = (old + inc) >> 16;
   }
   __syncthreads();
   if (!s_last) return;
+  if (s_bad != 0u) {   // a split of this (batch, head) is not valid
+    if (t < D) out[static_cast<size_t>(bhi) * D + t] = __int_as_float(0x7FC00000);
+    if (t == 0) counters[bhi] = 0u;
+    return;
+  }
 
   // ---- last CTA of this (batch, head): merge ----
   // Current token score q.k_cur, original domain [RQ §3.2, §4.2].

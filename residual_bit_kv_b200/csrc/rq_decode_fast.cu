@@ -19,7 +19,7 @@
 // the LS coefficients along the reference chain.
 // Values: a code masked out of its word (all other bits zero) is the exact
 // fp32 subnormal c * 2^(p-149), p its bit position; packed fp32 FMAs with
-// weights p_t * kappa * s~ * 2^(109-p) accumulate p_t * kappa * s~ * c * 2^-40
+// weights p_t * kappa * s~ * 2^(92-p) accumulate p_t * kappa * s~ * c * 2^-57
 // per channel, the offsets z~ going to separate accumulators.  Accumulation
 // is in the rotated domain; H^T is applied once in the merge.
 #include <type_traits>
@@ -188,8 +188,10 @@ struct VAcc {
   float mw[8];   // fixed means: sum of p_t * kappa_c per residual component (MU layouts)
 };
 
-constexpr int kPosBias = 109;                        // weights w * 2^(109 - p), p <= 14
-constexpr float kValueUnscale = 1099511627776.0f;    // 2^(149 - kPosBias) = 2^40
+// Weights w * 2^(92 - p), p <= 14: finite for w < 2^36, and products stay
+// normal down to w * c = 2^-69.
+constexpr int kPosBias = 92;
+constexpr float kValueUnscale = 144115188075855872.0f;   // 2^(149 - kPosBias) = 2^57
 
 __device__ __forceinline__ float pow2i(int e) {
   return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
@@ -202,7 +204,7 @@ __device__ __forceinline__ float2 masked_pair(uint32_t w, uint32_t ma, uint32_t 
 // acc += pk * D(c) over one lane's 32 channels of record token jl (codes
 // part; the z~ offsets go to cst).  A channel pair shares a word, and the
 // code positions (pa, pb) of the pair fix its weight pair
-// {w 2^(109-pa), w 2^(109-pb)}, w = pk * s~:
+// {w 2^(92-pa), w 2^(92-pb)}, w = pk * s~:
 //   b = 2: word k holds channels 16k + 2i, +1 at bits 4i, 4i+2 (i < 4), and
 //          channels 16k + 8 + 2i, +1 at the same bits of word >> 16;
 //   b = 4: word 2k + hh holds channels 16k + 2hh, +1 at bits 0, 4 and
@@ -345,7 +347,7 @@ __device__ __forceinline__ void rescale(VAcc& va, float f) {
 }
 
 // Final per-channel values: undo the 2^-40 code scale and add the z~ terms.
-// A weight past the scaled range (p_t * kappa * s~ >= 2^19) leaves an
+// A weight past the scaled range (p_t * kappa * s~ >= 2^36) leaves an
 // infinity or NaN here and is reported.
 __device__ __forceinline__ void finish_values(const VAcc& va, float (&acc)[32],
                                               uint32_t& range_err) {
@@ -606,6 +608,7 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   }
   __syncthreads();   // every warp has left the loop: s_abort is settled
   const bool aborted = s_abort != 0;
+  const bool range_bad = __syncthreads_or(range_err != 0u) != 0;
   if (range_err && !aborted) atomicOr(p.err, kErrRange);
   if (aborted) {
     m = kNegInf;
@@ -618,7 +621,8 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   finish_split<D, kCThreads, NSLOT, true>(m, l, acc, slice, warp * TPW + tw,
                                           reinterpret_cast<float*>(smem), bhi, split, p.splits,
                                           p.partials, p.counters, p.q, p.kcur, p.vcur,
-                                          p.scale_log2, p.rot_scale, p.out, svec, sred);
+                                          p.scale_log2, p.rot_scale, p.out, svec, sred,
+                                          aborted || range_bad);
 }
 
 // ---------------------------------------------------------------- BF16 --
@@ -766,10 +770,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
     }
   }
-  __syncthreads();
+  const bool aborted = __syncthreads_or(s_abort != 0) != 0;
   finish_split<D, kThreads, NSLOT, false>(m, l, acc, slice, slot, reinterpret_cast<float*>(smem),
                                           bhi, split, p.splits, p.partials, p.counters, p.q,
-                                          p.kcur, p.vcur, p.scale_log2, 1.0f, p.out, svec, sred);
+                                          p.kcur, p.vcur, p.scale_log2, 1.0f, p.out, svec, sred,
+                                          aborted);
 }
 
 template <typename K>

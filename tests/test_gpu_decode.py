@@ -152,3 +152,26 @@ def test_split_plan_invariants(cuda_dev, T, batch, heads):
     assert 1 <= s <= max(1, chunks)
     cps = -(-chunks // s)
     assert -(-chunks // cps) == s
+
+
+def test_value_range_limit_gives_nan_rows_and_a_flag(cuda_dev):
+    """A unit whose value weights p * alpha * s~ reach 2^36 (the limit of the
+    fast kernel's scaled accumulators) is reported (RQ_ERR_UNSUPPORTED) and its
+    output row is NaN; the other unit of the same call is exact to the oracle's
+    tolerance, and the anchor loop (alpha = 1) of the same cache is fine."""
+    import range_case as rc
+    bits = rc.inputs()
+    lay, cache, keep, q, kc, vc = rc.build(bits)
+    ws = Workspace(lay, rc.T)
+    sl = torch.full((rc.B,), rc.T, dtype=torch.int32, device="cuda")
+    for loop, bad in ((0, True), (1, False)):
+        out = torch.zeros(rc.B, rc.H, rc.D, dtype=torch.float32, device="cuda")
+        L.rq_decode_attention(cache, 0, loop, q, sl, rc.T, kc, vc, 0.0, out, ws.buf, ws.bytes)
+        status = L.rq_workspace_error(ws.buf, ws.bytes)
+        got = out.cpu().numpy().astype(np.float64)
+        assert status == (L.RQ_ERR_UNSUPPORTED if bad else L.RQ_OK), loop
+        assert np.all(np.isnan(got[0])) == bad and np.all(np.isfinite(got[0])) != bad
+        for b in ([1] if bad else [0, 1]):
+            ref = rc.oracle_out(bits, b, loop)
+            assert np.max(np.abs(got[b, 0] - ref)) <= attn_tolerance(ref), (loop, b)
+    assert np.all(np.isfinite(rc.oracle_out(bits, 0, 0)))   # the method itself is fine there
