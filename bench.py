@@ -363,17 +363,19 @@ class Engine:
         w = self.w
         return w.layers * w.loops + w.layers
 
-    def step(self, stream, ev=None, q=None, kc_layer=None, vc_layer=None):
+    def step(self, stream, ev=None, q=None, kc_layer=None, vc_layer=None, loops=None,
+             appends=True):
         """One decode step: the decode attention of every (layer, loop), then
         per layer one launch that quantises and appends the new token of every
         loop, K and V.  ev: optional list collecting (start, end) event pairs
-        around each decode-attention launch."""
+        around each decode-attention launch.  loops / appends=False select a
+        part of the step (the roofline's kernel-only timings)."""
         L, w, T = self.L, self.w, self.w.tokens
         q = q or self.q
         kcl = kc_layer or self.kc_layer
         vcl = vc_layer or self.vc_layer
         for layer in range(w.layers):
-            for loop in range(w.loops):
+            for loop in (range(w.loops) if loops is None else loops):
                 if ev is not None:
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
@@ -385,7 +387,9 @@ class Engine:
                     e1.record(stream)
                     ev.append((e0, e1, loop))
             # after the final loop: quantise and append the new token (position T)
-            L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1, stream)
+            if appends:
+                L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1,
+                                           stream)
 
     def bf16_step(self, stream, ev=None, nlayers_buf=4):
         L, w, T = self.L, self.w, self.w.tokens
@@ -637,45 +641,25 @@ def main():
     w = eng.w
     stream = torch.cuda.current_stream(dev)
 
-    # ---- the decode step launched eagerly, with CUDA events around every
-    # decode-attention launch (the roofline's kernel times)
-    ev = []
-    for _ in range(args.warmup):
-        eng.step(stream)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        eng.step(stream, ev)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    eager_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
-    dec_ms = sum(a.elapsed_time(b) for a, b, _ in ev)
-    dec_bytes = args.steps * w.layers * sum(decode_call_bytes(w, l, w.tokens) for l in range(w.loops))
-    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    per_loop = {}
-    for l in range(w.loops):
-        t_l = sum(a.elapsed_time(b) for a, b, ll in ev if ll == l) / (args.steps * w.layers)
-        per_loop[str(l)] = {"us": t_l * 1e3,
-                            "gbs": decode_call_bytes(w, l, w.tokens) / (t_l * 1e-3) / 1e9}
     hbm, hbm_kind = peaks()
     traffic = profile_traffic(DECODE_SOURCES, "decode_kernel_ouro_16k.md")
-
-    # ---- main timed region: the same step captured once as a CUDA graph
-    # (the launch sequence of one step: no host work or launch gaps between
-    # kernels) and replayed
-    graph = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream(dev)
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        eng.step(cap)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(graph, stream=cap):
-        eng.step(cap)
-    torch.cuda.synchronize()
+
+    def capture(fn):
+        """fn(stream) captured once as a CUDA graph (after one eager run)."""
+        g = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            fn(cap)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=cap):
+            fn(cap)
+        torch.cuda.synchronize()
+        return g
+
+    # ---- main timed region: the whole step (96 decode + 24 append launches)
+    # captured once as a CUDA graph (no host work or launch gaps) and replayed
+    graph = capture(lambda st: eng.step(st))
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -691,6 +675,26 @@ def main():
         torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     clocks = clk.summary()
+    del graph
+
+    # ---- the roofline's kernel time: the step's 96 decode launches alone,
+    # as one graph (back to back, the appends left out), and each loop's 24
+    # launches as its own graph
+    dec_bytes = w.layers * sum(decode_call_bytes(w, l, w.tokens) for l in range(w.loops))
+    g_dec = capture(lambda st: eng.step(st, appends=False))
+    dec_ms = timed(g_dec.replay, args.steps, args.warmup, stream, dist)
+    del g_dec
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    per_loop = {}
+    for l in range(w.loops):
+        g_l = capture(lambda st, l=l: eng.step(st, loops=[l], appends=False))
+        t_l = timed(g_l.replay, args.steps, args.warmup, stream, dist) / w.layers
+        del g_l
+        per_loop[str(l)] = {"us": t_l * 1e3,
+                            "gbs": decode_call_bytes(w, l, w.tokens) / (t_l * 1e-3) / 1e9}
+
+    # ---- the same step launched call by call (host launch gaps included)
+    eager_ms = timed(lambda: eng.step(stream), args.steps, args.warmup, stream, dist)
 
     # ---- end to end: host buffers, H2D of the step's inputs, D2H of the outputs
     pin = {k: v.cpu().pin_memory() for k, v in eng.q.items()}
@@ -701,16 +705,32 @@ def main():
     dkc = [torch.empty_like(t) for t in eng.kc_layer]
     dvc = [torch.empty_like(t) for t in eng.vc_layer]
 
-    def e2e_step():
+    def copy_in():
         for k in pin:
             dq[k].copy_(pin[k], non_blocking=True)
         for i in range(len(pkc)):
             dkc[i].copy_(pkc[i], non_blocking=True)
             dvc[i].copy_(pvc[i], non_blocking=True)
+
+    def e2e_eager_step():
+        copy_in()
         eng.step(stream, None, dq, dkc, dvc)
         hout.copy_(eng.out, non_blocking=True)
 
+    e2e_eager_ms = timed(e2e_eager_step, args.steps, args.warmup, stream, dist)
+
+    # the public-API step on the device input buffers captured once as a CUDA
+    # graph, as a serving loop would: per step the inputs are copied in from
+    # pinned host memory, the graph replays and the outputs are read back
+    graph_io = capture(lambda st: eng.step(st, None, dq, dkc, dvc))
+
+    def e2e_step():
+        copy_in()
+        graph_io.replay()
+        hout.copy_(eng.out, non_blocking=True)
+
     e2e_ms = timed(e2e_step, args.steps, args.warmup, stream, dist)
+    del graph_io
     h2d = (sum(v.numel() for v in pin.values()) + sum(t.numel() for t in pkc) +
            sum(t.numel() for t in pvc)) * 2
     d2h = hout.numel() * 4
@@ -759,7 +779,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
                          "kernel": "decode_fast_kernel (all loops of the step)", "peak_kind": hbm_kind,
-                         "bytes_per_step": dec_bytes / args.steps},
+                         "bytes_per_step": dec_bytes,
+                         "kernel_time": ("CUDA events around a graph of the step's "
+                                         f"{w.layers * w.loops} decode launches replayed "
+                                         f"back to back: {dec_ms:.3f} ms per step")},
             "decode_per_loop": per_loop,
             "step_launch": {"timed": f"one CUDA graph per step ({w.layers * w.loops} decode + "
                                      f"{w.layers} append launches)",
@@ -769,7 +792,10 @@ def main():
             "decode_hbm_frac_of_8tbs": achieved / 8000.0,
             "e2e": {"value": job_tokens_per_s(ws, w.batch, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "path": "public API per call (eager), inputs from pinned host memory"},
+                    "path": "public API step captured as a CUDA graph on device input buffers; "
+                            "per step: H2D of the inputs from pinned host memory, replay, D2H "
+                            "of the output",
+                    "eager_value": job_tokens_per_s(ws, w.batch, e2e_eager_ms)},
             "gpu_launches": launches,
             "clocks": clocks,
             "bf16_baseline": bf16,
