@@ -246,7 +246,9 @@ rq_status rq_decode_workspace_init(void* workspace, uint64_t ws_bytes,
  *            written as NaN
  *   workspace  >= rq_decode_workspace_bytes(layout, max_seq_len), zeroed by
  *            rq_decode_workspace_init once; calls sharing a workspace must be
- *            ordered on one stream. */
+ *            ordered on one stream, and a workspace moved to a layout with
+ *            another batch * kv_heads must be zeroed again (its per-row
+ *            counters sit where the other layout's partials were). */
 rq_status rq_decode_attention(const rq_cache* cache, int32_t layer,
                               int32_t loop, const void* q,
                               const int32_t* seq_lens, int32_t max_seq_len,
@@ -306,8 +308,8 @@ int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);
  *   threads) race on it and must be ordered by the caller.
  *   If the split partials of a shape do not fit, fewer splits are used; if
  *   one split per (batch, head) does not fit (batch * kv_heads * (head_dim+2)
- *   * 4 bytes above ~8 MiB) the call returns RQ_ERR_WORKSPACE without
- *   launching.  With no workspace there is no error word for the caller to
+ *   * 4 bytes above the 8 MiB less 256 KiB of per-row counters) the call
+ *   returns RQ_ERR_WORKSPACE without launching.  With no workspace there is no error word for the caller to
  *   read: a (batch, head) whose decode is not valid (a bounded wait ran out,
  *   or a value weight left the accumulator range) gets a NaN output row, as
  *   in rq_decode_attention; a seq_lens entry out of range is clamped without

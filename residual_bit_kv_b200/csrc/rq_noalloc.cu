@@ -16,9 +16,13 @@ using namespace rq;
 
 // Scratch of rq_decode_attention_noalloc: [error word | split counters |
 // split partials].  8 MiB, held by every device that loads the library until
-// the process exits.
+// the process exits.  The counters have a fixed region for the largest
+// batch * kv_heads a layout allows, so the partials of one call never land on
+// the counters of a later call with more rows (the counters must start at
+// zero; the kernels return every counter they use to zero).
 constexpr size_t kNoAllocScratchBytes = 8u << 20;
 constexpr size_t kHeaderAlign = 256;
+constexpr size_t kMaxRows = 65535;   // batch * kv_heads limit of rq_layout_validate
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
@@ -74,7 +78,7 @@ extern "C" rq_status rq_decode_attention_noalloc(const rq_cache* c, int32_t laye
   // Fit the split partials into the fixed scratch: fewer splits if needed,
   // an error if even one split per (batch, head) does not fit.
   const size_t counters_off = kHeaderAlign;
-  const size_t partials_off = align_up(counters_off + static_cast<size_t>(p.bh) * 4, kHeaderAlign);
+  const size_t partials_off = align_up(counters_off + kMaxRows * 4, kHeaderAlign);
   const size_t per_split = static_cast<size_t>(p.bh) * (D + 2) * sizeof(float);
   if (partials_off + per_split > kNoAllocScratchBytes) return RQ_ERR_WORKSPACE;
   const int fit = static_cast<int>((kNoAllocScratchBytes - partials_off) / per_split);

@@ -274,28 +274,30 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   constexpr int NG = G < 32 ? 2 : 1;        // group parts per lane
   constexpr int LPG = G > 32 ? G / 32 : 1;  // lanes sharing a group
-  float st[2], zt[2], inv[2], gmn[2], gmx[2];
+  float st[2], zt[2], inv[2];
   uint32_t metaw[2];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
-    float mn, mx;
-    if constexpr (NG == 2) {
-      mn = mx = gi == 0 ? v[0].x : v[0].y;
+    // min / max as trees (exact in any order; short dependency chains)
+    float tn[16], tx[16];
 #pragma unroll
-      for (int k = 1; k < 16; ++k) {
-        const float e = gi == 0 ? v[k].x : v[k].y;
-        mn = fminf(mn, e);
-        mx = fmaxf(mx, e);
-      }
-    } else {
-      mn = fminf(v[0].x, v[0].y);
-      mx = fmaxf(v[0].x, v[0].y);
-#pragma unroll
-      for (int k = 1; k < 16; ++k) {
-        mn = fminf(mn, fminf(v[k].x, v[k].y));
-        mx = fmaxf(mx, fmaxf(v[k].x, v[k].y));
+    for (int k = 0; k < 16; ++k) {
+      if constexpr (NG == 2) {
+        tn[k] = tx[k] = gi == 0 ? v[k].x : v[k].y;
+      } else {
+        tn[k] = fminf(v[k].x, v[k].y);
+        tx[k] = fmaxf(v[k].x, v[k].y);
       }
     }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+      for (int k = 0; k < w; ++k) {
+        tn[k] = fminf(tn[k], tn[k + w]);
+        tx[k] = fmaxf(tx[k], tx[k + w]);
+      }
+    }
+    float mn = tn[0], mx = tx[0];
 #pragma unroll
     for (int off = 1; off < LPG; off <<= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -303,8 +305,6 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     mn = __fadd_rn(mn, 0.0f);   // a zero end of the range is +0
     mx = __fadd_rn(mx, 0.0f);
-    gmn[gi] = mn;
-    gmx[gi] = mx;
     const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
     if (m16) {
       // 16-bit metadata: scale byte nearest to max(s, |mn| / 15.875), offset
@@ -335,16 +335,6 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
   }
-  // (x - z~) * (1/s~) is monotone in x, so when a group's ends map into
-  // [-1/2, 2^b - 1/2) every element rounds into [0, 2^b - 1] and the clamp
-  // changes nothing; the warp skips it when that holds for all its lanes.
-  bool in_range = true;
-#pragma unroll
-  for (int gi = 0; gi < NG; ++gi) {
-    const float ulo = __fmul_rn(__fsub_rn(gmn[gi], zt[gi]), inv[gi]);
-    const float uhi = __fmul_rn(__fsub_rn(gmx[gi], zt[gi]), inv[gi]);
-    in_range = in_range && ulo >= -0.5f && uhi < static_cast<float>(QMAX) + 0.5f;
-  }
   if constexpr (NG == 1) {
     st[1] = st[0];
     zt[1] = zt[0];
@@ -352,18 +342,10 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   }
   const float2 nz = make_float2(-zt[0], -zt[1]), iv = make_float2(inv[0], inv[1]);
   uint32_t words[BITS];
-  const bool fast = __all_sync(0xffffffffu, in_range);
-  if (levels == nullptr) {
-    if (fast)
-      pack_codes<BITS, false, false>(v, nz, iv, st, zt, words, levels);
-    else
-      pack_codes<BITS, true, false>(v, nz, iv, st, zt, words, levels);
-  } else {
-    if (fast)
-      pack_codes<BITS, false, true>(v, nz, iv, st, zt, words, levels);
-    else
-      pack_codes<BITS, true, true>(v, nz, iv, st, zt, words, levels);
-  }
+  if (levels == nullptr)
+    pack_codes<BITS, true, false>(v, nz, iv, st, zt, words, levels);
+  else
+    pack_codes<BITS, true, true>(v, nz, iv, st, zt, words, levels);
   if (!active) return;
   uint32_t* cw = codes_row + slice * BITS;
   if constexpr (BITS == 4) {
@@ -510,7 +492,7 @@ __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_
 // Z^_r = fma(alpha~_r, Z^_ref, D(c_r)) after loop r.  The anchor is read
 // once and never re-read from the cache; the arithmetic (and so every
 // stored bit) is that of the per-loop kernels.
-template <int D>
+template <int D, bool CHAINED>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_loops_kernel(const __grid_constant__ QuantLoopsParams p) {
   constexpr int P = D / 32;
@@ -546,8 +528,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
                    static_cast<int>(t % kBlock), c.meta16 ? 2 : 4) = __bfloat16_as_ushort(ab);
       float2 lv[16];   // stored levels, the next reference of a chain
-      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, p.chained ? lv : nullptr);
-      if (p.chained) {
+      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, CHAINED ? lv : nullptr);
+      if constexpr (CHAINED) {
         const float at = __bfloat162float(ab);
         const float2 a2 = make_float2(at, at);
 #pragma unroll
@@ -643,9 +625,11 @@ cudaError_t launch_quantize_loops(const QuantLoopsParams& p, int D, cudaStream_t
   if (rows == 0) return cudaSuccess;
   const dim3 grid(quant_grid(rows, D), 2);
   if (D == 64)
-    quantize_loops_kernel<64><<<grid, kQuantThreads, 0, s>>>(p);
+    p.chained ? quantize_loops_kernel<64, true><<<grid, kQuantThreads, 0, s>>>(p)
+              : quantize_loops_kernel<64, false><<<grid, kQuantThreads, 0, s>>>(p);
   else if (D == 128)
-    quantize_loops_kernel<128><<<grid, kQuantThreads, 0, s>>>(p);
+    p.chained ? quantize_loops_kernel<128, true><<<grid, kQuantThreads, 0, s>>>(p)
+              : quantize_loops_kernel<128, false><<<grid, kQuantThreads, 0, s>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

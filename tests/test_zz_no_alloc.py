@@ -68,8 +68,9 @@ def test_noalloc_marks_invalid_rows_nan(cuda_dev):
 
 def _noalloc_fit(bh, D=128):
     """Split partials that fit the no-allocation scratch (8 MiB: error word,
-    per-unit counters at 256 bytes, partials after the counters, 256-aligned)."""
-    poff = -(-(256 + bh * 4) // 256) * 256
+    a counter per row for up to 65535 rows at 256 bytes, then the partials,
+    256-aligned)."""
+    poff = -(-(256 + 65535 * 4) // 256) * 256
     return ((8 << 20) - poff) // (bh * (D + 2) * 4)
 
 
