@@ -368,22 +368,26 @@ class Engine:
 
     def step(self, stream, ev=None, q=None, kc_layer=None, vc_layer=None, loops=None,
              appends=True, side=None):
-        """One decode step: the decode attention of every (layer, loop), then
-        per layer one launch that quantises and appends the new token of every
-        loop, K and V.  ev: optional list collecting (start, end) event pairs
+        """One decode step of the looped model, in its own order: loop 1 runs
+        every layer, then loop 2 every layer, ..., so each (layer, loop) decode
+        call sees the query of its loop; after the final loop of a layer, one
+        launch quantises and appends the new token of every loop of that
+        layer, K and V.  ev: optional list collecting (start, end) event pairs
         around each decode-attention launch.  loops / appends=False select a
         part of the step (the roofline's kernel-only timings).  side: a second
-        stream for the appends; each waits for its layer's decode calls and
-        runs beside the next layers' (it writes position T, which no decode
-        call of this step reads), and the step ends when both streams have."""
+        stream for the appends; each waits for its layer's final-loop decode
+        and runs beside the next layers' (it writes position T, which no
+        decode call of this step reads), and the step ends when both streams
+        have."""
         L, w, T = self.L, self.w, self.w.tokens
         q = q or self.q
         kcl = kc_layer or self.kc_layer
         vcl = vc_layer or self.vc_layer
+        final = w.loops - 1
         if side is not None:
             side.wait_stream(stream)
-        for layer in range(w.layers):
-            for loop in (range(w.loops) if loops is None else loops):
+        for loop in (range(w.loops) if loops is None else loops):
+            for layer in range(w.layers):
                 if ev is not None:
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
@@ -394,21 +398,25 @@ class Engine:
                 if ev is not None:
                     e1.record(stream)
                     ev.append((e0, e1, loop))
-            # after the final loop: quantise and append the new token (position T)
-            if appends and side is None:
-                L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1,
-                                           stream)
-            elif appends:
-                side.wait_stream(stream)
-                L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1, side)
+                if loop != final or not appends:
+                    continue
+                # after the final loop: quantise and append the new token (position T)
+                if side is None:
+                    L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1,
+                                               stream)
+                else:
+                    side.wait_stream(stream)
+                    L.rq_quantize_append_loops(self.cache, layer, kcl[layer], vcl[layer], T, 1,
+                                               side)
         if side is not None:
             stream.wait_stream(side)
 
     def bf16_step(self, stream, ev=None, nlayers_buf=4):
+        """The same step on the uncompressed bf16 cache (loop-major, as step())."""
         L, w, T = self.L, self.w, self.w.tokens
-        for layer in range(w.layers):
-            lb = layer % nlayers_buf
-            for loop in range(w.loops):
+        for loop in range(w.loops):
+            for layer in range(w.layers):
+                lb = layer % nlayers_buf
                 k = self.bf16[(lb, 0, loop)]
                 v = self.bf16[(lb, 1, loop)]
                 if ev is not None:
@@ -422,9 +430,10 @@ class Engine:
                 if ev is not None:
                     e1.record(stream)
                     ev.append((e0, e1, loop))
-            for loop in range(w.loops):
-                self.bf16[(lb, 0, loop)][:, :, T].copy_(self.kc[(layer, loop)], non_blocking=True)
-                self.bf16[(lb, 1, loop)][:, :, T].copy_(self.vc[(layer, loop)], non_blocking=True)
+                if loop == w.loops - 1:
+                    for lp in range(w.loops):
+                        self.bf16[(lb, 0, lp)][:, :, T].copy_(self.kc[(layer, lp)], non_blocking=True)
+                        self.bf16[(lb, 1, lp)][:, :, T].copy_(self.vc[(layer, lp)], non_blocking=True)
 
 
 def timed(fn, steps, warmup, stream, dist=None):
@@ -805,9 +814,10 @@ def main():
                                          f"back to back: {dec_ms:.3f} ms per step")},
             "decode_per_loop": per_loop,
             "step_launch": {"timed": f"one CUDA graph per step ({w.layers * w.loops} decode + "
-                                     f"{w.layers} append launches; each append on a second stream "
-                                     "after its layer's decode calls, joined at the end of the "
-                                     "step)",
+                                     f"{w.layers} append launches in the looped model's order: "
+                                     "loop 1 over every layer, then loop 2, ...; each append on a "
+                                     "second stream after its layer's final-loop decode, joined "
+                                     "at the end of the step)",
                             "timed_launch_count": w.layers * w.loops + w.layers,
                             "eager_ms_per_step": eager_ms,
                             "eager_tokens_per_s": job_tokens_per_s(ws, w.batch, eager_ms)},
