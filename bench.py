@@ -644,6 +644,8 @@ def main():
     ap.add_argument("--no-quant", action="store_true", help="skip the prefill quantise leg")
     ap.add_argument("--no-ablation", action="store_true",
                     help="skip the shared-vs-chained deep-recurrence decode ablation")
+    ap.add_argument("--only-quant", action="store_true",
+                    help="run only the prefill quantise leg and print its numbers (profiling)")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -653,6 +655,10 @@ def main():
     dev = torch.device("cuda", local)
     from residual_bit_kv_b200 import build
     build.build()
+    if args.only_quant:
+        print(json.dumps({"quantize": bench_quantize(dev, torch.cuda.current_stream(dev), args,
+                                                     peaks()[0])}))
+        return 0
     w = synth.WORKLOADS[WORKLOAD]
     if args.layers:
         w = w.replace(layers=args.layers)
