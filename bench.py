@@ -645,7 +645,8 @@ def main():
     ap.add_argument("--no-ablation", action="store_true",
                     help="skip the shared-vs-chained deep-recurrence decode ablation")
     ap.add_argument("--only-quant", action="store_true",
-                    help="run only the prefill quantise leg and print its numbers (profiling)")
+                    help="run only the prefill quantise leg and print its numbers (profiling; "
+                         "--batch then sets its batch)")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -959,6 +960,8 @@ def bench_quantize(dev, stream, args, hbm):
     HBM for the bytes the pass must move."""
     import residual_bit_kv_b200.librq as L
     w = synth.WORKLOADS[QUANT_WORKLOAD]
+    if args.only_quant and args.batch:
+        w = w.replace(batch=args.batch)
     T = w.tokens
     lay = L.make_layout(1, w.loops, w.batch, w.heads, w.head_dim, T, w.bits, w.group,
                         L.RQ_POLICY_LAST_LOOP)
