@@ -11,9 +11,13 @@
 // the scaling, the residual and the quantisation run as packed fp32
 // operations (each element of a pair rounded exactly as its scalar op).  The Hadamard transform runs its
 // first five butterfly stages inside the lane and the remaining log2(P)
-// stages across lanes with xor-shuffles; group min/max and the two dot
-// products of the LS coefficient are lane-serial followed by xor-shuffle
-// butterflies.  Every floating-point step that decides a stored bit uses an
+// stages across lanes with xor-shuffles; the group min/max are trees of
+// three-input min/max (exact in any order) and the two dot products of the
+// LS coefficient are lane-serial followed by xor-shuffle butterflies.  The
+// fused all-loops kernel streams its input rows through a per-warp
+// shared-memory ring filled by cp.async ahead of use; the per-loop kernel
+// rebuilds a residual's reference before loading the row, which keeps it at
+// two CTAs of 256 threads per SM.  Every floating-point step that decides a stored bit uses an
 // explicitly rounded intrinsic (no contraction), in this fixed order:
 //   Hadamard stages h = 1, 2, ..., D/2 with (a + b, a - b), then one multiply
 //   by fp32(1/sqrt(D)); dots: per-lane serial fma from +0, then butterflies
@@ -73,16 +77,15 @@ __device__ __forceinline__ void fwht_row(float2 (&v)[16], int slice) {
   }
 }
 
-// Row of bf16 x -> fp32 -> Z = H x (normalised) in one lane's 16 pairs.
+// One lane's 32 bf16 channels (four 16-byte pieces, channels 8i .. 8i + 7 in
+// piece i) -> fp32 pairs -> Z = H x (normalised) in the lane's 16 pairs.
 template <int D>
-__device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, int slice,
-                                            float rot_scale, float2 (&v)[16]) {
+__device__ __forceinline__ void rotate_pieces(const uint4 (&q)[4], bool active, int slice,
+                                              float rot_scale, float2 (&v)[16]) {
   if (active) {
-    const uint4* src = reinterpret_cast<const uint4*>(xrow + slice * 32);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 q = src[i];
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c0 = i * 8 + 2 * j;   // channels c0, c0 + 1
@@ -104,6 +107,73 @@ __device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, i
   const float2 rs = make_float2(rot_scale, rot_scale);
 #pragma unroll
   for (int k = 0; k < 16; ++k) v[k] = __fmul2_rn(v[k], rs);
+}
+
+// Row of bf16 x (global memory) -> Z = H x in one lane's 16 pairs.
+template <int D>
+__device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, int slice,
+                                            float rot_scale, float2 (&v)[16]) {
+  uint4 q[4];
+  if (active) {
+    const uint4* src = reinterpret_cast<const uint4*>(xrow + slice * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = src[i];
+  }
+  rotate_pieces<D>(q, active, slice, rot_scale, v);
+}
+
+// Input staging of the fused kernel: each warp streams its rows through a
+// private ring of kQStages shared-memory slots of 32 x 64 bytes (the RPW
+// rows of one loop: 8 rows of 128 channels or 16 rows of 64), filled by
+// 16-byte cp.async copies kQStages - 1 jobs ahead of the job being
+// quantised, so every warp keeps about 6 KB of input in flight without
+// holding it in registers.  A copy instruction covers 512 contiguous bytes
+// (lane l: bytes 16 l of each 512-byte quarter); piece pi of the slice
+// that lane l of the row reads lands at pi ^ ((l >> 1) & 3), so the four
+// 16-byte reads of a quarter-warp hit eight distinct bank groups.
+constexpr int kQStages = 4;
+constexpr int kQSlotBytes = 2048;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Copies `rows` (<= RPW) consecutive rows of D bf16 from src into a slot.
+template <int D>
+__device__ __forceinline__ void stage_rows(uint32_t slot, const unsigned char* src, int rows,
+                                           int lane) {
+  constexpr int P = D / 32;
+  const int nbytes = rows * D * 2;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int o = i * 512 + lane * 16;
+    if (o < nbytes) {
+      const int rho = o / (2 * D), b = o % (2 * D);
+      const int sg = b / 64, pi = (b % 64) / 16;
+      const int l = rho * P + sg;
+      cp_async16(slot + rho * 2 * D + sg * 64 + ((pi ^ ((l >> 1) & 3)) << 4), src + o);
+    }
+  }
+}
+
+// This lane's four pieces of its row from a filled slot.
+template <int D>
+__device__ __forceinline__ void read_slot(uint32_t slot, int lane, uint4 (&q)[4]) {
+  constexpr int P = D / 32;
+  const uint32_t a = slot + (lane / P) * 2 * D + (lane % P) * 64;
+  const int f = (lane >> 1) & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(q[i].x), "=r"(q[i].y), "=r"(q[i].z), "=r"(q[i].w)
+                 : "r"(a + ((i ^ f) << 4)));
 }
 
 // Stored levels fma(s~, code, z~) of one lane's 32 channels of a component
@@ -231,12 +301,14 @@ __host__ __device__ constexpr uint32_t magic_pack_offset(int word) {
 }
 
 // Codes of one lane's 32 values packed into BITS words: u = (x - z~) * (1/s~)
-// (clamped to [0, 2^b - 1] when CLAMP); u + 1.5 * 2^23 rounds it to the
+// clamped to [0, 2^b - 1] (CLAMP 2), or to [0, inf) when the group's ends are
+// known to map into [-1/2, 2^b - 1/2) (CLAMP 1: every u then rounds into
+// [0, 2^b - 1], so the upper bound changes nothing); u + 1.5 * 2^23 rounds it to the
 // nearest integer (ties to even), held in the low mantissa bits of a float
 // whose bit pattern is kRoundMagicBits + code; packing adds that pattern
 // shifted into place (the magic offsets are subtracted up front), one
 // integer multiply-add per code.  LEVELS: `levels` receives fma(s~, code, z~).
-template <int BITS, bool CLAMP, bool LEVELS>
+template <int BITS, int CLAMP, bool LEVELS>
 __device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, float2 iv,
                                            const float (&st)[2], const float (&zt)[2],
                                            uint32_t (&words)[BITS], float2* levels) {
@@ -247,9 +319,15 @@ __device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, flo
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     float2 u = __fmul2_rn(__fadd2_rn(v[k], nz), iv);
-    if constexpr (CLAMP) {
+    if constexpr (CLAMP == 2) {
       u.x = fminf(fmaxf(u.x, 0.0f), static_cast<float>(QMAX));
       u.y = fminf(fmaxf(u.y, 0.0f), static_cast<float>(QMAX));
+    } else {
+      // the group's ends already map into [-1/2, 2^b - 1/2): only the
+      // lower bound is applied (it changes no code there), which also keeps
+      // the rounding add a separate operation from the multiply
+      u.x = fmaxf(u.x, 0.0f);
+      u.y = fmaxf(u.y, 0.0f);
     }
     const float2 r = __fadd2_rn(u, mg);
     const uint32_t b0 = __float_as_uint(r.x), b1 = __float_as_uint(r.y);
@@ -259,6 +337,40 @@ __device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, flo
       const float2 cf = __fadd2_rn(r, make_float2(-kRoundMagic, -kRoundMagic));   // exact codes
       levels[k] = __ffma2_rn(make_float2(st[0], st[1]), cf, make_float2(zt[0], zt[1]));
     }
+  }
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// In place: mn[0] = min and mx[0] = max of the N values, by passes of
+// three-input operations (a pass maps N values to ceil(N / 3)).
+template <int N>
+__device__ __forceinline__ void reduce_min_max(float* mn, float* mx) {
+  if constexpr (N > 1) {
+    constexpr int M = (N + 2) / 3;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      if (3 * i + 2 < N) {
+        mn[i] = min3f(mn[3 * i], mn[3 * i + 1], mn[3 * i + 2]);
+        mx[i] = max3f(mx[3 * i], mx[3 * i + 1], mx[3 * i + 2]);
+      } else if (3 * i + 1 < N) {
+        mn[i] = fminf(mn[3 * i], mn[3 * i + 1]);
+        mx[i] = fmaxf(mx[3 * i], mx[3 * i + 1]);
+      } else {
+        mn[i] = mn[3 * i];
+        mx[i] = mx[3 * i];
+      }
+    }
+    reduce_min_max<M>(mn, mx);
   }
 }
 
@@ -274,28 +386,26 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   constexpr int NG = G < 32 ? 2 : 1;        // group parts per lane
   constexpr int LPG = G > 32 ? G / 32 : 1;  // lanes sharing a group
-  float st[2], zt[2], inv[2];
+  float st[2], zt[2], inv[2], gmn[2], gmx[2];
   uint32_t metaw[2];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
-    // min / max as trees (exact in any order; short dependency chains)
+    // min / max as trees of three-input operations (exact in any order)
     float tn[16], tx[16];
+    if constexpr (NG == 2) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      if constexpr (NG == 2) {
-        tn[k] = tx[k] = gi == 0 ? v[k].x : v[k].y;
-      } else {
-        tn[k] = fminf(v[k].x, v[k].y);
-        tx[k] = fmaxf(v[k].x, v[k].y);
+      for (int k = 0; k < 16; ++k) tn[k] = tx[k] = gi == 0 ? v[k].x : v[k].y;
+      reduce_min_max<16>(tn, tx);
+    } else {
+      float un[32], ux[32];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        un[k] = ux[k] = v[k].x;
+        un[k + 16] = ux[k + 16] = v[k].y;
       }
-    }
-#pragma unroll
-    for (int w = 8; w >= 1; w >>= 1) {
-#pragma unroll
-      for (int k = 0; k < w; ++k) {
-        tn[k] = fminf(tn[k], tn[k + w]);
-        tx[k] = fmaxf(tx[k], tx[k + w]);
-      }
+      reduce_min_max<32>(un, ux);
+      tn[0] = un[0];
+      tx[0] = ux[0];
     }
     float mn = tn[0], mx = tx[0];
 #pragma unroll
@@ -305,6 +415,8 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     mn = __fadd_rn(mn, 0.0f);   // a zero end of the range is +0
     mx = __fadd_rn(mx, 0.0f);
+    gmn[gi] = mn;
+    gmx[gi] = mx;
     const float s = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
     if (m16) {
       // 16-bit metadata: scale byte nearest to max(s, |mn| / 15.875), offset
@@ -335,6 +447,16 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
     }
     inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
   }
+  // (x - z~) * (1/s~) is monotone in x: when both ends of every group of the
+  // warp map into [-1/2, 2^b - 1/2), the upper clamp can change no code
+  bool in_range = true;
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    const float ulo = __fmul_rn(__fsub_rn(gmn[gi], zt[gi]), inv[gi]);
+    const float uhi = __fmul_rn(__fsub_rn(gmx[gi], zt[gi]), inv[gi]);
+    in_range = in_range && ulo >= -0.5f && uhi < static_cast<float>(QMAX) + 0.5f;
+  }
+  const bool lower_only = __all_sync(0xffffffffu, in_range);
   if constexpr (NG == 1) {
     st[1] = st[0];
     zt[1] = zt[0];
@@ -342,10 +464,17 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   }
   const float2 nz = make_float2(-zt[0], -zt[1]), iv = make_float2(inv[0], inv[1]);
   uint32_t words[BITS];
-  if (levels == nullptr)
-    pack_codes<BITS, true, false>(v, nz, iv, st, zt, words, levels);
-  else
-    pack_codes<BITS, true, true>(v, nz, iv, st, zt, words, levels);
+  if (levels == nullptr) {
+    if (lower_only)
+      pack_codes<BITS, 1, false>(v, nz, iv, st, zt, words, levels);
+    else
+      pack_codes<BITS, 2, false>(v, nz, iv, st, zt, words, levels);
+  } else {
+    if (lower_only)
+      pack_codes<BITS, 1, true>(v, nz, iv, st, zt, words, levels);
+    else
+      pack_codes<BITS, 2, true>(v, nz, iv, st, zt, words, levels);
+  }
   if (!active) return;
   uint32_t* cw = codes_row + slice * BITS;
   if constexpr (BITS == 4) {
@@ -407,7 +536,7 @@ __device__ __forceinline__ __nv_bfloat16 ls_residual(float2 (&v)[16], const floa
 }
 
 template <int D, int BITS, int G>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_kernel(const __grid_constant__ QuantParams p) {
   constexpr int P = D / 32;
   constexpr int RPW = 32 / P;
@@ -420,17 +549,15 @@ __global__ void __launch_bounds__(kQuantThreads)
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    float2 v[16];
-    load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
-
     const int64_t bhi = active ? row / p.n : 0;
     const int64_t t = p.t0 + (active ? row % p.n : 0);
-
+    float2 v[16];
     if (p.dst.has_alpha) {
-      // Fixed mean removed first [RQ App. G.2]; least-squares coefficient
-      // against the reconstructed reference [RQ §3.2 scaling coefficient,
-      // App. G.1], then the residual.
-      if (p.dst.mean != nullptr && active) sub_mean(p.dst, bhi, slice, D, v);
+      // The reference is rebuilt from the cache first (its temporaries are
+      // dead before the input row is loaded).  Fixed mean removed from the
+      // input [RQ App. G.2]; least-squares coefficient against the
+      // reconstructed reference [RQ §3.2 scaling coefficient, App. G.1],
+      // then the residual.
       float2 ref[16];
       if (active) {
         chain_slice(p.ref, p.nref, bhi, p.nblk, t, slice, D, ref);
@@ -438,11 +565,15 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
         for (int k = 0; k < 16; ++k) ref[k] = make_float2(0.0f, 0.0f);
       }
+      load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
+      if (p.dst.mean != nullptr && active) sub_mean(p.dst, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
         *rec_alpha(comp_record(p.dst, bhi, p.nblk, t), D, BITS, G, static_cast<int>(t % kBlock),
                    p.dst.meta16 ? 2 : 4) =
             __bfloat16_as_ushort(ab);
+    } else {
+      load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
     }
     unsigned char* rec = comp_record(p.dst, bhi, p.nblk, t);
     const int i = static_cast<int>(t % kBlock);
@@ -497,6 +628,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_loops_kernel(const __grid_constant__ QuantLoopsParams p) {
   constexpr int P = D / 32;
   constexpr int RPW = 32 / P;
+  static_assert(RPW * D * 2 == kQSlotBytes, "a slot holds one job of RPW rows");
+  extern __shared__ __align__(128) unsigned char qsmem[];
   const int side = blockIdx.y;
   const uint16_t* xs = p.x[side];
   if (xs == nullptr) return;
@@ -507,21 +640,55 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) +
                        (threadIdx.x >> 5);
   const int a = p.anchor;
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(qsmem)) +
+                        (threadIdx.x >> 5) * (kQStages * kQSlotBytes);
+  // Job j of this warp: rows base_j .. base_j + RPW - 1 of loop li_j (li 0 is
+  // the anchor, li k >= 1 is p.order[k - 1]); jobs run row group by row
+  // group, every loop of a group in turn.
+  int64_t is_base = warp * RPW;
+  int is_li = 0, is_slot = 0;
+  auto issue_next = [&]() {
+    if (is_base < total) {
+      const int r = is_li == 0 ? a : p.order[is_li - 1];
+      const int64_t left = total - is_base;
+      stage_rows<D>(ring + is_slot * kQSlotBytes,
+                    reinterpret_cast<const unsigned char*>(
+                        xs + (static_cast<int64_t>(r) * total + is_base) * D),
+                    left < RPW ? static_cast<int>(left) : RPW, lane);
+    }
+    cp_async_commit();   // one group per job, empty past the end
+    if (++is_li == p.nloops) {
+      is_li = 0;
+      is_base += nwarps * RPW;
+    }
+    is_slot = is_slot + 1 == kQStages ? 0 : is_slot + 1;
+  };
+#pragma unroll
+  for (int s = 0; s + 1 < kQStages; ++s) issue_next();
+  int slot = 0;
+  // the job in `slot` has landed (this lane's copies, then the warp's); the
+  // slot read in the previous job is free again and takes the next issue
+  auto next_input = [&](bool active, float2 (&v)[16]) {
+    cp_async_wait<kQStages - 2>();
+    __syncwarp();
+    issue_next();
+    uint4 q[4];
+    read_slot<D>(ring + slot * kQSlotBytes, lane, q);
+    slot = slot + 1 == kQStages ? 0 : slot + 1;
+    rotate_pieces<D>(q, active, slice, p.rot_scale, v);
+  };
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    const int64_t r_in = active ? row : 0;
     const int64_t bhi = active ? row / p.n : 0;
     const int64_t t = p.t0 + (active ? row % p.n : 0);
     float2 ref[16], v[16];
-    load_rotate<D>(xs + (static_cast<int64_t>(a) * total + r_in) * D, active, slice, p.rot_scale,
-                   v);
+    next_input(active, v);
     quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, v, slice, active, ref);
     for (int k = 0; k + 1 < p.nloops; ++k) {
       const int r = p.order[k];
       const Comp& c = p.dst[side][r];
-      load_rotate<D>(xs + (static_cast<int64_t>(r) * total + r_in) * D, active, slice,
-                     p.rot_scale, v);
+      next_input(active, v);
       if (c.mean != nullptr && active) sub_mean(c, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
@@ -538,6 +705,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
       }
     }
   }
+  cp_async_wait<0>();   // nothing left in flight into the ring at exit
 }
 
 template <int D>
@@ -620,19 +788,23 @@ cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
   return cudaErrorInvalidValue;
 }
 
+template <int D, bool CHAINED>
+cudaError_t launch_loops(const QuantLoopsParams& p, dim3 grid, cudaStream_t s) {
+  constexpr int smem = (kQuantThreads / 32) * kQStages * kQSlotBytes;
+  const cudaError_t e = cudaFuncSetAttribute(quantize_loops_kernel<D, CHAINED>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  quantize_loops_kernel<D, CHAINED><<<grid, kQuantThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_loops(const QuantLoopsParams& p, int D, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(p.bh) * p.n;
   if (rows == 0) return cudaSuccess;
   const dim3 grid(quant_grid(rows, D), 2);
-  if (D == 64)
-    p.chained ? quantize_loops_kernel<64, true><<<grid, kQuantThreads, 0, s>>>(p)
-              : quantize_loops_kernel<64, false><<<grid, kQuantThreads, 0, s>>>(p);
-  else if (D == 128)
-    p.chained ? quantize_loops_kernel<128, true><<<grid, kQuantThreads, 0, s>>>(p)
-              : quantize_loops_kernel<128, false><<<grid, kQuantThreads, 0, s>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (D == 64) return p.chained ? launch_loops<64, true>(p, grid, s) : launch_loops<64, false>(p, grid, s);
+  if (D == 128) return p.chained ? launch_loops<128, true>(p, grid, s) : launch_loops<128, false>(p, grid, s);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_dequantize(const DequantParams& p, int D, cudaStream_t s) {
