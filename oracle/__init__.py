@@ -132,6 +132,14 @@ def lib() -> ctypes.CDLL:
                                            None),
             "rqo_encode_residual_rows_ex": ([_P, _P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P,
                                              _P], None),
+            "rqo_rotate_dense_row": ([_P, _P, _I, _P, _P], None),
+            "rqo_rotate_dense_rows": ([_P, _P, _I64, _I, _P, _P], None),
+            "rqo_quantize_box": ([_P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P], None),
+            "rqo_quantize_box_rows": ([_P, _P, _P, _I64, _I, _I, _I, _P, _P, _P, _P, _P], None),
+            "rqo_encode_residual_box": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P,
+                                         _P, _P, _P], None),
+            "rqo_encode_residual_box_rows": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P,
+                                              _P, _P, _P, _P, _P], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(h, name)
@@ -455,6 +463,172 @@ def decode_attention(khat: np.ndarray, vhat: np.ndarray, q_bits: np.ndarray,
         for h in range(H):
             out[b, h] = attention(q[b, h], khat[b, h, :n], vhat[b, h, :n], kc[b, h], vc[b, h],
                                   scale)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Dense rotation [RQ §3.3, App. G.1, App. G.2]
+# --------------------------------------------------------------------------
+
+def rotate_dense(u: np.ndarray, x: np.ndarray):
+    """z = U x for rows x (bf16 bits [n, D]) with U binary16 bits [D, D] (row i
+    = output channel i): x is rounded to binary16 and the exact products are
+    summed in fp64.  Returns (z fp64 [n, D], bound fp64 [n, D]): every order of
+    fp32 accumulation of those products lands within bound of z."""
+    u = np.ascontiguousarray(u, dtype=np.uint16)
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    D = _check_dim(x.shape[-1])
+    assert u.shape == (D, D)
+    n = x.size // D
+    z = np.zeros((n, D), np.float64)
+    b = np.zeros((n, D), np.float64)
+    lib().rqo_rotate_dense_rows(_ptr(u), _ptr(x), n, D, _ptr(z), _ptr(b))
+    return z.reshape(x.shape), b.reshape(x.shape)
+
+
+def f32_box(z: np.ndarray, bound: np.ndarray):
+    """fp32 (lo, hi, mid): lo <= z - bound and hi >= z + bound as fp32 values,
+    mid = fp32 rounding of z."""
+    lo = np.nextafter((z - bound).astype(np.float32), np.float32(-np.inf))
+    hi = np.nextafter((z + bound).astype(np.float32), np.float32(np.inf))
+    return (np.ascontiguousarray(lo), np.ascontiguousarray(hi),
+            np.ascontiguousarray(z.astype(np.float32)))
+
+
+def quantize_box(lo: np.ndarray, hi: np.ndarray, mid: np.ndarray, bits: int, group: int):
+    """Interval quantiser over rows [n, D] (binary16 metadata): (codes, meta,
+    deq, meta_ok [n, D/group], code_ok [n, D]); the flags mark the decisions
+    every fp32 row inside the box shares."""
+    lo, hi, mid = (np.ascontiguousarray(a, dtype=np.float32) for a in (lo, hi, mid))
+    D = _check_dim(mid.shape[-1])
+    n = mid.size // D
+    codes = np.zeros((n, D * bits // 32), np.uint32)
+    meta = np.zeros((n, D // group), np.uint32)
+    deq = np.zeros((n, D), np.float32)
+    mok = np.zeros((n, D // group), np.uint8)
+    cok = np.zeros((n, D), np.uint8)
+    lib().rqo_quantize_box_rows(_ptr(lo), _ptr(hi), _ptr(mid), n, D, bits, group, _ptr(codes),
+                                _ptr(meta), _ptr(deq), _ptr(mok), _ptr(cok))
+    return codes, meta, deq, mok.astype(bool), cok.astype(bool)
+
+
+def encode_side_dense(x: np.ndarray, u: np.ndarray, heads: int, tokens: int,
+                      bits: Sequence[int], group: Sequence[int], policy: str = POLICY_LAST,
+                      unit_alpha: bool = False,
+                      mu: Optional[np.ndarray] = None) -> List[Dict[str, np.ndarray]]:
+    """encode_side with the dense rotation of one (layer, K|V) side
+    [RQ §3.3, App. G.2]: u binary16 bits [heads, D, D], one matrix per head
+    shared by every loop; rows of x [L, N, D] are (b, h, t) with `tokens` rows
+    per (b, h).  Binary16 metadata.
+
+    The accumulation order of the rotation is not fixed by the pages, so the
+    encoder works on the box of fp32 rows that any order can produce
+    (rotate_dense's bound): 'codes', 'meta', 'alpha', 'zhat' are those of the
+    fp32-rounded exact rotation, and 'code_ok', 'meta_ok', 'alpha_ok' mark the
+    decisions that every row of the box shares (a row whose reference is not
+    fully determined gets no flag)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    L, N, D = x.shape
+    _check_dim(D)
+    u = np.ascontiguousarray(u, dtype=np.uint16)
+    assert u.shape == (heads, D, D) and N % (heads * tokens) == 0
+    head_of = (np.arange(N) // tokens) % heads
+    boxes = []
+    for l in range(L):
+        z = np.zeros((N, D), np.float64)
+        bd = np.zeros((N, D), np.float64)
+        for h in range(heads):
+            rows = np.nonzero(head_of == h)[0]
+            zh, bh = rotate_dense(u[h], x[l][rows])
+            z[rows], bd[rows] = zh, bh
+        boxes.append(f32_box(z, bd))
+    out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
+    a = anchor_loop(L, policy)
+    lo, hi, mid = boxes[a]
+    codes, meta, deq, mok, cok = quantize_box(lo, hi, mid, bits[a], group[a])
+    out[a] = {"codes": codes, "meta": meta, "alpha": None, "zhat": deq,
+              "meta_ok": mok, "code_ok": cok, "alpha_ok": None,
+              "clean": mok.all(axis=1) & cok.all(axis=1)}
+    for r in encode_order(L, policy):
+        ref_enc = out[reference_loop(L, r, policy)]
+        lo, hi, mid = boxes[r]
+        G = D // group[r]
+        enc = {"codes": np.zeros((N, D * bits[r] // 32), np.uint32),
+               "meta": np.zeros((N, G), np.uint32),
+               "alpha": np.zeros(N, np.uint16),
+               "zhat": np.zeros((N, D), np.float32)}
+        aok = np.zeros(N, np.uint8)
+        mok = np.zeros((N, G), np.uint8)
+        cok = np.zeros((N, D), np.uint8)
+        m = None if mu is None else np.ascontiguousarray(mu[r], dtype=np.float32)
+        lib().rqo_encode_residual_box_rows(
+            _ptr(lo), _ptr(hi), _ptr(mid), _ptr(np.ascontiguousarray(ref_enc["zhat"])),
+            None if m is None else _ptr(m), N, D, bits[r], group[r], int(unit_alpha),
+            _ptr(enc["codes"]), _ptr(enc["meta"]), _ptr(enc["alpha"]), _ptr(enc["zhat"]),
+            _ptr(aok), _ptr(mok), _ptr(cok))
+        ref_clean = ref_enc["clean"]
+        enc["alpha_ok"] = aok.astype(bool) & ref_clean
+        enc["meta_ok"] = mok.astype(bool) & ref_clean[:, None]
+        enc["code_ok"] = cok.astype(bool) & ref_clean[:, None]
+        enc["clean"] = enc["alpha_ok"] & enc["meta_ok"].all(axis=1) & enc["code_ok"].all(axis=1)
+        out[r] = enc
+    return out  # type: ignore[return-value]
+
+
+def f16_bits_to_f64(a: np.ndarray) -> np.ndarray:
+    return np.asarray(a, np.uint16).view(np.float16).astype(np.float64)
+
+
+def reconstruct_dense(encs, loop, bits, group, u: np.ndarray, heads: int, tokens: int,
+                      policy=POLICY_LAST, mu=None) -> np.ndarray:
+    """fp64 reconstruction in the original domain under the dense rotation:
+    X^ = U^T Z^ per row, U the row's head matrix [RQ App. G.2]."""
+    z = reconstruct_rotated(encs, loop, bits, group, policy, mu)
+    N = z.shape[0]
+    head_of = (np.arange(N) // tokens) % heads
+    uf = f16_bits_to_f64(u)
+    out = np.zeros_like(z)
+    for h in range(heads):
+        rows = head_of == h
+        out[rows] = z[rows] @ uf[h]          # row form of U^T z
+    return out
+
+
+def rotate_query_dense(q_bits: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """Exact U q of bf16 queries rounded to binary16 (the pages' FP16 inputs):
+    q_bits [..., D], u [D, D] binary16 bits -> fp64."""
+    qh = f16_bits_to_f64(np.asarray(
+        [f32_to_f16_bits(float(v)) for v in bf16_bits_to_f64(q_bits).ravel()],
+        np.uint16)).reshape(np.shape(q_bits))
+    return qh @ f16_bits_to_f64(u).T
+
+
+def decode_attention_dense(zk: np.ndarray, zv: np.ndarray, q_bits: np.ndarray,
+                           seq_lens: Sequence[int], kcur_bits: np.ndarray,
+                           vcur_bits: np.ndarray, uk: np.ndarray, uv: np.ndarray,
+                           scale: Optional[float] = None) -> np.ndarray:
+    """fp64 decode attention under dense rotations [RQ App. G.2]: scores
+    (U_K q~) . Z^_K with q~ the query rounded to binary16, values
+    U_V^T sum_t p_t Z^_V,t; the current token's k_cur / v_cur stay in the
+    original domain.  zk, zv: fp64 rotated reconstructions [B, H, T, D];
+    uk, uv: binary16 bits [H, D, D]; the rest as decode_attention."""
+    B, H, T, D = zk.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    kc = bf16_bits_to_f64(kcur_bits)
+    vc = bf16_bits_to_f64(vcur_bits)
+    out = np.zeros((B, H, D), np.float64)
+    for b in range(B):
+        n = int(seq_lens[b])
+        for h in range(H):
+            qr = rotate_query_dense(q_bits[b, h], uk[h])
+            s = np.concatenate([zk[b, h, :n] @ qr, [bf16_bits_to_f64(q_bits[b, h]) @ kc[b, h]]])
+            # the current token's score uses the unrotated query
+            s = s * scale
+            p = np.exp(s - s.max())
+            acc = p[:n] @ zv[b, h, :n]
+            o = f16_bits_to_f64(uv[h]).T @ acc + p[n] * vc[b, h]
+            out[b, h] = o / p.sum()
     return out
 
 

@@ -506,6 +506,167 @@ void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Dense rotation [RQ §3.3, App. G.1, App. G.2]                              */
+/* ------------------------------------------------------------------------ */
+
+/* z = U x for one row.  U is D x D in binary16, row i giving output channel
+ * i; x is the bf16 row rounded to binary16 (the pages: rotation matrices
+ * stored in FP16, multiplication with FP16 inputs and FP32 accumulation).
+ * A product of two binary16 values is exact in binary32 and in fp64.  The
+ * pages fix the accumulator's precision but not the order of its D
+ * additions, so the oracle returns the sum formed in fp64 together with a
+ * bound that every order of fp32 accumulation of the exact products meets:
+ *   bound_i = D 2^-23 sum_j |U_ij x_j|  (+ the fp64 sum's own D 2^-53 share),
+ * twice the textbook (D - 1) 2^-24, which also covers adders that truncate. */
+void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z,
+                          double* bound) {
+  double xh[256];
+  for (int j = 0; j < D; ++j) xh[j] = rqo_f16_to_f32(rqo_f32_to_f16(rqo_bf16_to_f32(x[j])));
+  for (int i = 0; i < D; ++i) {
+    double acc = 0.0, mag = 0.0;
+    for (int j = 0; j < D; ++j) {
+      const double t = (double)rqo_f16_to_f32(u[(size_t)i * D + j]) * xh[j];
+      acc += t;
+      mag += fabs(t);
+    }
+    z[i] = acc;
+    bound[i] = mag * ((double)D * 0x1p-23 + (double)D * 0x1p-53);
+  }
+}
+
+void rqo_rotate_dense_rows(const uint16_t* u, const uint16_t* x, int64_t n, int D,
+                           double* z, double* bound) {
+  for (int64_t r = 0; r < n; ++r)
+    rqo_rotate_dense_row(u, x + r * D, D, z + r * D, bound + r * D);
+}
+
+/* Interval form of rqo_quantize for a row known only to lie in the box
+ * [lo_i, hi_i]: which decisions every row of the box shares.  Each step is
+ * monotone in its inputs: the group min and max are non-decreasing in every
+ * element, the fp32 scale (mx - mn) / qmax is non-decreasing in mx and
+ * non-increasing in mn, binary16 rounding, the code's fsub / fmul by a
+ * non-negative inverse, the clamp and rint are non-decreasing.  So the
+ * group's metadata is the same for the whole box (meta_ok) when the ends of
+ * the offset's and the scale's intervals round to the same binary16 value,
+ * and a channel's code is the same (code_ok) when, besides, both ends of its
+ * own interval give the same code.  words / meta / deq are those of mid. */
+void rqo_quantize_box(const float* lo, const float* hi, const float* mid, int D,
+                      int bits, int group, uint32_t* words, uint32_t* meta, float* deq,
+                      uint8_t* meta_ok, uint8_t* code_ok) {
+  const int qmax = (1 << bits) - 1;
+  rqo_quantize(mid, D, bits, group, words, meta, deq);
+  for (int g0 = 0, j = 0; g0 < D; g0 += group, ++j) {
+    float mn_lo = lo[g0], mn_hi = hi[g0], mx_lo = lo[g0], mx_hi = hi[g0];
+    for (int i = g0 + 1; i < g0 + group; ++i) {
+      if (lo[i] < mn_lo) mn_lo = lo[i];
+      if (hi[i] < mn_hi) mn_hi = hi[i];
+      if (lo[i] > mx_lo) mx_lo = lo[i];
+      if (hi[i] > mx_hi) mx_hi = hi[i];
+    }
+    mn_lo = mn_lo + 0.0f;
+    mn_hi = mn_hi + 0.0f;
+    mx_lo = mx_lo + 0.0f;
+    mx_hi = mx_hi + 0.0f;
+    const float s_lo = (mx_lo - mn_hi) / (float)qmax;
+    const float s_hi = (mx_hi - mn_lo) / (float)qmax;
+    const int ok = rqo_f32_to_f16(mn_lo) == rqo_f32_to_f16(mn_hi) &&
+                   rqo_f32_to_f16(s_lo) == rqo_f32_to_f16(s_hi);
+    meta_ok[j] = (uint8_t)ok;
+    const float st = rqo_f16_to_f32((uint16_t)(meta[j] & 0xFFFFu));
+    const float zt = rqo_f16_to_f32((uint16_t)(meta[j] >> 16));
+    const float inv = (st > 0.0f) ? 1.0f / st : 0.0f;
+    for (int i = g0; i < g0 + group; ++i) {
+      float ua = (lo[i] - zt) * inv, ub = (hi[i] - zt) * inv;
+      if (ua < 0.0f) ua = 0.0f;
+      if (ua > (float)qmax) ua = (float)qmax;
+      if (ub < 0.0f) ub = 0.0f;
+      if (ub > (float)qmax) ub = (float)qmax;
+      code_ok[i] = (uint8_t)(ok && rintf(ua) == rintf(ub));
+    }
+  }
+}
+
+/* Interval form of the residual encoder (rqo_encode_residual_rot_ex with
+ * binary16 metadata) for a row z in the box [lo, hi] and an exactly known
+ * reference (and mean).  The mean's fsub is non-decreasing in z.  Any row of
+ * the box has a lane-serial fp32 dot <z - mu, ref> within
+ *   sum_i |ref_i| (hi_i - lo_i) + 35 2^-24 sum_i (|mid_i - mu_i| + hi_i - lo_i) |ref_i|
+ * of the fp64 dot of mid (32 serial fma roundings and at most 3 butterfly
+ * additions, each within 2^-24 of its partial sum); d_zr / d_rr is monotone
+ * in d_zr (d_rr > 0 is the same fp32 value for every row: ref is known), so
+ * alpha~ is the same for the whole box (alpha_ok) when bf16 rounding maps
+ * the quotients of the ends of that interval to one value.  With alpha~
+ * fixed the residual fma(-alpha~, ref_i, z_i) is non-decreasing in z_i and its
+ * box is the image of the ends; rqo_quantize_box takes it from there.
+ * With alpha~ not unique every flag of the row is cleared. */
+void rqo_encode_residual_box(const float* lo, const float* hi, const float* mid,
+                             const float* ref, const float* mu, int D, int bits, int group,
+                             int unit_alpha, uint32_t* words, uint32_t* meta,
+                             uint16_t* alpha, float* zhat, uint8_t* alpha_ok,
+                             uint8_t* meta_ok, uint8_t* code_ok) {
+  rqo_encode_residual_rot_ex(mid, ref, mu, D, bits, group, unit_alpha, 0, words, meta, alpha,
+                             zhat);
+  const float at = rqo_bf16_to_f32(*alpha);
+  int aok = 1;
+  if (!unit_alpha) {
+    const float d_rr = rqo_dot_f32(ref, ref, D);
+    if (d_rr > 0.0f) {
+      double c = 0.0, w = 0.0, m = 0.0;
+      for (int i = 0; i < D; ++i) {
+        const double zc = mu ? (double)mid[i] - (double)mu[i] : (double)mid[i];
+        const double wd = (double)hi[i] - (double)lo[i];
+        c += zc * (double)ref[i];
+        w += fabs((double)ref[i]) * wd;
+        m += (fabs(zc) + wd) * fabs((double)ref[i]);
+      }
+      const double dev = w + 35.0 * 0x1p-24 * m + (double)D * 0x1p-52 * m;
+      /* fp32 values bracketing every attainable d_zr */
+      const float dlo = nextafterf((float)(c - dev), -INFINITY);
+      const float dhi = nextafterf((float)(c + dev), INFINITY);
+      aok = rqo_f32_to_bf16(dlo / d_rr) == rqo_f32_to_bf16(dhi / d_rr);
+    }
+  }
+  *alpha_ok = (uint8_t)aok;
+  float elo[256], ehi[256], emid[256], deq[256];
+  uint32_t w2[64], m2[256];
+  for (int i = 0; i < D; ++i) {
+    const float zl = mu ? lo[i] - mu[i] : lo[i];
+    const float zh = mu ? hi[i] - mu[i] : hi[i];
+    const float zm = mu ? mid[i] - mu[i] : mid[i];
+    elo[i] = fmaf(-at, ref[i], zl);
+    ehi[i] = fmaf(-at, ref[i], zh);
+    emid[i] = fmaf(-at, ref[i], zm);
+  }
+  rqo_quantize_box(elo, ehi, emid, D, bits, group, w2, m2, deq, meta_ok, code_ok);
+  if (!aok) {
+    for (int j = 0; j < D / group; ++j) meta_ok[j] = 0;
+    for (int i = 0; i < D; ++i) code_ok[i] = 0;
+  }
+}
+
+void rqo_quantize_box_rows(const float* lo, const float* hi, const float* mid, int64_t n,
+                           int D, int bits, int group, uint32_t* words, uint32_t* meta,
+                           float* deq, uint8_t* meta_ok, uint8_t* code_ok) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r)
+    rqo_quantize_box(lo + r * D, hi + r * D, mid + r * D, D, bits, group, words + r * W,
+                     meta + r * G, deq + r * D, meta_ok + r * G, code_ok + r * D);
+}
+
+void rqo_encode_residual_box_rows(const float* lo, const float* hi, const float* mid,
+                                  const float* ref, const float* mu, int64_t n, int D,
+                                  int bits, int group, int unit_alpha, uint32_t* words,
+                                  uint32_t* meta, uint16_t* alpha, float* zhat,
+                                  uint8_t* alpha_ok, uint8_t* meta_ok, uint8_t* code_ok) {
+  const int W = D * bits / 32, G = D / group;
+  for (int64_t r = 0; r < n; ++r)
+    rqo_encode_residual_box(lo + r * D, hi + r * D, mid + r * D, ref + r * D,
+                            mu ? mu + r * D : NULL, D, bits, group, unit_alpha, words + r * W,
+                            meta + r * G, alpha + r, zhat + r * D, alpha_ok + r,
+                            meta_ok + r * G, code_ok + r * D);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Storage and access accounting [RQ §5.1, App. A.3, App. D]                */
 /* ------------------------------------------------------------------------ */
 

@@ -177,6 +177,33 @@ void rqo_encode_residual_rows_ex(const uint16_t* x, const float* ref,
  * App. G.1]: s_t = scale * q.k_t for t < T, plus the current token
  * s_cur = scale * q.k_cur; p = softmax(s); out = sum_t p_t v_t + p_cur v_cur.
  * khat and vhat are T x D row-major (original domain). */
+/* Dense rotation [RQ §3.3, App. G.2]: z = U x with U binary16 (row i =
+ * output channel i) and x rounded from bf16 to binary16; z in fp64 and, per
+ * channel, a bound on the error of any order of fp32 accumulation. */
+void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z,
+                          double* bound);
+void rqo_rotate_dense_rows(const uint16_t* u, const uint16_t* x, int64_t n, int D,
+                           double* z, double* bound);
+/* Interval forms of the quantiser and of the residual encoder (binary16
+ * metadata): the decisions shared by every row of the box [lo, hi]. */
+void rqo_quantize_box(const float* lo, const float* hi, const float* mid, int D,
+                      int bits, int group, uint32_t* words, uint32_t* meta, float* deq,
+                      uint8_t* meta_ok, uint8_t* code_ok);
+void rqo_encode_residual_box(const float* lo, const float* hi, const float* mid,
+                             const float* ref, const float* mu, int D, int bits, int group,
+                             int unit_alpha, uint32_t* words, uint32_t* meta,
+                             uint16_t* alpha, float* zhat, uint8_t* alpha_ok,
+                             uint8_t* meta_ok, uint8_t* code_ok);
+
+void rqo_quantize_box_rows(const float* lo, const float* hi, const float* mid, int64_t n,
+                           int D, int bits, int group, uint32_t* words, uint32_t* meta,
+                           float* deq, uint8_t* meta_ok, uint8_t* code_ok);
+void rqo_encode_residual_box_rows(const float* lo, const float* hi, const float* mid,
+                                  const float* ref, const float* mu, int64_t n, int D,
+                                  int bits, int group, int unit_alpha, uint32_t* words,
+                                  uint32_t* meta, uint16_t* alpha, float* zhat,
+                                  uint8_t* alpha_ok, uint8_t* meta_ok, uint8_t* code_ok);
+
 void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
                        int64_t T, const double* kcur, const double* vcur,
                        int D, double scale, double* out);
