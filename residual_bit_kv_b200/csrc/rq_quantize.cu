@@ -314,10 +314,17 @@ __device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, flo
                                            uint32_t (&words)[BITS], float2* levels) {
   constexpr uint32_t QMAX = (1u << BITS) - 1u;
   const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+  // two partial sums per word (even and odd k) keep the add chains short;
+  // the fields never overlap, so any grouping of the adds gives the same word
+  uint32_t odd[BITS];
 #pragma unroll
-  for (int i = 0; i < BITS; ++i) words[i] = 0u - magic_pack_offset<BITS>(i);
+  for (int i = 0; i < BITS; ++i) {
+    words[i] = 0u - magic_pack_offset<BITS>(i);
+    odd[i] = 0u;
+  }
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
+    uint32_t* wk = (k & 1) ? odd : words;
     float2 u = __fmul2_rn(__fadd2_rn(v[k], nz), iv);
     if constexpr (CLAMP == 2) {
       u.x = fminf(fmaxf(u.x, 0.0f), static_cast<float>(QMAX));
@@ -331,13 +338,15 @@ __device__ __forceinline__ void pack_codes(const float2 (&v)[16], float2 nz, flo
     }
     const float2 r = __fadd2_rn(u, mg);
     const uint32_t b0 = __float_as_uint(r.x), b1 = __float_as_uint(r.y);
-    words[slice_word<BITS>(k)] += b0 << slice_shift<BITS>(k);
-    words[slice_word<BITS>(k + 16)] += b1 << slice_shift<BITS>(k + 16);
+    wk[slice_word<BITS>(k)] += b0 << slice_shift<BITS>(k);
+    wk[slice_word<BITS>(k + 16)] += b1 << slice_shift<BITS>(k + 16);
     if constexpr (LEVELS) {
       const float2 cf = __fadd2_rn(r, make_float2(-kRoundMagic, -kRoundMagic));   // exact codes
       levels[k] = __ffma2_rn(make_float2(st[0], st[1]), cf, make_float2(zt[0], zt[1]));
     }
   }
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) words[i] += odd[i];
 }
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
@@ -502,6 +511,20 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
   }
 }
 
+// Batch-head row and token of a flattened row index (32-bit division when
+// every row index fits in 32 bits).
+__device__ __forceinline__ void split_row(int64_t row, int32_t n, bool narrow, int64_t& bhi,
+                                          int64_t& tn) {
+  if (narrow) {
+    const uint32_t r = static_cast<uint32_t>(row), q = r / static_cast<uint32_t>(n);
+    bhi = q;
+    tn = r - q * static_cast<uint32_t>(n);
+  } else {
+    bhi = row / n;
+    tn = row - bhi * n;
+  }
+}
+
 // Least-squares coefficient of z against the reference over the row
 // [RQ §3.2 scaling coefficient, App. G.1]: alpha~ = bf16(<z, ref> / <ref, ref>)
 // (0 for a zero reference; 1 without LS scaling); z becomes the residual
@@ -546,11 +569,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kQuantThreads / 32);
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) +
                        (threadIdx.x >> 5);
+  const bool narrow = total <= 0xFFFFFFFFll;
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    const int64_t bhi = active ? row / p.n : 0;
-    const int64_t t = p.t0 + (active ? row % p.n : 0);
+    int64_t bhi, tn;
+    split_row(active ? row : 0, p.n, narrow, bhi, tn);
+    const int64_t t = p.t0 + tn;
     float2 v[16];
     if (p.dst.has_alpha) {
       // The reference is rebuilt from the cache first (its temporaries are
@@ -585,31 +610,46 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   }
 }
 
+// Record of component c at token t of row `row`, geometry fixed at compile
+// time: codes, metadata and (residual loops) the LS coefficient's slot.
+template <int D, int BITS, int G>
+__device__ __forceinline__ void quantize_at(const Comp& c, int64_t row, int64_t nblk, int64_t t,
+                                            const float2 (&v)[16], int slice, bool active,
+                                            float2* levels, int alpha_bits) {
+  constexpr int CW = D * BITS / 32;   // code words per token
+  unsigned char* rec = comp_record(c, row, nblk, t);
+  const int i = static_cast<int>(t % kBlock);
+  const bool m16 = c.meta16 != 0;
+  const int mb = m16 ? 2 : 4;
+  uint32_t* cw = reinterpret_cast<uint32_t*>(rec) + i * CW;
+  unsigned char* mw = rec + kBlock * 4 * CW + i * (D / G) * mb;
+  if (alpha_bits >= 0 && active && slice == 0)
+    reinterpret_cast<uint16_t*>(rec + kBlock * (4 * CW + mb * (D / G)))[i] =
+        static_cast<uint16_t>(alpha_bits);
+  quantize_store<D, BITS, G>(v, slice, active, cw, mw, m16, levels);
+}
+
 // Quantisation of one component at token t (run-time bits / group): codes,
-// metadata and (if `levels`) the stored levels of this lane's 32 channels.
+// metadata, the LS coefficient's bf16 bits when alpha_bits >= 0, and (if
+// `levels`) the stored levels of this lane's 32 channels.
 template <int D>
 __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_t nblk, int64_t t,
                                               const float2 (&v)[16], int slice, bool active,
-                                              float2* levels) {
-  unsigned char* rec = comp_record(c, row, nblk, t);
-  const int i = static_cast<int>(t % kBlock);
-  uint32_t* cw = rec_codes(rec, D, c.bits, i);
-  unsigned char* mw =
-      c.meta16 ? reinterpret_cast<unsigned char*>(rec_meta16(rec, D, c.bits, c.group, i))
-               : reinterpret_cast<unsigned char*>(rec_meta(rec, D, c.bits, c.group, i));
-  const bool m16 = c.meta16 != 0;
+                                              float2* levels, int alpha_bits = -1) {
   const int key = c.bits * 1000 + c.group;
   switch (key) {
-    case 2016: quantize_store<D, 2, 16>(v, slice, active, cw, mw, m16, levels); break;
-    case 2032: quantize_store<D, 2, 32>(v, slice, active, cw, mw, m16, levels); break;
-    case 2064: quantize_store<D, 2, 64>(v, slice, active, cw, mw, m16, levels); break;
-    case 4016: quantize_store<D, 4, 16>(v, slice, active, cw, mw, m16, levels); break;
-    case 4032: quantize_store<D, 4, 32>(v, slice, active, cw, mw, m16, levels); break;
-    case 4064: quantize_store<D, 4, 64>(v, slice, active, cw, mw, m16, levels); break;
+    case 2016: quantize_at<D, 2, 16>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
+    case 2032: quantize_at<D, 2, 32>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
+    case 2064: quantize_at<D, 2, 64>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
+    case 4016: quantize_at<D, 4, 16>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
+    case 4032: quantize_at<D, 4, 32>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
+    case 4064: quantize_at<D, 4, 64>(c, row, nblk, t, v, slice, active, levels, alpha_bits); break;
     default:
       if constexpr (D >= 128) {
-        if (key == 2128) quantize_store<D, 2, 128>(v, slice, active, cw, mw, m16, levels);
-        else if (key == 4128) quantize_store<D, 4, 128>(v, slice, active, cw, mw, m16, levels);
+        if (key == 2128)
+          quantize_at<D, 2, 128>(c, row, nblk, t, v, slice, active, levels, alpha_bits);
+        else if (key == 4128)
+          quantize_at<D, 4, 128>(c, row, nblk, t, v, slice, active, levels, alpha_bits);
       }
       break;
   }
@@ -677,11 +717,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     slot = slot + 1 == kQStages ? 0 : slot + 1;
     rotate_pieces<D>(q, active, slice, p.rot_scale, v);
   };
+  const bool narrow = total <= 0xFFFFFFFFll;
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
-    const int64_t bhi = active ? row / p.n : 0;
-    const int64_t t = p.t0 + (active ? row % p.n : 0);
+    int64_t bhi, tn;
+    split_row(active ? row : 0, p.n, narrow, bhi, tn);
+    const int64_t t = p.t0 + tn;
     float2 ref[16], v[16];
     next_input(active, v);
     quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, v, slice, active, ref);
@@ -691,11 +733,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
       next_input(active, v);
       if (c.mean != nullptr && active) sub_mean(c, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
-      if (active && slice == 0)
-        *rec_alpha(comp_record(c, bhi, p.nblk, t), D, c.bits, c.group,
-                   static_cast<int>(t % kBlock), c.meta16 ? 2 : 4) = __bfloat16_as_ushort(ab);
       float2 lv[16];   // stored levels, the next reference of a chain
-      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, CHAINED ? lv : nullptr);
+      quantize_comp<D>(c, bhi, p.nblk, t, v, slice, active, CHAINED ? lv : nullptr,
+                       __bfloat16_as_ushort(ab));
       if constexpr (CHAINED) {
         const float at = __bfloat162float(ab);
         const float2 a2 = make_float2(at, at);
