@@ -854,10 +854,27 @@ def main():
 POLICY_NAMES = ("last", "next", "first", "previous")
 
 
-def policy_decode_step(w, policy, dev, stream, args, meta16=False):
+def random_rotations(w, seed):
+    """Binary16 orthogonal matrices [1, H, D, D] per side (QR of Gaussians):
+    stand-ins for calibrated rotations, which need model activations."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    rot = {}
+    for side in (0, 1):
+        m = np.zeros((1, w.heads, w.head_dim, w.head_dim), np.float16)
+        for h in range(w.heads):
+            q, r = np.linalg.qr(rng.standard_normal((w.head_dim, w.head_dim)))
+            m[0, h] = (q * np.sign(np.diag(r))).astype(np.float16)
+        rot[side] = torch.from_numpy(m)
+    return rot
+
+
+def policy_decode_step(w, policy, dev, stream, args, meta16=False, dense=False):
     """One layer of workload w stored under `policy` (16-bit metadata per
-    group if meta16): the time of a decode step over every loop (one call
-    per loop) and its algorithmic bytes."""
+    group if meta16; dense binary16 rotations instead of the Hadamard
+    transform if dense): the time of a decode step over every loop (one call
+    per loop), its algorithmic bytes, the component reads, and the time of the
+    fused prefill append of both sides."""
     import residual_bit_kv_b200.librq as L
     T = w.tokens
     code = {"last": L.RQ_POLICY_LAST_LOOP, "next": L.RQ_POLICY_NEXT_LOOP,
@@ -868,13 +885,18 @@ def policy_decode_step(w, policy, dev, stream, args, meta16=False):
     kb = torch.empty(nb, dtype=torch.uint8, device=dev)
     vb = torch.empty(nb, dtype=torch.uint8, device=dev)
     cache = L.rq_cache_bind(lay, kb, vb)
-    for side in (0, 1):
-        xs = torch.stack([synth.kv_full(w, 0, side, loop, 0, T, device=dev, chunk_b=2)
-                          for loop in range(w.loops)])
-        L.rq_quantize_append_loops(cache, 0, xs if side == 0 else None,
-                                   xs if side == 1 else None, 0, T, stream)
-        torch.cuda.synchronize()
-        del xs
+    rot = None
+    if dense:
+        rot = {k: v.to(dev) for k, v in random_rotations(w, 7).items()}
+        L.rq_cache_set_rotations(cache, rot[0], rot[1])
+    xk = torch.stack([synth.kv_full(w, 0, 0, loop, 0, T, device=dev, chunk_b=2)
+                      for loop in range(w.loops)])
+    xv = torch.stack([synth.kv_full(w, 0, 1, loop, 0, T, device=dev, chunk_b=2)
+                      for loop in range(w.loops)])
+    prefill_ms = timed(lambda: L.rq_quantize_append_loops(cache, 0, xk, xv, 0, T, stream),
+                       max(1, args.steps // 2), args.warmup, stream)
+    torch.cuda.synchronize()
+    del xk, xv
     q = [synth.query(w, 0, l, dev).contiguous() for l in range(w.loops)]
     kc = [synth.current_token(w, 0, 0, l, dev).contiguous() for l in range(w.loops)]
     vc = [synth.current_token(w, 0, 1, l, dev).contiguous() for l in range(w.loops)]
@@ -893,9 +915,9 @@ def policy_decode_step(w, policy, dev, stream, args, meta16=False):
     byt = sum(decode_call_bytes(w, l, T, policy, meta_bytes=2 if meta16 else 4)
               for l in range(w.loops))
     reads = sum(len(policy_chain(w.loops, l, policy)[0]) for l in range(w.loops))
-    del kb, vb, ws
+    del kb, vb, ws, rot
     torch.cuda.empty_cache()
-    return ms, byt, reads
+    return ms, byt, reads, prefill_ms
 
 
 def bench_ablation(dev, stream, args, hbm):
@@ -912,7 +934,7 @@ def bench_ablation(dev, stream, args, hbm):
     out = {"workload": f"{w.name}: 1 layer x {w.loops} loops, batch {w.batch}, {w.heads} heads, "
                        f"{T} past tokens, bits {list(w.bits)}, group {w.group[0]}"}
     for policy, name in (("last", "shared"), ("next", "chained")):
-        ms, byt, reads = policy_decode_step(w, policy, dev, stream, args)
+        ms, byt, reads, _ = policy_decode_step(w, policy, dev, stream, args)
         out[name] = {"ms_per_step": ms, "bytes_per_step": byt,
                      "gbs": byt / (ms * 1e-3) / 1e9, "frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
                      "component_reads": reads}
@@ -925,7 +947,7 @@ def bench_ablation(dev, stream, args, hbm):
     for policy in POLICY_NAMES:
         bits = tuple(wo.bits) if policy in ("last", "next") else tuple(wo.bits)[::-1]
         wp = wo.replace(bits=bits)
-        ms, byt, reads = policy_decode_step(wp, policy, dev, stream, args)
+        ms, byt, reads, _ = policy_decode_step(wp, policy, dev, stream, args)
         pol[policy] = {"bits": list(bits), "ms_per_step": ms, "bytes_per_step": byt,
                        "gbs": byt / (ms * 1e-3) / 1e9, "component_reads": reads}
     pol["throughput_last_over_previous"] = pol["previous"]["ms_per_step"] / pol["last"]["ms_per_step"]
@@ -937,7 +959,7 @@ def bench_ablation(dev, stream, args, hbm):
     m16 = {"workload": f"{wm.name}: 1 layer x {wm.loops} loops, batch {wm.batch}, {wm.heads} "
                        f"heads, {wm.tokens} past tokens, bits {list(wm.bits)}, group {wm.group[0]}"}
     for name, flag in (("meta32", False), ("meta16", True)):
-        ms, byt, _ = policy_decode_step(wm, "last", dev, stream, args, meta16=flag)
+        ms, byt, _, _ = policy_decode_step(wm, "last", dev, stream, args, meta16=flag)
         mb = 2 if flag else 4
         m16[name] = {"ms_per_step": ms, "bytes_per_step": byt, "gbs": byt / (ms * 1e-3) / 1e9,
                      "frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
@@ -951,6 +973,18 @@ def bench_ablation(dev, stream, args, hbm):
                          for l in range(wm.loops)]}
     m16["speedup_meta16_over_meta32"] = m16["meta32"]["ms_per_step"] / m16["meta16"]["ms_per_step"]
     out["metadata16_ouro_16k_layer"] = m16
+    # dense binary16 rotations (tensor-core product) against the Hadamard transform
+    dn = {"workload": m16["workload"],
+          "note": "random orthogonal binary16 matrices per head and side stand in for calibrated "
+                  "rotations; prefill = fused append of every loop, K and V"}
+    for name, flag in (("hadamard", False), ("dense", True)):
+        ms, byt, _, pms = policy_decode_step(wm, "last", dev, stream, args, dense=flag)
+        qb = 2 * quant_loops_bytes(wm, wm.tokens)
+        dn[name] = {"decode_ms_per_step": ms, "decode_gbs": byt / (ms * 1e-3) / 1e9,
+                    "decode_frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
+                    "prefill_ms": pms, "prefill_gbs": qb / (pms * 1e-3) / 1e9,
+                    "prefill_frac_of_hbm": qb / (pms * 1e-3) / 1e9 / hbm}
+    out["dense_rotation_ouro_16k_layer"] = dn
     return out
 
 

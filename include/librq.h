@@ -72,7 +72,7 @@
 extern "C" {
 #endif
 
-#define RQ_ABI_VERSION 2
+#define RQ_ABI_VERSION 3
 #define RQ_MAX_LOOPS 32
 #define RQ_BLOCK_TOKENS 32
 
@@ -139,6 +139,8 @@ typedef struct rq_cache {
   uint32_t rec_bytes[RQ_MAX_LOOPS];  /* bytes of one 32-token record of loop r */
   const float* k_means;              /* fixed means (rq_cache_set_means) or NULL */
   const float* v_means;
+  const void* k_rot;                 /* dense rotations (rq_cache_set_rotations) or NULL */
+  const void* v_rot;
 } rq_cache;
 
 /* ABI version of the loaded library (RQ_ABI_VERSION at build time). */
@@ -158,8 +160,6 @@ uint64_t rq_cache_bytes(const rq_layout* layout);
 /* Bytes of one (layer, side): the stride between layers inside a side. */
 uint64_t rq_layer_bytes(const rq_layout* layout);
 
-/* Binds device buffers of rq_cache_bytes() each (256-byte aligned) to `out`.
- * The buffers need no initialisation.  Host-only, launches nothing. */
 /* Fixed means of the residual loops [RQ App. G.2]: the reconstruction of a
  * residual loop r is Z^_r = alpha~_r R + D(c_r) + mu_r, and the encoder
  * removes mu_r before the LS coefficient (zc = Z_r - mu_r, alpha =
@@ -172,6 +172,26 @@ uint64_t rq_layer_bytes(const rq_layout* layout);
  * means. */
 rq_status rq_cache_set_means(rq_cache* cache, const float* k_means, const float* v_means);
 
+/* Dense rotations in place of the Sylvester-Hadamard transform [RQ §3.3,
+ * App. G.1, App. G.2]: one matrix per (layer, head) and side, shared by every
+ * loop, stored in binary16; the quantisers compute Z = U x with x rounded
+ * from bf16 to binary16 and fp32 accumulation on the tensor cores, decode
+ * scores use U_K q (q rounded to binary16, fp32 accumulation) and the output
+ * is U_V^T of the fp32 value sum; rq_dequantize returns U^T Z^.
+ *   k_rot, v_rot  device binary16 [num_layers][kv_heads][head_dim][head_dim],
+ *                 row i of a matrix giving output channel i (z_i = sum_j
+ *                 U_ij x_j), 16-byte aligned; NULL for a side keeps the
+ *                 Hadamard transform (the state after rq_cache_bind).
+ * head_dim must be 128 when either is set (RQ_ERR_UNSUPPORTED otherwise).
+ * The cache keeps the pointers; the caller keeps the matrices alive and
+ * unchanged while appends and decodes that use them are in flight.  The
+ * accumulation order of a tensor-core product is the hardware's, so the
+ * codes are those of some fp32 ordering of the exact binary16 products (the
+ * pages fix the formats, not the order). */
+rq_status rq_cache_set_rotations(rq_cache* cache, const void* k_rot, const void* v_rot);
+
+/* Binds device buffers of rq_cache_bytes() each (256-byte aligned) to `out`.
+ * The buffers need no initialisation.  Host-only, launches nothing. */
 rq_status rq_cache_bind(const rq_layout* layout, void* k_base, void* v_base,
                         rq_cache* out);
 

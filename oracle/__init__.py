@@ -488,11 +488,15 @@ def rotate_dense(u: np.ndarray, x: np.ndarray):
 
 def f32_box(z: np.ndarray, bound: np.ndarray):
     """fp32 (lo, hi, mid): lo <= z - bound and hi >= z + bound as fp32 values,
-    mid = fp32 rounding of z."""
+    mid = fp32 rounding of z.  A zero bound on a value exact in fp32 (every
+    accumulation order gives exactly z) is a box of one point."""
+    mid = z.astype(np.float32)
     lo = np.nextafter((z - bound).astype(np.float32), np.float32(-np.inf))
     hi = np.nextafter((z + bound).astype(np.float32), np.float32(np.inf))
-    return (np.ascontiguousarray(lo), np.ascontiguousarray(hi),
-            np.ascontiguousarray(z.astype(np.float32)))
+    point = (bound == 0.0) & (mid.astype(np.float64) == z)
+    lo = np.where(point, mid, lo)
+    hi = np.where(point, mid, hi)
+    return (np.ascontiguousarray(lo), np.ascontiguousarray(hi), np.ascontiguousarray(mid))
 
 
 def quantize_box(lo: np.ndarray, hi: np.ndarray, mid: np.ndarray, bits: int, group: int):

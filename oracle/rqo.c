@@ -517,20 +517,45 @@ void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
  * additions, so the oracle returns the sum formed in fp64 together with a
  * bound that every order of fp32 accumulation of the exact products meets:
  *   bound_i = D 2^-23 sum_j |U_ij x_j|  (+ the fp64 sum's own D 2^-53 share),
- * twice the textbook (D - 1) 2^-24, which also covers adders that truncate. */
+ * twice the textbook (D - 1) 2^-24, which also covers adders that truncate;
+ * the bound is 0 when every partial sum is exact in any order (below). */
+/* Exponent of the lowest set bit of a nonzero double. */
+static int low_bit_exponent(double t) {
+  int e;
+  const double m = frexp(fabs(t), &e);          /* |t| = m 2^e, m in [1/2, 1) */
+  uint64_t M = (uint64_t)ldexp(m, 53);           /* exact: 53-bit integer */
+  int k = 0;
+  while ((M & 1u) == 0u) {
+    M >>= 1;
+    ++k;
+  }
+  return e - 53 + k;
+}
+
 void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z,
                           double* bound) {
   double xh[256];
   for (int j = 0; j < D; ++j) xh[j] = rqo_f16_to_f32(rqo_f32_to_f16(rqo_bf16_to_f32(x[j])));
   for (int i = 0; i < D; ++i) {
     double acc = 0.0, mag = 0.0;
+    int emin = 1 << 20;
     for (int j = 0; j < D; ++j) {
       const double t = (double)rqo_f16_to_f32(u[(size_t)i * D + j]) * xh[j];
       acc += t;
       mag += fabs(t);
+      if (t != 0.0) {
+        const int e = low_bit_exponent(t);
+        if (e < emin) emin = e;
+      }
     }
     z[i] = acc;
-    bound[i] = mag * ((double)D * 0x1p-23 + (double)D * 0x1p-53);
+    /* Every term a multiple of 2^emin and sum |t| < 2^(24 + emin): each partial
+     * sum of any subset, in any order, is such a multiple below 2^(24 + emin),
+     * exact in fp32 (and in fp64): no rounding anywhere. */
+    if (mag == 0.0 || mag < ldexp(1.0, 24 + emin))
+      bound[i] = 0.0;
+    else
+      bound[i] = mag * ((double)D * 0x1p-23 + (double)D * 0x1p-53);
   }
 }
 
@@ -619,11 +644,14 @@ void rqo_encode_residual_box(const float* lo, const float* hi, const float* mid,
         w += fabs((double)ref[i]) * wd;
         m += (fabs(zc) + wd) * fabs((double)ref[i]);
       }
-      const double dev = w + 35.0 * 0x1p-24 * m + (double)D * 0x1p-52 * m;
-      /* fp32 values bracketing every attainable d_zr */
-      const float dlo = nextafterf((float)(c - dev), -INFINITY);
-      const float dhi = nextafterf((float)(c + dev), INFINITY);
-      aok = rqo_f32_to_bf16(dlo / d_rr) == rqo_f32_to_bf16(dhi / d_rr);
+      /* A box of zero width holds one row, whose fp32 dot is the oracle's own;
+       * otherwise the fp32 values bracketing every attainable d_zr. */
+      if (w > 0.0) {
+        const double dev = w + 35.0 * 0x1p-24 * m + (double)D * 0x1p-52 * m;
+        const float dlo = nextafterf((float)(c - dev), -INFINITY);
+        const float dhi = nextafterf((float)(c + dev), INFINITY);
+        aok = rqo_f32_to_bf16(dlo / d_rr) == rqo_f32_to_bf16(dhi / d_rr);
+      }
     }
   }
   *alpha_ok = (uint8_t)aok;

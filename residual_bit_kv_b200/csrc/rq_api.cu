@@ -180,6 +180,15 @@ int chain_of(const rq_cache* c, int layer, int kv, int loop, Comp* out) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Dense rotation of (layer, side) or nullptr (Hadamard).
+const uint16_t* rot_of(const rq_cache* c, int layer, int kv) {
+  const void* r = kv ? c->v_rot : c->k_rot;
+  if (r == nullptr) return nullptr;
+  const rq_layout& l = c->layout;
+  return static_cast<const uint16_t*>(r) +
+         static_cast<int64_t>(layer) * l.kv_heads * l.head_dim * l.head_dim;
+}
+
 rq_status check_cache(const rq_cache* c, int32_t layer, int32_t kv) {
   if (c == nullptr || c->k_base == nullptr || c->v_base == nullptr) return RQ_ERR_INVALID_ARG;
   if (rq_layout_validate(&c->layout) != RQ_OK) return RQ_ERR_INVALID_ARG;
@@ -275,6 +284,17 @@ rq_status rq_cache_set_means(rq_cache* c, const float* k_means, const float* v_m
   return RQ_OK;
 }
 
+rq_status rq_cache_set_rotations(rq_cache* c, const void* k_rot, const void* v_rot) {
+  if (c == nullptr) return RQ_ERR_INVALID_ARG;
+  if ((k_rot != nullptr && !aligned(k_rot, 16)) || (v_rot != nullptr && !aligned(v_rot, 16)))
+    return RQ_ERR_INVALID_ARG;
+  if ((k_rot != nullptr || v_rot != nullptr) && c->layout.head_dim != 128)
+    return RQ_ERR_UNSUPPORTED;
+  c->k_rot = k_rot;
+  c->v_rot = v_rot;
+  return RQ_OK;
+}
+
 rq_status rq_quantize_anchor(const rq_cache* c, int32_t layer, int32_t kv, const void* x,
                              int32_t t0, int32_t n, void* stream) {
   rq_status st = check_cache(c, layer, kv);
@@ -294,6 +314,8 @@ rq_status rq_quantize_anchor(const rq_cache* c, int32_t layer, int32_t kv, const
   p.dst = comp_of(c, layer, kv, a);
   p.nref = 0;
   p.rot_scale = rot_scale_of(l.head_dim);
+  p.urot = rot_of(c, layer, kv);
+  p.heads = l.kv_heads;
   return cuda_status(launch_quantize(p, l.head_dim, l.bits[a], l.group[a], as_stream(stream)));
 }
 
@@ -321,6 +343,8 @@ rq_status rq_quantize_append_residual(const rq_cache* c, int32_t layer, int32_t 
   for (int i = 1; i < len; ++i) p.ref[i - 1] = chain[i];
   p.unit_alpha = (l.flags & RQ_FLAG_UNIT_ALPHA) ? 1 : 0;
   p.rot_scale = rot_scale_of(l.head_dim);
+  p.urot = rot_of(c, layer, kv);
+  p.heads = l.kv_heads;
   return cuda_status(
       launch_quantize(p, l.head_dim, l.bits[loop], l.group[loop], as_stream(stream)));
 }
@@ -355,6 +379,9 @@ rq_status rq_quantize_append_loops(const rq_cache* c, int32_t layer, const void*
   for (int kv = 0; kv < 2; ++kv)
     for (int r = 0; r < l.num_loops; ++r) p.dst[kv][r] = comp_of(c, layer, kv, r);
   p.rot_scale = rot_scale_of(l.head_dim);
+  p.urot[0] = rot_of(c, layer, 0);
+  p.urot[1] = rot_of(c, layer, 1);
+  p.heads = l.kv_heads;
   return cuda_status(launch_quantize_loops(p, l.head_dim, as_stream(stream)));
 }
 
@@ -376,6 +403,8 @@ rq_status rq_dequantize(const rq_cache* c, int32_t layer, int32_t kv, int32_t lo
   p.ncomp = chain_of(c, layer, kv, loop, p.comp);
   p.rot_scale = rot_scale_of(l.head_dim);
   p.out = out;
+  p.urot = rot_of(c, layer, kv);
+  p.heads = l.kv_heads;
   return cuda_status(launch_dequantize(p, l.head_dim, as_stream(stream)));
 }
 
@@ -423,6 +452,8 @@ static rq_status fill_decode_params(const rq_cache* c, int32_t layer, int32_t lo
   (void)chain_of(c, layer, 1, loop, p->v);
   p->max_seq_len = max_seq_len;
   p->rot_scale = rot_scale_of(l.head_dim);
+  p->urot_k = rot_of(c, layer, 0);
+  p->urot_v = rot_of(c, layer, 1);
   *D = l.head_dim;
   int stages = 0, occ = 0, chunk = kChunk;
   if (fast_decode_plan(*p, *D, &stages, &chunk, &occ)) {

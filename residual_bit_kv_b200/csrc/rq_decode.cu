@@ -222,11 +222,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (t == 0) {
     for (; issued < min(S, nchunks); ++issued) issue(issued);
   }
-  smem_fwht<D>(svec);
+  const float qrs = rotate_query<D>(
+      svec, p.urot_k ? p.urot_k + static_cast<size_t>(bhi % p.heads) * D * D : nullptr,
+      p.rot_scale);
   float q[32];
   float qsa = 0.0f, qsb = 0.0f;
   {
-    const float sc = p.rot_scale * p.scale_log2;
+    const float sc = qrs * p.scale_log2;
 #pragma unroll
     for (int ch = 0; ch < 32; ++ch) {
       q[ch] = svec[slice * 32 + ch] * sc;
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   // Fixed means [RQ App. G.2]: q'.mu_c over each 32-channel slice.
   const int head = bhi % p.heads;
   {
-    const float sc = p.rot_scale * p.scale_log2;
+    const float sc = qrs * p.scale_log2;
     for (int e = t; e < p.ncomp * G::P; e += kDecodeThreads) {
       const int c = e / G::P, s = e % G::P;
       float sum = 0.0f;
@@ -355,7 +357,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const bool aborted = __syncthreads_or(s_abort != 0) != 0;
   finish_split<D, kDecodeThreads, Geom<D>::NSLOT, true>(
       m, l, acc, slice, slot, reinterpret_cast<float*>(smem), bhi, split, p.splits, p.partials,
-      p.counters, p.q, p.kcur, p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred, aborted);
+      p.counters, p.q, p.kcur, p.vcur, p.scale_log2, p.rot_scale, p.out, svec, sred, aborted,
+      p.urot_v ? p.urot_v + static_cast<size_t>(bhi % p.heads) * D * D : nullptr);
 }
 
 template <int D>

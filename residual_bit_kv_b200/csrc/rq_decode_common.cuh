@@ -44,6 +44,42 @@ __device__ __forceinline__ void smem_fwht(float* v) {
   }
 }
 
+// Rotated query in svec (which holds the bf16 query on entry), every thread
+// of the CTA calls it.  Hadamard: the unnormalised butterflies, and the
+// returned factor rot_scale normalises them.  Dense rotation [RQ App. G.2]
+// (urot: this head's binary16 D x D matrix, row i = output channel i):
+// U q~ with q~ the query rounded to binary16 and fp32 sums; returns 1.
+template <int D>
+__device__ __forceinline__ float rotate_query(float* svec, const uint16_t* urot,
+                                              float rot_scale) {
+  const int t = threadIdx.x;
+  if (urot == nullptr) {
+    smem_fwht<D>(svec);
+    return rot_scale;
+  }
+  if (t < D) svec[t] = __half2float(__float2half_rn(svec[t]));
+  __syncthreads();
+  float a = 0.0f;
+  if (t < D) {
+    const uint4* row = reinterpret_cast<const uint4*>(urot + static_cast<size_t>(t) * D);
+#pragma unroll 4
+    for (int j8 = 0; j8 < D / 8; ++j8) {
+      const uint4 w = __ldg(row + j8);
+      const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 u = __half22float2(*reinterpret_cast<const __half2*>(&h[e]));
+        a = fmaf(u.x, svec[8 * j8 + 2 * e], a);
+        a = fmaf(u.y, svec[8 * j8 + 2 * e + 1], a);
+      }
+    }
+  }
+  __syncthreads();
+  if (t < D) svec[t] = a;
+  __syncthreads();
+  return 1.0f;
+}
+
 // Sequence length of batch row b, clamped to [0, max_seq_len] and flagged.
 __device__ __forceinline__ int seq_len_of(const int32_t* seq_lens, int b, int max_seq_len,
                                           uint32_t* err) {
@@ -82,7 +118,8 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
                                              const uint16_t* q, const uint16_t* kcur,
                                              const uint16_t* vcur, float scale_log2,
                                              float rot_scale, float* out, float* svec,
-                                             float* sred, bool bad) {
+                                             float* sred, bool bad,
+                                             const uint16_t* urot = nullptr) {
   constexpr int RP = red_pitch<D>();
   float* red = scratch;                 // [NSLOT][D/32][36]
   float* mred = red + NSLOT * RP;       // [NSLOT]
@@ -186,10 +223,20 @@ __device__ __forceinline__ void finish_split(float m, float l, const float (&acc
   __syncthreads();   // everyone is done reading svec / the scratch
   if (t < D) svec[t] = ax;
   __syncthreads();
-  if constexpr (ROT) smem_fwht<D>(svec);
+  // Back to the original domain: the Hadamard butterflies, or U_V^T of the
+  // fp32 value sum under a dense rotation [RQ App. G.2] (column t of U).
+  float dv = 0.0f;
+  if (urot != nullptr) {
+    if (t < D)
+      for (int j = 0; j < D; ++j)
+        dv = fmaf(__half2float(__ushort_as_half(__ldg(urot + static_cast<size_t>(j) * D + t))),
+                  svec[j], dv);
+  } else if constexpr (ROT) {
+    smem_fwht<D>(svec);
+  }
   if (t < D) {
     const float pc = fast_exp2(s_cur - Mx);
-    const float v = ROT ? svec[t] * rot_scale : svec[t];
+    const float v = urot != nullptr ? dv : (ROT ? svec[t] * rot_scale : svec[t]);
     out[static_cast<size_t>(bhi) * D + t] =
         (v + pc * bf16_bits_to_f32(vcur[static_cast<size_t>(bhi) * D + t])) / Lx;
   }

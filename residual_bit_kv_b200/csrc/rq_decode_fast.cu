@@ -472,8 +472,11 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
   __shared__ float s_amax[kCWarps];
   if (t < D) svec[t] = bf16_bits_to_f32(p.q[static_cast<size_t>(bhi) * D + t]);
   __syncthreads();
-  smem_fwht<D>(svec);
-  const float qscale = p.rot_scale * p.scale_log2;
+  const int qhead = bhi % p.heads;
+  const float qscale =
+      rotate_query<D>(svec, p.urot_k ? p.urot_k + static_cast<size_t>(qhead) * D * D : nullptr,
+                      p.rot_scale) *
+      p.scale_log2;
   const float qv = t < D ? svec[t] * qscale : 0.0f;
   float amax = fabsf(qv);
 #pragma unroll
@@ -622,7 +625,10 @@ __global__ void __launch_bounds__(kCThreads, kCMinCtas)
                                           reinterpret_cast<float*>(smem), bhi, split, p.splits,
                                           p.partials, p.counters, p.q, p.kcur, p.vcur,
                                           p.scale_log2, p.rot_scale, p.out, svec, sred,
-                                          aborted || range_bad);
+                                          aborted || range_bad,
+                                          p.urot_v ? p.urot_v + static_cast<size_t>(bhi % p.heads) *
+                                                                    D * D
+                                                   : nullptr);
 }
 
 // ---------------------------------------------------------------- BF16 --

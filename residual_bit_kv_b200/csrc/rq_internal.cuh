@@ -128,6 +128,10 @@ struct QuantParams {
   int32_t nref;
   Comp ref[RQ_MAX_LOOPS];
   float rot_scale;         // fp32(1/sqrt(D))
+  // Dense rotation of this (layer, side): binary16 [heads][D][D], or nullptr
+  // for the Hadamard transform.
+  const uint16_t* urot;
+  int32_t heads;
 };
 
 // Every loop of one (layer, token range), both sides, in one launch.
@@ -141,6 +145,8 @@ struct QuantLoopsParams {
   int64_t t0, nblk;
   Comp dst[2][RQ_MAX_LOOPS];
   float rot_scale;
+  const uint16_t* urot[2]; // dense rotations per side (binary16 [heads][D][D]) or nullptr
+  int32_t heads;
 };
 
 struct DequantParams {
@@ -150,6 +156,8 @@ struct DequantParams {
   Comp comp[RQ_MAX_LOOPS];
   float rot_scale;
   float* out;              // fp32 [B*H][n][D]
+  const uint16_t* urot;    // dense rotation (binary16 [heads][D][D]) or nullptr
+  int32_t heads;
 };
 
 struct DecodeParams {
@@ -177,6 +185,10 @@ struct DecodeParams {
   int32_t stages;
   uint32_t stage_bytes;
   int32_t use_fast;        // warp-specialised kernel for a compiled layout
+  // Dense rotations of the layer (binary16 [heads][D][D]) or nullptr for the
+  // Hadamard transform.
+  const uint16_t* urot_k;
+  const uint16_t* urot_v;
 };
 
 struct DecodeBf16Params {

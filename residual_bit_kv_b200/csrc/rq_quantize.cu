@@ -122,6 +122,89 @@ __device__ __forceinline__ void load_rotate(const uint16_t* xrow, bool active, i
   rotate_pieces<D>(q, active, slice, rot_scale, v);
 }
 
+// Dense rotation [RQ §3.3, App. G.1, App. G.2]: Z = U x for the warp's eight
+// rows (head_dim 128; the row of lane l is l / 4, its slice l % 4), U the
+// binary16 matrix of the row's head (row i = output channel i), x rounded
+// from bf16 to binary16, fp32 accumulation on the tensor cores
+// (mma.m16n8k16, rows 8..15 of A unused).  Both contraction indices are
+// permuted so that no data moves between lanes:
+//   k: step ks, A/B fragment column 2t + e (+8) <-> channel 32t + 4ks + e (+2),
+//      so a lane's A fragments are its own slice, words 2ks and 2ks + 1;
+//   n: tile nt, column c <-> output channel 32 (c >> 1) + 2 nt + (c & 1),
+//      so the accumulators of lane (g, t) are channels 32t + 2nt + {0, 1} of
+//      its own row, and its B fragments are 64 contiguous bytes of U row
+//      32 (g >> 1) + 2 nt + (g & 1).
+// A warp whose rows belong to several heads runs one pass per head; a lane
+// keeps the pass of its own head (rows are independent in the product).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// Per-lane staging of the dense rotation's accumulators (a stride of 34
+// floats keeps the float2 stores of a warp on distinct bank pairs).
+constexpr int kDenseLaneFloats = 34;
+constexpr int kDenseTileBytes = (kQuantThreads) * kDenseLaneFloats * 4;
+
+template <int D>
+__device__ __forceinline__ void rotate_dense(const uint4 (&q)[4], bool active, int lane, int head,
+                                             const uint16_t* urot, float* tile,
+                                             float2 (&v)[16]) {
+  static_assert(D == 128, "the dense rotation is built for head_dim 128");
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t a[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a[4 * i + j] = active ? bf16x2_to_f16x2(w[j]) : 0u;
+  }
+  uint32_t todo = __ballot_sync(0xffffffffu, active);
+  while (todo != 0u) {
+    const int h = __shfl_sync(0xffffffffu, head, __ffs(todo) - 1);
+    const bool mine = active && head == h;
+    todo &= ~__ballot_sync(0xffffffffu, mine);
+    // U row of n-tile nt for this lane: 64 bytes; the next tile's row is
+    // loaded while the current one's products run
+    const uint4* up = reinterpret_cast<const uint4*>(
+        urot + static_cast<size_t>(h) * D * D + 32 * t +
+        static_cast<size_t>(32 * (g >> 1) + (g & 1)) * D);
+    uint4 bn[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bn[i] = __ldg(up + i);
+#pragma unroll 1
+    for (int nt = 0; nt < 16; ++nt) {
+      uint4 bc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bc[i] = bn[i];
+      if (nt + 1 < 16) {
+        const uint4* un = up + (nt + 1) * (2 * D / 8);   // two U rows further per tile
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bn[i] = __ldg(un + i);
+      }
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {   // 16 bytes of U serve two k-steps
+        mma_16816(d, a[4 * i], a[4 * i + 1], bc[i].x, bc[i].y);
+        mma_16816(d, a[4 * i + 2], a[4 * i + 3], bc[i].z, bc[i].w);
+      }
+      if (mine) *reinterpret_cast<float2*>(tile + 2 * nt) = make_float2(d[0], d[1]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    v[k] = active ? make_float2(tile[k], tile[k + 16]) : make_float2(0.0f, 0.0f);
+}
+
 // Input staging of the fused kernel: each warp streams its rows through a
 // private ring of kQStages shared-memory slots of 32 x 64 bytes (the RPW
 // rows of one loop: 8 rows of 128 channels or 16 rows of 64), filled by
@@ -454,7 +537,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&v)[16], int slice,
       metaw[gi] = static_cast<uint32_t>(__half_as_ushort(sh)) |
                   (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
     }
-    inv[gi] = (st[gi] > 0.0f) ? __fdiv_rn(1.0f, st[gi]) : 0.0f;
+    inv[gi] = (st[gi] > 0.0f) ? __frcp_rn(st[gi]) : 0.0f;
   }
   // (x - z~) * (1/s~) is monotone in x: when both ends of every group of the
   // warp map into [-1/2, 2^b - 1/2), the upper clamp can change no code
@@ -558,7 +641,25 @@ __device__ __forceinline__ __nv_bfloat16 ls_residual(float2 (&v)[16], const floa
   return ab;
 }
 
-template <int D, int BITS, int G>
+// Row of bf16 x -> Z in one lane's 16 pairs: the Hadamard transform, or the
+// dense rotation of the row's head (DENSE).
+template <int D, bool DENSE>
+__device__ __forceinline__ void load_input(const QuantParams& p, int64_t row, int64_t bhi,
+                                           bool active, int lane, float* tile, float2 (&v)[16]) {
+  if constexpr (DENSE) {
+    uint4 q[4];
+    if (active) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + row * D + (lane % (D / 32)) * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) q[i] = src[i];
+    }
+    rotate_dense<D>(q, active, lane, static_cast<int>(bhi % p.heads), p.urot, tile, v);
+  } else {
+    load_rotate<D>(p.x + (active ? row : 0) * D, active, lane % (D / 32), p.rot_scale, v);
+  }
+}
+
+template <int D, int BITS, int G, bool DENSE>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_kernel(const __grid_constant__ QuantParams p) {
   constexpr int P = D / 32;
@@ -570,6 +671,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) +
                        (threadIdx.x >> 5);
   const bool narrow = total <= 0xFFFFFFFFll;
+  float* tile = nullptr;
+  if constexpr (DENSE) {
+    __shared__ __align__(16) float dense_tile[kQuantThreads * kDenseLaneFloats];
+    tile = dense_tile + threadIdx.x * kDenseLaneFloats;
+  }
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
     const int64_t row = base + lane / P;
     const bool active = row < total;
@@ -590,7 +696,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
 #pragma unroll
         for (int k = 0; k < 16; ++k) ref[k] = make_float2(0.0f, 0.0f);
       }
-      load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
+      load_input<D, DENSE>(p, row, bhi, active, lane, tile, v);
       if (p.dst.mean != nullptr && active) sub_mean(p.dst, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       if (active && slice == 0)
@@ -598,7 +704,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                    p.dst.meta16 ? 2 : 4) =
             __bfloat16_as_ushort(ab);
     } else {
-      load_rotate<D>(p.x + (active ? row : 0) * D, active, slice, p.rot_scale, v);
+      load_input<D, DENSE>(p, row, bhi, active, lane, tile, v);
     }
     unsigned char* rec = comp_record(p.dst, bhi, p.nblk, t);
     const int i = static_cast<int>(t % kBlock);
@@ -663,7 +769,7 @@ __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_
 // Z^_r = fma(alpha~_r, Z^_ref, D(c_r)) after loop r.  The anchor is read
 // once and never re-read from the cache; the arithmetic (and so every
 // stored bit) is that of the per-loop kernels.
-template <int D, bool CHAINED>
+template <int D, bool CHAINED, bool DENSE>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_loops_kernel(const __grid_constant__ QuantLoopsParams p) {
   constexpr int P = D / 32;
@@ -708,14 +814,21 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   int slot = 0;
   // the job in `slot` has landed (this lane's copies, then the warp's); the
   // slot read in the previous job is free again and takes the next issue
-  auto next_input = [&](bool active, float2 (&v)[16]) {
+  auto next_input = [&](bool active, int head, float2 (&v)[16]) {
     cp_async_wait<kQStages - 2>();
     __syncwarp();
     issue_next();
     uint4 q[4];
     read_slot<D>(ring + slot * kQSlotBytes, lane, q);
     slot = slot + 1 == kQStages ? 0 : slot + 1;
-    rotate_pieces<D>(q, active, slice, p.rot_scale, v);
+    if constexpr (DENSE)
+      rotate_dense<D>(q, active, lane, head, p.urot[side],
+                      reinterpret_cast<float*>(qsmem + (kQuantThreads / 32) * kQStages *
+                                                           kQSlotBytes) +
+                          threadIdx.x * kDenseLaneFloats,
+                      v);
+    else
+      rotate_pieces<D>(q, active, slice, p.rot_scale, v);
   };
   const bool narrow = total <= 0xFFFFFFFFll;
   for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
@@ -724,13 +837,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     int64_t bhi, tn;
     split_row(active ? row : 0, p.n, narrow, bhi, tn);
     const int64_t t = p.t0 + tn;
+    const int head = static_cast<int>(bhi % p.heads);
     float2 ref[16], v[16];
-    next_input(active, v);
+    next_input(active, head, v);
     quantize_comp<D>(p.dst[side][a], bhi, p.nblk, t, v, slice, active, ref);
     for (int k = 0; k + 1 < p.nloops; ++k) {
       const int r = p.order[k];
       const Comp& c = p.dst[side][r];
-      next_input(active, v);
+      next_input(active, head, v);
       if (c.mean != nullptr && active) sub_mean(c, bhi, slice, D, v);
       const __nv_bfloat16 ab = ls_residual<D>(v, ref, p.unit_alpha != 0);
       float2 lv[16];   // stored levels, the next reference of a chain
@@ -769,6 +883,45 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
       for (int k = 0; k < 16; ++k) v[k] = make_float2(0.0f, 0.0f);
     }
+    if (p.urot != nullptr) {
+      // X^ = U^T Z^ [RQ App. G.2]: the row through shared memory, fp32 sums
+      // over j ascending, lane `slice` writing channels [32 slice, +32).
+      if constexpr (D == 128) {
+        __shared__ float zrow[kQuantThreads / 32][RPW][D];
+        float* zr = zrow[threadIdx.x >> 5][lane / P];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) zr[slice * 32 + k] = ch_of(v, k);
+        __syncwarp();
+        float o[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = 0.0f;
+        const uint16_t* uh = p.urot + static_cast<size_t>(active ? (row / p.n) % p.heads : 0) *
+                                          D * D + slice * 32;
+        for (int j = 0; j < D; ++j) {
+          const float zj = zr[j];
+          const uint4* up = reinterpret_cast<const uint4*>(uh + static_cast<size_t>(j) * D);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = __ldg(up + i);
+            const uint32_t hw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 u = __half22float2(*reinterpret_cast<const __half2*>(&hw[e]));
+              o[8 * i + 2 * e] = fmaf(u.x, zj, o[8 * i + 2 * e]);
+              o[8 * i + 2 * e + 1] = fmaf(u.y, zj, o[8 * i + 2 * e + 1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (active) {
+          float4* dst = reinterpret_cast<float4*>(p.out + row * D + slice * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+      }
+      continue;
+    }
     // X^ = H^T Z^ = H Z^ (the normalised Sylvester matrix is symmetric).
     fwht_row<D>(v, slice);
     if (active) {
@@ -796,7 +949,14 @@ int quant_grid(int64_t rows, int D) {
 template <int D, int BITS, int G>
 cudaError_t launch_q(const QuantParams& p, cudaStream_t s) {
   const int grid = quant_grid(static_cast<int64_t>(p.bh) * p.n, D);
-  quantize_kernel<D, BITS, G><<<grid, kQuantThreads, 0, s>>>(p);
+  if (p.urot != nullptr) {
+    if constexpr (D == 128)
+      quantize_kernel<D, BITS, G, true><<<grid, kQuantThreads, 0, s>>>(p);
+    else
+      return cudaErrorInvalidValue;
+  } else {
+    quantize_kernel<D, BITS, G, false><<<grid, kQuantThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -828,14 +988,38 @@ cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
   return cudaErrorInvalidValue;
 }
 
-template <int D, bool CHAINED>
-cudaError_t launch_loops(const QuantLoopsParams& p, dim3 grid, cudaStream_t s) {
-  constexpr int smem = (kQuantThreads / 32) * kQStages * kQSlotBytes;
-  const cudaError_t e = cudaFuncSetAttribute(quantize_loops_kernel<D, CHAINED>,
+template <int D, bool CHAINED, bool DENSE>
+cudaError_t launch_loops_t(const QuantLoopsParams& p, dim3 grid, cudaStream_t s) {
+  constexpr int smem = (kQuantThreads / 32) * kQStages * kQSlotBytes + (DENSE ? kDenseTileBytes : 0);
+  const cudaError_t e = cudaFuncSetAttribute(quantize_loops_kernel<D, CHAINED, DENSE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  quantize_loops_kernel<D, CHAINED><<<grid, kQuantThreads, smem, s>>>(p);
+  quantize_loops_kernel<D, CHAINED, DENSE><<<grid, kQuantThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+// Both sides of a fused call use the same transform kind (a cache sets its
+// K and V rotations together or not at all on a side: a side without one
+// keeps the Hadamard transform and runs in a second launch).
+template <int D, bool CHAINED>
+cudaError_t launch_loops(const QuantLoopsParams& p, dim3 grid, cudaStream_t s) {
+  const bool dk = p.urot[0] != nullptr && p.x[0] != nullptr;
+  const bool dv = p.urot[1] != nullptr && p.x[1] != nullptr;
+  if (!dk && !dv) return launch_loops_t<D, CHAINED, false>(p, grid, s);
+  if constexpr (D != 128) {
+    return cudaErrorInvalidValue;
+  } else {
+    // one launch per transform kind; a side of the other kind is skipped
+    QuantLoopsParams pd = p, ph = p;
+    pd.x[0] = dk ? p.x[0] : nullptr;
+    pd.x[1] = dv ? p.x[1] : nullptr;
+    ph.x[0] = dk ? nullptr : p.x[0];
+    ph.x[1] = dv ? nullptr : p.x[1];
+    cudaError_t e = launch_loops_t<D, CHAINED, true>(pd, grid, s);
+    if (e == cudaSuccess && (ph.x[0] != nullptr || ph.x[1] != nullptr))
+      e = launch_loops_t<D, CHAINED, false>(ph, grid, s);
+    return e;
+  }
 }
 
 cudaError_t launch_quantize_loops(const QuantLoopsParams& p, int D, cudaStream_t s) {

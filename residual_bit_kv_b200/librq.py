@@ -39,6 +39,7 @@ SYMBOLS = (
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
     "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
     "rq_quantize_append_loops", "rq_selftest_wait_timeout", "rq_cache_set_means",
+    "rq_cache_set_rotations",
 )
 
 
@@ -59,6 +60,7 @@ class rq_cache(ctypes.Structure):
         ("comp_off", ctypes.c_uint64 * RQ_MAX_LOOPS),
         ("rec_bytes", ctypes.c_uint32 * RQ_MAX_LOOPS),
         ("k_means", ctypes.c_void_p), ("v_means", ctypes.c_void_p),
+        ("k_rot", ctypes.c_void_p), ("v_rot", ctypes.c_void_p),
     ]
 
 
@@ -95,6 +97,7 @@ def load() -> ctypes.CDLL:
         "rq_layer_bytes": ([LP], _U64),
         "rq_cache_bind": ([LP, _P, _P, CP], ctypes.c_int),
         "rq_cache_set_means": ([CP, _P, _P], ctypes.c_int),
+        "rq_cache_set_rotations": ([CP, _P, _P], ctypes.c_int),
         "rq_quantize_anchor": ([CP, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_residual": ([CP, _I32, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_loops": ([CP, _I32, _P, _P, _I32, _I32, _P], ctypes.c_int),
@@ -193,6 +196,16 @@ def rq_cache_set_means(cache: rq_cache, k_means, v_means) -> None:
                                      None if k_means is None else _ptr(k_means),
                                      None if v_means is None else _ptr(v_means)),
            "rq_cache_set_means")
+
+
+def rq_cache_set_rotations(cache: rq_cache, k_rot, v_rot) -> None:
+    """k_rot, v_rot: binary16 (torch.float16 or 16-bit words) device tensors
+    [num_layers, kv_heads, head_dim, head_dim], row i of a matrix giving
+    output channel i, or None for the Hadamard transform of that side."""
+    _check(load().rq_cache_set_rotations(ctypes.byref(cache),
+                                         None if k_rot is None else _ptr(k_rot),
+                                         None if v_rot is None else _ptr(v_rot)),
+           "rq_cache_set_rotations")
 
 
 def rq_quantize_anchor(cache: rq_cache, layer: int, kv: int, x, t0: int, n: int,

@@ -54,6 +54,7 @@ class GpuCache:
     unit_alpha: bool = False
     meta16: bool = False
     means: Optional[Dict] = None   # side -> fp32 [layers, loops, H, D] cuda tensor
+    rot: Optional[Dict] = None     # side -> binary16 [layers, H, D, D] cuda tensor (or None)
 
 
 def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[int] = (0,),
@@ -61,7 +62,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     max_tokens: Optional[int] = None, append_chunks: Optional[Sequence[int]] = None,
                     fused: bool = False, unit_alpha: bool = False,
                     gen_device: str = "cuda", meta16: bool = False,
-                    means_seed: Optional[int] = None) -> GpuCache:
+                    means_seed: Optional[int] = None,
+                    rotations: Optional[Dict] = None) -> GpuCache:
     """Generates every loop's K/V on the GPU and quantise-appends them through
     the C ABI in the order the policy requires (fused: every loop and both
     sides of a chunk in one rq_quantize_append_loops call).  append_chunks
@@ -82,6 +84,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
         means = {side: (torch.randn(lay.num_layers, w.loops, w.heads, w.head_dim, generator=g) *
                         0.5).to("cuda") for side in SIDES}
         L.rq_cache_set_means(cache, means[0], means[1])
+    if rotations is not None:
+        L.rq_cache_set_rotations(cache, rotations.get(0), rotations.get(1))
     inputs = {}
     bounds = [0] + list(np.cumsum(append_chunks)) if append_chunks else [0, T]
     assert bounds[-1] == T
@@ -119,7 +123,8 @@ def build_gpu_cache(w: synth.Workload, policy: str = "last", layers: Sequence[in
                     inputs[(layer, side, loop)] = x
             del xs
     torch.cuda.synchronize()
-    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha, meta16, means)
+    return GpuCache(w, policy, lay, cache, kbuf, vbuf, inputs, unit_alpha, meta16, means,
+                    rotations)
 
 
 def gpu_component(gc: GpuCache, layer: int, side: int, loop: int,

@@ -27,7 +27,7 @@ def test_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(L.SYMBOLS)
-    assert L.rq_abi_version() == 2
+    assert L.rq_abi_version() == 3
 
 
 def test_status_strings(L):
@@ -181,6 +181,26 @@ def test_host_checks_reject_before_launch(L):
         with pytest.raises(L.RQError) as e:
             L.rq_selftest_wait_timeout(*args, stream=0)
         assert e.value.status == L.RQ_ERR_INVALID_ARG, args
+
+
+def test_rotation_setter_checks(L):
+    """rq_cache_set_rotations: NULL keeps the Hadamard transform, pointers must
+    be 16-byte aligned, and head_dim must be 128 (host checks, no launch)."""
+    lay = L.make_layout(2, 4, 2, 3, 128, 100, (2, 2, 2, 4), (32,) * 4)
+    cache = L.rq_cache_bind(lay, 1 << 20, 1 << 30)
+    assert cache.k_rot is None and cache.v_rot is None
+    L.rq_cache_set_rotations(cache, 1 << 16, None)
+    assert cache.k_rot == 1 << 16 and cache.v_rot is None
+    L.rq_cache_set_rotations(cache, None, None)
+    assert cache.k_rot is None
+    with pytest.raises(L.RQError) as e:
+        L.rq_cache_set_rotations(cache, (1 << 16) + 8, None)
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+    lay64 = L.make_layout(1, 4, 1, 2, 64, 100, (2, 2, 2, 4), (32,) * 4)
+    c64 = L.rq_cache_bind(lay64, 1 << 20, 1 << 30)
+    with pytest.raises(L.RQError) as e:
+        L.rq_cache_set_rotations(c64, None, 1 << 16)
+    assert e.value.status == L.RQ_ERR_UNSUPPORTED
 
 
 def test_no_cpu_fallback_in_product():

@@ -45,7 +45,7 @@ def test_dense_rotation_orientation_and_fp16_inputs(oracle_mod):
     want = sign * xb[perm].astype(np.float16).astype(np.float64)
     np.testing.assert_array_equal(z[0], want)
     assert np.any(xb[perm].astype(np.float16).astype(np.float32) != xb[perm])   # rounding happened
-    np.testing.assert_allclose(bound[0], D * 2.0 ** -23 * np.abs(want), rtol=1e-9)
+    assert np.all(bound[0] == 0.0)          # one term per output: nothing is rounded
 
 
 def test_dense_bound_covers_fp32_orders(oracle_mod):
@@ -79,6 +79,37 @@ def _narrow_range_rows(rng, n, D):
     mag = np.exp2(rng.uniform(-3, 3, (n, D)))
     v = (mag * rng.choice([-1.0, 1.0], (n, D))).astype(np.float32)
     return _bf16_bits(v) & np.uint16(0xFFFF)   # truncation keeps |x| inside the range
+
+
+def test_dense_exact_sums_have_zero_bound(oracle_mod):
+    """U = P H_128 / 8 (signed row permutation of a Hadamard matrix, entries
+    +-1/8 exact in binary16) on bf16 rows with |x| in [1/8, 8): every product
+    is a multiple of 2^-13 and their magnitudes sum below 2^11, so every order
+    of fp32 accumulation is exact.  The oracle returns a zero bound and z
+    equals the sequential, reversed and pairwise fp32 sums bit for bit; a
+    random orthogonal U on the same rows gets a positive bound."""
+    rng = np.random.default_rng(7)
+    D = 128
+    perm = rng.permutation(D)
+    sign = rng.choice([-1.0, 1.0], D)
+    u = (sign[:, None] * scipy.linalg.hadamard(D)[perm] / 8).astype(np.float16)
+    x = _narrow_range_rows(rng, 4, D)
+    z, bound = oracle_mod.rotate_dense(u.view(np.uint16), x)
+    assert np.all(bound == 0.0)
+    lo, hi, mid = oracle_mod.f32_box(z, bound)          # boxes of one point
+    assert np.array_equal(lo, mid) and np.array_equal(hi, mid)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    prods = u.astype(np.float32)[None, :, :] * xf[:, None, :]
+    seq = np.zeros((4, D), np.float32)
+    rev = np.zeros((4, D), np.float32)
+    for j in range(D):
+        seq = (seq + prods[:, :, j]).astype(np.float32)
+        rev = (rev + prods[:, :, D - 1 - j]).astype(np.float32)
+    np.testing.assert_array_equal(seq.astype(np.float64), z)
+    np.testing.assert_array_equal(rev.astype(np.float64), z)
+    q, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    _, b2 = oracle_mod.rotate_dense(q.astype(np.float16).view(np.uint16), x)
+    assert np.all(b2 > 0.0)
 
 
 @pytest.mark.parametrize("policy", ["last", "next"])
