@@ -155,10 +155,24 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 constexpr int kDenseLaneFloats = 34;
 constexpr int kDenseTileBytes = (kQuantThreads) * kDenseLaneFloats * 4;
 
+// A CTA's copy of one head's matrix in shared memory: rows of 128 binary16
+// padded to 136 (272 bytes), so the four 16-byte loads of a quarter-warp
+// (two U rows, four lanes) fall in at most two wavefronts.
+constexpr int kUshStride = 136;
+constexpr int kUshBytes = 128 * kUshStride * 2;
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+  return r;
+}
+
 template <int D>
 __device__ __forceinline__ void rotate_dense(const uint4 (&q)[4], bool active, int lane, int head,
                                              const uint16_t* urot, float* tile,
-                                             float2 (&v)[16]) {
+                                             float2 (&v)[16], uint32_t ush = 0u,
+                                             int ush_head = -1) {
   static_assert(D == 128, "the dense rotation is built for head_dim 128");
   const int g = lane >> 2, t = lane & 3;
   uint32_t a[16];
@@ -173,6 +187,23 @@ __device__ __forceinline__ void rotate_dense(const uint4 (&q)[4], bool active, i
     const int h = __shfl_sync(0xffffffffu, head, __ffs(todo) - 1);
     const bool mine = active && head == h;
     todo &= ~__ballot_sync(0xffffffffu, mine);
+    if (h == ush_head) {
+      // the CTA's shared copy of this head's matrix
+      const uint32_t ub = ush + ((32 * (g >> 1) + (g & 1)) * kUshStride + 32 * t) * 2;
+#pragma unroll 2
+      for (int nt = 0; nt < 16; ++nt) {
+        const uint32_t un = ub + nt * 2 * kUshStride * 2;
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 bw = lds128(un + 16 * i);
+          mma_16816(d, a[4 * i], a[4 * i + 1], bw.x, bw.y);
+          mma_16816(d, a[4 * i + 2], a[4 * i + 3], bw.z, bw.w);
+        }
+        if (mine) *reinterpret_cast<float2*>(tile + 2 * nt) = make_float2(d[0], d[1]);
+      }
+      continue;
+    }
     // U row of n-tile nt for this lane: 64 bytes; the next tile's row is
     // loaded while the current one's products run
     const uint4* up = reinterpret_cast<const uint4*>(
@@ -769,11 +800,22 @@ __device__ __forceinline__ void quantize_comp(const Comp& c, int64_t row, int64_
 // Z^_r = fma(alpha~_r, Z^_ref, D(c_r)) after loop r.  The anchor is read
 // once and never re-read from the cache; the arithmetic (and so every
 // stored bit) is that of the per-loop kernels.
+// The fused kernel's dense instantiation keeps two ring slots per warp and a
+// CTA copy of the current head's matrix.
+template <bool DENSE>
+constexpr int loops_stages() { return DENSE ? 2 : kQStages; }
+template <bool DENSE>
+constexpr int loops_smem() {
+  return (kQuantThreads / 32) * loops_stages<DENSE>() * kQSlotBytes +
+         (DENSE ? kDenseTileBytes + kUshBytes : 0);
+}
+
 template <int D, bool CHAINED, bool DENSE>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quantize_loops_kernel(const __grid_constant__ QuantLoopsParams p) {
   constexpr int P = D / 32;
   constexpr int RPW = 32 / P;
+  constexpr int NS = loops_stages<DENSE>();
   static_assert(RPW * D * 2 == kQSlotBytes, "a slot holds one job of RPW rows");
   extern __shared__ __align__(128) unsigned char qsmem[];
   const int side = blockIdx.y;
@@ -787,7 +829,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                        (threadIdx.x >> 5);
   const int a = p.anchor;
   const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(qsmem)) +
-                        (threadIdx.x >> 5) * (kQStages * kQSlotBytes);
+                        (threadIdx.x >> 5) * (NS * kQSlotBytes);
   // Job j of this warp: rows base_j .. base_j + RPW - 1 of loop li_j (li 0 is
   // the anchor, li k >= 1 is p.order[k - 1]); jobs run row group by row
   // group, every loop of a group in turn.
@@ -807,31 +849,60 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
       is_li = 0;
       is_base += nwarps * RPW;
     }
-    is_slot = is_slot + 1 == kQStages ? 0 : is_slot + 1;
+    is_slot = is_slot + 1 == NS ? 0 : is_slot + 1;
   };
 #pragma unroll
-  for (int s = 0; s + 1 < kQStages; ++s) issue_next();
+  for (int s = 0; s + 1 < NS; ++s) issue_next();
   int slot = 0;
   // the job in `slot` has landed (this lane's copies, then the warp's); the
   // slot read in the previous job is free again and takes the next issue
+  // dense: the CTA's shared matrix (head ush_head, -1 when the CTA's rows of
+  // this pass span several heads)
+  const uint32_t ush = static_cast<uint32_t>(__cvta_generic_to_shared(qsmem)) +
+                       (kQuantThreads / 32) * NS * kQSlotBytes + (DENSE ? kDenseTileBytes : 0);
+  int ush_head = -1;
   auto next_input = [&](bool active, int head, float2 (&v)[16]) {
-    cp_async_wait<kQStages - 2>();
+    cp_async_wait<NS - 2>();
     __syncwarp();
     issue_next();
     uint4 q[4];
     read_slot<D>(ring + slot * kQSlotBytes, lane, q);
-    slot = slot + 1 == kQStages ? 0 : slot + 1;
+    slot = slot + 1 == NS ? 0 : slot + 1;
     if constexpr (DENSE)
       rotate_dense<D>(q, active, lane, head, p.urot[side],
-                      reinterpret_cast<float*>(qsmem + (kQuantThreads / 32) * kQStages *
+                      reinterpret_cast<float*>(qsmem + (kQuantThreads / 32) * NS *
                                                            kQSlotBytes) +
                           threadIdx.x * kDenseLaneFloats,
-                      v);
+                      v, ush, ush_head);
     else
       rotate_pieces<D>(q, active, slice, p.rot_scale, v);
   };
   const bool narrow = total <= 0xFFFFFFFFll;
-  for (int64_t base = warp * RPW; base < total; base += nwarps * RPW) {
+  // CTA-uniform passes: every warp of the CTA takes part in each pass (its
+  // rows may lie past the end), so the dense form can share one matrix
+  constexpr int64_t kCtaRows = (kQuantThreads / 32) * RPW;
+  for (int64_t cbase = static_cast<int64_t>(blockIdx.x) * kCtaRows; cbase < total;
+       cbase += nwarps * RPW) {
+    const int64_t base = cbase + (threadIdx.x >> 5) * RPW;
+    if constexpr (DENSE) {
+      __syncthreads();   // the previous pass is done with the shared matrix
+      const int64_t last = (cbase + kCtaRows < total ? cbase + kCtaRows : total) - 1;
+      const int64_t b0 = cbase / p.n, b1 = last / p.n;
+      ush_head = b0 == b1 ? static_cast<int>(b0 % p.heads) : -1;
+      if (ush_head >= 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.urot[side] + static_cast<size_t>(ush_head) * D * D);
+        for (int c = threadIdx.x; c < D * D / 8; c += kQuantThreads) {
+          const uint4 w = __ldg(src + c);
+          const uint32_t dst = ush + ((c >> 4) * kUshStride + (c & 15) * 8) * 2;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w.x),
+                       "r"(w.y), "r"(w.z), "r"(w.w)
+                       : "memory");
+        }
+      }
+      __syncthreads();
+    }
+    if (base >= total) continue;
     const int64_t row = base + lane / P;
     const bool active = row < total;
     int64_t bhi, tn;
@@ -990,7 +1061,7 @@ cudaError_t launch_quantize(const QuantParams& p, int D, int bits, int group,
 
 template <int D, bool CHAINED, bool DENSE>
 cudaError_t launch_loops_t(const QuantLoopsParams& p, dim3 grid, cudaStream_t s) {
-  constexpr int smem = (kQuantThreads / 32) * kQStages * kQSlotBytes + (DENSE ? kDenseTileBytes : 0);
+  constexpr int smem = loops_smem<DENSE>();
   const cudaError_t e = cudaFuncSetAttribute(quantize_loops_kernel<D, CHAINED, DENSE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
