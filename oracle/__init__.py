@@ -518,19 +518,21 @@ def quantize_box(lo: np.ndarray, hi: np.ndarray, mid: np.ndarray, bits: int, gro
 
 def encode_side_dense(x: np.ndarray, u: np.ndarray, heads: int, tokens: int,
                       bits: Sequence[int], group: Sequence[int], policy: str = POLICY_LAST,
-                      unit_alpha: bool = False,
-                      mu: Optional[np.ndarray] = None) -> List[Dict[str, np.ndarray]]:
+                      unit_alpha: bool = False, mu: Optional[np.ndarray] = None,
+                      meta16: bool = False) -> List[Dict[str, np.ndarray]]:
     """encode_side with the dense rotation of one (layer, K|V) side
     [RQ §3.3, App. G.2]: u binary16 bits [heads, D, D], one matrix per head
     shared by every loop; rows of x [L, N, D] are (b, h, t) with `tokens` rows
-    per (b, h).  Binary16 metadata.
+    per (b, h); mu as in encode_side.
 
     The accumulation order of the rotation is not fixed by the pages, so the
     encoder works on the box of fp32 rows that any order can produce
     (rotate_dense's bound): 'codes', 'meta', 'alpha', 'zhat' are those of the
     fp32-rounded exact rotation, and 'code_ok', 'meta_ok', 'alpha_ok' mark the
     decisions that every row of the box shares (a row whose reference is not
-    fully determined gets no flag)."""
+    fully determined gets no flag).  The interval form covers binary16
+    metadata; with meta16 (16-bit metadata, R22) every rotation must be exact
+    (boxes of one point), and the point encoders give the one answer."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     L, N, D = x.shape
     _check_dim(D)
@@ -546,6 +548,8 @@ def encode_side_dense(x: np.ndarray, u: np.ndarray, heads: int, tokens: int,
             zh, bh = rotate_dense(u[h], x[l][rows])
             z[rows], bd[rows] = zh, bh
         boxes.append(f32_box(z, bd))
+    if meta16:
+        return _encode_points_m8(boxes, bits, group, policy, unit_alpha, mu)
     out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
     a = anchor_loop(L, policy)
     lo, hi, mid = boxes[a]
@@ -577,6 +581,43 @@ def encode_side_dense(x: np.ndarray, u: np.ndarray, heads: int, tokens: int,
         enc["clean"] = enc["alpha_ok"] & enc["meta_ok"].all(axis=1) & enc["code_ok"].all(axis=1)
         out[r] = enc
     return out  # type: ignore[return-value]
+
+
+def _encode_points_m8(boxes, bits, group, policy, unit_alpha, mu):
+    """encode_side_dense with 16-bit metadata on exact rotations."""
+    L = len(boxes)
+    for lo, hi, mid in boxes:
+        if not (np.array_equal(lo, mid) and np.array_equal(hi, mid)):
+            raise ValueError("16-bit metadata with a dense rotation needs exact sums")
+    N, D = boxes[0][2].shape
+    out: List[Optional[Dict[str, np.ndarray]]] = [None] * L
+    a = anchor_loop(L, policy)
+    z = boxes[a][2]
+    enc = {"codes": np.zeros((N, D * bits[a] // 32), np.uint32),
+           "meta": np.zeros((N, D // group[a]), np.uint16), "alpha": None,
+           "zhat": np.zeros((N, D), np.float32)}
+    for n in range(N):
+        enc["codes"][n], enc["meta"][n], enc["zhat"][n] = quantize_m8(z[n], bits[a], group[a])
+    out[a] = enc
+    for r in encode_order(L, policy):
+        ref = out[reference_loop(L, r, policy)]["zhat"]
+        z = boxes[r][2]
+        enc = {"codes": np.zeros((N, D * bits[r] // 32), np.uint32),
+               "meta": np.zeros((N, D // group[r]), np.uint16),
+               "alpha": np.zeros(N, np.uint16), "zhat": np.zeros((N, D), np.float32)}
+        for n in range(N):
+            m = None if mu is None else mu[r][n]
+            w_, m_, al, zh = encode_residual_rot_ex(z[n], ref[n], m, bits[r], group[r],
+                                                    unit_alpha, meta16=True)
+            enc["codes"][n], enc["meta"][n], enc["alpha"][n], enc["zhat"][n] = w_, m_, al, zh
+        out[r] = enc
+    for l in range(L):
+        e = out[l]
+        e["code_ok"] = np.ones((N, D), bool)
+        e["meta_ok"] = np.ones(e["meta"].shape, bool)
+        e["alpha_ok"] = None if e["alpha"] is None else np.ones(N, bool)
+        e["clean"] = np.ones(N, bool)
+    return out
 
 
 def f16_bits_to_f64(a: np.ndarray) -> np.ndarray:

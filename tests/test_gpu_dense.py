@@ -63,14 +63,18 @@ class Case:
     """A one-layer cache built through the ABI from host rows x[side] (bf16
     bits [L, B, H, T, D]) with rotations rot[side] (None: Hadamard)."""
 
-    def __init__(self, w, x, rot, policy="last", fused=True):
+    def __init__(self, w, x, rot, policy="last", fused=True, meta16=False, means=None):
         self.w, self.x, self.rot, self.policy = w, x, rot, policy
-        self.lay = layout_of(w, policy, layers=1)
+        self.meta16, self.means = meta16, means
+        self.lay = layout_of(w, policy, layers=1, meta16=meta16)
         nb = L.rq_cache_bytes(self.lay)
         self.kbuf = torch.empty(nb, dtype=torch.uint8, device="cuda")
         self.vbuf = torch.empty(nb, dtype=torch.uint8, device="cuda")
         self.cache = L.rq_cache_bind(self.lay, self.kbuf, self.vbuf)
         L.rq_cache_set_rotations(self.cache, *(None if rot[s] is None else rot[s][0] for s in SIDES))
+        if means is not None:
+            self.means_dev = {sd: torch.from_numpy(means[sd]).to("cuda") for sd in SIDES}
+            L.rq_cache_set_means(self.cache, self.means_dev[0], self.means_dev[1])
         dev = {s: torch.from_numpy(x[s].view(np.int16)).to("cuda") for s in SIDES}
         T = w.tokens
         if fused:
@@ -86,17 +90,28 @@ class Case:
                         L.rq_quantize_append_residual(self.cache, 0, side, loop, xl, 0, T)
         torch.cuda.synchronize()
         self.gc = type("G", (), {"cache": self.cache, "w": w, "kbuf": self.kbuf,
-                                 "vbuf": self.vbuf, "meta16": False, "policy": policy})
+                                 "vbuf": self.vbuf, "meta16": meta16, "policy": policy})
 
     def rows(self, side):
         return self.x[side].reshape(self.w.loops, -1, D)
 
+    def mu_rows(self, side):
+        """The fixed means of one side expanded to the oracle's rows [L, N, D]."""
+        if self.means is None:
+            return None
+        w = self.w
+        m = self.means[side][0]                                  # [L, H, D]
+        return np.ascontiguousarray(np.stack(
+            [np.repeat(np.tile(m[l], (w.batch, 1)), w.tokens, axis=0) for l in range(w.loops)]))
+
     def encode(self, side):
         w = self.w
         if self.rot[side] is None:
-            return oracle.encode_side(self.rows(side), w.bits, w.group, self.policy)
+            return oracle.encode_side(self.rows(side), w.bits, w.group, self.policy,
+                                      meta16=self.meta16, mu=self.mu_rows(side))
         return oracle.encode_side_dense(self.rows(side), self.rot[side][1][0], w.heads, w.tokens,
-                                        w.bits, w.group, self.policy)
+                                        w.bits, w.group, self.policy, mu=self.mu_rows(side),
+                                        meta16=self.meta16)
 
 
 def _narrow_rows(rng, w):
@@ -199,7 +214,8 @@ def _decode_case(case, loop, seq):
     L.rq_decode_attention(case.cache, 0, loop, q, sl, T, kc, vc, 0.0, out, ws.buf, ws.bytes)
     torch.cuda.synchronize()
     assert L.rq_workspace_error(ws.buf, ws.bytes) == L.RQ_OK
-    z = {s: oracle.reconstruct_rotated(case.encode(s), loop, w.bits, w.group, case.policy)
+    z = {s: oracle.reconstruct_rotated(case.encode(s), loop, w.bits, w.group, case.policy,
+                                       case.mu_rows(s))
          .reshape(w.batch, w.heads, w.tokens, D) for s in SIDES}
     ref = oracle.decode_attention_dense(z[0], z[1], synth.bits_of(q.cpu()).reshape(w.batch, w.heads, D),
                                         seq, synth.bits_of(kc.cpu()), synth.bits_of(vc.cpu()),
@@ -221,6 +237,26 @@ def test_dense_decode_matches_oracle(cuda_dev, policy, groups):
     for loop in range(w.loops):
         out, ref = _decode_case(case, loop, [400, 177])
         assert np.max(np.abs(out - ref)) <= attn_tolerance(ref), loop
+
+
+@pytest.mark.parametrize("policy", ["last", "next"])
+def test_dense_meta16_and_means_exact(cuda_dev, policy):
+    """Dense rotations with 16-bit metadata, and with fixed means (multiples of
+    1/64, so the mean's subtraction is exact too): codes, metadata and LS
+    coefficients bit for bit, decode within tolerance."""
+    rng = np.random.default_rng(27)
+    w = synth.WORKLOADS["ouro_layer"].replace(batch=2, heads=3, tokens=160)
+    x = {s: _narrow_rows(rng, w) for s in SIDES}
+    rot = {s: _rot(_perm_hadamard_f16(rng, w.heads), 1, w.heads) for s in SIDES}
+    means = {s: (rng.integers(-64, 64, (1, w.loops, w.heads, D)) / 64).astype(np.float32)
+             for s in SIDES}
+    for meta16, mu in ((True, None), (False, means)):
+        case = Case(w, x, rot, policy, fused=True, meta16=meta16, means=mu)
+        for side in SIDES:
+            _assert_exact(case, side, case.encode(side))
+        for loop in range(w.loops):
+            out, ref = _decode_case(case, loop, [160, 97])
+            assert np.max(np.abs(out - ref)) <= attn_tolerance(ref), (meta16, loop)
 
 
 def test_dense_dequantize_is_u_transpose_z(cuda_dev):

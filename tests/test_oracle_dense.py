@@ -113,10 +113,12 @@ def test_dense_exact_sums_have_zero_bound(oracle_mod):
 
 
 @pytest.mark.parametrize("policy", ["last", "next"])
-def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy):
+@pytest.mark.parametrize("meta16", [False, True])
+def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy, meta16):
     """U = H_64 / 8 (exact in binary16), on rows whose Hadamard sums are exact
     in any order: the dense encoder's codes, metadata and LS coefficients equal
-    the Sylvester-Hadamard (FWHT) encoder's bit for bit."""
+    the Sylvester-Hadamard (FWHT) encoder's bit for bit, with either metadata
+    form, and every decision is certified."""
     rng = np.random.default_rng(3)
     D, L, H, T = 64, 4, 2, 40
     xa = _narrow_range_rows(rng, H * T, D)
@@ -128,16 +130,21 @@ def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy):
                   for a in (0.8, 1.1, 0.9)] + [xa])
     u = np.stack([_hadamard_f16(D)] * H)
     bits, group = (2, 2, 2, 4), (32, 32, 32, 32)
-    want = oracle_mod.encode_side(x, bits, group, policy)
-    got = oracle_mod.encode_side_dense(x, u, H, T, bits, group, policy)
+    want = oracle_mod.encode_side(x, bits, group, policy, meta16=meta16)
+    got = oracle_mod.encode_side_dense(x, u, H, T, bits, group, policy, meta16=meta16)
     for l in range(L):
         np.testing.assert_array_equal(got[l]["codes"], want[l]["codes"])
         np.testing.assert_array_equal(got[l]["meta"], want[l]["meta"])
         if want[l]["alpha"] is not None:
             np.testing.assert_array_equal(got[l]["alpha"], want[l]["alpha"])
-    # the interval encoder still certifies most of the anchor's decisions at
-    # the order-free accumulation bound
-    assert got[3]["code_ok"].mean() > 0.8 and got[3]["meta_ok"].mean() > 0.8
+    # every sum here is exact in any order: every decision is certified
+    for l in range(L):
+        assert got[l]["clean"].all(), l
+    if meta16:   # 16-bit metadata needs exact sums
+        q, _ = np.linalg.qr(rng.standard_normal((D, D)))
+        uq = np.stack([q.astype(np.float16).view(np.uint16)] * H)
+        with pytest.raises(ValueError):
+            oracle_mod.encode_side_dense(x, uq, H, T, bits, group, policy, meta16=True)
 
 
 def _box_samples(rng, lo, hi, k):
