@@ -241,7 +241,8 @@ __device__ __forceinline__ void rotate_dense(const uint4 (&q)[4], bool active, i
 // rows of one loop: 8 rows of 128 channels or 16 rows of 64), filled by
 // 16-byte cp.async copies kQStages - 1 jobs ahead of the job being
 // quantised, so every warp keeps about 6 KB of input in flight without
-// holding it in registers.  A copy instruction covers 512 contiguous bytes
+// holding it in registers (the dense-rotation instantiation keeps two slots,
+// to leave room for its shared matrix).  A copy instruction covers 512 contiguous bytes
 // (lane l: bytes 16 l of each 512-byte quarter); piece pi of the slice
 // that lane l of the row reads lands at pi ^ ((l >> 1) & 3), so the four
 // 16-byte reads of a quarter-warp hit eight distinct bank groups.
