@@ -644,6 +644,9 @@ def main():
     ap.add_argument("--no-quant", action="store_true", help="skip the prefill quantise leg")
     ap.add_argument("--no-ablation", action="store_true",
                     help="skip the shared-vs-chained deep-recurrence decode ablation")
+    ap.add_argument("--only-dense", action="store_true",
+                    help="run only the dense-rotation leg on one 16k layer and print its numbers "
+                         "(profiling; --batch then sets its batch)")
     ap.add_argument("--only-quant", action="store_true",
                     help="run only the prefill quantise leg and print its numbers (profiling; "
                          "--batch then sets its batch)")
@@ -656,6 +659,13 @@ def main():
     dev = torch.device("cuda", local)
     from residual_bit_kv_b200 import build
     build.build()
+    if args.only_dense:
+        wd = synth.WORKLOADS[WORKLOAD].replace(layers=1)
+        if args.batch:
+            wd = wd.replace(batch=args.batch)
+        print(json.dumps({"dense_rotation": bench_dense(wd, dev, torch.cuda.current_stream(dev),
+                                                        args, peaks()[0])}))
+        return 0
     if args.only_quant:
         print(json.dumps({"quantize": bench_quantize(dev, torch.cuda.current_stream(dev), args,
                                                      peaks()[0])}))
@@ -973,8 +983,16 @@ def bench_ablation(dev, stream, args, hbm):
                          for l in range(wm.loops)]}
     m16["speedup_meta16_over_meta32"] = m16["meta32"]["ms_per_step"] / m16["meta16"]["ms_per_step"]
     out["metadata16_ouro_16k_layer"] = m16
-    # dense binary16 rotations (tensor-core product) against the Hadamard transform
-    dn = {"workload": m16["workload"],
+    out["dense_rotation_ouro_16k_layer"] = bench_dense(wm, dev, stream, args, hbm)
+    return out
+
+
+def bench_dense(wm, dev, stream, args, hbm):
+    """Dense binary16 rotations (tensor-core product) against the Hadamard
+    transform on one layer of workload wm: the decode step over every loop and
+    the fused prefill append of every loop, K and V."""
+    dn = {"workload": f"{wm.name}: 1 layer x {wm.loops} loops, batch {wm.batch}, {wm.heads} "
+                      f"heads, {wm.tokens} past tokens, bits {list(wm.bits)}, group {wm.group[0]}",
           "note": "random orthogonal binary16 matrices per head and side stand in for calibrated "
                   "rotations; prefill = fused append of every loop, K and V"}
     for name, flag in (("hadamard", False), ("dense", True)):
@@ -984,8 +1002,7 @@ def bench_ablation(dev, stream, args, hbm):
                     "decode_frac_of_hbm": byt / (ms * 1e-3) / 1e9 / hbm,
                     "prefill_ms": pms, "prefill_gbs": qb / (pms * 1e-3) / 1e9,
                     "prefill_frac_of_hbm": qb / (pms * 1e-3) / 1e9 / hbm}
-    out["dense_rotation_ouro_16k_layer"] = dn
-    return out
+    return dn
 
 
 def bench_quantize(dev, stream, args, hbm):
