@@ -21,6 +21,9 @@
  *   consecutive channels, s = (max - min)/(2^b - 1), s~ = fp16(s),
  *   z~ = fp16(min), code = rint_even(clamp((z - z~) * (1/s~), 0, 2^b - 1)).
  *   Reconstruction: Z^_r = alpha~_r R + s~ c + z~ and X^_r = H^T Z^_r.
+ *   With fixed means (rq_cache_set_means) a residual loop stores the codes
+ *   of Z_r - mu_r - alpha~ R and adds mu_r back; with dense rotations
+ *   (rq_cache_set_rotations) Z = U x replaces H x and X^ = U^T Z^.
  *
  * Storage contract (per layer and per side K | V):
  *   Tokens are stored in records of RQ_BLOCK_TOKENS = 32 consecutive tokens.
