@@ -519,32 +519,33 @@ void rqo_attention_f64(const double* q, const double* khat, const double* vhat,
  *   bound_i = D 2^-23 sum_j |U_ij x_j|  (+ the fp64 sum's own D 2^-53 share),
  * twice the textbook (D - 1) 2^-24, which also covers adders that truncate;
  * the bound is 0 when every partial sum is exact in any order (below). */
-/* Exponent of the lowest set bit of a nonzero double. */
-static int low_bit_exponent(double t) {
-  int e;
-  const double m = frexp(fabs(t), &e);          /* |t| = m 2^e, m in [1/2, 1) */
-  uint64_t M = (uint64_t)ldexp(m, 53);           /* exact: 53-bit integer */
-  int k = 0;
-  while ((M & 1u) == 0u) {
-    M >>= 1;
-    ++k;
-  }
-  return e - 53 + k;
+/* Exponent of the lowest set bit of a nonzero binary16 value (from its bits):
+ * a normal value is (1024 + m) 2^(e - 25), a subnormal one m 2^-24. */
+static int f16_low_bit(uint16_t h) {
+  const int e = (h >> 10) & 0x1F, m = h & 0x3FF;
+  return e == 0 ? -24 + __builtin_ctz((unsigned)m) : e - 25 + __builtin_ctz((unsigned)(m | 1024));
 }
 
-void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z,
-                          double* bound) {
+/* One row against a matrix already decoded: ud[i*D + j] = U_ij as a double,
+ * ulow[i*D + j] = the exponent of its lowest set bit. */
+static void rotate_dense_decoded(const double* ud, const int* ulow, const uint16_t* x, int D,
+                                 double* z, double* bound) {
   double xh[256];
-  for (int j = 0; j < D; ++j) xh[j] = rqo_f16_to_f32(rqo_f32_to_f16(rqo_bf16_to_f32(x[j])));
+  int xlow[256];
+  for (int j = 0; j < D; ++j) {
+    const uint16_t hb = rqo_f32_to_f16(rqo_bf16_to_f32(x[j]));
+    xh[j] = rqo_f16_to_f32(hb);
+    xlow[j] = (hb & 0x7FFF) ? f16_low_bit(hb) : 0;
+  }
   for (int i = 0; i < D; ++i) {
     double acc = 0.0, mag = 0.0;
     int emin = 1 << 20;
     for (int j = 0; j < D; ++j) {
-      const double t = (double)rqo_f16_to_f32(u[(size_t)i * D + j]) * xh[j];
+      const double t = ud[(size_t)i * D + j] * xh[j];
       acc += t;
       mag += fabs(t);
-      if (t != 0.0) {
-        const int e = low_bit_exponent(t);
+      if (t != 0.0) {   /* the product's lowest bit: the sum of its factors' */
+        const int e = ulow[(size_t)i * D + j] + xlow[j];
         if (e < emin) emin = e;
       }
     }
@@ -559,10 +560,27 @@ void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z
   }
 }
 
+static void decode_matrix(const uint16_t* u, int D, double* ud, int* ulow) {
+  for (int k = 0; k < D * D; ++k) {
+    ud[k] = rqo_f16_to_f32(u[k]);
+    ulow[k] = (u[k] & 0x7FFF) ? f16_low_bit(u[k]) : 0;
+  }
+}
+
+void rqo_rotate_dense_row(const uint16_t* u, const uint16_t* x, int D, double* z,
+                          double* bound) {
+  rqo_rotate_dense_rows(u, x, 1, D, z, bound);
+}
+
 void rqo_rotate_dense_rows(const uint16_t* u, const uint16_t* x, int64_t n, int D,
                            double* z, double* bound) {
+  double* ud = (double*)malloc(sizeof(double) * (size_t)D * D);
+  int* ulow = (int*)malloc(sizeof(int) * (size_t)D * D);
+  decode_matrix(u, D, ud, ulow);
   for (int64_t r = 0; r < n; ++r)
-    rqo_rotate_dense_row(u, x + r * D, D, z + r * D, bound + r * D);
+    rotate_dense_decoded(ud, ulow, x + r * D, D, z + r * D, bound + r * D);
+  free(ud);
+  free(ulow);
 }
 
 /* Interval form of rqo_quantize for a row known only to lie in the box
