@@ -113,12 +113,13 @@ def test_dense_exact_sums_have_zero_bound(oracle_mod):
 
 
 @pytest.mark.parametrize("policy", ["last", "next"])
-@pytest.mark.parametrize("meta16", [False, True])
-def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy, meta16):
+@pytest.mark.parametrize("meta16,means", [(False, False), (True, False), (False, True),
+                                          (True, True)])
+def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy, meta16, means):
     """U = H_64 / 8 (exact in binary16), on rows whose Hadamard sums are exact
     in any order: the dense encoder's codes, metadata and LS coefficients equal
     the Sylvester-Hadamard (FWHT) encoder's bit for bit, with either metadata
-    form, and every decision is certified."""
+    form and with or without fixed means, and every decision is certified."""
     rng = np.random.default_rng(3)
     D, L, H, T = 64, 4, 2, 40
     xa = _narrow_range_rows(rng, H * T, D)
@@ -130,8 +131,11 @@ def test_dense_hadamard_reproduces_fwht_path_bit_for_bit(oracle_mod, policy, met
                   for a in (0.8, 1.1, 0.9)] + [xa])
     u = np.stack([_hadamard_f16(D)] * H)
     bits, group = (2, 2, 2, 4), (32, 32, 32, 32)
-    want = oracle_mod.encode_side(x, bits, group, policy, meta16=meta16)
-    got = oracle_mod.encode_side_dense(x, u, H, T, bits, group, policy, meta16=meta16)
+    mu = None
+    if means:   # fixed means on a 1/64 grid: their subtraction is exact as well
+        mu = (rng.integers(-64, 64, (L, H * T, D)) / 64).astype(np.float32)
+    want = oracle_mod.encode_side(x, bits, group, policy, meta16=meta16, mu=mu)
+    got = oracle_mod.encode_side_dense(x, u, H, T, bits, group, policy, meta16=meta16, mu=mu)
     for l in range(L):
         np.testing.assert_array_equal(got[l]["codes"], want[l]["codes"])
         np.testing.assert_array_equal(got[l]["meta"], want[l]["meta"])
