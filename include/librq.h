@@ -315,6 +315,17 @@ rq_status rq_selftest_wait_timeout(void* workspace, uint64_t ws_bytes, int32_t l
  * the current device (for tests and benchmarks). */
 int32_t rq_decode_splits(const rq_layout* layout, int32_t max_seq_len);
 
+/* The split plan alone, for a device with `sms` multiprocessors running
+ * `ctas_per_sm` decode CTAs each (host logic, no device access; tests):
+ * `rows` = batch * kv_heads units, 64-token chunks.  *splits >= 1 partitions of
+ * *chunks_per_split chunks each, none empty, at most one per chunk (and at most
+ * the workspace's bound); the count fills every resident slot at least once
+ * when the sequence is long enough and minimises (waves of resident CTAs) x
+ * (chunks per CTA + a fixed per-CTA cost).  RQ_ERR_INVALID_ARG for rows,
+ * ctas_per_sm or sms below 1, a negative length or NULL outputs. */
+rq_status rq_plan_splits(int32_t rows, int32_t max_seq_len, int32_t ctas_per_sm, int32_t sms,
+                         int32_t* splits, int32_t* chunks_per_split);
+
 /* rq_decode_attention for callers that cannot allocate device memory -- code
  * embedded in a host framework that owns every allocation, or a serving loop
  * that may not call cudaMalloc -- and so cannot provide a workspace.  The

@@ -96,15 +96,24 @@ int max_splits_of(int32_t max_seq_len) {
 // the count that fills every resident slot once, so a small batch still
 // occupies the whole GPU.  Splits never exceed max_splits_of() (the
 // workspace bound) and never leave an empty split.
+void choose_splits_on(int bh, int32_t max_seq_len, int chunk, int ctas_per_sm, int sms,
+                      int* splits, int* cps);
+
 void choose_splits(int bh, int32_t max_seq_len, int chunk, int ctas_per_sm, int* splits,
                    int* cps) {
+  choose_splits_on(bh, max_seq_len, chunk, ctas_per_sm, device_sms(), splits, cps);
+}
+
+// The plan for a device with `sms` multiprocessors (host logic only).
+void choose_splits_on(int bh, int32_t max_seq_len, int chunk, int ctas_per_sm, int sms,
+                      int* splits, int* cps) {
   const int chunks = (max_seq_len + chunk - 1) / chunk;
   if (chunks == 0) {
     *splits = 1;
     *cps = 0;
     return;
   }
-  const int64_t slots = static_cast<int64_t>(device_sms()) * (ctas_per_sm > 0 ? ctas_per_sm : 1);
+  const int64_t slots = static_cast<int64_t>(sms > 0 ? sms : 1) * (ctas_per_sm > 0 ? ctas_per_sm : 1);
   int smax = max_splits_of(max_seq_len);
   if (smax > chunks) smax = chunks;
   int smin = static_cast<int>((slots + bh - 1) / bh);
@@ -498,6 +507,18 @@ int32_t rq_decode_splits(const rq_layout* l, int32_t max_seq_len) {
   const int far = anchor_of(l) == 0 ? l->num_loops - 1 : 0;
   if (fill_decode_params(&c, 0, far, max_seq_len, &p, &D) != RQ_OK) return 0;
   return p.splits;
+}
+
+rq_status rq_plan_splits(int32_t rows, int32_t max_seq_len, int32_t ctas_per_sm, int32_t sms,
+                         int32_t* splits, int32_t* chunks_per_split) {
+  if (rows < 1 || max_seq_len < 0 || ctas_per_sm < 1 || sms < 1 || splits == nullptr ||
+      chunks_per_split == nullptr)
+    return RQ_ERR_INVALID_ARG;
+  int s = 0, c = 0;
+  choose_splits_on(rows, max_seq_len, kChunk, ctas_per_sm, sms, &s, &c);
+  *splits = s;
+  *chunks_per_split = c;
+  return RQ_OK;
 }
 
 rq_status rq_decode_attention(const rq_cache* c, int32_t layer, int32_t loop, const void* q,

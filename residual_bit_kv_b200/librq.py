@@ -39,7 +39,7 @@ SYMBOLS = (
     "rq_decode_attention", "rq_decode_bf16_workspace_bytes", "rq_decode_attention_bf16",
     "rq_workspace_error", "rq_decode_splits", "rq_decode_attention_noalloc",
     "rq_quantize_append_loops", "rq_selftest_wait_timeout", "rq_cache_set_means",
-    "rq_cache_set_rotations",
+    "rq_cache_set_rotations", "rq_plan_splits",
 )
 
 
@@ -98,6 +98,9 @@ def load() -> ctypes.CDLL:
         "rq_cache_bind": ([LP, _P, _P, CP], ctypes.c_int),
         "rq_cache_set_means": ([CP, _P, _P], ctypes.c_int),
         "rq_cache_set_rotations": ([CP, _P, _P], ctypes.c_int),
+        "rq_plan_splits": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)],
+                           ctypes.c_int),
         "rq_quantize_anchor": ([CP, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_residual": ([CP, _I32, _I32, _I32, _P, _I32, _I32, _P], ctypes.c_int),
         "rq_quantize_append_loops": ([CP, _I32, _P, _P, _I32, _I32, _P], ctypes.c_int),
@@ -264,6 +267,16 @@ def rq_decode_attention_bf16(batch: int, heads: int, head_dim: int, q, k, v, tok
                                            token_stride, _ptr(seq_lens), max_seq_len, _ptr(k_cur),
                                            _ptr(v_cur), softmax_scale, _ptr(out), _ptr(workspace),
                                            ws_bytes, _stream(stream)), "rq_decode_attention_bf16")
+
+
+def rq_plan_splits(rows: int, max_seq_len: int, ctas_per_sm: int, sms: int):
+    """(splits, chunks_per_split) of the decode split plan for a device with
+    `sms` multiprocessors (host logic only)."""
+    s = ctypes.c_int32()
+    c = ctypes.c_int32()
+    _check(load().rq_plan_splits(rows, max_seq_len, ctas_per_sm, sms, ctypes.byref(s),
+                                 ctypes.byref(c)), "rq_plan_splits")
+    return s.value, c.value
 
 
 def rq_workspace_error(workspace, ws_bytes: int, stream=None) -> int:

@@ -203,6 +203,36 @@ def test_rotation_setter_checks(L):
     assert e.value.status == L.RQ_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("sms,ctas", [(148, 5), (148, 6), (132, 4), (1, 1)])
+def test_split_plan_host_logic(L, sms, ctas):
+    """The decode split plan (host logic, no device): at least one split, none
+    empty, no more than one per 64-token chunk or the 1024 the counters hold,
+    and every resident CTA slot filled once when the sequence allows it."""
+    for rows in (1, 3, 16, 128, 256, 1280, 40960):
+        for T in (0, 1, 63, 64, 65, 777, 4096, 16384, 65536, 1 << 20):
+            s, cps = L.rq_plan_splits(rows, T, ctas, sms)
+            chunks = (T + 63) // 64
+            assert 1 <= s <= max(1, min(chunks, 1024)), (rows, T, s)
+            if chunks:
+                assert -(-chunks // cps) == s, (rows, T, s, cps)     # no empty split
+                assert s * cps >= chunks and (s - 1) * cps < chunks
+                want = min(-(-(sms * ctas) // rows), chunks, 1024)
+                assert s >= want, (rows, T, s, want)
+            else:
+                assert (s, cps) == (1, 0)
+
+
+def test_split_plan_matches_the_measured_launches(L):
+    """The plans the benchmark's launches showed on a 148-SM B200 at five
+    CTAs per SM: 8 splits for 256 rows and 11 for 128 rows at 16384 tokens."""
+    assert L.rq_plan_splits(256, 16384, 5, 148) == (8, 32)
+    assert L.rq_plan_splits(128, 16384, 5, 148) == (11, 24)
+    for args in [(0, 100, 5, 148), (4, -1, 5, 148), (4, 100, 0, 148), (4, 100, 5, 0)]:
+        with pytest.raises(L.RQError) as e:
+            L.rq_plan_splits(*args)
+        assert e.value.status == L.RQ_ERR_INVALID_ARG
+
+
 def test_no_cpu_fallback_in_product():
     """The product package never imports the oracle."""
     pkg = os.path.join(ROOT, "residual_bit_kv_b200")
