@@ -233,6 +233,33 @@ def test_split_plan_matches_the_measured_launches(L):
         assert e.value.status == L.RQ_ERR_INVALID_ARG
 
 
+def test_workspace_holds_every_split_plan(L):
+    """The decode workspace holds the error word, one counter per (batch, head)
+    and the partials (m, l, acc[D]) of the largest split count any device's plan
+    can use (one split per 64-token chunk, at most 1024)."""
+    for batch, heads, D in ((1, 1, 128), (16, 16, 128), (3, 5, 64), (64, 40, 128)):
+        for T in (0, 1, 100, 4096, 16384, 1 << 17):
+            lay = L.make_layout(1, 4, batch, heads, D, max(T, 1), (2, 2, 2, 4), (32,) * 4)
+            rows = batch * heads
+            need = 256 + rows * 4 + rows * max(1, min((T + 63) // 64, 1024)) * (D + 2) * 4
+            assert L.rq_decode_workspace_bytes(lay, T) >= need, (batch, heads, D, T)
+            for sms, ctas in ((148, 5), (1, 1), (1000, 8)):
+                s, _ = L.rq_plan_splits(rows, T, ctas, sms)
+                assert 256 + rows * 4 + rows * s * (D + 2) * 4 <= L.rq_decode_workspace_bytes(lay, T)
+
+
+def test_means_setter_checks(L):
+    """rq_cache_set_means: NULL clears, pointers must be 16-byte aligned."""
+    cache = L.rq_cache_bind(_lay(L), 1 << 20, 1 << 30)
+    L.rq_cache_set_means(cache, 1 << 16, 1 << 17)
+    assert cache.k_means == 1 << 16 and cache.v_means == 1 << 17
+    L.rq_cache_set_means(cache, None, None)
+    assert cache.k_means is None and cache.v_means is None
+    with pytest.raises(L.RQError) as e:
+        L.rq_cache_set_means(cache, (1 << 16) + 4, None)
+    assert e.value.status == L.RQ_ERR_INVALID_ARG
+
+
 def test_no_cpu_fallback_in_product():
     """The product package never imports the oracle."""
     pkg = os.path.join(ROOT, "residual_bit_kv_b200")
